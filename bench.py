@@ -1,0 +1,485 @@
+#!/usr/bin/env python
+"""Benchmark of the Muon optimizer step on B200.
+
+One step = one Muon step over every hidden 2-D weight of the workload (Nesterov
+momentum, Frobenius normalisation, 5 quintic Newton-Schulz iterations in bf16
+on tcgen05 tensor cores, shape scale, decoupled decay, update) plus the aux
+AdamW step over the non-2-D parameters, all through the C ABI of
+libmuon_b200.so.
+
+Default workload: the GPT-2-small hidden set (12 layers x Q, K, V, O 768x768,
+MLP 3072x768 and 768x3072 = 72 matrices, 85 M parameters), bf16 gradients
+N(0, 1e-3) drawn fresh for each of 10 steps and cycled, fp32 weights
+N(0, 0.02), momentum carried; aux AdamW over a GPT-2-small-sized set (token and
+position embeddings, layer-norm gains and biases, linear biases; 39.5 M
+parameters).
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+                    [--workload gpt2-small|llama3-8b|single-256|sweep-4096|...]
+
+Prints one JSON line (rank 0).  Multi-GPU (torchrun): every rank steps an
+independent replica of the workload (weak scaling, no data-path collective).
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as wl  # noqa: E402
+
+AUX_GPT2 = [("wte", 50257 * 768), ("wpe", 1024 * 768)] + \
+    [(f"h{l}.{n}", 768) for l in range(12) for n in ("ln1.g", "ln1.b", "ln2.g", "ln2.b",
+                                                     "attn.proj.b", "mlp.proj.b")] + \
+    [(f"h{l}.attn.qkv.b", 3 * 768) for l in range(12)] + \
+    [(f"h{l}.mlp.fc.b", 3072) for l in range(12)] + [("lnf.g", 768), ("lnf.b", 768)]
+
+AUX_LLAMA = [("embed", 128256 * 4096), ("lm_head", 128256 * 4096)] + \
+    [(f"l{l}.{n}", 4096) for l in range(32) for n in ("attn_norm", "mlp_norm")] + [("norm", 4096)]
+
+GRAD_CYCLE = 10
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sus=d["bf16_tflops_sustained"],
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, source="fallback")
+
+
+def workload_def(name):
+    w = wl.WORKLOADS[name]()
+    aux = {"gpt2-small": AUX_GPT2, "llama3-8b": AUX_LLAMA}.get(name, [])
+    return w, aux
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work per step
+# ---------------------------------------------------------------------------
+
+def step_work(w, aux, ns_steps=5):
+    """Nominal NS FLOPs per kernel class and algorithmic HBM bytes of the
+    elementwise kernels, per step."""
+    gram = poly = upd = 0
+    elems = 0
+    for m in w.mats:
+        a, b = min(m.rows, m.cols), max(m.rows, m.cols)
+        gram += 2 * a * a * b * ns_steps
+        poly += 2 * a ** 3 * ns_steps
+        upd += 2 * a * a * b * ns_steps
+        elems += m.rows * m.cols
+    gbytes = 2 if w.grad_dtype == "bf16" else 4
+    aux_el = sum(n for _, n in aux)
+    return {
+        "gram": ("flop", gram), "poly": ("flop", poly), "update": ("flop", upd),
+        # momentum: read grad + buf, write buf + bf16 U
+        "momentum": ("byte", elems * (gbytes + 4 + 4 + 2)),
+        # apply: read bf16 O + W, write W
+        "apply": ("byte", elems * (2 + 4 + 4)),
+        # adamw: read bf16 grad, read+write param, m, v
+        "adamw": ("byte", aux_el * (2 + 3 * 8)),
+    }, elems, aux_el
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            threading.Thread(target=self._read, daemon=True).start()
+            time.sleep(1.0)
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append((time.time(), ln.strip()))
+
+    def mark(self, which):
+        if which == 0:
+            self.t0 = time.time()
+        else:
+            self.t1 = time.time()
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.3)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = [ln for t, ln in self.lines if self.t0 - 0.15 <= t <= self.t1 + 0.15]
+        if not rows:
+            rows = [ln for _, ln in self.lines[-3:]]
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            f = [x.strip() for x in r.split(",")]
+            if len(f) < 10:
+                continue
+            try:
+                sm.append(float(f[2]))
+                mx.append(float(f[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[6:10]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the fp64 oracle on a bounded sample of the workload
+# ---------------------------------------------------------------------------
+
+def cpu_baseline(w, aux, budget_s=12.0):
+    """Oracle Muon step over whole layers (6 matrices each for GPT-2) until
+    about budget_s seconds of CPU work, plus AdamW on the same share of the
+    aux parameters; scaled to one full step."""
+    import numpy as np
+    import oracle
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [os.cpu_count()])
+    except Exception:
+        threads = os.cpu_count()
+    per_layer = 6 if len(w.mats) % 6 == 0 else 1
+    t_total, done = 0.0, 0
+    rng = np.random.default_rng(0)
+    while done < len(w.mats) and t_total < budget_s:
+        mats = w.mats[done:done + per_layer]
+        ins = [(rng.standard_normal((m.rows, m.cols)) * 0.02, rng.standard_normal((m.rows, m.cols)) * 1e-3,
+                np.zeros((m.rows, m.cols))) for m in mats]
+        t0 = time.perf_counter()
+        for W, G, B in ins:
+            oracle.muon_step(W, G, B)
+        t_total += time.perf_counter() - t0
+        done += len(mats)
+    frac = done / len(w.mats)
+    aux_el = sum(n for _, n in aux)
+    if aux_el:
+        n = max(1, int(aux_el * frac))
+        p, g = rng.standard_normal(n), rng.standard_normal(n) * 1e-2
+        t0 = time.perf_counter()
+        oracle.adamw_step(p, g, np.zeros(n), np.zeros(n), 1)
+        t_total += time.perf_counter() - t0
+    step_s = t_total / frac
+    return {"value": 1.0 / step_s, "unit": "Muon step/s", "cores": threads, "kind": "oracle",
+            "sample": f"{done} of {len(w.mats)} hidden matrices (whole layers) and the same share "
+                      f"of the aux AdamW elements, fp64 NumPy, scaled by {1 / frac:.2f}",
+            "sample_seconds": round(t_total, 3)}
+
+
+def run_reference(args, w, aux):
+    """The oracle as it stands, timed on the host: each step is one hidden
+    matrix (cycling through the workload in order) plus its share of the aux
+    AdamW elements; the full-step rate is extrapolated by the matrix count."""
+    import numpy as np
+    import oracle
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    rng = np.random.default_rng(0)
+    aux_el = sum(n for _, n in aux)
+    share = max(1, aux_el // len(w.mats)) if aux_el else 0
+    times = []
+    for k in range(args.warmup + args.steps):
+        m = w.mats[k % len(w.mats)]
+        W = rng.standard_normal((m.rows, m.cols)) * 0.02
+        G = rng.standard_normal((m.rows, m.cols)) * 1e-3
+        B = np.zeros((m.rows, m.cols))
+        t0 = time.perf_counter()
+        oracle.muon_step(W, G, B)
+        if share:
+            oracle.adamw_step(np.zeros(share), np.ones(share), np.zeros(share), np.zeros(share), 1)
+        dt = time.perf_counter() - t0
+        if k >= args.warmup:
+            times.append(dt)
+    step_s = len(w.mats) * statistics.mean(times)
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [os.cpu_count()])
+    except Exception:
+        threads = os.cpu_count()
+    v = 1.0 / step_s
+    out = {"impl": "reference", "metric": "Muon step/s", "value": v, "unit": "Muon step/s",
+           "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": w.name, "matrices": len(w.mats)},
+           "cpu_baseline": {"value": v, "unit": "Muon step/s", "cores": threads, "kind": "oracle",
+                            "sample": f"one hidden matrix per step, cycling through the {len(w.mats)} "
+                                      f"in order, plus 1/{len(w.mats)} of the aux AdamW elements; "
+                                      f"full step = {len(w.mats)} x mean sample time"},
+           "e2e": {"value": v, "unit": "Muon step/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# the CUDA path
+# ---------------------------------------------------------------------------
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in ("ns_gemm.cuh", "sm100_ptx.cuh", "elementwise.cuh"):
+        h.update(open(os.path.join(ROOT, "matrix_aware_optimizer_step_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def read_traffic(kind):
+    """DRAM bytes per launch of `kind` from the committed ncu summary, if it
+    was taken on the current kernel source."""
+    p = os.path.join(ROOT, "profiles", "ns_gemm_dram_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    vals, src = {}, None
+    for ln in open(p):
+        ln = ln.strip()
+        if ln.startswith("kernel_source_sha256_16"):
+            src = ln.split()[-1]
+        elif ln.startswith("dram_bytes_per_step."):
+            k, v = ln.split()
+            vals[k.split(".", 1)[1]] = float(v)
+    if src != kernel_source_hash() or kind not in vals:
+        return None
+    return vals[kind]
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="muon", choices=["muon", "reference"])
+    ap.add_argument("--workload", default="gpt2-small", choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    w, aux = workload_def(args.workload)
+    if args.impl == "reference":
+        run_reference(args, w, aux)
+        return
+
+    import torch
+    import matrix_aware_optimizer_step_b200 as mx
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    seed = 1000 + rank
+
+    # ---- resident inputs ----
+    tdt = torch.bfloat16 if w.grad_dtype == "bf16" else torch.float32
+    Ws = [wl.torch_normal((m.rows, m.cols), w.weight_std, seed, 0, i, wl.ROLE_WEIGHT, device=dev)
+          for i, m in enumerate(w.mats)]
+    Bs = [torch.zeros((m.rows, m.cols), device=dev) for m in w.mats]
+    n_cycle = min(GRAD_CYCLE, max(1, w.steps)) if args.workload != "llama3-8b" else 1
+    Gs = [[wl.torch_normal((m.rows, m.cols), w.grad_std, seed, s, i, wl.ROLE_GRAD, dtype=tdt, device=dev)
+           for i, m in enumerate(w.mats)] for s in range(n_cycle)]
+    Ps = [wl.torch_normal((n,), 0.02, seed, 0, 10000 + i, wl.ROLE_WEIGHT, device=dev) for i, (_, n) in enumerate(aux)]
+    Ms = [torch.zeros(n, device=dev) for _, n in aux]
+    Vs = [torch.zeros(n, device=dev) for _, n in aux]
+    AGs = [[wl.torch_normal((n,), 1e-3, seed, s, 10000 + i, wl.ROLE_AUX, dtype=torch.bfloat16, device=dev)
+            for i, (_, n) in enumerate(aux)] for s in range(n_cycle)]
+
+    by_shape = {}
+    for i, m in enumerate(w.mats):
+        by_shape.setdefault((m.rows, m.cols), []).append(i)
+
+    def groups_for(s):
+        return [dict(weights=[Ws[i] for i in ix], grads=[Gs[s][i] for i in ix],
+                     momentum=[Bs[i] for i in ix]) for ix in by_shape.values()]
+
+    ctx = mx.MuonContext(local)
+    hp = mx.default_hparams()
+    ahp = mx.default_adamw_hparams()
+    stream = torch.cuda.current_stream()
+    pre_groups = [groups_for(s) for s in range(n_cycle)]
+    adam_step = [0]
+
+    def one_step(k):
+        ctx.step(pre_groups[k % n_cycle], hp, stream)
+        if aux:
+            adam_step[0] += 1
+            ctx.adamw_step(Ps, AGs[k % n_cycle], Ms, Vs, adam_step[0], ahp, stream)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if dist is None:
+            return x
+        t = torch.tensor([x], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def timed(k_steps, body):
+        barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for k in range(k_steps):
+            body(k)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        return max_over_ranks(e0.elapsed_time(e1))
+
+    for k in range(args.warmup):
+        one_step(k)
+    torch.cuda.synchronize()
+    ctx.check_device()
+
+    # ---- headline: device-resident inputs ----
+    clocks = ClockSampler(local)
+    clocks.start()
+    l0 = ctx.launch_count
+    clocks.mark(0)
+    ms = timed(args.steps, lambda k: one_step(args.warmup + k))
+    clocks.mark(1)
+    launches = ctx.launch_count - l0
+    clk = clocks.stop()
+    ctx.check_device()
+    ms_per_step = ms / args.steps
+    value = world * 1e3 / ms_per_step
+
+    # ---- per-kernel device times (events on the launching stream) ----
+    ctx.profile(True)
+    timed(args.steps, lambda k: one_step(args.warmup + args.steps + k))
+    kt = ctx.profile_read()
+    ctx.profile(False)
+    work, elems, aux_el = step_work(w, aux, hp.ns_steps)
+    pk = peaks()
+    kernels = {}
+    for kind, (t_ms, nl) in kt.items():
+        if nl == 0 or kind not in work:
+            continue
+        unit, per_step = work[kind]
+        tot = per_step * args.steps
+        if unit == "flop":
+            ach = tot / (t_ms * 1e-3) / 1e12
+            kernels[kind] = {"ms_per_step": t_ms / args.steps, "launches": nl, "achieved": ach,
+                             "unit": "TFLOP/s", "frac": ach / pk["bf16"]}
+        else:
+            ach = tot / (t_ms * 1e-3) / 1e9
+            kernels[kind] = {"ms_per_step": t_ms / args.steps, "launches": nl, "achieved": ach,
+                             "unit": "GB/s", "frac": ach / pk["hbm"]}
+    tot_ms = sum(v["ms_per_step"] for v in kernels.values())
+    for v in kernels.values():
+        v["share"] = v["ms_per_step"] / tot_ms if tot_ms else 0.0
+    dom = max(kernels, key=lambda k: kernels[k]["ms_per_step"])
+    d = kernels[dom]
+    traffic = read_traffic(dom)
+    roofline = {"bound": "tensor" if d["unit"] == "TFLOP/s" else "hbm", "kernel": dom,
+                "achieved": d["achieved"], "peak": pk["bf16"] if d["unit"] == "TFLOP/s" else pk["hbm"],
+                "unit": d["unit"], "frac": d["frac"],
+                "traffic": (traffic / d["launches"] * args.steps) if traffic is not None else None,
+                "peak_source": pk["source"] + (" burst bf16 (torch.matmul 8192^3)" if d["unit"] == "TFLOP/s"
+                                               else " HBM copy")}
+    ns_flops = work["gram"][1] + work["poly"][1] + work["update"][1]
+    ns_ms = sum(kernels.get(k, {"ms_per_step": 0})["ms_per_step"] for k in ("gram", "poly", "update"))
+    ew_bytes = work["momentum"][1] + work["apply"][1] + (work["adamw"][1] if aux else 0)
+    ew_ms = sum(kernels.get(k, {"ms_per_step": 0})["ms_per_step"] for k in ("momentum", "apply", "adamw"))
+
+    # ---- end to end through the public API with host buffers ----
+    e2e = None
+    if not args.no_e2e:
+        hG = [[t.cpu().pin_memory() for t in Gs[s]] for s in range(n_cycle)]
+        hAG = [[t.cpu().pin_memory() for t in AGs[s]] for s in range(n_cycle)]
+        hW = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in Ws]
+        hP = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in Ps]
+        h2d = sum(t.numel() * t.element_size() for t in hG[0]) + sum(t.numel() * t.element_size() for t in hAG[0])
+        d2h = sum(t.numel() * t.element_size() for t in hW) + sum(t.numel() * t.element_size() for t in hP)
+        k_e2e = max(3, min(args.steps, 50))
+
+        def e2e_step(k):
+            s = k % n_cycle
+            for dst, src in zip(Gs[s], hG[s]):
+                dst.copy_(src, non_blocking=True)
+            for dst, src in zip(AGs[s], hAG[s]):
+                dst.copy_(src, non_blocking=True)
+            one_step(k)
+            for dst, src in zip(hW, Ws):
+                dst.copy_(src, non_blocking=True)
+            for dst, src in zip(hP, Ps):
+                dst.copy_(src, non_blocking=True)
+
+        ms_e2e = timed(k_e2e, e2e_step)
+        e2e = {"value": world * 1e3 * k_e2e / ms_e2e, "unit": "Muon step/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h,
+               "note": "gradients copied host->device and updated weights device->host every step"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, aux)
+
+    out = {
+        "metric": "Muon step/s", "value": value, "unit": "Muon step/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "elementwise_dtype": "f32", "data": "synthetic",
+        "config": {"workload": w.name, "matrices": len(w.mats), "hidden_params": elems,
+                   "aux_params": aux_el, "grad_dtype": w.grad_dtype, "ns_steps": hp.ns_steps,
+                   "grad_sets_cycled": n_cycle, "l2": "inputs larger than L2 (no flush)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single"},
+        "ns_tflops": ns_flops / (ns_ms * 1e-3) / 1e12 if ns_ms else None,
+        "ns_tflops_of_step": ns_flops / (ms_per_step * 1e-3) / 1e12,
+        "ns_frac_bf16_peak": (ns_flops / (ns_ms * 1e-3) / 1e12) / pk["bf16"] if ns_ms else None,
+        "elementwise_gbs": ew_bytes / (ew_ms * 1e-3) / 1e9 if ew_ms else None,
+        "elementwise_frac_hbm": (ew_bytes / (ew_ms * 1e-3) / 1e9) / pk["hbm"] if ew_ms else None,
+        "roofline": roofline, "kernels": kernels, "gpu_launches": launches,
+        "launches_per_step": launches / args.steps,
+        "clocks": clk, "e2e": e2e, "cpu_baseline": cpu,
+    }
+    ctx.close()
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,256 @@
+/*
+ * muon.h -- C ABI of the B200 (sm_100a) Muon optimizer step.
+ *
+ * The operation, by source:
+ *
+ *   "Muon: An optimizer for the hidden layers of neural networks" (README of
+ *   the KellerJordan/Muon repository), sections "Usage" and "Hyperparameter
+ *   tuning": hidden 2-D weights are stepped by Muon (lr 0.02, weight decay
+ *   0.01, momentum 0.95, Nesterov, 5 Newton-Schulz steps); every other
+ *   parameter by AdamW (lr 3e-4, betas (0.9, 0.95), weight decay 0.01).
+ *
+ *   "Muon: when the LLM optimizer treats weight matrices as matrices" (blog),
+ *   section 3: X = G / ||G||_F, then X <- a X + b (X X^T) X + c (X X^T)^2 X
+ *   with a, b, c = 3.4445, -4.7750, 2.0315; PyTorch set-up after section 4:
+ *   shape-dependent scaling conventions and decoupled weight decay.
+ *
+ *   "The Newton-Muon Optimizer" (README of zhehangdu/Newton-Muon), section
+ *   "What Is Newton-Muon?": the gradient is right-multiplied by an inverse
+ *   activation second moment S^-1 (one d x d estimate, or four d x d blocks
+ *   for the MLP contraction) before the standard Muon step.
+ *
+ * Conventions for every entry point:
+ *
+ *   - Tensors are caller-owned, contiguous, row-major, on the device the
+ *     context was created for, and 16-byte aligned.  Arrays of tensor
+ *     pointers (the `weights`, `grads`, ... fields) are HOST arrays whose
+ *     elements are DEVICE pointers.  Descriptor structs are read on the host
+ *     during the call only; nothing is retained after the call returns.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Work is enqueued on it asynchronously; a call returns before
+ *     the GPU finishes.  Calls sharing one context must be ordered (one
+ *     stream, or externally synchronised streams): the context's workspace
+ *     and descriptor tables are reused from call to call.
+ *   - Errors are status codes; nothing throws across the ABI.  Argument
+ *     errors are detected on the host before anything is enqueued and leave
+ *     every tensor untouched.  muon_last_error() then describes the error.
+ *     CUDA errors of earlier asynchronous work surface as MUON_ERR_CUDA on a
+ *     later call.  A kernel whose internal wait runs past its limit records
+ *     MUON_ERR_TIMEOUT in a device flag read by muon_check_device().
+ */
+#ifndef MUON_B200_H
+#define MUON_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MUON_API __attribute__((visibility("default")))
+#else
+#define MUON_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MUON_OK = 0,
+  MUON_ERR_INVALID_ARG = 1,   /* bad shape, count, pointer, alignment or hyper-parameter */
+  MUON_ERR_UNSUPPORTED = 2,   /* valid request this build does not implement */
+  MUON_ERR_WORKSPACE = 3,     /* a caller-given workspace is too small for one matrix */
+  MUON_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed (also earlier async faults) */
+  MUON_ERR_NONFINITE = 5,     /* check_finite was set and a gradient held NaN/Inf */
+  MUON_ERR_TIMEOUT = 6        /* a bounded device-side wait gave up */
+} muon_status;
+
+typedef enum { MUON_F32 = 0, MUON_BF16 = 1 } muon_dtype;
+
+/* Shape-dependent factor multiplying the learning rate (blog, PyTorch
+ * set-up after section 4).  ORIGINAL: max(1, rows/cols)^0.5, the convention
+ * of the first page's lr 0.02.  MATCH_RMS_ADAMW: 0.2 * sqrt(max(rows, cols)).
+ * NONE: 1. */
+typedef enum {
+  MUON_SCALE_ORIGINAL = 0,
+  MUON_SCALE_MATCH_RMS_ADAMW = 1,
+  MUON_SCALE_NONE = 2
+} muon_scale_mode;
+
+/* Hyper-parameters of one Muon step; muon_default_hparams() fills the
+ * sources' defaults.  momentum in [0, 1); ns_steps >= 0; eps > 0 guards the
+ * Frobenius normalisation; check_finite != 0 scans the gradients first and,
+ * when one holds NaN/Inf, leaves every weight and momentum buffer untouched
+ * and returns MUON_ERR_NONFINITE (this synchronises the stream). */
+typedef struct {
+  float lr;
+  float momentum;
+  float weight_decay;
+  float eps;
+  float ns_a, ns_b, ns_c;
+  int32_t nesterov;
+  int32_t ns_steps;
+  int32_t scale_mode;   /* muon_scale_mode */
+  int32_t check_finite;
+} muon_hparams;
+
+/* A group of `count` hidden weights of one shape rows x cols.
+ *   weights[i]   fp32 rows x cols, updated in place.
+ *   grads[i]     grad_dtype rows x cols, read only.
+ *   momentum[i]  fp32 rows x cols, updated in place (EMA convention:
+ *                buf <- beta buf + (1 - beta) g).
+ *   update_out   optional (NULL = off): update_out[i] receives the
+ *                orthogonalised update O (fp32 rows x cols) before scale and
+ *                learning rate, for inspection and staged checking.
+ *   precond      optional (NULL = plain Muon): precond[i] points at
+ *                precond_blocks consecutive fp32 d x d matrices S_b^-1,
+ *                d = cols / precond_blocks; the gradient is right-multiplied
+ *                block-diagonally by them before momentum (Newton-Muon).
+ *                Several matrices may share one S^-1 (the shared QKV
+ *                estimate).  Requires grad_dtype == MUON_BF16. */
+typedef struct {
+  int64_t rows;
+  int64_t cols;
+  int32_t count;
+  int32_t grad_dtype;              /* muon_dtype */
+  float* const* weights;
+  const void* const* grads;
+  float* const* momentum;
+  float* const* update_out;
+  const float* const* precond;
+  int32_t precond_blocks;
+  int32_t reserved;
+} muon_group;
+
+/* Newton-Schulz only: outputs[i] (fp32 rows x cols) = NS(inputs[i]). */
+typedef struct {
+  int64_t rows;
+  int64_t cols;
+  int32_t count;
+  int32_t in_dtype;                /* muon_dtype */
+  const void* const* inputs;
+  float* const* outputs;
+} muon_ns_group;
+
+/* One non-2-D parameter for the aux AdamW step; all buffers have numel
+ * elements. */
+typedef struct {
+  int64_t numel;
+  int32_t grad_dtype;              /* muon_dtype */
+  int32_t reserved;
+  float* param;
+  const void* grad;
+  float* exp_avg;
+  float* exp_avg_sq;
+} muon_adamw_tensor;
+
+typedef struct {
+  float lr, beta1, beta2, eps, weight_decay;
+} muon_adamw_hparams;
+
+/* One activation matrix feeding a Newton-Muon refresh: acts is tokens x
+ * width (act_dtype), split into nblocks column blocks of d = width / nblocks;
+ * s_inv receives nblocks consecutive fp32 d x d matrices
+ * (X_b^T X_b / tokens + damping I)^-1. */
+typedef struct {
+  const void* acts;
+  int32_t act_dtype;               /* muon_dtype; MUON_BF16 only in this build */
+  int32_t nblocks;
+  int64_t tokens;
+  int64_t width;
+  float* s_inv;
+} muon_act_desc;
+
+typedef struct muon_ctx muon_ctx;
+
+/* Defaults of the first page ("Usage", "Hyperparameter tuning") and the
+ * blog's coefficients: lr 0.02, momentum 0.95, weight decay 0.01, eps 1e-7,
+ * a b c = 3.4445 -4.7750 2.0315, Nesterov on, 5 steps, ORIGINAL scale. */
+MUON_API void muon_default_hparams(muon_hparams* hp);
+/* AdamW defaults of the first page: lr 3e-4, betas 0.9 / 0.95, eps 1e-8,
+ * weight decay 0.01. */
+MUON_API void muon_default_adamw_hparams(muon_adamw_hparams* hp);
+
+/* Create a context on CUDA device `device`.  workspace_bytes == 0: the
+ * library allocates and grows its own workspace as needed.  Otherwise the
+ * library allocates exactly that much once and splits larger requests into
+ * chunks that fit; a single matrix that does not fit returns
+ * MUON_ERR_WORKSPACE.  *ctx is NULL on failure. */
+MUON_API muon_status muon_init(muon_ctx** ctx, int device, size_t workspace_bytes);
+
+/* Release the context, its workspace and tables (synchronises the device). */
+MUON_API void muon_destroy(muon_ctx* ctx);
+
+/* Human-readable description of the context's last error ("" if none). */
+MUON_API const char* muon_last_error(const muon_ctx* ctx);
+MUON_API const char* muon_status_string(muon_status s);
+
+/* Workspace bytes a muon_step / muon_orthogonalize over these groups needs
+ * to run in one chunk. */
+MUON_API muon_status muon_query_workspace(const muon_group* groups, int32_t ngroups, size_t* bytes);
+
+/* Hand the context a caller-owned device workspace (e.g. a torch tensor).
+ * It is used instead of the library's own until replaced; the caller keeps
+ * it alive and unmodified while work enqueued with it may run.  ptr must be
+ * 256-byte aligned.  ptr == NULL returns to library-owned workspace. */
+MUON_API muon_status muon_set_workspace(muon_ctx* ctx, void* ptr, size_t bytes);
+
+/* One Muon step over ngroups groups: for every matrix, Nesterov momentum,
+ * Frobenius normalisation, hp->ns_steps quintic Newton-Schulz iterations in
+ * bf16 with fp32 accumulation (on the transpose when rows > cols), then
+ * W <- W (1 - lr wd) - lr scale O. */
+MUON_API muon_status muon_step(muon_ctx* ctx, const muon_group* groups, int32_t ngroups,
+                      const muon_hparams* hp, void* stream);
+
+/* Frobenius normalisation plus hp->ns_steps Newton-Schulz iterations only
+ * (uses hp->eps, ns_a/b/c, ns_steps). */
+MUON_API muon_status muon_orthogonalize(muon_ctx* ctx, const muon_ns_group* groups, int32_t ngroups,
+                               const muon_hparams* hp, void* stream);
+
+/* Aux AdamW over n tensors; step counts from 1 (bias correction). */
+MUON_API muon_status muon_adamw_step(muon_ctx* ctx, const muon_adamw_tensor* tensors, int32_t n,
+                            const muon_adamw_hparams* hp, int64_t step, void* stream);
+
+/* Newton-Muon refresh: for each descriptor, the second moment of each
+ * column block and its inverse (Cholesky in fp32). */
+MUON_API muon_status muon_newton_refresh(muon_ctx* ctx, const muon_act_desc* acts, int32_t n,
+                                float damping, void* stream);
+
+/* Synchronise the context's last stream and report device-side flags:
+ * MUON_ERR_TIMEOUT if a bounded wait gave up since the last check (the flag
+ * is cleared), MUON_ERR_CUDA on an asynchronous CUDA error, else MUON_OK. */
+MUON_API muon_status muon_check_device(muon_ctx* ctx);
+
+/* Number of kernels this context has launched since creation. */
+MUON_API uint64_t muon_launch_count(const muon_ctx* ctx);
+
+/* Kernel classes timed by the context's profiler. */
+typedef enum {
+  MUON_K_MOMENTUM = 0,   /* momentum + cast + Frobenius partial sums      */
+  MUON_K_GRAM = 1,       /* A = X X^T                                     */
+  MUON_K_POLY = 2,       /* B = b A + c A A                               */
+  MUON_K_UPDATE = 3,     /* X <- a X + B X                                */
+  MUON_K_APPLY = 4,      /* decay + scaled update of the weights          */
+  MUON_K_ADAMW = 5,
+  MUON_K_NEWTON_REFRESH = 6,
+  MUON_K_PRECONDITION = 7,
+  MUON_K_OTHER = 8,      /* finite scan                                    */
+  MUON_K_COUNT = 9
+} muon_kernel_kind;
+
+typedef struct {
+  double ms[MUON_K_COUNT];          /* summed device time of the launches  */
+  uint64_t launches[MUON_K_COUNT];
+} muon_kernel_times;
+
+/* enable != 0: bracket every launch with CUDA events on its stream (a few
+ * microseconds of host time per launch; the GPU work is unchanged). */
+MUON_API muon_status muon_profile_enable(muon_ctx* ctx, int enable);
+/* Wait for the recorded launches, add their event-measured durations into
+ * *out (zeroed first) and reset the accumulators. */
+MUON_API muon_status muon_profile_read(muon_ctx* ctx, muon_kernel_times* out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MUON_B200_H */

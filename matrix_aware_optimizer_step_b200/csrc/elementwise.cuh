@@ -1,0 +1,399 @@
+// elementwise.cuh -- the HBM-bound kernels of the Muon step.
+//
+//   momentum_kernel   Nesterov momentum in place on the fp32 buffer, the
+//                     look-ahead U cast to bf16 and written in the wide
+//                     (rows <= cols) layout the Newton-Schulz engine reads,
+//                     transposing through shared memory for tall matrices,
+//                     and the per-matrix sum of U^2 (block reduction + one
+//                     atomic per block).  12 B/element with bf16 gradients.
+//   apply_kernel      W <- W (1 - lr wd) - lr scale O, O read from the final
+//                     wide bf16 X (transposed back through shared memory for
+//                     tall matrices); optionally O to an fp32 output.
+//                     10 B/element.
+//   finite_kernel     read-only NaN/Inf scan of the gradients.
+//   adamw_kernel      fused AdamW over a list of tensors, bias-corrected.
+//
+// Sources: momentum 0.95 with Nesterov (first page, "Hyperparameter
+// tuning"); EMA convention of the blog's section 1; decoupled decay and the
+// shape scale (blog, PyTorch set-up after section 4); AdamW (first page,
+// "Usage"; blog section 1).
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "sm100_ptx.cuh"
+
+namespace muon {
+
+constexpr int EW_TILE = 64;        // 64 x 64 element tiles
+constexpr int EW_THREADS = 256;
+
+// One matrix as the elementwise kernels see it.  Lives in a device table.
+struct MatDesc {
+  const void* grad;          // rows x cols, grad_dtype (momentum) / input (export)
+  float* weight;             // rows x cols
+  float* momentum;           // rows x cols
+  float* update_out;         // rows x cols fp32 or nullptr
+  __nv_bfloat16* x_in;       // wide layout (m x ld), where U is written
+  const __nv_bfloat16* x_out;  // wide layout, final Newton-Schulz output
+  float* norm2;              // this matrix's ||U||^2 slot
+  float* partials;           // one partial sum per tile of the launch (indexed by tile)
+  unsigned int* counter;     // tiles of this matrix finished so far (starts at 0)
+  int64_t rows, cols;
+  int64_t ld;                // leading dimension of the wide layout
+  int64_t tile_start;        // first 64x64 tile of this matrix in the launch
+  int32_t tiles_c;           // ceil(cols / 64)
+  int32_t transposed;        // rows > cols: wide layout is the transpose
+  int32_t grad_dtype;        // 0 f32, 1 bf16
+  float lr_scale;            // lr * shape scale
+  float decay;               // 1 - lr * wd
+  int32_t pad;
+};
+
+__device__ __forceinline__ int find_mat(const MatDesc* __restrict__ d, int n, int64_t tile) {
+  int lo = 0, hi = n - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (d[mid].tile_start <= tile) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ void load8_grad(const void* g, int dtype, int64_t idx, float (&x)[8]) {
+  if (dtype == 1) {
+    const uint4 w = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(g) + idx);
+    float2 f;
+    f = unpack_bf16x2(w.x); x[0] = f.x; x[1] = f.y;
+    f = unpack_bf16x2(w.y); x[2] = f.x; x[3] = f.y;
+    f = unpack_bf16x2(w.z); x[4] = f.x; x[5] = f.y;
+    f = unpack_bf16x2(w.w); x[6] = f.x; x[7] = f.y;
+  } else {
+    const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(g) + idx);
+    const float4 a = p[0], b = p[1];
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+  }
+}
+
+__device__ __forceinline__ float load1_grad(const void* g, int dtype, int64_t idx) {
+  return dtype == 1 ? __bfloat162float(static_cast<const __nv_bfloat16*>(g)[idx])
+                    : static_cast<const float*>(g)[idx];
+}
+
+__device__ __forceinline__ float block_sum(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  __syncthreads();
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  float s = 0.f;
+  if (w == 0) {
+    s = (l < EW_THREADS / 32) ? red[l] : 0.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  }
+  return s;   // valid in thread 0
+}
+
+// mode 0: momentum (buf updated, U = Nesterov look-ahead or buf)
+// mode 1: plain load (U = input), for Newton-Schulz only
+template <int MODE>
+__global__ void __launch_bounds__(EW_THREADS)
+    momentum_kernel(const MatDesc* __restrict__ descs, int nmat, float beta, int nesterov,
+                    const int* skip) {
+  if (skip != nullptr && *skip) return;
+  __shared__ __align__(16) __nv_bfloat16 tile[EW_TILE][EW_TILE + 8];
+  __shared__ float red[EW_THREADS / 32];
+  const int64_t gt = blockIdx.x;
+  const MatDesc& d = descs[find_mat(descs, nmat, gt)];
+  const int64_t lt = gt - d.tile_start;
+  const int64_t r0 = (lt / d.tiles_c) * EW_TILE;
+  const int64_t c0 = (lt % d.tiles_c) * EW_TILE;
+  const bool vec_ok = (d.cols % 8 == 0) && (d.ld % 8 == 0);
+  float ss = 0.f;
+  // 64 rows x 8 vectors of 8 columns = 512 vectors, 2 per thread
+#pragma unroll
+  for (int it = 0; it < 2; ++it) {
+    const int v = threadIdx.x + it * EW_THREADS;
+    const int rl = v >> 3, cl = (v & 7) * 8;
+    const int64_t r = r0 + rl, c = c0 + cl;
+    if (r >= d.rows) continue;
+    float u[8];
+    if (vec_ok && c + 8 <= d.cols) {
+      const int64_t idx = r * d.cols + c;
+      float g[8];
+      load8_grad(d.grad, d.grad_dtype, idx, g);
+      if (MODE == 0) {
+        float4* bp = reinterpret_cast<float4*>(d.momentum + idx);
+        float4 b0 = bp[0], b1 = bp[1];
+        float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          b[k] = beta * b[k] + (1.f - beta) * g[k];
+          u[k] = nesterov ? (1.f - beta) * g[k] + beta * b[k] : b[k];
+        }
+        bp[0] = make_float4(b[0], b[1], b[2], b[3]);
+        bp[1] = make_float4(b[4], b[5], b[6], b[7]);
+      } else {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) u[k] = g[k];
+      }
+#pragma unroll
+      for (int k = 0; k < 8; ++k) ss += u[k] * u[k];
+      if (!d.transposed) {
+        uint4 w;
+        w.x = pack_bf16x2(u[0], u[1]); w.y = pack_bf16x2(u[2], u[3]);
+        w.z = pack_bf16x2(u[4], u[5]); w.w = pack_bf16x2(u[6], u[7]);
+        *reinterpret_cast<uint4*>(d.x_in + r * d.ld + c) = w;
+      } else {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) tile[cl + k][rl] = __float2bfloat16_rn(u[k]);
+      }
+    } else {
+      for (int k = 0; k < 8; ++k) {
+        const int64_t cc = c + k;
+        if (cc >= d.cols) break;
+        const int64_t idx = r * d.cols + cc;
+        const float g = load1_grad(d.grad, d.grad_dtype, idx);
+        float uk;
+        if (MODE == 0) {
+          const float b = beta * d.momentum[idx] + (1.f - beta) * g;
+          d.momentum[idx] = b;
+          uk = nesterov ? (1.f - beta) * g + beta * b : b;
+        } else {
+          uk = g;
+        }
+        ss += uk * uk;
+        if (!d.transposed) d.x_in[r * d.ld + cc] = __float2bfloat16_rn(uk);
+        else tile[cl + k][rl] = __float2bfloat16_rn(uk);
+      }
+    }
+  }
+  if (d.transposed) {
+    __syncthreads();
+    // wide row = original column c0 + cl, wide columns = original rows r0 .. r0+63
+#pragma unroll
+    for (int it = 0; it < 2; ++it) {
+      const int v = threadIdx.x + it * EW_THREADS;
+      const int cl = v >> 3, rl = (v & 7) * 8;
+      const int64_t wr = c0 + cl, wc = r0 + rl;
+      if (wr >= d.cols) continue;
+      __nv_bfloat16* dst = d.x_in + wr * d.ld + wc;
+      if (wc + 8 <= d.rows && (d.ld % 8 == 0)) {
+        *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(&tile[cl][rl]);
+      } else {
+        for (int k = 0; k < 8 && wc + k < d.rows; ++k) dst[k] = tile[cl][rl + k];
+      }
+    }
+  }
+  // Deterministic sum of U^2: every block stores its partial; the last block
+  // of the matrix to finish adds all partials in tile order.
+  __shared__ bool is_last;
+  const float tot = block_sum(ss, red);
+  if (threadIdx.x == 0) {
+    d.partials[gt] = tot;
+    __threadfence();
+    const unsigned ntiles = static_cast<unsigned>(((d.rows + EW_TILE - 1) / EW_TILE) * d.tiles_c);
+    is_last = atomicAdd(d.counter, 1u) == ntiles - 1;
+  }
+  __syncthreads();
+  if (is_last) {
+    __threadfence();
+    const int64_t ntiles = ((d.rows + EW_TILE - 1) / EW_TILE) * d.tiles_c;
+    float acc = 0.f;
+    for (int64_t t = threadIdx.x; t < ntiles; t += EW_THREADS)
+      acc += *reinterpret_cast<volatile float*>(&d.partials[d.tile_start + t]);
+    const float all = block_sum(acc, red);
+    if (threadIdx.x == 0) {
+      *d.norm2 = all;
+      *d.counter = 0u;     // ready for the next call
+    }
+  }
+}
+
+// mode 0: apply update to W (and optionally write O)
+// mode 1: export O only (Newton-Schulz only path)
+// norm_scale: when no iteration ran, O = U / (||U|| + eps) is formed here.
+template <int MODE>
+__global__ void __launch_bounds__(EW_THREADS)
+    apply_kernel(const MatDesc* __restrict__ descs, int nmat, int normalise, float eps,
+                 const int* skip) {
+  if (skip != nullptr && *skip) return;
+  __shared__ __align__(16) __nv_bfloat16 tile[EW_TILE][EW_TILE + 8];
+  const int64_t gt = blockIdx.x;
+  const MatDesc& d = descs[find_mat(descs, nmat, gt)];
+  const int64_t lt = gt - d.tile_start;
+  const int64_t r0 = (lt / d.tiles_c) * EW_TILE;
+  const int64_t c0 = (lt % d.tiles_c) * EW_TILE;
+  const float s = normalise ? 1.0f / (sqrtf(*d.norm2) + eps) : 1.0f;
+  if (d.transposed) {
+    // stage the 64x64 block of the wide X (rows c0.., cols r0..) in smem
+#pragma unroll
+    for (int it = 0; it < 2; ++it) {
+      const int v = threadIdx.x + it * EW_THREADS;
+      const int cl = v >> 3, rl = (v & 7) * 8;
+      const int64_t wr = c0 + cl, wc = r0 + rl;
+      if (wr >= d.cols) continue;
+      const __nv_bfloat16* src = d.x_out + wr * d.ld + wc;
+      if (wc + 8 <= d.rows && (d.ld % 8 == 0)) {
+        *reinterpret_cast<uint4*>(&tile[cl][rl]) = *reinterpret_cast<const uint4*>(src);
+      } else {
+        for (int k = 0; k < 8 && wc + k < d.rows; ++k) tile[cl][rl + k] = src[k];
+      }
+    }
+    __syncthreads();
+  }
+  const bool vec_ok = (d.cols % 8 == 0) && (d.ld % 8 == 0);
+#pragma unroll
+  for (int it = 0; it < 2; ++it) {
+    const int v = threadIdx.x + it * EW_THREADS;
+    const int rl = v >> 3, cl = (v & 7) * 8;
+    const int64_t r = r0 + rl, c = c0 + cl;
+    if (r >= d.rows) continue;
+    if (vec_ok && c + 8 <= d.cols) {
+      float o[8];
+      if (!d.transposed) {
+        const uint4 w = *reinterpret_cast<const uint4*>(d.x_out + r * d.ld + c);
+        float2 f;
+        f = unpack_bf16x2(w.x); o[0] = f.x; o[1] = f.y;
+        f = unpack_bf16x2(w.y); o[2] = f.x; o[3] = f.y;
+        f = unpack_bf16x2(w.z); o[4] = f.x; o[5] = f.y;
+        f = unpack_bf16x2(w.w); o[6] = f.x; o[7] = f.y;
+      } else {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) o[k] = __bfloat162float(tile[cl + k][rl]);
+      }
+#pragma unroll
+      for (int k = 0; k < 8; ++k) o[k] *= s;
+      const int64_t idx = r * d.cols + c;
+      if (MODE == 0) {
+        float4* wp = reinterpret_cast<float4*>(d.weight + idx);
+        float4 w0 = wp[0], w1 = wp[1];
+        w0.x = w0.x * d.decay - d.lr_scale * o[0]; w0.y = w0.y * d.decay - d.lr_scale * o[1];
+        w0.z = w0.z * d.decay - d.lr_scale * o[2]; w0.w = w0.w * d.decay - d.lr_scale * o[3];
+        w1.x = w1.x * d.decay - d.lr_scale * o[4]; w1.y = w1.y * d.decay - d.lr_scale * o[5];
+        w1.z = w1.z * d.decay - d.lr_scale * o[6]; w1.w = w1.w * d.decay - d.lr_scale * o[7];
+        wp[0] = w0; wp[1] = w1;
+      }
+      if (d.update_out != nullptr) {
+        float4* op = reinterpret_cast<float4*>(d.update_out + idx);
+        op[0] = make_float4(o[0], o[1], o[2], o[3]);
+        op[1] = make_float4(o[4], o[5], o[6], o[7]);
+      }
+    } else {
+      for (int k = 0; k < 8; ++k) {
+        const int64_t cc = c + k;
+        if (cc >= d.cols) break;
+        const float ok = s * (d.transposed ? __bfloat162float(tile[cl + k][rl])
+                                           : __bfloat162float(d.x_out[r * d.ld + cc]));
+        const int64_t idx = r * d.cols + cc;
+        if (MODE == 0) d.weight[idx] = d.weight[idx] * d.decay - d.lr_scale * ok;
+        if (d.update_out != nullptr) d.update_out[idx] = ok;
+      }
+    }
+  }
+}
+
+// Sets *flag when any gradient element is NaN or Inf.  One 64x64 tile per
+// block, same tiling as momentum_kernel.
+__global__ void __launch_bounds__(EW_THREADS)
+    finite_kernel(const MatDesc* __restrict__ descs, int nmat, int* flag) {
+  const int64_t gt = blockIdx.x;
+  const MatDesc& d = descs[find_mat(descs, nmat, gt)];
+  const int64_t lt = gt - d.tile_start;
+  const int64_t r0 = (lt / d.tiles_c) * EW_TILE;
+  const int64_t c0 = (lt % d.tiles_c) * EW_TILE;
+  bool bad = false;
+  for (int e = threadIdx.x; e < EW_TILE * EW_TILE; e += EW_THREADS) {
+    const int64_t r = r0 + e / EW_TILE, c = c0 + e % EW_TILE;
+    if (r < d.rows && c < d.cols) bad |= !isfinite(load1_grad(d.grad, d.grad_dtype, r * d.cols + c));
+  }
+  if (__syncthreads_or(bad) && threadIdx.x == 0) atomicOr(flag, 1);
+}
+
+// ----------------------------------------------------------------------------
+// AdamW
+// ----------------------------------------------------------------------------
+constexpr int ADAM_CHUNK = 8192;   // elements per block
+
+struct AdamDesc {
+  float* param;
+  const void* grad;
+  float* m;
+  float* v;
+  int64_t numel;
+  int64_t chunk_start;
+  int32_t grad_dtype;
+  int32_t pad;
+};
+
+struct AdamScalars {
+  float lr, beta1, beta2, eps, decay;   // decay = 1 - lr * wd
+  float bc1, bc2_sqrt;                  // 1 - beta1^t, sqrt(1 - beta2^t)
+};
+
+__device__ __forceinline__ int find_adam(const AdamDesc* __restrict__ d, int n, int64_t chunk) {
+  int lo = 0, hi = n - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (d[mid].chunk_start <= chunk) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ void adam_one(float& p, float g, float& m, float& v, const AdamScalars& s) {
+  m = s.beta1 * m + (1.f - s.beta1) * g;
+  v = s.beta2 * v + (1.f - s.beta2) * g * g;
+  const float denom = sqrtf(v) / s.bc2_sqrt + s.eps;
+  p = p * s.decay - (s.lr / s.bc1) * (m / denom);
+}
+
+__global__ void __launch_bounds__(EW_THREADS)
+    adamw_kernel(const AdamDesc* __restrict__ descs, int n, AdamScalars s) {
+  const int64_t ch = blockIdx.x;
+  const AdamDesc& d = descs[find_adam(descs, n, ch)];
+  const int64_t base = (ch - d.chunk_start) * ADAM_CHUNK;
+  const int64_t end = min(base + ADAM_CHUNK, d.numel);
+  const bool vec_ok = ((reinterpret_cast<uintptr_t>(d.param) | reinterpret_cast<uintptr_t>(d.m) |
+                        reinterpret_cast<uintptr_t>(d.v)) & 15) == 0 &&
+                      (reinterpret_cast<uintptr_t>(d.grad) & (d.grad_dtype == 1 ? 7 : 15)) == 0;
+  if (vec_ok) {
+    const int64_t vend = base + ((end - base) / 4) * 4;
+    for (int64_t i = base + threadIdx.x * 4; i < vend; i += EW_THREADS * 4) {
+      float4 p = *reinterpret_cast<float4*>(d.param + i);
+      float4 m = *reinterpret_cast<float4*>(d.m + i);
+      float4 v = *reinterpret_cast<float4*>(d.v + i);
+      float g[4];
+      if (d.grad_dtype == 1) {
+        const uint2 w = *reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(d.grad) + i);
+        const float2 a = unpack_bf16x2(w.x), b = unpack_bf16x2(w.y);
+        g[0] = a.x; g[1] = a.y; g[2] = b.x; g[3] = b.y;
+      } else {
+        const float4 q = *reinterpret_cast<const float4*>(static_cast<const float*>(d.grad) + i);
+        g[0] = q.x; g[1] = q.y; g[2] = q.z; g[3] = q.w;
+      }
+      adam_one(p.x, g[0], m.x, v.x, s);
+      adam_one(p.y, g[1], m.y, v.y, s);
+      adam_one(p.z, g[2], m.z, v.z, s);
+      adam_one(p.w, g[3], m.w, v.w, s);
+      *reinterpret_cast<float4*>(d.param + i) = p;
+      *reinterpret_cast<float4*>(d.m + i) = m;
+      *reinterpret_cast<float4*>(d.v + i) = v;
+    }
+    const int64_t j = vend + threadIdx.x;   // at most 3 trailing elements
+    if (j < end) {
+      float p = d.param[j], m = d.m[j], v = d.v[j];
+      adam_one(p, load1_grad(d.grad, d.grad_dtype, j), m, v, s);
+      d.param[j] = p; d.m[j] = m; d.v[j] = v;
+    }
+  } else {
+    for (int64_t j = base + threadIdx.x; j < end; j += EW_THREADS) {
+      float p = d.param[j], m = d.m[j], v = d.v[j];
+      adam_one(p, load1_grad(d.grad, d.grad_dtype, j), m, v, s);
+      d.param[j] = p; d.m[j] = m; d.v[j] = v;
+    }
+  }
+}
+
+}  // namespace muon

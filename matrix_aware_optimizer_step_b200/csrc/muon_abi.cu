@@ -1,0 +1,1001 @@
+// muon_abi.cu -- host side of the library: argument checks, the grouping
+// scheduler, workspace planning, TMA descriptor encoding, kernel launches
+// and the extern "C" entry points declared in include/muon.h.
+//
+// Scheduling.  Every hidden weight is handled in its wide orientation
+// (m = min(rows, cols) rows, n = max columns; a tall matrix is transposed by
+// the momentum kernel on its way into the workspace).  Matrices of one wide
+// shape form a run; each Newton-Schulz product of a run is ONE batched launch
+// whose tile list covers every matrix of the run, so small layers fill the
+// 148 SMs together.  When a caller-bounded workspace cannot hold everything,
+// the matrices are processed in chunks that fit.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "../../include/muon.h"
+#include "elementwise.cuh"
+#include "newton.cuh"
+#include "ns_gemm.cuh"
+
+using namespace muon;
+
+struct muon_ctx {
+  int device = 0;
+  size_t ws_cap = 0;            // 0: grow on demand
+  void* ws_own = nullptr;
+  size_t ws_own_bytes = 0;
+  void* ws_user = nullptr;
+  size_t ws_user_bytes = 0;
+  void* dtable = nullptr;       // device descriptor table
+  size_t dtable_bytes = 0;
+  void* htable[2] = {nullptr, nullptr};   // pinned staging, double-buffered
+  size_t htable_bytes[2] = {0, 0};
+  cudaEvent_t hevent[2] = {nullptr, nullptr};
+  int hslot = 0;
+  int* dflags = nullptr;        // [0] error bits, [1] non-finite, [2..] spare
+  uint64_t launches = 0;
+  cudaStream_t last_stream = nullptr;
+  std::string err;
+  // profiler: event pairs per kernel class, recycled through a pool
+  bool prof = false;
+  std::vector<std::pair<cudaEvent_t, cudaEvent_t>> prof_pending[MUON_K_COUNT];
+  std::vector<cudaEvent_t> prof_pool;
+  double prof_ms[MUON_K_COUNT] = {};
+  uint64_t prof_n[MUON_K_COUNT] = {};
+};
+
+namespace {
+
+// ---------------------------------------------------------------------------
+// errors
+// ---------------------------------------------------------------------------
+muon_status fail(muon_ctx* ctx, muon_status st, const char* fmt, ...) {
+  if (ctx) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    ctx->err = buf;
+  }
+  return st;
+}
+
+#define CUDA_TRY(ctx, expr)                                                                    \
+  do {                                                                                         \
+    cudaError_t e_ = (expr);                                                                   \
+    if (e_ != cudaSuccess)                                                                     \
+      return fail((ctx), MUON_ERR_CUDA, "%s failed: %s (%s:%d)", #expr, cudaGetErrorString(e_), \
+                  __FILE__, __LINE__);                                                         \
+  } while (0)
+
+// ---------------------------------------------------------------------------
+// TMA descriptors through the driver entry point (no link against libcuda)
+// ---------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// bf16 tensor [batch][rows][ld] viewed as (cols, rows, batch), 128-byte swizzle.
+bool encode_bf16_3d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, uint64_t batch,
+                    uint64_t ld, uint32_t box_cols, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {cols, rows, batch};
+  cuuint64_t strides[2] = {ld * 2, rows * ld * 2};
+  cuuint32_t box[3] = {box_cols, box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------------------
+// small helpers
+// ---------------------------------------------------------------------------
+inline int64_t round_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
+inline int64_t cdiv(int64_t x, int64_t a) { return (x + a - 1) / a; }
+
+float shape_scale(int64_t rows, int64_t cols, int mode) {
+  switch (mode) {
+    case MUON_SCALE_ORIGINAL: return std::sqrt(std::max(1.0, double(rows) / double(cols)));
+    case MUON_SCALE_MATCH_RMS_ADAMW: return float(0.2 * std::sqrt(double(std::max(rows, cols))));
+    default: return 1.0f;
+  }
+}
+
+// One matrix after validation, in scheduling order.
+struct Item {
+  int64_t rows, cols, m, n;
+  bool transposed;
+  int grad_dtype;
+  const void* grad;
+  float* weight;
+  float* momentum;
+  float* update_out;
+  const float* precond;
+  int precond_blocks;
+};
+
+// A run of matrices sharing one wide shape, inside one chunk.
+struct Run {
+  int64_t m, n, ld_n, ld_m;
+  int first, count;              // item range
+  size_t off_x0, off_x1, off_a, off_b;
+};
+
+struct Chunk {
+  int first, count;              // item range
+  size_t off_norm;               // count floats, then count counters, then per-tile partials
+  size_t off_partials;
+  size_t off_pgrad;              // preconditioned gradients (fp32), if any
+  std::vector<Run> runs;
+  size_t bytes;
+};
+
+constexpr size_t kAlign = 256;
+
+// Lay the chunk out in workspace; returns its total bytes.
+size_t layout_chunk(Chunk& c, const std::vector<Item>& items) {
+  size_t off = 0;
+  c.off_norm = off;
+  off += round_up(c.count * (sizeof(float) + sizeof(unsigned)), kAlign);
+  c.off_partials = off;
+  int64_t tiles = 0;
+  for (int i = c.first; i < c.first + c.count; ++i)
+    tiles += cdiv(items[i].rows, EW_TILE) * cdiv(items[i].cols, EW_TILE);
+  off += round_up(size_t(tiles) * sizeof(float), kAlign);
+  c.off_pgrad = off;
+  for (int i = c.first; i < c.first + c.count; ++i)
+    if (items[i].precond) off += round_up(size_t(items[i].rows) * items[i].cols * 4, kAlign);
+  c.runs.clear();
+  int i = c.first;
+  while (i < c.first + c.count) {
+    Run r{};
+    r.m = items[i].m;
+    r.n = items[i].n;
+    r.ld_n = round_up(r.n, 8);
+    r.ld_m = round_up(r.m, 8);
+    r.first = i;
+    int j = i;
+    while (j < c.first + c.count && items[j].m == r.m && items[j].n == r.n) ++j;
+    r.count = j - i;
+    const size_t xb = round_up(size_t(r.count) * r.m * r.ld_n * 2, kAlign);
+    const size_t ab = round_up(size_t(r.count) * r.m * r.ld_m * 2, kAlign);
+    r.off_x0 = off; off += xb;
+    r.off_x1 = off; off += xb;
+    r.off_a = off; off += ab;
+    r.off_b = off; off += ab;
+    c.runs.push_back(r);
+    i = j;
+  }
+  c.bytes = off;
+  return off;
+}
+
+// Split items into chunks whose layout fits `cap` bytes (cap == 0: one chunk).
+bool plan_chunks(const std::vector<Item>& items, size_t cap, std::vector<Chunk>& out) {
+  out.clear();
+  int i = 0;
+  const int n = int(items.size());
+  while (i < n) {
+    Chunk c{};
+    c.first = i;
+    c.count = cap == 0 ? n - i : 1;
+    if (cap != 0 && layout_chunk(c, items) > cap) return false;
+    // grow greedily
+    while (i + c.count < n) {
+      Chunk t = c;
+      t.count = c.count + 1;
+      if (cap != 0 && layout_chunk(t, items) > cap) break;
+      c.count = t.count;
+    }
+    layout_chunk(c, items);
+    out.push_back(c);
+    i += c.count;
+  }
+  return true;
+}
+
+// ---------------------------------------------------------------------------
+// context resources
+// ---------------------------------------------------------------------------
+muon_status ensure_workspace(muon_ctx* ctx, size_t need, void** base) {
+  if (ctx->ws_user) {
+    if (need > ctx->ws_user_bytes)
+      return fail(ctx, MUON_ERR_WORKSPACE, "workspace of %zu bytes is smaller than the %zu needed",
+                  ctx->ws_user_bytes, need);
+    *base = ctx->ws_user;
+    return MUON_OK;
+  }
+  if (need > ctx->ws_own_bytes) {
+    if (ctx->ws_cap != 0)
+      return fail(ctx, MUON_ERR_WORKSPACE, "workspace cap %zu < %zu", ctx->ws_cap, need);
+    if (ctx->ws_own) {
+      CUDA_TRY(ctx, cudaDeviceSynchronize());
+      CUDA_TRY(ctx, cudaFree(ctx->ws_own));
+      ctx->ws_own = nullptr;
+      ctx->ws_own_bytes = 0;
+    }
+    const size_t grow = round_up(need, size_t(1) << 20);
+    CUDA_TRY(ctx, cudaMalloc(&ctx->ws_own, grow));
+    ctx->ws_own_bytes = grow;
+  }
+  *base = ctx->ws_own;
+  return MUON_OK;
+}
+
+size_t ws_limit(const muon_ctx* ctx) {
+  if (ctx->ws_user) return ctx->ws_user_bytes;
+  return ctx->ws_cap;   // 0 = unbounded
+}
+
+// Copy `bytes` of host data to the device table through pinned staging.
+muon_status upload_table(muon_ctx* ctx, const void* data, size_t bytes, cudaStream_t st, void** dptr) {
+  if (bytes > ctx->dtable_bytes) {
+    if (ctx->dtable) {
+      CUDA_TRY(ctx, cudaDeviceSynchronize());
+      CUDA_TRY(ctx, cudaFree(ctx->dtable));
+      ctx->dtable = nullptr;
+    }
+    const size_t nb = round_up(std::max<size_t>(bytes, 1 << 16), 1 << 16);
+    CUDA_TRY(ctx, cudaMalloc(&ctx->dtable, nb));
+    ctx->dtable_bytes = nb;
+  }
+  const int s = ctx->hslot;
+  ctx->hslot ^= 1;
+  CUDA_TRY(ctx, cudaEventSynchronize(ctx->hevent[s]));   // previous copy from this slot done
+  if (bytes > ctx->htable_bytes[s]) {
+    if (ctx->htable[s]) CUDA_TRY(ctx, cudaFreeHost(ctx->htable[s]));
+    ctx->htable[s] = nullptr;
+    const size_t nb = round_up(std::max<size_t>(bytes, 1 << 16), 1 << 16);
+    CUDA_TRY(ctx, cudaMallocHost(&ctx->htable[s], nb));
+    ctx->htable_bytes[s] = nb;
+  }
+  std::memcpy(ctx->htable[s], data, bytes);
+  CUDA_TRY(ctx, cudaMemcpyAsync(ctx->dtable, ctx->htable[s], bytes, cudaMemcpyHostToDevice, st));
+  CUDA_TRY(ctx, cudaEventRecord(ctx->hevent[s], st));
+  *dptr = ctx->dtable;
+  return MUON_OK;
+}
+
+// Profiler brackets: begin records an event before the launch, end after it.
+cudaEvent_t prof_event(muon_ctx* ctx) {
+  if (!ctx->prof_pool.empty()) {
+    cudaEvent_t e = ctx->prof_pool.back();
+    ctx->prof_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+struct ProfScope {
+  muon_ctx* ctx;
+  int kind;
+  cudaStream_t st;
+  cudaEvent_t a = nullptr;
+  ProfScope(muon_ctx* c, int k, cudaStream_t s) : ctx(c), kind(k), st(s) {
+    if (ctx->prof) {
+      a = prof_event(ctx);
+      cudaEventRecord(a, st);
+    }
+  }
+  ~ProfScope() {
+    if (a) {
+      cudaEvent_t b = prof_event(ctx);
+      cudaEventRecord(b, st);
+      ctx->prof_pending[kind].push_back({a, b});
+    }
+  }
+};
+
+muon_status set_device(muon_ctx* ctx) {
+  CUDA_TRY(ctx, cudaSetDevice(ctx->device));
+  return MUON_OK;
+}
+
+// ---------------------------------------------------------------------------
+// launches
+// ---------------------------------------------------------------------------
+template <int KIND, bool BMN>
+cudaError_t launch_gemm(muon_ctx* ctx, const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& g,
+                        cudaStream_t st) {
+  static bool attr_done[64] = {};
+  const int dev = ctx->device & 63;
+  if (!attr_done[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(ns_gemm_kernel<KIND, BMN>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, gemm_cfg::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_done[dev] = true;
+  }
+  const int64_t grid = int64_t(g.batch) * g.tiles_per_mat;
+  if (grid <= 0) return cudaSuccess;
+  ns_gemm_kernel<KIND, BMN><<<unsigned(grid), gemm_cfg::THREADS, gemm_cfg::SMEM_BYTES, st>>>(a, b, g);
+  ctx->launches++;
+  return cudaGetLastError();
+}
+
+struct RunMaps {
+  CUtensorMap x_r128[2], x_r256[2], x_mn[2], a_r128, a_r256, b_r128;
+};
+
+// ns_steps quintic iterations on one run, X starting in x0.  Returns the
+// buffer index (0/1) holding the result.
+muon_status run_newton_schulz(muon_ctx* ctx, uint8_t* ws, const Run& r, const float* norm2,
+                              const muon_hparams* hp, const int* skip, cudaStream_t st, int* final_buf) {
+  __nv_bfloat16* x[2] = {reinterpret_cast<__nv_bfloat16*>(ws + r.off_x0),
+                         reinterpret_cast<__nv_bfloat16*>(ws + r.off_x1)};
+  __nv_bfloat16* A = reinterpret_cast<__nv_bfloat16*>(ws + r.off_a);
+  __nv_bfloat16* B = reinterpret_cast<__nv_bfloat16*>(ws + r.off_b);
+  RunMaps mp;
+  bool ok = true;
+  for (int k = 0; k < 2; ++k) {
+    ok &= encode_bf16_3d(&mp.x_r128[k], x[k], r.n, r.m, r.count, r.ld_n, 64, 128);
+    ok &= encode_bf16_3d(&mp.x_r256[k], x[k], r.n, r.m, r.count, r.ld_n, 64, 256);
+    ok &= encode_bf16_3d(&mp.x_mn[k], x[k], r.n, r.m, r.count, r.ld_n, 64, 64);
+  }
+  ok &= encode_bf16_3d(&mp.a_r128, A, r.m, r.m, r.count, r.ld_m, 64, 128);
+  ok &= encode_bf16_3d(&mp.a_r256, A, r.m, r.m, r.count, r.ld_m, 64, 256);
+  ok &= encode_bf16_3d(&mp.b_r128, B, r.m, r.m, r.count, r.ld_m, 64, 128);
+  if (!ok) return fail(ctx, MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed (run %lldx%lld)",
+                       (long long)r.m, (long long)r.n);
+
+  const int tm = int(cdiv(r.m, gemm_cfg::BM));
+  const int tn_sym = int(cdiv(r.m, gemm_cfg::BN));
+  const int tn_upd = int(cdiv(r.n, gemm_cfg::BN));
+  int cur = 0;
+  for (int it = 0; it < hp->ns_steps; ++it) {
+    const bool first = (it == 0);
+    GemmArgs g{};
+    g.batch = r.count;
+    g.eps = hp->eps;
+    g.err = ctx->dflags;
+    g.skip = skip;
+    // A = alpha X X^T
+    g.M = int(r.m); g.N = int(r.m); g.K = int(r.n);
+    g.tiles_m = tm; g.tiles_n = tn_sym;
+    g.tiles_per_mat = gemm_tiles_per_mat(EPI_GRAM, tm, tn_sym);
+    g.out = A; g.out_ld = r.ld_m; g.out_bs = r.m * r.ld_m;
+    g.aux = nullptr;
+    g.norm2 = first ? norm2 : nullptr;
+    g.alpha_pow = 2;
+    {
+      ProfScope ps(ctx, MUON_K_GRAM, st);
+      CUDA_TRY(ctx, (launch_gemm<EPI_GRAM, false>(ctx, mp.x_r128[cur], mp.x_r256[cur], g, st)));
+    }
+    // B = b A + c A A
+    g.K = int(r.m);
+    g.tiles_per_mat = gemm_tiles_per_mat(EPI_POLY, tm, tn_sym);
+    g.out = B;
+    g.aux = A; g.aux_ld = r.ld_m; g.aux_bs = r.m * r.ld_m;
+    g.norm2 = nullptr;
+    g.c0 = hp->ns_b; g.c1 = hp->ns_c;
+    {
+      ProfScope ps(ctx, MUON_K_POLY, st);
+      CUDA_TRY(ctx, (launch_gemm<EPI_POLY, false>(ctx, mp.a_r128, mp.a_r256, g, st)));
+    }
+    // X' = alpha (a X + B X)
+    g.M = int(r.m); g.N = int(r.n); g.K = int(r.m);
+    g.tiles_n = tn_upd;
+    g.tiles_per_mat = gemm_tiles_per_mat(EPI_UPDATE, tm, tn_upd);
+    g.out = x[cur ^ 1]; g.out_ld = r.ld_n; g.out_bs = r.m * r.ld_n;
+    g.aux = x[cur]; g.aux_ld = r.ld_n; g.aux_bs = r.m * r.ld_n;
+    g.norm2 = first ? norm2 : nullptr;
+    g.alpha_pow = 1;
+    g.c0 = hp->ns_a;
+    {
+      ProfScope ps(ctx, MUON_K_UPDATE, st);
+      CUDA_TRY(ctx, (launch_gemm<EPI_UPDATE, true>(ctx, mp.b_r128, mp.x_mn[cur], g, st)));
+    }
+    cur ^= 1;
+  }
+  *final_buf = cur;
+  return MUON_OK;
+}
+
+muon_status check_hparams(muon_ctx* ctx, const muon_hparams* hp) {
+  if (!hp) return fail(ctx, MUON_ERR_INVALID_ARG, "hparams is NULL");
+  if (hp->ns_steps < 0 || hp->ns_steps > 100)
+    return fail(ctx, MUON_ERR_INVALID_ARG, "ns_steps %d out of [0, 100]", hp->ns_steps);
+  if (!(hp->momentum >= 0.f && hp->momentum < 1.f))
+    return fail(ctx, MUON_ERR_INVALID_ARG, "momentum %g out of [0, 1)", hp->momentum);
+  if (!(hp->eps > 0.f)) return fail(ctx, MUON_ERR_INVALID_ARG, "eps must be > 0");
+  if (!std::isfinite(hp->lr) || !std::isfinite(hp->weight_decay) || !std::isfinite(hp->ns_a) ||
+      !std::isfinite(hp->ns_b) || !std::isfinite(hp->ns_c))
+    return fail(ctx, MUON_ERR_INVALID_ARG, "non-finite hyper-parameter");
+  if (hp->scale_mode < 0 || hp->scale_mode > 2)
+    return fail(ctx, MUON_ERR_INVALID_ARG, "scale_mode %d unknown", hp->scale_mode);
+  return MUON_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// Validate groups and flatten them into items sorted by wide shape.
+muon_status collect_items(muon_ctx* ctx, const muon_group* groups, int32_t ngroups, std::vector<Item>& items,
+                          bool for_step) {
+  items.clear();
+  if (ngroups < 0) return fail(ctx, MUON_ERR_INVALID_ARG, "ngroups < 0");
+  if (ngroups > 0 && !groups) return fail(ctx, MUON_ERR_INVALID_ARG, "groups is NULL");
+  for (int gi = 0; gi < ngroups; ++gi) {
+    const muon_group& g = groups[gi];
+    if (g.rows < 1 || g.cols < 1)
+      return fail(ctx, MUON_ERR_INVALID_ARG, "group %d: shape %lldx%lld", gi, (long long)g.rows, (long long)g.cols);
+    if (g.rows > (int64_t(1) << 20) || g.cols > (int64_t(1) << 20) || std::min(g.rows, g.cols) > 32768)
+      return fail(ctx, MUON_ERR_UNSUPPORTED, "group %d: shape %lldx%lld beyond the supported range", gi,
+                  (long long)g.rows, (long long)g.cols);
+    if (g.count < 0) return fail(ctx, MUON_ERR_INVALID_ARG, "group %d: count < 0", gi);
+    if (g.count == 0) continue;
+    if (g.grad_dtype != MUON_F32 && g.grad_dtype != MUON_BF16)
+      return fail(ctx, MUON_ERR_INVALID_ARG, "group %d: grad_dtype %d", gi, g.grad_dtype);
+    if (!g.grads || (for_step && (!g.weights || !g.momentum)))
+      return fail(ctx, MUON_ERR_INVALID_ARG, "group %d: NULL pointer array", gi);
+    if (g.precond) {
+      if (g.precond_blocks < 1 || g.cols % g.precond_blocks != 0)
+        return fail(ctx, MUON_ERR_INVALID_ARG, "group %d: precond_blocks %d does not divide cols", gi,
+                    g.precond_blocks);
+      if (g.grad_dtype != MUON_BF16)
+        return fail(ctx, MUON_ERR_UNSUPPORTED, "group %d: preconditioning needs bf16 gradients", gi);
+      if ((g.cols / g.precond_blocks) % 8 != 0)
+        return fail(ctx, MUON_ERR_UNSUPPORTED, "group %d: preconditioner block width must be a multiple of 8", gi);
+    }
+    for (int k = 0; k < g.count; ++k) {
+      Item it{};
+      it.rows = g.rows;
+      it.cols = g.cols;
+      it.transposed = g.rows > g.cols;
+      it.m = std::min(g.rows, g.cols);
+      it.n = std::max(g.rows, g.cols);
+      it.grad_dtype = g.grad_dtype;
+      it.grad = g.grads[k];
+      it.weight = for_step ? g.weights[k] : nullptr;
+      it.momentum = for_step ? g.momentum[k] : nullptr;
+      it.update_out = g.update_out ? g.update_out[k] : nullptr;
+      it.precond = g.precond ? g.precond[k] : nullptr;
+      it.precond_blocks = g.precond ? g.precond_blocks : 0;
+      if (!it.grad || (for_step && (!it.weight || !it.momentum)) || (g.precond && !it.precond) ||
+          (g.update_out && !it.update_out))
+        return fail(ctx, MUON_ERR_INVALID_ARG, "group %d matrix %d: NULL tensor pointer", gi, k);
+      if (!aligned16(it.grad) || (it.weight && !aligned16(it.weight)) || (it.momentum && !aligned16(it.momentum)) ||
+          (it.update_out && !aligned16(it.update_out)) || (it.precond && !aligned16(it.precond)))
+        return fail(ctx, MUON_ERR_INVALID_ARG, "group %d matrix %d: tensor not 16-byte aligned", gi, k);
+      items.push_back(it);
+    }
+  }
+  std::stable_sort(items.begin(), items.end(), [](const Item& a, const Item& b) {
+    return a.m != b.m ? a.m > b.m : a.n > b.n;
+  });
+  return MUON_OK;
+}
+
+// The full pipeline over validated items.  mode 0: Muon step.  mode 1:
+// Newton-Schulz only (grad = input, update_out = output).
+muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_hparams* hp, int mode,
+                      cudaStream_t st) {
+  if (items.empty()) return MUON_OK;
+  std::vector<Chunk> chunks;
+  if (!plan_chunks(items, ws_limit(ctx), chunks))
+    return fail(ctx, MUON_ERR_WORKSPACE, "one matrix needs more workspace than the %zu bytes available",
+                ws_limit(ctx));
+  size_t need = 0;
+  for (auto& c : chunks) need = std::max(need, c.bytes);
+  void* wsv = nullptr;
+  muon_status s = ensure_workspace(ctx, need, &wsv);
+  if (s != MUON_OK) return s;
+  uint8_t* ws = static_cast<uint8_t*>(wsv);
+
+  // Descriptor table: all chunks' MatDescs (the device copy is read by
+  // kernels in stream order, so one upload per call suffices), then the
+  // Newton-Muon precondition descriptors.
+  std::vector<MatDesc> descs(items.size());
+  std::vector<PrecondDesc> pdescs;
+  std::vector<int64_t> chunk_tiles(chunks.size(), 0);
+  std::vector<int> chunk_pbegin(chunks.size(), 0), chunk_pcount(chunks.size(), 0);
+  std::vector<int64_t> chunk_ptiles(chunks.size(), 0);
+  const bool check = mode == 0 && hp->check_finite;
+  for (size_t ci = 0; ci < chunks.size(); ++ci) {
+    Chunk& c = chunks[ci];
+    int64_t tiles = 0;
+    size_t pg_off = c.off_pgrad;
+    chunk_pbegin[ci] = int(pdescs.size());
+    int64_t ptiles = 0;
+    for (const Run& r : c.runs) {
+      for (int k = 0; k < r.count; ++k) {
+        const int idx = r.first + k;
+        const Item& it = items[idx];
+        MatDesc& d = descs[idx];
+        d.grad = it.grad;
+        d.grad_dtype = it.grad_dtype;
+        if (it.precond) {
+          float* pg = reinterpret_cast<float*>(ws + pg_off);
+          pg_off += round_up(size_t(it.rows) * it.cols * 4, kAlign);
+          PrecondDesc p{};
+          p.grad = static_cast<const __nv_bfloat16*>(it.grad);
+          p.s_inv = it.precond;
+          p.out = pg;
+          p.rows = it.rows;
+          p.cols = it.cols;
+          p.d = it.cols / it.precond_blocks;
+          p.tiles_r = int(cdiv(it.rows, PRE_BM));
+          p.tiles_c = int(cdiv(p.d, PRE_BN));
+          p.tile_start = ptiles;
+          ptiles += int64_t(p.tiles_r) * p.tiles_c * it.precond_blocks;
+          pdescs.push_back(p);
+          d.grad = pg;
+          d.grad_dtype = MUON_F32;
+        }
+        d.weight = it.weight;
+        d.momentum = it.momentum;
+        d.update_out = it.update_out;
+        d.x_in = reinterpret_cast<__nv_bfloat16*>(ws + r.off_x0) + int64_t(k) * r.m * r.ld_n;
+        const int final_buf = hp->ns_steps % 2;
+        d.x_out = reinterpret_cast<__nv_bfloat16*>(ws + (final_buf ? r.off_x1 : r.off_x0)) +
+                  int64_t(k) * r.m * r.ld_n;
+        d.norm2 = reinterpret_cast<float*>(ws + c.off_norm) + (idx - c.first);
+        d.counter = reinterpret_cast<unsigned*>(ws + c.off_norm + c.count * sizeof(float)) + (idx - c.first);
+        d.partials = reinterpret_cast<float*>(ws + c.off_partials);
+        d.rows = it.rows;
+        d.cols = it.cols;
+        d.ld = r.ld_n;
+        d.tile_start = tiles;
+        d.tiles_c = int(cdiv(it.cols, EW_TILE));
+        d.transposed = it.transposed ? 1 : 0;
+        const float scale = shape_scale(it.rows, it.cols, hp->scale_mode);
+        d.lr_scale = hp->lr * scale;
+        d.decay = 1.0f - hp->lr * hp->weight_decay;
+        tiles += cdiv(it.rows, EW_TILE) * d.tiles_c;
+      }
+    }
+    chunk_tiles[ci] = tiles;
+    chunk_pcount[ci] = int(pdescs.size()) - chunk_pbegin[ci];
+    chunk_ptiles[ci] = ptiles;
+  }
+  const size_t mat_bytes = round_up(descs.size() * sizeof(MatDesc), kAlign);
+  std::vector<uint8_t> table(mat_bytes + pdescs.size() * sizeof(PrecondDesc));
+  std::memcpy(table.data(), descs.data(), descs.size() * sizeof(MatDesc));
+  if (!pdescs.empty()) std::memcpy(table.data() + mat_bytes, pdescs.data(), pdescs.size() * sizeof(PrecondDesc));
+  void* dtab = nullptr;
+  s = upload_table(ctx, table.data(), table.size(), st, &dtab);
+  if (s != MUON_OK) return s;
+  const MatDesc* ddesc = static_cast<const MatDesc*>(dtab);
+  const PrecondDesc* dpdesc = reinterpret_cast<const PrecondDesc*>(static_cast<uint8_t*>(dtab) + mat_bytes);
+
+  const int* skip = nullptr;
+  if (check) {
+    CUDA_TRY(ctx, cudaMemsetAsync(ctx->dflags + 1, 0, sizeof(int), st));
+    int64_t tiles = 0;
+    for (size_t i = 0; i < items.size(); ++i) tiles += cdiv(items[i].rows, EW_TILE) * cdiv(items[i].cols, EW_TILE);
+    // finite_kernel reads the caller's gradients: give it a table with those
+    std::vector<MatDesc> raw(descs);
+    int64_t t = 0;
+    for (size_t i = 0; i < items.size(); ++i) {
+      raw[i].grad = items[i].grad;
+      raw[i].grad_dtype = items[i].grad_dtype;
+      raw[i].tile_start = t;
+      t += cdiv(items[i].rows, EW_TILE) * cdiv(items[i].cols, EW_TILE);
+    }
+    // second table region after the main one
+    const size_t off = round_up(table.size(), kAlign);
+    std::vector<uint8_t> both(off + raw.size() * sizeof(MatDesc));
+    std::memcpy(both.data(), table.data(), table.size());
+    std::memcpy(both.data() + off, raw.data(), raw.size() * sizeof(MatDesc));
+    s = upload_table(ctx, both.data(), both.size(), st, &dtab);
+    if (s != MUON_OK) return s;
+    ddesc = static_cast<const MatDesc*>(dtab);
+    dpdesc = reinterpret_cast<const PrecondDesc*>(static_cast<uint8_t*>(dtab) + mat_bytes);
+    const MatDesc* draw = reinterpret_cast<const MatDesc*>(static_cast<uint8_t*>(dtab) + off);
+    {
+      ProfScope ps(ctx, MUON_K_OTHER, st);
+      finite_kernel<<<unsigned(tiles), EW_THREADS, 0, st>>>(draw, int(items.size()), ctx->dflags + 1);
+    }
+    ctx->launches++;
+    CUDA_TRY(ctx, cudaGetLastError());
+    skip = ctx->dflags + 1;
+  }
+
+  for (size_t ci = 0; ci < chunks.size(); ++ci) {
+    const Chunk& c = chunks[ci];
+    float* norm2 = reinterpret_cast<float*>(ws + c.off_norm);
+    CUDA_TRY(ctx, cudaMemsetAsync(norm2, 0, c.count * (sizeof(float) + sizeof(unsigned)), st));
+    if (chunk_pcount[ci] > 0) {
+      ProfScope ps(ctx, MUON_K_PRECONDITION, st);
+      precond_kernel<<<unsigned(chunk_ptiles[ci]), PRE_THREADS, 0, st>>>(dpdesc + chunk_pbegin[ci],
+                                                                        chunk_pcount[ci], skip);
+      ctx->launches++;
+      CUDA_TRY(ctx, cudaGetLastError());
+    }
+    {
+      ProfScope ps(ctx, MUON_K_MOMENTUM, st);
+      if (mode == 0)
+        momentum_kernel<0><<<unsigned(chunk_tiles[ci]), EW_THREADS, 0, st>>>(
+            ddesc + c.first, c.count, hp->momentum, hp->nesterov, skip);
+      else
+        momentum_kernel<1><<<unsigned(chunk_tiles[ci]), EW_THREADS, 0, st>>>(ddesc + c.first, c.count, 0.f,
+                                                                             0, skip);
+    }
+    ctx->launches++;
+    CUDA_TRY(ctx, cudaGetLastError());
+    for (const Run& r : c.runs) {
+      int fb = 0;
+      s = run_newton_schulz(ctx, ws, r, norm2 + (r.first - c.first), hp, skip, st, &fb);
+      if (s != MUON_OK) return s;
+    }
+    {
+      ProfScope ps(ctx, MUON_K_APPLY, st);
+      if (mode == 0)
+        apply_kernel<0><<<unsigned(chunk_tiles[ci]), EW_THREADS, 0, st>>>(ddesc + c.first, c.count,
+                                                                         hp->ns_steps == 0, hp->eps, skip);
+      else
+        apply_kernel<1><<<unsigned(chunk_tiles[ci]), EW_THREADS, 0, st>>>(ddesc + c.first, c.count,
+                                                                         hp->ns_steps == 0, hp->eps, skip);
+    }
+    ctx->launches++;
+    CUDA_TRY(ctx, cudaGetLastError());
+  }
+
+  if (check) {
+    int flag = 0;
+    CUDA_TRY(ctx, cudaMemcpyAsync(&flag, ctx->dflags + 1, sizeof(int), cudaMemcpyDeviceToHost, st));
+    CUDA_TRY(ctx, cudaStreamSynchronize(st));
+    if (flag) return fail(ctx, MUON_ERR_NONFINITE, "a gradient holds NaN or Inf; nothing was updated");
+  }
+  return MUON_OK;
+}
+
+}  // namespace
+
+// ===========================================================================
+// extern "C"
+// ===========================================================================
+extern "C" {
+
+void muon_default_hparams(muon_hparams* hp) {
+  if (!hp) return;
+  hp->lr = 0.02f;
+  hp->momentum = 0.95f;
+  hp->weight_decay = 0.01f;
+  hp->eps = 1e-7f;
+  hp->ns_a = 3.4445f;
+  hp->ns_b = -4.7750f;
+  hp->ns_c = 2.0315f;
+  hp->nesterov = 1;
+  hp->ns_steps = 5;
+  hp->scale_mode = MUON_SCALE_ORIGINAL;
+  hp->check_finite = 0;
+}
+
+void muon_default_adamw_hparams(muon_adamw_hparams* hp) {
+  if (!hp) return;
+  hp->lr = 3e-4f;
+  hp->beta1 = 0.9f;
+  hp->beta2 = 0.95f;
+  hp->eps = 1e-8f;
+  hp->weight_decay = 0.01f;
+}
+
+const char* muon_status_string(muon_status s) {
+  switch (s) {
+    case MUON_OK: return "MUON_OK";
+    case MUON_ERR_INVALID_ARG: return "MUON_ERR_INVALID_ARG";
+    case MUON_ERR_UNSUPPORTED: return "MUON_ERR_UNSUPPORTED";
+    case MUON_ERR_WORKSPACE: return "MUON_ERR_WORKSPACE";
+    case MUON_ERR_CUDA: return "MUON_ERR_CUDA";
+    case MUON_ERR_NONFINITE: return "MUON_ERR_NONFINITE";
+    case MUON_ERR_TIMEOUT: return "MUON_ERR_TIMEOUT";
+  }
+  return "unknown muon_status";
+}
+
+muon_status muon_init(muon_ctx** out, int device, size_t workspace_bytes) {
+  if (!out) return MUON_ERR_INVALID_ARG;
+  *out = nullptr;
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev) return MUON_ERR_INVALID_ARG;
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, device) != cudaSuccess) return MUON_ERR_CUDA;
+  if (prop.major != 10 || prop.minor != 0) return MUON_ERR_UNSUPPORTED;   // built for sm_100a only
+  if (encode_fn() == nullptr) return MUON_ERR_CUDA;
+  muon_ctx* ctx = new muon_ctx();
+  ctx->device = device;
+  ctx->ws_cap = workspace_bytes;
+  auto bail = [&](muon_status s) { muon_destroy(ctx); return s; };
+  if (cudaSetDevice(device) != cudaSuccess) return bail(MUON_ERR_CUDA);
+  if (cudaMalloc(&ctx->dflags, 16 * sizeof(int)) != cudaSuccess) return bail(MUON_ERR_CUDA);
+  if (cudaMemset(ctx->dflags, 0, 16 * sizeof(int)) != cudaSuccess) return bail(MUON_ERR_CUDA);
+  for (int k = 0; k < 2; ++k)
+    if (cudaEventCreateWithFlags(&ctx->hevent[k], cudaEventDisableTiming) != cudaSuccess) return bail(MUON_ERR_CUDA);
+  if (workspace_bytes != 0) {
+    if (cudaMalloc(&ctx->ws_own, workspace_bytes) != cudaSuccess) return bail(MUON_ERR_CUDA);
+    ctx->ws_own_bytes = workspace_bytes;
+  }
+  *out = ctx;
+  return MUON_OK;
+}
+
+void muon_destroy(muon_ctx* ctx) {
+  if (!ctx) return;
+  cudaSetDevice(ctx->device);
+  cudaDeviceSynchronize();
+  if (ctx->ws_own) cudaFree(ctx->ws_own);
+  if (ctx->dtable) cudaFree(ctx->dtable);
+  for (int k = 0; k < 2; ++k) {
+    if (ctx->htable[k]) cudaFreeHost(ctx->htable[k]);
+    if (ctx->hevent[k]) cudaEventDestroy(ctx->hevent[k]);
+  }
+  if (ctx->dflags) cudaFree(ctx->dflags);
+  for (int k = 0; k < MUON_K_COUNT; ++k)
+    for (auto& pr : ctx->prof_pending[k]) {
+      cudaEventDestroy(pr.first);
+      cudaEventDestroy(pr.second);
+    }
+  for (auto e : ctx->prof_pool) cudaEventDestroy(e);
+  delete ctx;
+}
+
+const char* muon_last_error(const muon_ctx* ctx) { return ctx ? ctx->err.c_str() : "NULL context"; }
+
+muon_status muon_query_workspace(const muon_group* groups, int32_t ngroups, size_t* bytes) {
+  if (!bytes) return MUON_ERR_INVALID_ARG;
+  std::vector<Item> items;
+  muon_status s = collect_items(nullptr, groups, ngroups, items, false);
+  if (s != MUON_OK) return s;
+  std::vector<Chunk> chunks;
+  plan_chunks(items, 0, chunks);
+  *bytes = chunks.empty() ? 0 : chunks[0].bytes;
+  return MUON_OK;
+}
+
+muon_status muon_set_workspace(muon_ctx* ctx, void* ptr, size_t bytes) {
+  if (!ctx) return MUON_ERR_INVALID_ARG;
+  if (ptr && (reinterpret_cast<uintptr_t>(ptr) & 255))
+    return fail(ctx, MUON_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  ctx->ws_user = ptr;
+  ctx->ws_user_bytes = ptr ? bytes : 0;
+  return MUON_OK;
+}
+
+muon_status muon_step(muon_ctx* ctx, const muon_group* groups, int32_t ngroups, const muon_hparams* hp,
+                      void* stream) {
+  if (!ctx) return MUON_ERR_INVALID_ARG;
+  muon_status s = check_hparams(ctx, hp);
+  if (s != MUON_OK) return s;
+  std::vector<Item> items;
+  s = collect_items(ctx, groups, ngroups, items, true);
+  if (s != MUON_OK) return s;
+  s = set_device(ctx);
+  if (s != MUON_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  ctx->last_stream = st;
+  CUDA_TRY(ctx, cudaGetLastError());
+  return run_items(ctx, items, hp, 0, st);
+}
+
+muon_status muon_orthogonalize(muon_ctx* ctx, const muon_ns_group* groups, int32_t ngroups,
+                               const muon_hparams* hp, void* stream) {
+  if (!ctx) return MUON_ERR_INVALID_ARG;
+  muon_status s = check_hparams(ctx, hp);
+  if (s != MUON_OK) return s;
+  if (ngroups < 0 || (ngroups > 0 && !groups)) return fail(ctx, MUON_ERR_INVALID_ARG, "bad groups");
+  std::vector<muon_group> gs(ngroups);
+  for (int i = 0; i < ngroups; ++i) {
+    gs[i] = muon_group{};
+    gs[i].rows = groups[i].rows;
+    gs[i].cols = groups[i].cols;
+    gs[i].count = groups[i].count;
+    gs[i].grad_dtype = groups[i].in_dtype;
+    gs[i].grads = groups[i].inputs;
+    gs[i].update_out = groups[i].outputs;
+    if (groups[i].count > 0 && !groups[i].outputs)
+      return fail(ctx, MUON_ERR_INVALID_ARG, "group %d: outputs is NULL", i);
+  }
+  std::vector<Item> items;
+  s = collect_items(ctx, gs.data(), ngroups, items, false);
+  if (s != MUON_OK) return s;
+  s = set_device(ctx);
+  if (s != MUON_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  ctx->last_stream = st;
+  CUDA_TRY(ctx, cudaGetLastError());
+  return run_items(ctx, items, hp, 1, st);
+}
+
+muon_status muon_adamw_step(muon_ctx* ctx, const muon_adamw_tensor* tensors, int32_t n,
+                            const muon_adamw_hparams* hp, int64_t step, void* stream) {
+  if (!ctx) return MUON_ERR_INVALID_ARG;
+  if (!hp) return fail(ctx, MUON_ERR_INVALID_ARG, "hparams is NULL");
+  if (n < 0 || (n > 0 && !tensors)) return fail(ctx, MUON_ERR_INVALID_ARG, "bad tensor list");
+  if (step < 1) return fail(ctx, MUON_ERR_INVALID_ARG, "step counts from 1");
+  if (!(hp->beta1 >= 0.f && hp->beta1 < 1.f && hp->beta2 >= 0.f && hp->beta2 < 1.f && hp->eps > 0.f))
+    return fail(ctx, MUON_ERR_INVALID_ARG, "betas must lie in [0,1), eps > 0");
+  std::vector<AdamDesc> descs;
+  int64_t chunks = 0;
+  for (int i = 0; i < n; ++i) {
+    const muon_adamw_tensor& t = tensors[i];
+    if (t.numel < 0) return fail(ctx, MUON_ERR_INVALID_ARG, "tensor %d: numel < 0", i);
+    if (t.numel == 0) continue;
+    if (!t.param || !t.grad || !t.exp_avg || !t.exp_avg_sq)
+      return fail(ctx, MUON_ERR_INVALID_ARG, "tensor %d: NULL pointer", i);
+    if (t.grad_dtype != MUON_F32 && t.grad_dtype != MUON_BF16)
+      return fail(ctx, MUON_ERR_INVALID_ARG, "tensor %d: grad_dtype %d", i, t.grad_dtype);
+    AdamDesc d{};
+    d.param = t.param;
+    d.grad = t.grad;
+    d.m = t.exp_avg;
+    d.v = t.exp_avg_sq;
+    d.numel = t.numel;
+    d.grad_dtype = t.grad_dtype;
+    d.chunk_start = chunks;
+    chunks += cdiv(t.numel, ADAM_CHUNK);
+    descs.push_back(d);
+  }
+  if (descs.empty()) return MUON_OK;
+  muon_status s = set_device(ctx);
+  if (s != MUON_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  ctx->last_stream = st;
+  CUDA_TRY(ctx, cudaGetLastError());
+  void* dtab = nullptr;
+  s = upload_table(ctx, descs.data(), descs.size() * sizeof(AdamDesc), st, &dtab);
+  if (s != MUON_OK) return s;
+  AdamScalars sc;
+  sc.lr = hp->lr;
+  sc.beta1 = hp->beta1;
+  sc.beta2 = hp->beta2;
+  sc.eps = hp->eps;
+  sc.decay = 1.0f - hp->lr * hp->weight_decay;
+  sc.bc1 = float(1.0 - std::pow(double(hp->beta1), double(step)));
+  sc.bc2_sqrt = float(std::sqrt(1.0 - std::pow(double(hp->beta2), double(step))));
+  {
+    ProfScope ps(ctx, MUON_K_ADAMW, st);
+    adamw_kernel<<<unsigned(chunks), EW_THREADS, 0, st>>>(static_cast<const AdamDesc*>(dtab), int(descs.size()),
+                                                          sc);
+  }
+  ctx->launches++;
+  CUDA_TRY(ctx, cudaGetLastError());
+  return MUON_OK;
+}
+
+muon_status muon_newton_refresh(muon_ctx* ctx, const muon_act_desc* acts, int32_t n, float damping,
+                                void* stream) {
+  if (!ctx) return MUON_ERR_INVALID_ARG;
+  if (n < 0 || (n > 0 && !acts)) return fail(ctx, MUON_ERR_INVALID_ARG, "bad activation list");
+  if (!(damping >= 0.f) || !std::isfinite(damping)) return fail(ctx, MUON_ERR_INVALID_ARG, "damping must be >= 0");
+  std::vector<GramDesc> gd;
+  std::vector<CholDesc> cd;
+  int64_t gtiles = 0;
+  size_t scratch = 0;
+  int max_d = 0;
+  for (int i = 0; i < n; ++i) {
+    const muon_act_desc& a = acts[i];
+    if (!a.acts || !a.s_inv) return fail(ctx, MUON_ERR_INVALID_ARG, "activation %d: NULL pointer", i);
+    if (a.act_dtype != MUON_BF16) return fail(ctx, MUON_ERR_UNSUPPORTED, "activation %d: bf16 only", i);
+    if (a.tokens < 1 || a.width < 1 || a.nblocks < 1 || a.width % a.nblocks != 0)
+      return fail(ctx, MUON_ERR_INVALID_ARG, "activation %d: bad shape", i);
+    const int64_t d = a.width / a.nblocks;
+    if (d > CHOL_MAX_D)
+      return fail(ctx, MUON_ERR_UNSUPPORTED, "activation %d: block width %lld > %d", i, (long long)d, CHOL_MAX_D);
+    if (!aligned16(a.acts) || !aligned16(a.s_inv))
+      return fail(ctx, MUON_ERR_INVALID_ARG, "activation %d: not 16-byte aligned", i);
+    for (int b = 0; b < a.nblocks; ++b) {
+      GramDesc g{};
+      g.acts = static_cast<const __nv_bfloat16*>(a.acts);
+      g.tokens = a.tokens;
+      g.width = a.width;
+      g.col0 = b * d;
+      g.d = d;
+      g.tiles = int(cdiv(d, GRAM_T));
+      g.tile_start = gtiles;
+      g.s_out = reinterpret_cast<float*>(scratch);          // offset, rebased below
+      gtiles += int64_t(g.tiles) * g.tiles;
+      gd.push_back(g);
+      CholDesc c{};
+      c.a = reinterpret_cast<float*>(scratch);
+      c.inv = a.s_inv + size_t(b) * d * d;
+      c.d = int(d);
+      cd.push_back(c);
+      scratch += round_up(size_t(d) * d * 4, kAlign);
+      max_d = std::max(max_d, int(d));
+    }
+  }
+  if (gd.empty()) return MUON_OK;
+  muon_status s = set_device(ctx);
+  if (s != MUON_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  ctx->last_stream = st;
+  CUDA_TRY(ctx, cudaGetLastError());
+  void* wsv = nullptr;
+  s = ensure_workspace(ctx, scratch, &wsv);
+  if (s != MUON_OK) return s;
+  uint8_t* ws = static_cast<uint8_t*>(wsv);
+  for (auto& g : gd) g.s_out = reinterpret_cast<float*>(ws + reinterpret_cast<size_t>(g.s_out));
+  for (auto& c : cd) c.a = reinterpret_cast<float*>(ws + reinterpret_cast<size_t>(c.a));
+  const size_t gbytes = round_up(gd.size() * sizeof(GramDesc), kAlign);
+  std::vector<uint8_t> table(gbytes + cd.size() * sizeof(CholDesc));
+  std::memcpy(table.data(), gd.data(), gd.size() * sizeof(GramDesc));
+  std::memcpy(table.data() + gbytes, cd.data(), cd.size() * sizeof(CholDesc));
+  void* dtab = nullptr;
+  s = upload_table(ctx, table.data(), table.size(), st, &dtab);
+  if (s != MUON_OK) return s;
+  const GramDesc* dg = static_cast<const GramDesc*>(dtab);
+  const CholDesc* dc = reinterpret_cast<const CholDesc*>(static_cast<uint8_t*>(dtab) + gbytes);
+  ProfScope ps(ctx, MUON_K_NEWTON_REFRESH, st);
+  act_gram_kernel<<<unsigned(gtiles), GRAM_THREADS, 0, st>>>(dg, int(gd.size()));
+  ctx->launches++;
+  CUDA_TRY(ctx, cudaGetLastError());
+  cholesky_kernel<<<unsigned(cd.size()), CHOL_THREADS, 0, st>>>(dc, damping, ctx->dflags);
+  ctx->launches++;
+  CUDA_TRY(ctx, cudaGetLastError());
+  const int parts = int(cdiv(max_d, SOLVE_ROWS_PER_BLOCK));
+  chol_solve_kernel<<<unsigned(cd.size() * parts), SOLVE_THREADS, 0, st>>>(dc, parts);
+  ctx->launches++;
+  CUDA_TRY(ctx, cudaGetLastError());
+  return MUON_OK;
+}
+
+muon_status muon_check_device(muon_ctx* ctx) {
+  if (!ctx) return MUON_ERR_INVALID_ARG;
+  muon_status s = set_device(ctx);
+  if (s != MUON_OK) return s;
+  CUDA_TRY(ctx, cudaDeviceSynchronize());
+  int flags = 0;
+  CUDA_TRY(ctx, cudaMemcpy(&flags, ctx->dflags, sizeof(int), cudaMemcpyDeviceToHost));
+  if (flags) {
+    CUDA_TRY(ctx, cudaMemset(ctx->dflags, 0, sizeof(int)));
+    if (flags & kDevErrTimeout) return fail(ctx, MUON_ERR_TIMEOUT, "a device-side wait gave up (flags 0x%x)", flags);
+    if (flags & kDevErrNotSPD)
+      return fail(ctx, MUON_ERR_INVALID_ARG, "a second moment was not positive definite (flags 0x%x)", flags);
+    return fail(ctx, MUON_ERR_CUDA, "device error flags 0x%x", flags);
+  }
+  return MUON_OK;
+}
+
+uint64_t muon_launch_count(const muon_ctx* ctx) { return ctx ? ctx->launches : 0; }
+
+muon_status muon_profile_enable(muon_ctx* ctx, int enable) {
+  if (!ctx) return MUON_ERR_INVALID_ARG;
+  ctx->prof = enable != 0;
+  return MUON_OK;
+}
+
+muon_status muon_profile_read(muon_ctx* ctx, muon_kernel_times* out) {
+  if (!ctx || !out) return MUON_ERR_INVALID_ARG;
+  muon_status s = set_device(ctx);
+  if (s != MUON_OK) return s;
+  for (int k = 0; k < MUON_K_COUNT; ++k) {
+    for (auto& pr : ctx->prof_pending[k]) {
+      CUDA_TRY(ctx, cudaEventSynchronize(pr.second));
+      float ms = 0.f;
+      CUDA_TRY(ctx, cudaEventElapsedTime(&ms, pr.first, pr.second));
+      ctx->prof_ms[k] += ms;
+      ctx->prof_n[k] += 1;
+      ctx->prof_pool.push_back(pr.first);
+      ctx->prof_pool.push_back(pr.second);
+    }
+    ctx->prof_pending[k].clear();
+    out->ms[k] = ctx->prof_ms[k];
+    out->launches[k] = ctx->prof_n[k];
+    ctx->prof_ms[k] = 0.0;
+    ctx->prof_n[k] = 0;
+  }
+  return MUON_OK;
+}
+
+}  // extern "C"

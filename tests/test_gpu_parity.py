@@ -1,0 +1,301 @@
+"""CUDA path against the fp64 oracle, through the C ABI, on seeded inputs.
+
+Bars: bf16 Newton-Schulz output within 2e-2 relative Frobenius error per
+matrix; fp32 momentum buffer, staged apply (the oracle's apply fed the GPU's
+own orthogonalised update) and AdamW within 1e-5.
+"""
+
+import numpy as np
+import pytest
+
+import oracle
+import workloads as wl
+from helpers import EW_TOL, NS_TOL, ns_tol, rel_fro, to_np
+
+torch = pytest.importorskip("torch")
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def mx():
+    import matrix_aware_optimizer_step_b200 as m
+    return m
+
+
+@pytest.fixture(scope="module")
+def ctx(mx):
+    c = mx.MuonContext(0)
+    yield c
+    c.close()
+
+
+def dev(a, dtype=torch.float32):
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to("cuda").to(dtype).contiguous()
+
+
+NS_SHAPES = [(256, 256), (5, 3), (3, 5), (1, 1), (1, 7), (127, 129), (129, 127), (300, 200),
+             (200, 300), (768, 768), (768, 3072), (3072, 768), (1024, 1024), (640, 2000),
+             (136, 1000), (520, 520)]
+
+
+@pytest.mark.parametrize("shape", NS_SHAPES, ids=lambda s: f"{s[0]}x{s[1]}")
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_orthogonalize_vs_oracle(ctx, shape, dtype):
+    x = wl.np_normal(shape, 1.0, seed=7, index=shape[0] * 10007 + shape[1])
+    if dtype == "bf16":
+        x = wl.bf16_round_np(x)
+    xt = dev(x, torch.bfloat16 if dtype == "bf16" else torch.float32)
+    out = torch.empty(shape, dtype=torch.float32, device="cuda")
+    ctx.orthogonalize([xt], [out])
+    torch.cuda.synchronize()
+    ctx.check_device()
+    want = oracle.newton_schulz(x.astype(np.float64), 5)
+    err = rel_fro(to_np(out), want)
+    assert err < ns_tol(shape), f"{shape} {dtype}: {err}"
+
+
+def test_orthogonalize_batched_groups(ctx):
+    """Many matrices of mixed shapes in one call: every one matches."""
+    shapes = [(384, 384)] * 5 + [(384, 1536)] * 3 + [(1536, 384)] * 3 + [(64, 64)] * 7
+    xs, outs = [], []
+    for i, s in enumerate(shapes):
+        x = wl.np_normal(s, 1e-3, seed=8, index=i)
+        xs.append(x)
+    xt = [dev(x) for x in xs]
+    outs = [torch.empty(s, dtype=torch.float32, device="cuda") for s in shapes]
+    ctx.orthogonalize(xt, outs)
+    torch.cuda.synchronize()
+    for x, o in zip(xs, outs):
+        assert rel_fro(to_np(o), oracle.newton_schulz(x, 5)) < ns_tol(x.shape)
+
+
+@pytest.mark.parametrize("steps", [0, 1, 2, 3, 7])
+def test_orthogonalize_ns_steps(ctx, mx, steps):
+    x = wl.np_normal((200, 456), 1.0, seed=9)
+    out = torch.empty((200, 456), dtype=torch.float32, device="cuda")
+    ctx.orthogonalize([dev(x)], [out], mx.default_hparams(ns_steps=steps))
+    torch.cuda.synchronize()
+    assert rel_fro(to_np(out), oracle.newton_schulz(x, steps)) < NS_TOL
+
+
+def _step_case(ctx, mx, shapes, steps, grad_dtype, hp_over=None, seed=0, grad_std=1e-3):
+    """Run `steps` Muon steps on GPU and oracle side by side; check momentum
+    and staged apply every step, and the update against the oracle's."""
+    hp_over = hp_over or {}
+    hp = mx.default_hparams(**hp_over)
+    ohp = {"scale": {0: "original", 1: "match_rms_adamw", 2: "none"}[hp.scale_mode],
+           "lr": hp.lr, "weight_decay": hp.weight_decay, "momentum": hp.momentum,
+           "nesterov": bool(hp.nesterov), "ns_steps": hp.ns_steps}
+    tdt = torch.bfloat16 if grad_dtype == "bf16" else torch.float32
+    w = [wl.np_normal(s, 0.02, seed=seed, index=i, role=wl.ROLE_WEIGHT).astype(np.float64)
+         for i, s in enumerate(shapes)]
+    buf = [np.zeros(s) for s in shapes]
+    wt = [dev(x) for x in w]
+    bt = [torch.zeros(s, dtype=torch.float32, device="cuda") for s in shapes]
+    ot = [torch.empty(s, dtype=torch.float32, device="cuda") for s in shapes]
+    for step in range(steps):
+        g = []
+        for i, s in enumerate(shapes):
+            x = wl.np_normal(s, grad_std, seed=seed, step=step, index=i)
+            g.append(wl.bf16_round_np(x) if grad_dtype == "bf16" else x)
+        gt = [dev(x, tdt) for x in g]
+        w_prev = [to_np(t) for t in wt]
+        by = {}
+        for i, s in enumerate(shapes):
+            by.setdefault(s, []).append(i)
+        groups = [dict(weights=[wt[i] for i in ix], grads=[gt[i] for i in ix],
+                       momentum=[bt[i] for i in ix], update_out=[ot[i] for i in ix])
+                  for ix in by.values()]
+        ctx.step(groups, hp)
+        torch.cuda.synchronize()
+        for i, s in enumerate(shapes):
+            nb, u = oracle.nesterov_momentum(g[i], buf[i], ohp["momentum"], ohp["nesterov"])
+            assert rel_fro(to_np(bt[i]), nb) < EW_TOL, f"momentum {s} step {step}"
+            o_ref = oracle.newton_schulz(u, ohp["ns_steps"])
+            o_gpu = to_np(ot[i])
+            assert rel_fro(o_gpu, o_ref) < ns_tol(s), f"update {s} step {step}"
+            scale = oracle.shape_scale(s[0], s[1], ohp["scale"])
+            w_staged = oracle.apply_update(w_prev[i], o_gpu, ohp["lr"], ohp["weight_decay"], scale)
+            assert rel_fro(to_np(wt[i]), w_staged) < EW_TOL, f"apply {s} step {step}"
+            buf[i] = nb
+        # carry the oracle buffer from its own arithmetic; weights from the GPU
+    return wt, bt
+
+
+def test_step_single_256_f32(ctx, mx):
+    """One 256x256 fp32 gradient N(0,1), weights N(0,0.02), zero momentum,
+    one step with the defaults."""
+    _step_case(ctx, mx, [(256, 256)], 1, "f32", grad_std=1.0)
+
+
+def test_step_gpt2_layer_bf16_multi_step(ctx, mx):
+    """One GPT-2-small layer (Q, K, V, O, MLP in/out), bf16 gradients, three
+    steps with momentum carried."""
+    shapes = [(768, 768)] * 4 + [(3072, 768), (768, 3072)]
+    _step_case(ctx, mx, shapes, 3, "bf16")
+
+
+@pytest.mark.parametrize("over", [dict(scale_mode="match_rms_adamw"), dict(scale_mode="none"),
+                                  dict(nesterov=0), dict(ns_steps=0), dict(ns_steps=3),
+                                  dict(momentum=0.0, weight_decay=0.0),
+                                  dict(lr=0.1, weight_decay=0.3)])
+def test_step_hparam_variants(ctx, mx, over):
+    _step_case(ctx, mx, [(96, 160), (160, 96), (33, 33)], 2, "f32", hp_over=over)
+
+
+def test_step_ragged_edge_shapes(ctx, mx):
+    shapes = [(1, 1), (1, 9), (9, 1), (3, 5), (5, 3), (65, 63), (130, 260), (260, 130), (257, 513)]
+    _step_case(ctx, mx, shapes, 2, "bf16", grad_std=1.0)
+
+
+def test_empty_and_zero(ctx, mx):
+    # no groups, and a group of count 0, are no-ops
+    ctx.step([], mx.default_hparams())
+    # zero gradient: O = 0, W only decays
+    w = torch.full((16, 24), 1.0, device="cuda")
+    g = torch.zeros((16, 24), device="cuda")
+    b = torch.zeros((16, 24), device="cuda")
+    ctx.step([dict(weights=[w], grads=[g], momentum=[b])])
+    torch.cuda.synchronize()
+    assert torch.allclose(w, torch.full_like(w, 1.0 - 0.02 * 0.01), rtol=0, atol=1e-7)
+
+
+def test_invalid_arguments_leave_tensors_untouched(ctx, mx):
+    w = torch.ones((8, 8), device="cuda")
+    g = torch.ones((8, 8), device="cuda")
+    b = torch.zeros((8, 8), device="cuda")
+    with pytest.raises(mx.MuonError) as e:
+        ctx.step([dict(weights=[w], grads=[g], momentum=[b])], mx.default_hparams(ns_steps=-1))
+    assert e.value.status == 1
+    with pytest.raises(mx.MuonError):
+        ctx.step([dict(weights=[w], grads=[g], momentum=[b])], mx.default_hparams(momentum=1.0))
+    with pytest.raises(ValueError):
+        ctx.step([dict(weights=[w], grads=[g[1:].contiguous()[:, :7].contiguous()], momentum=[b])])
+    # the C ABI itself rejects a NULL tensor pointer
+    import ctypes
+    lib = mx.load_library()
+    arr = (mx.binding.Group * 1)()
+    arr[0].rows, arr[0].cols, arr[0].count, arr[0].grad_dtype = 8, 8, 1, 0
+    nul = (ctypes.c_void_p * 1)(None)
+    ok = (ctypes.c_void_p * 1)(w.data_ptr())
+    arr[0].weights = ctypes.cast(ok, ctypes.c_void_p)
+    arr[0].grads = ctypes.cast(nul, ctypes.c_void_p)
+    arr[0].momentum = ctypes.cast(ok, ctypes.c_void_p)
+    hp = mx.default_hparams()
+    assert lib.muon_step(ctx._ctx, arr, 1, ctypes.byref(hp), None) == 1
+    torch.cuda.synchronize()
+    assert torch.all(w == 1) and torch.all(b == 0)
+
+
+def test_nonfinite_gradient_is_rejected(ctx, mx):
+    w = torch.ones((64, 96), device="cuda")
+    g = torch.randn((64, 96), device="cuda")
+    g[3, 5] = float("nan")
+    b = torch.zeros((64, 96), device="cuda")
+    with pytest.raises(mx.MuonError) as e:
+        ctx.step([dict(weights=[w], grads=[g], momentum=[b])], mx.default_hparams(check_finite=1))
+    assert e.value.status == 5
+    assert torch.all(w == 1) and torch.all(b == 0)
+    g[3, 5] = 0.0
+    ctx.step([dict(weights=[w], grads=[g], momentum=[b])], mx.default_hparams(check_finite=1))
+    torch.cuda.synchronize()
+    assert not torch.all(w == 1)
+
+
+def test_workspace_cap_and_caller_workspace(ctx, mx):
+    """A bounded workspace (chunked execution) and a caller-owned workspace
+    give the same result as the library's own."""
+    shapes = [(256, 512)] * 6 + [(512, 256)] * 3 + [(128, 128)] * 4
+    xs = [dev(wl.np_normal(s, 1.0, seed=10, index=i)) for i, s in enumerate(shapes)]
+    ref = [torch.empty(s, device="cuda") for s in shapes]
+    ctx.orthogonalize(xs, ref)
+    per = 2 * 256 * 512 * 2 + 2 * 256 * 256 * 2 + 4096
+    small = mx.MuonContext(0, workspace_bytes=3 * per)
+    out = [torch.empty(s, device="cuda") for s in shapes]
+    small.orthogonalize(xs, out)
+    torch.cuda.synchronize()
+    for a, b in zip(ref, out):
+        assert torch.equal(a, b)
+    small.close()
+    wst = torch.empty(64 << 20, dtype=torch.uint8, device="cuda")
+    ctx.set_workspace(wst)
+    out2 = [torch.empty(s, device="cuda") for s in shapes]
+    ctx.orthogonalize(xs, out2)
+    torch.cuda.synchronize()
+    ctx.set_workspace(None)
+    for a, b in zip(ref, out2):
+        assert torch.equal(a, b)
+
+
+def test_adamw_vs_oracle(ctx, mx):
+    sizes = [1, 3, 768, 1000, 50257 * 8 + 3, 12345]
+    ps = [wl.np_normal((n,), 0.02, seed=11, index=i, role=wl.ROLE_WEIGHT) for i, n in enumerate(sizes)]
+    pt = [dev(p) for p in ps]
+    mt = [torch.zeros(n, device="cuda") for n in sizes]
+    vt = [torch.zeros(n, device="cuda") for n in sizes]
+    m = [np.zeros(n) for n in sizes]
+    v = [np.zeros(n) for n in sizes]
+    w = [p.astype(np.float64) for p in ps]
+    for step in range(1, 4):
+        gs = [wl.bf16_round_np(wl.np_normal((n,), 1e-2, seed=11, step=step, index=i))
+              for i, n in enumerate(sizes)]
+        gt = [dev(g, torch.bfloat16) if i % 2 == 0 else dev(g) for i, g in enumerate(gs)]
+        ctx.adamw_step(pt, gt, mt, vt, step)
+        torch.cuda.synchronize()
+        for i in range(len(sizes)):
+            w_prev = to_np(pt[i]) if False else None
+            w[i], m[i], v[i] = oracle.adamw_step(w[i], gs[i], m[i], v[i], step)
+            assert rel_fro(to_np(mt[i]), m[i]) < EW_TOL
+            assert rel_fro(to_np(vt[i]), v[i]) < EW_TOL
+            assert rel_fro(to_np(pt[i]), w[i]) < EW_TOL
+
+
+def test_newton_refresh_vs_oracle(ctx, mx):
+    """S^-1 of the activation second moment, one block and four blocks."""
+    tokens = 2048
+    acts = [wl.bf16_round_np(wl.np_normal((tokens, 192), 1.0, seed=12, index=0, role=wl.ROLE_ACT)),
+            wl.bf16_round_np(wl.np_normal((tokens, 4 * 96), 1.0, seed=12, index=1, role=wl.ROLE_ACT))]
+    nblocks = [1, 4]
+    at = [dev(a, torch.bfloat16) for a in acts]
+    si = [torch.empty((nb, a.shape[1] // nb, a.shape[1] // nb), device="cuda") for a, nb in zip(acts, nblocks)]
+    ctx.newton_refresh(at, si, nblocks)
+    torch.cuda.synchronize()
+    ctx.check_device()
+    for a, nb, s in zip(acts, nblocks, si):
+        d = a.shape[1] // nb
+        for b in range(nb):
+            want = oracle.spd_inverse(oracle.second_moment(a[:, b * d:(b + 1) * d]))
+            assert rel_fro(to_np(s[b]), want) < 1e-4
+
+
+def test_newton_muon_step_vs_oracle(ctx, mx):
+    """Right-preconditioned step: shared S^-1 for Q/K/V-like matrices and a
+    four-block S^-1 for the contraction."""
+    d = 128
+    tokens = 1024
+    rng_acts = [wl.bf16_round_np(wl.np_normal((tokens, d), 1.0, seed=13, index=0, role=wl.ROLE_ACT)),
+                wl.bf16_round_np(wl.np_normal((tokens, 4 * d), 1.0, seed=13, index=1, role=wl.ROLE_ACT))]
+    s_in = [oracle.spd_inverse(oracle.second_moment(rng_acts[0]))]
+    s_out = [oracle.spd_inverse(oracle.second_moment(rng_acts[1][:, b * d:(b + 1) * d])) for b in range(4)]
+    si_a = dev(np.stack(s_in))
+    si_b = dev(np.stack(s_out))
+    shapes = [(d, d), (d, d), (d, d), (d, 4 * d)]
+    ws = [wl.np_normal(s, 0.02, seed=13, index=i, role=wl.ROLE_WEIGHT) for i, s in enumerate(shapes)]
+    gs = [wl.bf16_round_np(wl.np_normal(s, 1e-3, seed=13, index=i)) for i, s in enumerate(shapes)]
+    wt = [dev(x) for x in ws]
+    gt = [dev(x, torch.bfloat16) for x in gs]
+    bt = [torch.zeros(s, device="cuda") for s in shapes]
+    ot = [torch.empty(s, device="cuda") for s in shapes]
+    groups = [dict(weights=wt[:3], grads=gt[:3], momentum=bt[:3], update_out=ot[:3],
+                   precond=[si_a] * 3, precond_blocks=1),
+              dict(weights=wt[3:], grads=gt[3:], momentum=bt[3:], update_out=ot[3:],
+                   precond=[si_b], precond_blocks=4)]
+    ctx.step(groups)
+    torch.cuda.synchronize()
+    for i, s in enumerate(shapes):
+        blocks = s_in if i < 3 else s_out
+        pg = oracle.right_precondition(gs[i], blocks)
+        nb, u = oracle.nesterov_momentum(pg, np.zeros(s))
+        assert rel_fro(to_np(bt[i]), nb) < 1e-4, f"preconditioned momentum {i}"
+        assert rel_fro(to_np(ot[i]), oracle.newton_schulz(u, 5)) < NS_TOL
