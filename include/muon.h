@@ -249,6 +249,42 @@ MUON_API muon_status muon_profile_enable(muon_ctx* ctx, int enable);
  * *out (zeroed first) and reset the accumulators. */
 MUON_API muon_status muon_profile_read(muon_ctx* ctx, muon_kernel_times* out);
 
+/* Newton-Schulz of ONE matrix for callers that cannot allocate device
+ * memory -- code running where cudaMalloc is off limits, such as inside a
+ * host that manages every device byte itself, a custom allocator's
+ * callback, or a process whose memory pool must not grow.  The sources have
+ * no counterpart of this entry point; it computes what muon_orthogonalize
+ * computes for a one-matrix group, without a context.
+ *
+ *   input   rows x cols, in_dtype (MUON_F32 or MUON_BF16), device, 16-byte
+ *           aligned, read only.
+ *   output  rows x cols fp32, device, 16-byte aligned: the orthogonalised
+ *           matrix (Frobenius normalisation + hp->ns_steps iterations).
+ *   hp      read on the host during the call (eps, ns_a/b/c, ns_steps).
+ *   stream  cudaStream_t as void* (NULL = legacy default stream).
+ *
+ * Scratch is a fixed 32 MiB device array inside this library (every GPU that
+ * loads the library holds it until the process exits); no call allocates.
+ * A matrix fits when, with m = min(rows, cols), n = max(rows, cols),
+ * ld_n = n rounded up to 8 and ld_m = m rounded up to 8, the bf16 buffers
+ * (4 m ld_n + 4 m ld_m bytes) plus one float per 64 x 64 tile and about
+ * 1 KiB of bookkeeping stay within it (e.g. 1024 x 4096 fits, 2048 x 2048
+ * does not); a larger one returns MUON_ERR_WORKSPACE before anything is
+ * enqueued.  Bad pointers, shapes, dtypes or hyper-parameters return
+ * MUON_ERR_INVALID_ARG.
+ *
+ * The first call on a device looks the array's device address up (once, with
+ * that device current); make that first call before any stream capture.
+ * Each device has its own copy of the array, shared by every call on that
+ * device: calls whose work overlaps on one GPU (different streams, or
+ * threads without ordering) race and corrupt each other's results, so order
+ * them on one stream.  The array keeps the last call's contents; each call
+ * clears the parts that must start at zero.  Device-side wait timeouts are
+ * not reported by this entry point. */
+MUON_API muon_status muon_orthogonalize_noalloc(const void* input, int32_t in_dtype, int64_t rows,
+                                                int64_t cols, float* output, const muon_hparams* hp,
+                                                void* stream);
+
 #ifdef __cplusplus
 }
 #endif

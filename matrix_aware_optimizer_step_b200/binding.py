@@ -34,6 +34,7 @@ EXPORTED = [
     "muon_last_error", "muon_status_string", "muon_query_workspace", "muon_set_workspace",
     "muon_step", "muon_orthogonalize", "muon_adamw_step", "muon_newton_refresh",
     "muon_check_device", "muon_launch_count", "muon_profile_enable", "muon_profile_read",
+    "muon_orthogonalize_noalloc",
 ]
 
 KERNEL_KINDS = ["momentum", "gram", "poly", "update", "apply", "adamw", "newton_refresh",
@@ -122,6 +123,7 @@ def load_library() -> ctypes.CDLL:
         "muon_launch_count": (ctypes.c_uint64, [vp]),
         "muon_profile_enable": (st, [vp, ctypes.c_int]),
         "muon_profile_read": (st, [vp, ctypes.POINTER(KernelTimes)]),
+        "muon_orthogonalize_noalloc": (st, [vp, i32, i64, i64, vp, ctypes.POINTER(Hparams), vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -154,6 +156,20 @@ def default_adamw_hparams(**over) -> AdamwHparams:
 # ---------------------------------------------------------------------------
 # marshalling helpers
 # ---------------------------------------------------------------------------
+
+def orthogonalize_noalloc(x, out, hp: Optional[Hparams] = None, stream=None):
+    """out (fp32) = Newton-Schulz of x, without a context and without any
+    device allocation (the library's fixed scratch array is used)."""
+    hp = hp or default_hparams()
+    _check_cuda([x, out], "orthogonalize_noalloc")
+    if tuple(out.shape) != tuple(x.shape) or x.dim() != 2:
+        raise ValueError("x and out must be matrices of one shape")
+    lib = load_library()
+    st = lib.muon_orthogonalize_noalloc(x.data_ptr(), _dtype_code(x), x.shape[0], x.shape[1],
+                                        out.data_ptr(), ctypes.byref(hp), _stream_ptr(stream))
+    if st != MUON_OK:
+        raise MuonError(st, f"muon_orthogonalize_noalloc: {lib.muon_status_string(st).decode()}")
+
 
 def _dtype_code(t) -> int:
     import torch

@@ -18,6 +18,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -660,6 +661,31 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
   return MUON_OK;
 }
 
+// ---------------------------------------------------------------------------
+// Scratch for muon_orthogonalize_noalloc: a fixed device array that is part of
+// the module, so that entry point never asks the CUDA allocator for memory.
+// Every GPU that loads this library holds these bytes until the process exits.
+// ---------------------------------------------------------------------------
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;   // 32 MiB
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch on `device`.  In host code the array's
+// name only stands for the symbol; the usable address comes from
+// cudaGetSymbolAddress, looked up once per device with that device current.
+muon_status noalloc_scratch_address(int device, uint8_t** out) {
+  static std::mutex mu;
+  static void* addr[64] = {};
+  if (device < 0 || device >= 64) return MUON_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[device] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return MUON_ERR_CUDA;
+    addr[device] = p;
+  }
+  *out = static_cast<uint8_t*>(addr[device]);
+  return MUON_OK;
+}
+
 }  // namespace
 
 // ===========================================================================
@@ -995,6 +1021,83 @@ muon_status muon_profile_read(muon_ctx* ctx, muon_kernel_times* out) {
     ctx->prof_ms[k] = 0.0;
     ctx->prof_n[k] = 0;
   }
+  return MUON_OK;
+}
+
+// Newton-Schulz of one matrix without any device allocation: all scratch
+// lives in g_noalloc_scratch (see include/muon.h for the contract).
+muon_status muon_orthogonalize_noalloc(const void* input, int32_t in_dtype, int64_t rows, int64_t cols,
+                                       float* output, const muon_hparams* hp, void* stream) {
+  if (!input || !output || !hp) return MUON_ERR_INVALID_ARG;
+  if (rows < 1 || cols < 1) return MUON_ERR_INVALID_ARG;
+  if (in_dtype != MUON_F32 && in_dtype != MUON_BF16) return MUON_ERR_INVALID_ARG;
+  if (!aligned16(input) || !aligned16(output)) return MUON_ERR_INVALID_ARG;
+  muon_ctx tmp;   // host-side bookkeeping only; no device resources
+  muon_status s = check_hparams(&tmp, hp);
+  if (s != MUON_OK) return s;
+  int device = 0;
+  if (cudaGetDevice(&device) != cudaSuccess) return MUON_ERR_CUDA;
+  uint8_t* base = nullptr;
+  s = noalloc_scratch_address(device, &base);
+  if (s != MUON_OK) return s;
+  tmp.device = device;
+
+  // Layout: flags | descriptor | norm + counter | partials | X0 | X1 | A | B
+  Item it{};
+  it.rows = rows;
+  it.cols = cols;
+  it.transposed = rows > cols;
+  it.m = std::min(rows, cols);
+  it.n = std::max(rows, cols);
+  it.grad_dtype = in_dtype;
+  it.grad = input;
+  it.update_out = output;
+  std::vector<Item> items(1, it);
+  Chunk c{};
+  c.first = 0;
+  c.count = 1;
+  const size_t body = layout_chunk(c, items);
+  const size_t head = 2 * kAlign;   // flags, descriptor
+  if (head + body > kNoAllocScratchBytes) return MUON_ERR_WORKSPACE;
+  int* flags = reinterpret_cast<int*>(base);
+  MatDesc* ddesc = reinterpret_cast<MatDesc*>(base + kAlign);
+  uint8_t* ws = base + head;
+  const Run& r = c.runs[0];
+
+  MatDesc d{};
+  d.grad = input;
+  d.grad_dtype = in_dtype;
+  d.update_out = output;
+  d.x_in = reinterpret_cast<__nv_bfloat16*>(ws + r.off_x0);
+  d.x_out = reinterpret_cast<__nv_bfloat16*>(ws + ((hp->ns_steps % 2) ? r.off_x1 : r.off_x0));
+  d.norm2 = reinterpret_cast<float*>(ws + c.off_norm);
+  d.counter = reinterpret_cast<unsigned*>(ws + c.off_norm + sizeof(float));
+  d.partials = reinterpret_cast<float*>(ws + c.off_partials);
+  d.rows = rows;
+  d.cols = cols;
+  d.ld = r.ld_n;
+  d.tile_start = 0;
+  d.tiles_c = int(cdiv(cols, EW_TILE));
+  d.transposed = it.transposed ? 1 : 0;
+  const int64_t tiles = cdiv(rows, EW_TILE) * d.tiles_c;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // The descriptor is copied from this stack frame; the runtime stages a
+  // pageable source before the call returns.
+  if (cudaMemcpyAsync(ddesc, &d, sizeof(MatDesc), cudaMemcpyHostToDevice, st) != cudaSuccess) return MUON_ERR_CUDA;
+  // Previous calls leave their values behind: zero the flags, the norm and
+  // the tile counter (everything else is fully overwritten before it is read).
+  if (cudaMemsetAsync(flags, 0, sizeof(int) * 4, st) != cudaSuccess) return MUON_ERR_CUDA;
+  if (cudaMemsetAsync(ws + c.off_norm, 0, sizeof(float) + sizeof(unsigned), st) != cudaSuccess) return MUON_ERR_CUDA;
+  momentum_kernel<1><<<unsigned(tiles), EW_THREADS, 0, st>>>(ddesc, 1, 0.f, 0, nullptr);
+  if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;
+  tmp.dflags = flags;
+  int fb = 0;
+  s = run_newton_schulz(&tmp, ws, r, d.norm2, hp, nullptr, st, &fb);
+  tmp.dflags = nullptr;
+  if (s != MUON_OK) return s;
+  apply_kernel<1><<<unsigned(tiles), EW_THREADS, 0, st>>>(ddesc, 1, hp->ns_steps == 0, hp->eps, nullptr);
+  if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;
   return MUON_OK;
 }
 
