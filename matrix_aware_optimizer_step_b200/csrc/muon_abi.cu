@@ -328,8 +328,15 @@ cudaError_t launch_gemm(muon_ctx* ctx, const CUtensorMap& a, const CUtensorMap& 
     if (e != cudaSuccess) return e;
     attr_done[dev] = true;
   }
-  const int64_t grid = int64_t(g.batch) * g.tiles_per_mat;
-  if (grid <= 0) return cudaSuccess;
+  static int sms[64] = {};
+  if (sms[dev] == 0) {
+    cudaError_t e = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, ctx->device);
+    if (e != cudaSuccess) return e;
+  }
+  const int64_t tiles = int64_t(g.batch) * g.tiles_per_mat;
+  if (tiles <= 0) return cudaSuccess;
+  if (tiles > INT32_MAX) return cudaErrorInvalidValue;
+  const int64_t grid = std::min<int64_t>(tiles, sms[dev]);   // persistent: one CTA per SM
   ns_gemm_kernel<KIND, BMN><<<unsigned(grid), gemm_cfg::THREADS, gemm_cfg::SMEM_BYTES, st>>>(a, b, g);
   ctx->launches++;
   return cudaGetLastError();
