@@ -49,6 +49,7 @@ AUX_LLAMA = [("embed", 128256 * 4096), ("lm_head", 128256 * 4096)] + \
     [(f"l{l}.{n}", 4096) for l in range(32) for n in ("attn_norm", "mlp_norm")] + [("norm", 4096)]
 
 GRAD_CYCLE = 10
+FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12   # CUDA-core fp32 FMA peak at max clock
 
 
 def peaks():
@@ -72,9 +73,21 @@ def workload_def(name):
 
 def step_work(w, aux, ns_steps=5):
     """Nominal NS FLOPs per kernel class and algorithmic HBM bytes of the
-    elementwise kernels, per step."""
+    elementwise kernels, per step (Newton-Muon: fp32 FMA FLOPs of the
+    preconditioner per step and of the refresh amortised over its period)."""
     gram = poly = upd = 0
     elems = 0
+    pre = 0
+    for m in w.mats:
+        if m.name in w.precond:
+            nb = w.precond[m.name][1]
+            d = m.cols // nb
+            pre += 2 * m.rows * m.cols * d
+    refresh = 0
+    for _, tokens, width in w.acts:
+        nb = 4 if width > 768 else 1
+        d = width // nb
+        refresh += nb * (2 * tokens * d * d + d ** 3 // 3 * 2 + 2 * d ** 3)
     for m in w.mats:
         a, b = min(m.rows, m.cols), max(m.rows, m.cols)
         gram += 2 * a * a * b * ns_steps
@@ -91,6 +104,8 @@ def step_work(w, aux, ns_steps=5):
         "apply": ("byte", elems * (2 + 4 + 4)),
         # adamw: read bf16 grad, read+write param, m, v
         "adamw": ("byte", aux_el * (2 + 3 * 8)),
+        "precondition": ("fflop", pre),
+        "newton_refresh": ("fflop", refresh / max(1, w.refresh_every)),
     }, elems, aux_el
 
 
@@ -253,28 +268,37 @@ def run_reference(args, w, aux):
 # the CUDA path
 # ---------------------------------------------------------------------------
 
-def kernel_source_hash():
+SOURCE_GROUPS = {"gram": "ns_gemm", "poly": "ns_gemm", "update": "ns_gemm",
+                 "momentum": "elementwise", "apply": "elementwise", "adamw": "elementwise"}
+
+
+def kernel_source_hash(group):
+    files = {"ns_gemm": ("ns_gemm.cuh", "sm100_ptx.cuh"),
+             "elementwise": ("elementwise.cuh", "sm100_ptx.cuh")}[group]
     h = hashlib.sha256()
-    for f in ("ns_gemm.cuh", "sm100_ptx.cuh", "elementwise.cuh"):
+    for f in files:
         h.update(open(os.path.join(ROOT, "matrix_aware_optimizer_step_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
 
-def read_traffic(kind):
-    """DRAM bytes per launch of `kind` from the committed ncu summary, if it
-    was taken on the current kernel source."""
+def read_traffic(kind, workload):
+    """DRAM bytes per step of kernel class `kind` from the committed ncu
+    summary, if it was taken on this workload and on the current source of
+    that kernel (else None)."""
     p = os.path.join(ROOT, "profiles", "ns_gemm_dram_traffic.txt")
-    if not os.path.exists(p):
+    if not os.path.exists(p) or kind not in SOURCE_GROUPS or workload != "gpt2-small":
         return None
-    vals, src = {}, None
+    vals, src = {}, {}
     for ln in open(p):
         ln = ln.strip()
-        if ln.startswith("kernel_source_sha256_16"):
-            src = ln.split()[-1]
+        if ln.startswith("kernel_source_sha256_16."):
+            k, v = ln.split()
+            src[k.split(".", 1)[1]] = v
         elif ln.startswith("dram_bytes_per_step."):
             k, v = ln.split()
             vals[k.split(".", 1)[1]] = float(v)
-    if src != kernel_source_hash() or kind not in vals:
+    group = SOURCE_GROUPS[kind]
+    if src.get(group) != kernel_source_hash(group) or kind not in vals:
         return None
     return vals[kind]
 
@@ -328,9 +352,27 @@ def main():
     for i, m in enumerate(w.mats):
         by_shape.setdefault((m.rows, m.cols), []).append(i)
 
+    # Newton-Muon: activations per layer input, one S^-1 buffer per input
+    newton = bool(w.acts)
+    Acts, Sinv, nblk = [], [], []
+    if newton:
+        for a, (_, tokens, width) in enumerate(w.acts):
+            nb = 4 if width > 768 else 1
+            Acts.append(wl.torch_normal((tokens, width), 1.0, seed, 0, 20000 + a, wl.ROLE_ACT,
+                                        dtype=torch.bfloat16, device=dev))
+            Sinv.append(torch.empty((nb, width // nb, width // nb), device=dev))
+            nblk.append(nb)
+
     def groups_for(s):
-        return [dict(weights=[Ws[i] for i in ix], grads=[Gs[s][i] for i in ix],
-                     momentum=[Bs[i] for i in ix]) for ix in by_shape.values()]
+        gs = []
+        for ix in by_shape.values():
+            g = dict(weights=[Ws[i] for i in ix], grads=[Gs[s][i] for i in ix],
+                     momentum=[Bs[i] for i in ix])
+            if newton:
+                g["precond"] = [Sinv[w.precond[w.mats[i].name][0]] for i in ix]
+                g["precond_blocks"] = w.precond[w.mats[ix[0]].name][1]
+            gs.append(g)
+        return gs
 
     ctx = mx.MuonContext(local)
     hp = mx.default_hparams()
@@ -340,6 +382,8 @@ def main():
     adam_step = [0]
 
     def one_step(k):
+        if newton and k % w.refresh_every == 0:
+            ctx.newton_refresh(Acts, Sinv, nblk, 0.0, stream)
         ctx.step(pre_groups[k % n_cycle], hp, stream)
         if aux:
             adam_step[0] += 1
@@ -403,6 +447,11 @@ def main():
             ach = tot / (t_ms * 1e-3) / 1e12
             kernels[kind] = {"ms_per_step": t_ms / args.steps, "launches": nl, "achieved": ach,
                              "unit": "TFLOP/s", "frac": ach / pk["bf16"]}
+        elif unit == "fflop":
+            # fp32 FMA on CUDA cores: 148 SMs x 128 lanes x 2 FLOP x 1.965 GHz
+            ach = tot / (t_ms * 1e-3) / 1e12
+            kernels[kind] = {"ms_per_step": t_ms / args.steps, "launches": nl, "achieved": ach,
+                             "unit": "TFLOP/s", "bound": "alu", "frac": ach / FP32_PEAK_TFLOPS}
         else:
             ach = tot / (t_ms * 1e-3) / 1e9
             kernels[kind] = {"ms_per_step": t_ms / args.steps, "launches": nl, "achieved": ach,
@@ -412,7 +461,7 @@ def main():
         v["share"] = v["ms_per_step"] / tot_ms if tot_ms else 0.0
     dom = max(kernels, key=lambda k: kernels[k]["ms_per_step"])
     d = kernels[dom]
-    traffic = read_traffic(dom)
+    traffic = read_traffic(dom, args.workload)
     roofline = {"bound": "tensor" if d["unit"] == "TFLOP/s" else "hbm", "kernel": dom,
                 "achieved": d["achieved"], "peak": pk["bf16"] if d["unit"] == "TFLOP/s" else pk["hbm"],
                 "unit": d["unit"], "frac": d["frac"],
