@@ -51,13 +51,22 @@ struct MatDesc {
   int32_t pad;
 };
 
-__device__ __forceinline__ int find_mat(const MatDesc* __restrict__ d, int n, int64_t tile) {
-  int lo = 0, hi = n - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (d[mid].tile_start <= tile) lo = mid; else hi = mid - 1;
-  }
-  return lo;
+// Segments of equal-shape matrices in one launch (kernel parameter space,
+// no global memory round trip): tile -> matrix is a short scan plus one
+// division instead of a search through the descriptor table.
+constexpr int MAX_SEGS = 32;
+struct SegTable {
+  int n;
+  int first_mat[MAX_SEGS];        // descriptor index of the segment's first matrix
+  int64_t tile_start[MAX_SEGS];   // first tile of the segment (launch numbering)
+  int64_t tiles_per_mat[MAX_SEGS];
+};
+
+__device__ __forceinline__ int seg_find(const SegTable& t, int64_t tile) {
+  int s = 0;
+#pragma unroll 1
+  while (s + 1 < t.n && t.tile_start[s + 1] <= tile) ++s;
+  return t.first_mat[s] + static_cast<int>((tile - t.tile_start[s]) / t.tiles_per_mat[s]);
 }
 
 __device__ __forceinline__ void load8_grad(const void* g, int dtype, int64_t idx, float (&x)[8]) {
@@ -100,13 +109,13 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
 // mode 1: plain load (U = input), for Newton-Schulz only
 template <int MODE>
 __global__ void __launch_bounds__(EW_THREADS)
-    momentum_kernel(const MatDesc* __restrict__ descs, int nmat, float beta, int nesterov,
-                    const int* skip) {
+    momentum_kernel(const MatDesc* __restrict__ descs, const __grid_constant__ SegTable segs, int64_t tile_base,
+                    float beta, int nesterov, const int* skip) {
   if (skip != nullptr && *skip) return;
   __shared__ __align__(16) __nv_bfloat16 tile[EW_TILE][EW_TILE + 8];
   __shared__ float red[EW_THREADS / 32];
-  const int64_t gt = blockIdx.x;
-  const MatDesc& d = descs[find_mat(descs, nmat, gt)];
+  const int64_t gt = tile_base + blockIdx.x;
+  const MatDesc& d = descs[seg_find(segs, gt)];
   const int64_t lt = gt - d.tile_start;
   const int64_t r0 = (lt / d.tiles_c) * EW_TILE;
   const int64_t c0 = (lt % d.tiles_c) * EW_TILE;
@@ -217,12 +226,12 @@ __global__ void __launch_bounds__(EW_THREADS)
 // norm_scale: when no iteration ran, O = U / (||U|| + eps) is formed here.
 template <int MODE>
 __global__ void __launch_bounds__(EW_THREADS)
-    apply_kernel(const MatDesc* __restrict__ descs, int nmat, int normalise, float eps,
-                 const int* skip) {
+    apply_kernel(const MatDesc* __restrict__ descs, const __grid_constant__ SegTable segs, int64_t tile_base,
+                 int normalise, float eps, const int* skip) {
   if (skip != nullptr && *skip) return;
   __shared__ __align__(16) __nv_bfloat16 tile[EW_TILE][EW_TILE + 8];
-  const int64_t gt = blockIdx.x;
-  const MatDesc& d = descs[find_mat(descs, nmat, gt)];
+  const int64_t gt = tile_base + blockIdx.x;
+  const MatDesc& d = descs[seg_find(segs, gt)];
   const int64_t lt = gt - d.tile_start;
   const int64_t r0 = (lt / d.tiles_c) * EW_TILE;
   const int64_t c0 = (lt % d.tiles_c) * EW_TILE;
@@ -298,9 +307,10 @@ __global__ void __launch_bounds__(EW_THREADS)
 // Sets *flag when any gradient element is NaN or Inf.  One 64x64 tile per
 // block, same tiling as momentum_kernel.
 __global__ void __launch_bounds__(EW_THREADS)
-    finite_kernel(const MatDesc* __restrict__ descs, int nmat, int* flag) {
-  const int64_t gt = blockIdx.x;
-  const MatDesc& d = descs[find_mat(descs, nmat, gt)];
+    finite_kernel(const MatDesc* __restrict__ descs, const __grid_constant__ SegTable segs, int64_t tile_base,
+                  int* flag) {
+  const int64_t gt = tile_base + blockIdx.x;
+  const MatDesc& d = descs[seg_find(segs, gt)];
   const int64_t lt = gt - d.tile_start;
   const int64_t r0 = (lt / d.tiles_c) * EW_TILE;
   const int64_t c0 = (lt % d.tiles_c) * EW_TILE;

@@ -122,6 +122,38 @@ float shape_scale(int64_t rows, int64_t cols, int mode) {
   }
 }
 
+// Elementwise launches over descriptors d[0..n) whose tile_start fields are
+// set: each launch covers up to MAX_SEGS segments of equal-shape matrices.
+struct SegLaunch {
+  SegTable t;
+  int64_t tile_base;
+  int64_t tiles;
+};
+
+inline int64_t desc_tiles(const MatDesc& d) { return ((d.rows + EW_TILE - 1) / EW_TILE) * d.tiles_c; }
+
+std::vector<SegLaunch> build_seg_launches(const MatDesc* d, int n) {
+  std::vector<SegLaunch> out;
+  SegLaunch cur{};
+  auto close = [&](int64_t end_tile) {
+    cur.tiles = end_tile - cur.tile_base;
+    out.push_back(cur);
+    cur = SegLaunch{};
+  };
+  for (int i = 0; i < n; ++i) {
+    const bool fresh = i == 0 || d[i].rows != d[i - 1].rows || d[i].cols != d[i - 1].cols;
+    if (!fresh) continue;
+    if (cur.t.n == MAX_SEGS) close(d[i].tile_start);
+    if (cur.t.n == 0) cur.tile_base = d[i].tile_start;
+    const int s = cur.t.n++;
+    cur.t.first_mat[s] = i;
+    cur.t.tile_start[s] = d[i].tile_start;
+    cur.t.tiles_per_mat[s] = desc_tiles(d[i]);
+  }
+  if (n > 0) close(d[n - 1].tile_start + desc_tiles(d[n - 1]));
+  return out;
+}
+
 // One matrix after validation, in scheduling order.
 struct Item {
   int64_t rows, cols, m, n;
@@ -612,9 +644,11 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
     const MatDesc* draw = reinterpret_cast<const MatDesc*>(static_cast<uint8_t*>(dtab) + off);
     {
       ProfScope ps(ctx, MUON_K_OTHER, st);
-      finite_kernel<<<unsigned(tiles), EW_THREADS, 0, st>>>(draw, int(items.size()), ctx->dflags + 1);
+      for (const SegLaunch& L : build_seg_launches(raw.data(), int(raw.size()))) {
+      finite_kernel<<<unsigned(L.tiles), EW_THREADS, 0, st>>>(draw, L.t, L.tile_base, ctx->dflags + 1);
+      ctx->launches++;
     }
-    ctx->launches++;
+    }
     CUDA_TRY(ctx, cudaGetLastError());
     skip = ctx->dflags + 1;
   }
@@ -630,16 +664,19 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
       ctx->launches++;
       CUDA_TRY(ctx, cudaGetLastError());
     }
+    const std::vector<SegLaunch> segl = build_seg_launches(descs.data() + c.first, c.count);
     {
       ProfScope ps(ctx, MUON_K_MOMENTUM, st);
-      if (mode == 0)
-        momentum_kernel<0><<<unsigned(chunk_tiles[ci]), EW_THREADS, 0, st>>>(
-            ddesc + c.first, c.count, hp->momentum, hp->nesterov, skip);
-      else
-        momentum_kernel<1><<<unsigned(chunk_tiles[ci]), EW_THREADS, 0, st>>>(ddesc + c.first, c.count, 0.f,
-                                                                             0, skip);
+      for (const SegLaunch& L : segl) {
+        if (mode == 0)
+          momentum_kernel<0><<<unsigned(L.tiles), EW_THREADS, 0, st>>>(ddesc + c.first, L.t, L.tile_base,
+                                                                       hp->momentum, hp->nesterov, skip);
+        else
+          momentum_kernel<1><<<unsigned(L.tiles), EW_THREADS, 0, st>>>(ddesc + c.first, L.t, L.tile_base, 0.f,
+                                                                       0, skip);
+      }
     }
-    ctx->launches++;
+    ctx->launches += segl.size();
     CUDA_TRY(ctx, cudaGetLastError());
     for (const Run& r : c.runs) {
       int fb = 0;
@@ -648,14 +685,16 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
     }
     {
       ProfScope ps(ctx, MUON_K_APPLY, st);
-      if (mode == 0)
-        apply_kernel<0><<<unsigned(chunk_tiles[ci]), EW_THREADS, 0, st>>>(ddesc + c.first, c.count,
-                                                                         hp->ns_steps == 0, hp->eps, skip);
-      else
-        apply_kernel<1><<<unsigned(chunk_tiles[ci]), EW_THREADS, 0, st>>>(ddesc + c.first, c.count,
-                                                                         hp->ns_steps == 0, hp->eps, skip);
+      for (const SegLaunch& L : segl) {
+        if (mode == 0)
+          apply_kernel<0><<<unsigned(L.tiles), EW_THREADS, 0, st>>>(ddesc + c.first, L.t, L.tile_base,
+                                                                    hp->ns_steps == 0, hp->eps, skip);
+        else
+          apply_kernel<1><<<unsigned(L.tiles), EW_THREADS, 0, st>>>(ddesc + c.first, L.t, L.tile_base,
+                                                                    hp->ns_steps == 0, hp->eps, skip);
+      }
     }
-    ctx->launches++;
+    ctx->launches += segl.size();
     CUDA_TRY(ctx, cudaGetLastError());
   }
 
@@ -1096,14 +1135,16 @@ muon_status muon_orthogonalize_noalloc(const void* input, int32_t in_dtype, int6
   // the tile counter (everything else is fully overwritten before it is read).
   if (cudaMemsetAsync(flags, 0, sizeof(int) * 4, st) != cudaSuccess) return MUON_ERR_CUDA;
   if (cudaMemsetAsync(ws + c.off_norm, 0, sizeof(float) + sizeof(unsigned), st) != cudaSuccess) return MUON_ERR_CUDA;
-  momentum_kernel<1><<<unsigned(tiles), EW_THREADS, 0, st>>>(ddesc, 1, 0.f, 0, nullptr);
+  const std::vector<SegLaunch> segl = build_seg_launches(&d, 1);
+  momentum_kernel<1><<<unsigned(tiles), EW_THREADS, 0, st>>>(ddesc, segl[0].t, 0, 0.f, 0, nullptr);
   if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;
   tmp.dflags = flags;
   int fb = 0;
   s = run_newton_schulz(&tmp, ws, r, d.norm2, hp, nullptr, st, &fb);
   tmp.dflags = nullptr;
   if (s != MUON_OK) return s;
-  apply_kernel<1><<<unsigned(tiles), EW_THREADS, 0, st>>>(ddesc, 1, hp->ns_steps == 0, hp->eps, nullptr);
+  apply_kernel<1><<<unsigned(tiles), EW_THREADS, 0, st>>>(ddesc, segl[0].t, 0, hp->ns_steps == 0, hp->eps,
+                                                          nullptr);
   if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;
   return MUON_OK;
 }
