@@ -122,6 +122,18 @@ float shape_scale(int64_t rows, int64_t cols, int mode) {
   }
 }
 
+// Multiprocessor count of a device (cached).
+int device_sms(int device) {
+  static int sms[64] = {};
+  const int dev = device & 63;
+  if (sms[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || n <= 0) n = 148;
+    sms[dev] = n;
+  }
+  return sms[dev];
+}
+
 // Elementwise launches over descriptors d[0..n) whose tile_start fields are
 // set: each launch covers up to MAX_SEGS segments of equal-shape matrices.
 struct SegLaunch {
@@ -350,32 +362,40 @@ muon_status set_device(muon_ctx* ctx) {
 // launches
 // ---------------------------------------------------------------------------
 template <int KIND, bool BMN>
-cudaError_t launch_gemm(muon_ctx* ctx, const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& g,
-                        cudaStream_t st) {
+cudaError_t launch_gemm(muon_ctx* ctx, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& aux,
+                        const CUtensorMap& out, const GemmArgs& g, cudaStream_t st) {
   static bool attr_done[64] = {};
+  static int max_pairs[64] = {};
   const int dev = ctx->device & 63;
   if (!attr_done[dev]) {
     cudaError_t e = cudaFuncSetAttribute(ns_gemm_kernel<KIND, BMN>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, gemm_cfg::SMEM_BYTES);
     if (e != cudaSuccess) return e;
+    // how many CTA pairs can be resident at once (one CTA per SM)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (device_sms(ctx->device) / 2));
+    cfg.blockDim = dim3(gemm_cfg::THREADS);
+    cfg.dynamicSmemBytes = gemm_cfg::SMEM_BYTES;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, ns_gemm_kernel<KIND, BMN>, &cfg) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      n = device_sms(ctx->device) / 2;
+    }
+    max_pairs[dev] = n;
     attr_done[dev] = true;
-  }
-  static int sms[64] = {};
-  if (sms[dev] == 0) {
-    cudaError_t e = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, ctx->device);
-    if (e != cudaSuccess) return e;
   }
   const int64_t tiles = int64_t(g.batch) * g.tiles_per_mat;
   if (tiles <= 0) return cudaSuccess;
   if (tiles > INT32_MAX) return cudaErrorInvalidValue;
-  const int64_t grid = std::min<int64_t>(tiles, sms[dev]);   // persistent: one CTA per SM
-  ns_gemm_kernel<KIND, BMN><<<unsigned(grid), gemm_cfg::THREADS, gemm_cfg::SMEM_BYTES, st>>>(a, b, g);
+  const int64_t pairs = std::min<int64_t>(tiles, max_pairs[dev]);   // persistent pairs
+  ns_gemm_kernel<KIND, BMN><<<unsigned(2 * pairs), gemm_cfg::THREADS, gemm_cfg::SMEM_BYTES, st>>>(a, b, aux, out,
+                                                                                               g);
   ctx->launches++;
   return cudaGetLastError();
 }
 
 struct RunMaps {
-  CUtensorMap x_r128[2], x_r256[2], x_mn[2], a_r128, a_r256, b_r128;
+  CUtensorMap x_r128[2], x_mn[2], x_r32[2], a_r128, a_r32, b_r128, b_r32;
 };
 
 // ns_steps quintic iterations on one run, X starting in x0.  Returns the
@@ -390,18 +410,18 @@ muon_status run_newton_schulz(muon_ctx* ctx, uint8_t* ws, const Run& r, const fl
   bool ok = true;
   for (int k = 0; k < 2; ++k) {
     ok &= encode_bf16_3d(&mp.x_r128[k], x[k], r.n, r.m, r.count, r.ld_n, 64, 128);
-    ok &= encode_bf16_3d(&mp.x_r256[k], x[k], r.n, r.m, r.count, r.ld_n, 64, 256);
     ok &= encode_bf16_3d(&mp.x_mn[k], x[k], r.n, r.m, r.count, r.ld_n, 64, 64);
+    ok &= encode_bf16_3d(&mp.x_r32[k], x[k], r.n, r.m, r.count, r.ld_n, 64, 32);
   }
   ok &= encode_bf16_3d(&mp.a_r128, A, r.m, r.m, r.count, r.ld_m, 64, 128);
-  ok &= encode_bf16_3d(&mp.a_r256, A, r.m, r.m, r.count, r.ld_m, 64, 256);
+  ok &= encode_bf16_3d(&mp.a_r32, A, r.m, r.m, r.count, r.ld_m, 64, 32);
   ok &= encode_bf16_3d(&mp.b_r128, B, r.m, r.m, r.count, r.ld_m, 64, 128);
+  ok &= encode_bf16_3d(&mp.b_r32, B, r.m, r.m, r.count, r.ld_m, 64, 32);
   if (!ok) return fail(ctx, MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed (run %lldx%lld)",
                        (long long)r.m, (long long)r.n);
 
-  const int tm = int(cdiv(r.m, gemm_cfg::BM));
-  const int tn_sym = int(cdiv(r.m, gemm_cfg::BN));
-  const int tn_upd = int(cdiv(r.n, gemm_cfg::BN));
+  const int tm = int(cdiv(r.m, gemm_cfg::TM));
+  const int tn_upd = int(cdiv(r.n, gemm_cfg::TN));
   int cur = 0;
   for (int it = 0; it < hp->ns_steps; ++it) {
     const bool first = (it == 0);
@@ -412,39 +432,37 @@ muon_status run_newton_schulz(muon_ctx* ctx, uint8_t* ws, const Run& r, const fl
     g.skip = skip;
     // A = alpha X X^T
     g.M = int(r.m); g.N = int(r.m); g.K = int(r.n);
-    g.tiles_m = tm; g.tiles_n = tn_sym;
-    g.tiles_per_mat = gemm_tiles_per_mat(EPI_GRAM, tm, tn_sym);
+    g.tiles_m = tm; g.tiles_n = tm;
+    g.tiles_per_mat = gemm_tiles_per_mat(EPI_GRAM, tm, tm);
     g.out = A; g.out_ld = r.ld_m; g.out_bs = r.m * r.ld_m;
-    g.aux = nullptr;
     g.norm2 = first ? norm2 : nullptr;
     g.alpha_pow = 2;
     {
       ProfScope ps(ctx, MUON_K_GRAM, st);
-      CUDA_TRY(ctx, (launch_gemm<EPI_GRAM, false>(ctx, mp.x_r128[cur], mp.x_r256[cur], g, st)));
+      CUDA_TRY(ctx, (launch_gemm<EPI_GRAM, false>(ctx, mp.x_r128[cur], mp.x_r128[cur], mp.a_r32, mp.a_r32, g, st)));
     }
     // B = b A + c A A
     g.K = int(r.m);
-    g.tiles_per_mat = gemm_tiles_per_mat(EPI_POLY, tm, tn_sym);
+    g.tiles_per_mat = gemm_tiles_per_mat(EPI_POLY, tm, tm);
     g.out = B;
-    g.aux = A; g.aux_ld = r.ld_m; g.aux_bs = r.m * r.ld_m;
     g.norm2 = nullptr;
     g.c0 = hp->ns_b; g.c1 = hp->ns_c;
     {
       ProfScope ps(ctx, MUON_K_POLY, st);
-      CUDA_TRY(ctx, (launch_gemm<EPI_POLY, false>(ctx, mp.a_r128, mp.a_r256, g, st)));
+      CUDA_TRY(ctx, (launch_gemm<EPI_POLY, false>(ctx, mp.a_r128, mp.a_r128, mp.a_r32, mp.b_r32, g, st)));
     }
     // X' = alpha (a X + B X)
     g.M = int(r.m); g.N = int(r.n); g.K = int(r.m);
     g.tiles_n = tn_upd;
     g.tiles_per_mat = gemm_tiles_per_mat(EPI_UPDATE, tm, tn_upd);
     g.out = x[cur ^ 1]; g.out_ld = r.ld_n; g.out_bs = r.m * r.ld_n;
-    g.aux = x[cur]; g.aux_ld = r.ld_n; g.aux_bs = r.m * r.ld_n;
     g.norm2 = first ? norm2 : nullptr;
     g.alpha_pow = 1;
     g.c0 = hp->ns_a;
     {
       ProfScope ps(ctx, MUON_K_UPDATE, st);
-      CUDA_TRY(ctx, (launch_gemm<EPI_UPDATE, true>(ctx, mp.b_r128, mp.x_mn[cur], g, st)));
+      CUDA_TRY(ctx, (launch_gemm<EPI_UPDATE, true>(ctx, mp.b_r128, mp.x_mn[cur], mp.x_r32[cur], mp.x_r32[cur ^ 1],
+                                                   g, st)));
     }
     cur ^= 1;
   }

@@ -16,14 +16,27 @@
 // polynomial terms are added.  alpha folds the Frobenius normalisation of the
 // first iteration in (alpha = s^2 for GRAM, s for UPDATE, s = 1/(||U||+eps)).
 //
-// Persistent CTAs, one per SM, stride over the tile list.  Warp 0 issues TMA
-// loads into a 4-stage smem ring that runs across tile boundaries, warp 1
-// owns TMEM (two 128x256 fp32 accumulators) and issues tcgen05.mma from one
-// thread, warps 2..9 drain the other accumulator meanwhile: the epilogue of
-// one tile overlaps the main loop of the next.  Epilogue warp w reads TMEM
-// lanes 32*(w%4) .. +31 and one 128-column half of the tile; its stores are
-// staged through shared memory so that global writes (direct and mirrored)
-// are whole 64-byte row segments.
+// CTA pairs.  A cluster of two CTAs on two SMs computes one 256x256 output
+// tile with tcgen05.mma.cta_group::2: CTA r holds rows [128r, 128r+128) of
+// the A tile and rows [128r, 128r+128) of the B tile (N side) in its own
+// shared memory and receives rows [128r, 128r+128) of the accumulator in its
+// own TMEM.  Per SM this halves the operand bytes per FLOP of a 128x256 tile.
+// Both CTAs load their halves with TMA (no multicast) and signal the leader's
+// (rank 0) "full" barrier; the leader's single MMA thread waits for both
+// halves, issues the MMAs and commits to the "empty"/"accumulator ready"
+// barriers of both CTAs at once; both CTAs' epilogue warps report a drained
+// accumulator to the leader.
+//
+// Pairs are persistent (one CTA per SM) and stride over the tile list; two
+// 128x256 fp32 accumulators per CTA (512 TMEM columns) let eight epilogue
+// warps drain one tile while the next is computed.  Epilogue warp w reads
+// TMEM lanes 32*(w%4) .. +31 and one 128-column half of the CTA's 128x256
+// accumulator.  Its 32x128 slice of the epilogue input (A for the poly, X for
+// the update) arrives by TMA into a 128-byte-swizzled shared region before
+// the accumulator is ready; the warp reads it and writes its output back in
+// place (the swizzle keeps both conflict-free), then one lane stores the
+// slice with TMA.  Mirrored blocks of the symmetric products leave through a
+// small staging buffer as 64-byte row segments.
 #pragma once
 
 #include "sm100_ptx.cuh"
@@ -33,33 +46,37 @@ namespace muon {
 enum EpiKind : int { EPI_GRAM = 0, EPI_POLY = 1, EPI_UPDATE = 2 };
 
 namespace gemm_cfg {
-constexpr int BM = 128;
-constexpr int BN = 256;
+constexpr int TM = 256;                              // pair tile rows (128 per CTA)
+constexpr int TN = 256;                              // pair tile columns
+constexpr int HM = 128;                              // rows per CTA
+constexpr int HN = 128;                              // B rows (N side) per CTA
 constexpr int BK = 64;
 constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BK * 2;                 // 16 KB
-constexpr int B_BYTES = BN * BK * 2;                 // 32 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;       // 48 KB
+constexpr int A_BYTES = HM * BK * 2;                 // 16 KB
+constexpr int B_BYTES = HN * BK * 2;                 // 16 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;       // 32 KB per CTA
 constexpr int MN_CHUNK_BYTES = BK * 128;             // one 64-wide MN chunk of B (MN-major)
 constexpr int EPI_WARPS = 8;
 constexpr int THREADS = 64 + EPI_WARPS * 32;         // producer, MMA, 8 epilogue warps
-constexpr int STG_PITCH = 80;                        // staged row: 64 B of data + 16 B pad
-constexpr int STG_BYTES = 32 * STG_PITCH;            // one 32x32 bf16 block per epilogue warp
+constexpr int EPI_BOX_BYTES = 32 * 128;              // 32 rows x 64 bf16, 128-byte swizzle
+constexpr int EPI_BYTES = 2 * EPI_BOX_BYTES;         // a warp's 32x128 slice
+constexpr int STG_PITCH = 64;                        // mirror staging: 32 rows x 64 B
+constexpr int STG_BYTES = 32 * STG_PITCH;
 constexpr int BAR_BYTES = 256;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_WARPS * STG_BYTES + BAR_BYTES + 1024;
-constexpr int ACC_COLS = 256;                        // one fp32 128x256 accumulator
+constexpr int SMEM_BYTES =
+    STAGES * STAGE_BYTES + EPI_WARPS * (EPI_BYTES + STG_BYTES) + BAR_BYTES + 1024;   // + alignment slack
+constexpr int ACC_COLS = 256;                        // one fp32 128x256 accumulator per CTA
 constexpr int TMEM_COLS = 2 * ACC_COLS;              // double-buffered
+static_assert(SMEM_BYTES <= 232448, "shared memory per block");
 }  // namespace gemm_cfg
 
 struct GemmArgs {
   int M, N, K;               // per-matrix extents
   int batch;                 // matrices in this launch
-  int tiles_m, tiles_n;      // ceil(M/128), ceil(N/256)
+  int tiles_m, tiles_n;      // ceil(M/256), ceil(N/256)
   int tiles_per_mat;
   __nv_bfloat16* out;        // output, ld out_ld, batch stride out_bs (elements)
   int64_t out_ld, out_bs;
-  const __nv_bfloat16* aux;  // POLY: A (same layout as out); UPDATE: X
-  int64_t aux_ld, aux_bs;
   const float* norm2;        // per-matrix ||U||_F^2 (nullptr: alpha = 1)
   int alpha_pow;             // alpha = s^alpha_pow
   float eps;
@@ -68,12 +85,10 @@ struct GemmArgs {
   const int* skip;           // non-null and set: do nothing (non-finite gradient)
 };
 
-// Number of 128x256 tiles per matrix that the GEMM kind computes.
+// Number of 256x256 pair tiles per matrix that the GEMM kind computes.
 __host__ __device__ inline int gemm_tiles_per_mat(int kind, int tiles_m, int tiles_n) {
   if (kind == EPI_UPDATE) return tiles_m * tiles_n;
-  int t = 0;
-  for (int i = 0; i < tiles_m; ++i) t += tiles_n - (i >> 1);
-  return t;
+  return tiles_m * (tiles_m + 1) / 2;     // upper triangle of 256-blocks (tiles_n == tiles_m)
 }
 
 __device__ __forceinline__ void decode_tile(int kind, const GemmArgs& a, int t, int& bidx, int& ti,
@@ -81,14 +96,14 @@ __device__ __forceinline__ void decode_tile(int kind, const GemmArgs& a, int t, 
   bidx = t / a.tiles_per_mat;
   t -= bidx * a.tiles_per_mat;
   if (kind == EPI_UPDATE) {
-    ti = t % a.tiles_m;          // row tiles fastest: CTAs in flight share X columns
+    ti = t % a.tiles_m;          // row tiles fastest: pairs in flight share X columns
     tj = t / a.tiles_m;
     return;
   }
   ti = 0;
   while (true) {
-    const int cnt = a.tiles_n - (ti >> 1);
-    if (t < cnt) { tj = (ti >> 1) + t; return; }
+    const int cnt = a.tiles_n - ti;
+    if (t < cnt) { tj = ti + t; return; }
     t -= cnt;
     ++ti;
   }
@@ -115,27 +130,37 @@ __device__ __forceinline__ void store_staged(const uint8_t* stg, __nv_bfloat16* 
   }
 }
 
+// tmA: A operand rows (box 64 x 128), tmB: B operand (K-major box 64 x 128
+// rows, or MN-major box 64 x 64), tmAux: epilogue input (box 64 x 32),
+// tmOut: output (box 64 x 32).  Launched in clusters of two CTAs.
 template <int KIND, bool B_MN_MAJOR>
-__global__ void __launch_bounds__(gemm_cfg::THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1)
     ns_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmAux, const __grid_constant__ CUtensorMap tmOut,
                    const GemmArgs args) {
   using namespace gemm_cfg;
   extern __shared__ uint8_t smem_raw[];
-  if (args.skip != nullptr && *args.skip) return;
+  if (args.skip != nullptr && *args.skip) return;   // uniform over the grid
 
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t* smem_epi = smem + STAGES * STAGE_BYTES;
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem_epi + EPI_WARPS * STG_BYTES);
+  uint8_t* smem_epi = smem + STAGES * STAGE_BYTES;             // 1024-aligned slices
+  uint8_t* smem_stg = smem_epi + EPI_WARPS * EPI_BYTES;
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem_stg + EPI_WARPS * STG_BYTES);
   uint64_t* empty_bar = full_bar + STAGES;
-  uint64_t* tfull_bar = empty_bar + STAGES;     // accumulator ready   (MMA -> epilogue)
-  uint64_t* tempty_bar = tfull_bar + 2;         // accumulator drained (epilogue -> MMA)
+  uint64_t* tfull_bar = empty_bar + STAGES;     // accumulator ready   (leader MMA -> both epilogues)
+  uint64_t* tempty_bar = tfull_bar + 2;         // accumulator drained (both epilogues -> leader MMA)
   uint64_t* drain_bar = tempty_bar + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  uint64_t* aux_bar = drain_bar + 1;            // one per epilogue warp
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(aux_bar + EPI_WARPS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();      // 0: leader of the pair
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
   const int total = args.batch * args.tiles_per_mat;
   const int nk = (args.K + BK - 1) / BK;
 
@@ -146,30 +171,34 @@ __global__ void __launch_bounds__(gemm_cfg::THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull_bar[a], 1);
-      mbar_init(&tempty_bar[a], EPI_WARPS);
+      mbar_init(&tempty_bar[a], 2 * EPI_WARPS);
     }
     mbar_init(drain_bar, 1);
+    for (int w = 0; w < EPI_WARPS; ++w) mbar_init(&aux_bar[w], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, TMEM_COLS);
-    tmem_relinquish();
+    tmem_alloc_pair(tmem_slot, TMEM_COLS);
+    tmem_relinquish_pair();
   }
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmB);
+    prefetch_tensormap(&tmOut);
+    if (KIND != EPI_GRAM) prefetch_tensormap(&tmAux);
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();              // both CTAs' barriers exist before any remote use
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    // ---------------- TMA producer ----------------
+    // ---------------- TMA producer (both CTAs load their halves) ----------------
     if (lane == 0) {
+      const uint32_t full0 = map_to_cta(smem_u32(full_bar), 0);   // leader's full_bar[0]
       int it = 0;
-      for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
+      for (int t = pair; t < total && !*abort_flag; t += npairs) {
         int bidx, ti, tj;
         decode_tile(KIND, args, t, bidx, ti, tj);
         for (int kb = 0; kb < nk; ++kb) {
@@ -178,33 +207,33 @@ __global__ void __launch_bounds__(gemm_cfg::THREADS, 1)
           if (!mbar_wait(&empty_bar[s], ph ^ 1, args.err, abort_flag)) break;
           uint8_t* a_dst = smem + s * STAGE_BYTES;
           uint8_t* b_dst = a_dst + A_BYTES;
-          mbar_arrive_expect_tx(&full_bar[s], STAGE_BYTES);
-          tma_load_3d(a_dst, &tmA, &full_bar[s], kb * BK, ti * BM, bidx);
+          const uint32_t fb = full0 + s * 8;
+          if (leader) mbar_arrive_expect_tx(&full_bar[s], 2 * STAGE_BYTES);
+          tma_load_3d_pair(a_dst, &tmA, fb, kb * BK, ti * TM + rank * HM, bidx);
           if (B_MN_MAJOR) {
 #pragma unroll
-            for (int c = 0; c < BN / 64; ++c)
-              tma_load_3d(b_dst + c * MN_CHUNK_BYTES, &tmB, &full_bar[s], tj * BN + c * 64, kb * BK,
-                          bidx);
+            for (int c = 0; c < HN / 64; ++c)
+              tma_load_3d_pair(b_dst + c * MN_CHUNK_BYTES, &tmB, fb, tj * TN + rank * HN + c * 64, kb * BK, bidx);
           } else {
-            tma_load_3d(b_dst, &tmB, &full_bar[s], kb * BK, tj * BN, bidx);
+            tma_load_3d_pair(b_dst, &tmB, fb, kb * BK, tj * TN + rank * HN, bidx);
           }
           ++it;
         }
       }
-      if (*abort_flag) {
-        // Let every copy this thread started land before the CTA exits.
+      if (*abort_flag && leader) {
+        // Let every copy that signals this CTA's barriers land before exit.
         volatile int no_abort = 0;
         for (int k = (it > STAGES ? it - STAGES : 0); k < it; ++k)
           mbar_wait(&full_bar[k % STAGES], (k / STAGES) & 1, args.err, &no_abort);
       }
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, B_MN_MAJOR);
+    // ---------------- MMA issuer (leader CTA only) ----------------
+    if (leader && lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(TM, TN, B_MN_MAJOR);
       int it = 0, lt = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++lt) {
+      for (int t = pair; t < total && ok; t += npairs, ++lt) {
         const int acc = lt & 1;
         if (!mbar_wait(&tempty_bar[acc], ((lt >> 1) & 1) ^ 1, args.err, abort_flag)) break;
         tc_fence_after();
@@ -221,56 +250,76 @@ __global__ void __launch_bounds__(gemm_cfg::THREADS, 1)
             const uint64_t adesc = sdesc_kmajor_sw128(a_base + kk * 32);
             const uint64_t bdesc = B_MN_MAJOR ? sdesc_mnmajor_sw128(b_base + kk * 16 * 128, MN_CHUNK_BYTES)
                                               : sdesc_kmajor_sw128(b_base + kk * 32);
-            mma_bf16_ss(d_tmem, adesc, bdesc, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+            mma_bf16_ss_pair(d_tmem, adesc, bdesc, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
           }
-          mma_commit(&empty_bar[s]);
+          mma_commit_pair_mc(&empty_bar[s], 0x3);
           ++it;
         }
-        if (ok) mma_commit(&tfull_bar[acc]);
+        if (ok) mma_commit_pair_mc(&tfull_bar[acc], 0x3);
       }
       if (*abort_flag) {
         // wait for the MMAs already issued before TMEM is released
         volatile int no_abort = 0;
-        mma_commit(drain_bar);
+        mma_commit_pair_mc(drain_bar, 0x1);
         mbar_wait(drain_bar, 0, args.err, &no_abort);
       }
     }
     __syncwarp();
   } else {
-    // ---------------- epilogue (warps 2..9) ----------------
+    // ---------------- epilogue (warps 2..9, both CTAs) ----------------
     const int ew = warp - 2;
     const int q = warp & 3;                 // TMEM lane quarter this warp may read
     const int half = ew >> 2;               // 128-column half of the tile
-    uint8_t* stg = smem_epi + ew * STG_BYTES;
+    uint8_t* slice = smem_epi + ew * EPI_BYTES;
+    uint8_t* stg = smem_stg + ew * STG_BYTES;
+    const uint32_t tempty0 = map_to_cta(smem_u32(tempty_bar), 0);
+    uint32_t aux_phase = 0;
+    bool aux_pending = false;
     int lt = 0;
-    for (int t = blockIdx.x; t < total; t += gridDim.x, ++lt) {
+    for (int t = pair; t < total; t += npairs, ++lt) {
       int bidx, ti, tj;
       decode_tile(KIND, args, t, bidx, ti, tj);
       const int acc = lt & 1;
+      const int rb = ti * 2 + static_cast<int>(rank);   // 128-row block index of this CTA
+      const int rbase = rb * HM + q * 32;
+      const int cb = tj * 2 + half;          // 128-column block index
+      const int col0 = cb * 128;
+      bool active = col0 < args.N && rbase < args.M;
+      bool mirror = false;
+      if (KIND != EPI_UPDATE) {
+        if (cb < rb) active = false;         // below the diagonal: mirrored by another tile
+        mirror = cb > rb;
+      }
+      const bool two_boxes = col0 + 64 < args.N;
+      // the slice is free once the previous tile's TMA store has read it;
+      // then fetch this tile's epilogue input into it
+      if (lane == 0) {
+        bulk_wait_group_read0();
+        if (KIND != EPI_GRAM && active) {
+          mbar_arrive_expect_tx(&aux_bar[ew], EPI_BYTES);
+          tma_load_3d(slice, &tmAux, &aux_bar[ew], col0, rbase, bidx);
+          tma_load_3d(slice + EPI_BOX_BYTES, &tmAux, &aux_bar[ew], col0 + 64, rbase, bidx);
+        }
+      }
+      if (KIND != EPI_GRAM && active) aux_pending = true;
+      __syncwarp();
       // warp-uniform decision: tcgen05.ld below is warp-collective
       const bool got = mbar_wait(&tfull_bar[acc], (lt >> 1) & 1, args.err, abort_flag);
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
-      const int rbase = ti * BM + q * 32;
-      const int r = rbase + lane;
-      const bool row_ok = r < args.M;
-      float alpha = 1.0f;
-      if (args.norm2 != nullptr) {
-        const float sc = 1.0f / (sqrtf(args.norm2[bidx]) + args.eps);
-        alpha = (args.alpha_pow == 2) ? sc * sc : sc;
-      }
-      __nv_bfloat16* out = args.out + static_cast<int64_t>(bidx) * args.out_bs;
-      const __nv_bfloat16* aux =
-          (KIND == EPI_GRAM) ? nullptr : args.aux + static_cast<int64_t>(bidx) * args.aux_bs;
-      const int cb = tj * 2 + half;          // 128-column block index
-      const int col0 = cb * 128;
-      bool active = col0 < args.N;
-      bool mirror = false;
-      if (KIND != EPI_UPDATE) {
-        if (cb < ti) active = false;         // below the diagonal: mirrored by another tile
-        mirror = cb > ti;
+      if (active && KIND != EPI_GRAM) {
+        const bool ok = mbar_wait(&aux_bar[ew], aux_phase, args.err, abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        aux_phase ^= 1;
+        aux_pending = false;
       }
       if (active) {
+        float alpha = 1.0f;
+        if (args.norm2 != nullptr) {
+          const float sc = 1.0f / (sqrtf(args.norm2[bidx]) + args.eps);
+          alpha = (args.alpha_pow == 2) ? sc * sc : sc;
+        }
+        __nv_bfloat16* out = args.out + static_cast<int64_t>(bidx) * args.out_bs;
 #pragma unroll 1
         for (int c32 = 0; c32 < 4; ++c32) {
           const int cbase = col0 + c32 * 32;
@@ -279,55 +328,45 @@ __global__ void __launch_bounds__(gemm_cfg::THREADS, 1)
           tmem_ld_32x32b_x32(tmem + acc * ACC_COLS + (static_cast<uint32_t>(q * 32) << 16) + half * 128 + c32 * 32,
                              raw);
           tmem_ld_wait();
+          // this thread's row `lane`, 4 x 16 B at columns c32*32 + u*8 of the slice
+          uint4* cell[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int cc = c32 * 32 + u * 8;
+            const int j = (cc & 63) >> 3;
+            cell[u] = reinterpret_cast<uint4*>(slice + (cc >> 6) * EPI_BOX_BYTES + lane * 128 +
+                                               ((j ^ (lane & 7)) << 4));
+          }
           float v[32];
-          const bool full = (cbase + 32 <= args.N);
           if (KIND == EPI_GRAM) {
 #pragma unroll
             for (int k = 0; k < 32; ++k) v[k] = alpha * __uint_as_float(raw[k]);
           } else {
-            float in[32];
-            if (row_ok && full) {
-              const uint4* src = reinterpret_cast<const uint4*>(aux + static_cast<int64_t>(r) * args.aux_ld + cbase);
-#pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                const uint4 w = src[u];
-                float2 f;
-                f = unpack_bf16x2(w.x); in[u * 8 + 0] = f.x; in[u * 8 + 1] = f.y;
-                f = unpack_bf16x2(w.y); in[u * 8 + 2] = f.x; in[u * 8 + 3] = f.y;
-                f = unpack_bf16x2(w.z); in[u * 8 + 4] = f.x; in[u * 8 + 5] = f.y;
-                f = unpack_bf16x2(w.w); in[u * 8 + 6] = f.x; in[u * 8 + 7] = f.y;
-              }
-            } else {
-#pragma unroll
-              for (int k = 0; k < 32; ++k)
-                in[k] = (row_ok && cbase + k < args.N)
-                            ? __bfloat162float(aux[static_cast<int64_t>(r) * args.aux_ld + cbase + k])
-                            : 0.0f;
-            }
-            if (KIND == EPI_POLY) {
-#pragma unroll
-              for (int k = 0; k < 32; ++k) v[k] = args.c0 * in[k] + args.c1 * __uint_as_float(raw[k]);
-            } else {
-#pragma unroll
-              for (int k = 0; k < 32; ++k) v[k] = alpha * (args.c0 * in[k] + __uint_as_float(raw[k]));
-            }
-          }
-          // direct: row `lane` of the staged block, then whole row segments out
-          {
-            uint4* srow = reinterpret_cast<uint4*>(stg + lane * STG_PITCH);
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-              uint4 w;
-              w.x = pack_bf16x2(v[u * 8 + 0], v[u * 8 + 1]);
-              w.y = pack_bf16x2(v[u * 8 + 2], v[u * 8 + 3]);
-              w.z = pack_bf16x2(v[u * 8 + 4], v[u * 8 + 5]);
-              w.w = pack_bf16x2(v[u * 8 + 6], v[u * 8 + 7]);
-              srow[u] = w;
+              const uint4 w = *cell[u];
+              float in[8];
+              float2 f;
+              f = unpack_bf16x2(w.x); in[0] = f.x; in[1] = f.y;
+              f = unpack_bf16x2(w.y); in[2] = f.x; in[3] = f.y;
+              f = unpack_bf16x2(w.z); in[4] = f.x; in[5] = f.y;
+              f = unpack_bf16x2(w.w); in[6] = f.x; in[7] = f.y;
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const float a = __uint_as_float(raw[u * 8 + e]);
+                v[u * 8 + e] = (KIND == EPI_POLY) ? args.c0 * in[e] + args.c1 * a : alpha * (args.c0 * in[e] + a);
+              }
             }
           }
-          __syncwarp();
-          store_staged(stg, out, args.out_ld, rbase, cbase, args.M, args.N, lane);
-          __syncwarp();
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            uint4 w;
+            w.x = pack_bf16x2(v[u * 8 + 0], v[u * 8 + 1]);
+            w.y = pack_bf16x2(v[u * 8 + 2], v[u * 8 + 3]);
+            w.z = pack_bf16x2(v[u * 8 + 4], v[u * 8 + 5]);
+            w.w = pack_bf16x2(v[u * 8 + 6], v[u * 8 + 7]);
+            *cell[u] = w;
+          }
           if (mirror) {
             // transposed block: staged row k holds column cbase+k of the tile
 #pragma unroll
@@ -338,19 +377,37 @@ __global__ void __launch_bounds__(gemm_cfg::THREADS, 1)
             __syncwarp();
           }
         }
+        // the slice now holds the output: make it visible to the TMA unit, store it
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_3d(&tmOut, slice, col0, rbase, bidx);
+          if (two_boxes) tma_store_3d(&tmOut, slice + EPI_BOX_BYTES, col0 + 64, rbase, bidx);
+          bulk_commit_group();
+        }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty_bar[acc]);
+      if (lane == 0) mbar_arrive_cluster(tempty0 + acc * 8);   // leader's tempty_bar[acc]
     }
+    if (lane == 0) {
+      if (aux_pending) {
+        volatile int no_abort = 0;
+        mbar_wait(&aux_bar[ew], aux_phase, args.err, &no_abort);   // let the copy land
+      }
+      bulk_wait_group0();
+    }
+    __syncwarp();
   }
 
-  // ---- teardown: TMEM is freed by the warp that allocated it ----
+  // ---- teardown: both CTAs done with each other's barriers and smem, then
+  // TMEM is freed by the warp that allocated it ----
   tc_fence_before();
   __syncthreads();
+  cluster_sync();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, TMEM_COLS);
+    tmem_dealloc_pair(tmem, TMEM_COLS);
   }
 }
 
