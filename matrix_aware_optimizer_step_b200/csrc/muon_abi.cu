@@ -362,20 +362,19 @@ muon_status set_device(muon_ctx* ctx) {
 // launches
 // ---------------------------------------------------------------------------
 template <int KIND, bool BMN>
-cudaError_t launch_gemm(muon_ctx* ctx, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& aux,
-                        const CUtensorMap& out, const GemmArgs& g, cudaStream_t st) {
+cudaError_t launch_gemm(muon_ctx* ctx, const GemmMaps& maps, const GemmArgs& g, cudaStream_t st) {
   static bool attr_done[64] = {};
   static int max_pairs[64] = {};
   const int dev = ctx->device & 63;
   if (!attr_done[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(ns_gemm_kernel<KIND, BMN>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, gemm_cfg::SMEM_BYTES);
+    cudaError_t e = cudaFuncSetAttribute(ns_gemm_kernel<KIND, BMN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         gemm_cfg::smem_bytes(KIND));
     if (e != cudaSuccess) return e;
     // how many CTA pairs can be resident at once (one CTA per SM)
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * (device_sms(ctx->device) / 2));
     cfg.blockDim = dim3(gemm_cfg::THREADS);
-    cfg.dynamicSmemBytes = gemm_cfg::SMEM_BYTES;
+    cfg.dynamicSmemBytes = gemm_cfg::smem_bytes(KIND);
     int n = 0;
     if (cudaOccupancyMaxActiveClusters(&n, ns_gemm_kernel<KIND, BMN>, &cfg) != cudaSuccess || n <= 0) {
       cudaGetLastError();
@@ -384,89 +383,112 @@ cudaError_t launch_gemm(muon_ctx* ctx, const CUtensorMap& a, const CUtensorMap& 
     max_pairs[dev] = n;
     attr_done[dev] = true;
   }
-  const int64_t tiles = int64_t(g.batch) * g.tiles_per_mat;
-  if (tiles <= 0) return cudaSuccess;
-  if (tiles > INT32_MAX) return cudaErrorInvalidValue;
-  const int64_t pairs = std::min<int64_t>(tiles, max_pairs[dev]);   // persistent pairs
-  ns_gemm_kernel<KIND, BMN><<<unsigned(2 * pairs), gemm_cfg::THREADS, gemm_cfg::SMEM_BYTES, st>>>(a, b, aux, out,
-                                                                                               g);
+  if (g.total <= 0) return cudaSuccess;
+  const int pairs = std::min(g.total, max_pairs[dev]);   // persistent pairs
+  ns_gemm_kernel<KIND, BMN><<<unsigned(2 * pairs), gemm_cfg::THREADS, gemm_cfg::smem_bytes(KIND), st>>>(maps, g);
   ctx->launches++;
   return cudaGetLastError();
 }
 
+// Device buffers and tensor maps of one shape run.
 struct RunMaps {
+  __nv_bfloat16 *x[2], *A, *B;
   CUtensorMap x_r128[2], x_mn[2], x_r32[2], a_r128, a_r32, b_r128, b_r32;
 };
 
-// ns_steps quintic iterations on one run, X starting in x0.  Returns the
-// buffer index (0/1) holding the result.
-muon_status run_newton_schulz(muon_ctx* ctx, uint8_t* ws, const Run& r, const float* norm2,
-                              const muon_hparams* hp, const int* skip, cudaStream_t st, int* final_buf) {
-  __nv_bfloat16* x[2] = {reinterpret_cast<__nv_bfloat16*>(ws + r.off_x0),
-                         reinterpret_cast<__nv_bfloat16*>(ws + r.off_x1)};
-  __nv_bfloat16* A = reinterpret_cast<__nv_bfloat16*>(ws + r.off_a);
-  __nv_bfloat16* B = reinterpret_cast<__nv_bfloat16*>(ws + r.off_b);
-  RunMaps mp;
+bool encode_run(uint8_t* ws, const Run& r, RunMaps& mp) {
+  mp.x[0] = reinterpret_cast<__nv_bfloat16*>(ws + r.off_x0);
+  mp.x[1] = reinterpret_cast<__nv_bfloat16*>(ws + r.off_x1);
+  mp.A = reinterpret_cast<__nv_bfloat16*>(ws + r.off_a);
+  mp.B = reinterpret_cast<__nv_bfloat16*>(ws + r.off_b);
   bool ok = true;
   for (int k = 0; k < 2; ++k) {
-    ok &= encode_bf16_3d(&mp.x_r128[k], x[k], r.n, r.m, r.count, r.ld_n, 64, 128);
-    ok &= encode_bf16_3d(&mp.x_mn[k], x[k], r.n, r.m, r.count, r.ld_n, 64, 64);
-    ok &= encode_bf16_3d(&mp.x_r32[k], x[k], r.n, r.m, r.count, r.ld_n, 64, 32);
+    ok &= encode_bf16_3d(&mp.x_r128[k], mp.x[k], r.n, r.m, r.count, r.ld_n, 64, 128);
+    ok &= encode_bf16_3d(&mp.x_mn[k], mp.x[k], r.n, r.m, r.count, r.ld_n, 64, 64);
+    ok &= encode_bf16_3d(&mp.x_r32[k], mp.x[k], r.n, r.m, r.count, r.ld_n, 64, 32);
   }
-  ok &= encode_bf16_3d(&mp.a_r128, A, r.m, r.m, r.count, r.ld_m, 64, 128);
-  ok &= encode_bf16_3d(&mp.a_r32, A, r.m, r.m, r.count, r.ld_m, 64, 32);
-  ok &= encode_bf16_3d(&mp.b_r128, B, r.m, r.m, r.count, r.ld_m, 64, 128);
-  ok &= encode_bf16_3d(&mp.b_r32, B, r.m, r.m, r.count, r.ld_m, 64, 32);
-  if (!ok) return fail(ctx, MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed (run %lldx%lld)",
-                       (long long)r.m, (long long)r.n);
+  ok &= encode_bf16_3d(&mp.a_r128, mp.A, r.m, r.m, r.count, r.ld_m, 64, 128);
+  ok &= encode_bf16_3d(&mp.a_r32, mp.A, r.m, r.m, r.count, r.ld_m, 64, 32);
+  ok &= encode_bf16_3d(&mp.b_r128, mp.B, r.m, r.m, r.count, r.ld_m, 64, 128);
+  ok &= encode_bf16_3d(&mp.b_r32, mp.B, r.m, r.m, r.count, r.ld_m, 64, 32);
+  return ok;
+}
 
-  const int tm = int(cdiv(r.m, gemm_cfg::TM));
-  const int tn_upd = int(cdiv(r.n, gemm_cfg::TN));
-  int cur = 0;
-  for (int it = 0; it < hp->ns_steps; ++it) {
-    const bool first = (it == 0);
-    GemmArgs g{};
-    g.batch = r.count;
-    g.eps = hp->eps;
-    g.err = ctx->dflags;
-    g.skip = skip;
-    // A = alpha X X^T
-    g.M = int(r.m); g.N = int(r.m); g.K = int(r.n);
-    g.tiles_m = tm; g.tiles_n = tm;
-    g.tiles_per_mat = gemm_tiles_per_mat(EPI_GRAM, tm, tm);
-    g.out = A; g.out_ld = r.ld_m; g.out_bs = r.m * r.ld_m;
-    g.norm2 = first ? norm2 : nullptr;
-    g.alpha_pow = 2;
-    {
-      ProfScope ps(ctx, MUON_K_GRAM, st);
-      CUDA_TRY(ctx, (launch_gemm<EPI_GRAM, false>(ctx, mp.x_r128[cur], mp.x_r128[cur], mp.a_r32, mp.a_r32, g, st)));
+// ns_steps quintic iterations on the runs of one chunk (X of each run starts
+// in its x0; after the call it is in x[ns_steps % 2]).  norm2s[j] is run j's
+// per-matrix ||U||^2.  Each product of an iteration is one launch over up to
+// MAX_PROBLEMS runs.
+muon_status run_newton_schulz(muon_ctx* ctx, uint8_t* ws, const Run* runs, int nruns,
+                              const float* const* norm2s, const muon_hparams* hp, const int* skip,
+                              cudaStream_t st) {
+  std::vector<RunMaps> mp(nruns);
+  for (int j = 0; j < nruns; ++j)
+    if (!encode_run(ws, runs[j], mp[j]))
+      return fail(ctx, MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed (run %lldx%lld)", (long long)runs[j].m,
+                  (long long)runs[j].n);
+  for (int b0 = 0; b0 < nruns; b0 += MAX_PROBLEMS) {
+    const int nb = std::min(MAX_PROBLEMS, nruns - b0);
+    int cur = 0;
+    for (int it = 0; it < hp->ns_steps; ++it) {
+      const bool first = (it == 0);
+      for (int kind = EPI_GRAM; kind <= EPI_UPDATE; ++kind) {
+        GemmMaps maps;
+        GemmArgs g{};
+        g.nprob = nb;
+        g.eps = hp->eps;
+        g.err = ctx->dflags;
+        g.skip = skip;
+        g.alpha_pow = kind == EPI_GRAM ? 2 : 1;
+        g.c0 = kind == EPI_POLY ? hp->ns_b : hp->ns_a;
+        g.c1 = hp->ns_c;
+        int tile = 0;
+        for (int j = 0; j < nb; ++j) {
+          const Run& r = runs[b0 + j];
+          const RunMaps& m = mp[b0 + j];
+          GemmProblem& P = g.p[j];
+          const int tm = int(cdiv(r.m, gemm_cfg::TM));
+          P.batch = r.count;
+          P.tiles_m = tm;
+          P.tile_start = tile;
+          if (kind == EPI_GRAM) {          // A = alpha X X^T
+            P.M = int(r.m); P.N = int(r.m); P.K = int(r.n);
+            P.tiles_n = tm;
+            P.out = m.A; P.out_ld = r.ld_m; P.out_bs = r.m * r.ld_m;
+            P.norm2 = first ? norm2s[b0 + j] : nullptr;
+            maps.a[j] = m.x_r128[cur]; maps.b[j] = m.x_r128[cur]; maps.aux[j] = m.a_r32; maps.out[j] = m.a_r32;
+          } else if (kind == EPI_POLY) {   // B = b A + c A A
+            P.M = int(r.m); P.N = int(r.m); P.K = int(r.m);
+            P.tiles_n = tm;
+            P.out = m.B; P.out_ld = r.ld_m; P.out_bs = r.m * r.ld_m;
+            P.norm2 = nullptr;
+            maps.a[j] = m.a_r128; maps.b[j] = m.a_r128; maps.aux[j] = m.a_r32; maps.out[j] = m.b_r32;
+          } else {                         // X' = alpha (a X + B X)
+            P.M = int(r.m); P.N = int(r.n); P.K = int(r.m);
+            P.tiles_n = int(cdiv(r.n, gemm_cfg::TN));
+            P.out = m.x[cur ^ 1]; P.out_ld = r.ld_n; P.out_bs = r.m * r.ld_n;
+            P.norm2 = first ? norm2s[b0 + j] : nullptr;
+            maps.a[j] = m.b_r128; maps.b[j] = m.x_mn[cur]; maps.aux[j] = m.x_r32[cur]; maps.out[j] = m.x_r32[cur ^ 1];
+          }
+          P.tiles_per_mat = gemm_tiles_per_mat(kind, P.tiles_m, P.tiles_n);
+          const int64_t tt = int64_t(tile) + int64_t(P.batch) * P.tiles_per_mat;
+          if (tt > INT32_MAX) return fail(ctx, MUON_ERR_UNSUPPORTED, "too many tiles in one launch");
+          tile = int(tt);
+        }
+        g.total = tile;
+        if (kind == EPI_GRAM) {
+          ProfScope ps(ctx, MUON_K_GRAM, st);
+          CUDA_TRY(ctx, (launch_gemm<EPI_GRAM, false>(ctx, maps, g, st)));
+        } else if (kind == EPI_POLY) {
+          ProfScope ps(ctx, MUON_K_POLY, st);
+          CUDA_TRY(ctx, (launch_gemm<EPI_POLY, false>(ctx, maps, g, st)));
+        } else {
+          ProfScope ps(ctx, MUON_K_UPDATE, st);
+          CUDA_TRY(ctx, (launch_gemm<EPI_UPDATE, true>(ctx, maps, g, st)));
+        }
+      }
+      cur ^= 1;
     }
-    // B = b A + c A A
-    g.K = int(r.m);
-    g.tiles_per_mat = gemm_tiles_per_mat(EPI_POLY, tm, tm);
-    g.out = B;
-    g.norm2 = nullptr;
-    g.c0 = hp->ns_b; g.c1 = hp->ns_c;
-    {
-      ProfScope ps(ctx, MUON_K_POLY, st);
-      CUDA_TRY(ctx, (launch_gemm<EPI_POLY, false>(ctx, mp.a_r128, mp.a_r128, mp.a_r32, mp.b_r32, g, st)));
-    }
-    // X' = alpha (a X + B X)
-    g.M = int(r.m); g.N = int(r.n); g.K = int(r.m);
-    g.tiles_n = tn_upd;
-    g.tiles_per_mat = gemm_tiles_per_mat(EPI_UPDATE, tm, tn_upd);
-    g.out = x[cur ^ 1]; g.out_ld = r.ld_n; g.out_bs = r.m * r.ld_n;
-    g.norm2 = first ? norm2 : nullptr;
-    g.alpha_pow = 1;
-    g.c0 = hp->ns_a;
-    {
-      ProfScope ps(ctx, MUON_K_UPDATE, st);
-      CUDA_TRY(ctx, (launch_gemm<EPI_UPDATE, true>(ctx, mp.b_r128, mp.x_mn[cur], mp.x_r32[cur], mp.x_r32[cur ^ 1],
-                                                   g, st)));
-    }
-    cur ^= 1;
   }
-  *final_buf = cur;
   return MUON_OK;
 }
 
@@ -696,9 +718,10 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
     }
     ctx->launches += segl.size();
     CUDA_TRY(ctx, cudaGetLastError());
-    for (const Run& r : c.runs) {
-      int fb = 0;
-      s = run_newton_schulz(ctx, ws, r, norm2 + (r.first - c.first), hp, skip, st, &fb);
+    {
+      std::vector<const float*> n2(c.runs.size());
+      for (size_t j = 0; j < c.runs.size(); ++j) n2[j] = norm2 + (c.runs[j].first - c.first);
+      s = run_newton_schulz(ctx, ws, c.runs.data(), int(c.runs.size()), n2.data(), hp, skip, st);
       if (s != MUON_OK) return s;
     }
     {
@@ -1157,8 +1180,8 @@ muon_status muon_orthogonalize_noalloc(const void* input, int32_t in_dtype, int6
   momentum_kernel<1><<<unsigned(tiles), EW_THREADS, 0, st>>>(ddesc, segl[0].t, 0, 0.f, 0, nullptr);
   if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;
   tmp.dflags = flags;
-  int fb = 0;
-  s = run_newton_schulz(&tmp, ws, r, d.norm2, hp, nullptr, st, &fb);
+  const float* n2 = d.norm2;
+  s = run_newton_schulz(&tmp, ws, &r, 1, &n2, hp, nullptr, st);
   tmp.dflags = nullptr;
   if (s != MUON_OK) return s;
   apply_kernel<1><<<unsigned(tiles), EW_THREADS, 0, st>>>(ddesc, segl[0].t, 0, hp->ns_steps == 0, hp->eps,

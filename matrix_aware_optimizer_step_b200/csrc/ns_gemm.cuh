@@ -51,7 +51,10 @@ constexpr int TN = 256;                              // pair tile columns
 constexpr int HM = 128;                              // rows per CTA
 constexpr int HN = 128;                              // B rows (N side) per CTA
 constexpr int BK = 64;
-constexpr int STAGES = 4;
+// Pipeline depth per product: the update product has no mirrored blocks and
+// spends the mirror staging space on a fifth stage.
+__host__ __device__ constexpr int stages_for(int kind) { return kind == 2 ? 5 : 4; }
+__host__ __device__ constexpr bool mirrors(int kind) { return kind != 2; }
 constexpr int A_BYTES = HM * BK * 2;                 // 16 KB
 constexpr int B_BYTES = HN * BK * 2;                 // 16 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;       // 32 KB per CTA
@@ -63,26 +66,48 @@ constexpr int EPI_BYTES = 2 * EPI_BOX_BYTES;         // a warp's 32x128 slice
 constexpr int STG_PITCH = 64;                        // mirror staging: 32 rows x 64 B
 constexpr int STG_BYTES = 32 * STG_PITCH;
 constexpr int BAR_BYTES = 256;
-constexpr int SMEM_BYTES =
-    STAGES * STAGE_BYTES + EPI_WARPS * (EPI_BYTES + STG_BYTES) + BAR_BYTES + 1024;   // + alignment slack
+__host__ __device__ constexpr int smem_bytes(int kind) {
+  return stages_for(kind) * STAGE_BYTES + EPI_WARPS * (EPI_BYTES + (mirrors(kind) ? STG_BYTES : 0)) + BAR_BYTES +
+         1024;   // + alignment slack
+}
 constexpr int ACC_COLS = 256;                        // one fp32 128x256 accumulator per CTA
 constexpr int TMEM_COLS = 2 * ACC_COLS;              // double-buffered
-static_assert(SMEM_BYTES <= 232448, "shared memory per block");
+static_assert(smem_bytes(0) <= 232448 && smem_bytes(1) <= 232448 && smem_bytes(2) <= 232448,
+              "shared memory per block");
 }  // namespace gemm_cfg
 
-struct GemmArgs {
+// One batched problem of a launch: `batch` equal-shape matrices.
+struct GemmProblem {
   int M, N, K;               // per-matrix extents
-  int batch;                 // matrices in this launch
+  int batch;                 // matrices
   int tiles_m, tiles_n;      // ceil(M/256), ceil(N/256)
   int tiles_per_mat;
+  int tile_start;            // first tile of this problem in the launch
   __nv_bfloat16* out;        // output, ld out_ld, batch stride out_bs (elements)
   int64_t out_ld, out_bs;
   const float* norm2;        // per-matrix ||U||_F^2 (nullptr: alpha = 1)
+};
+
+// A launch covers up to MAX_PROBLEMS problems of one product kind (the shape
+// runs of a chunk); their tensor maps travel in parameter space.
+constexpr int MAX_PROBLEMS = 4;
+
+struct GemmArgs {
+  int nprob;
+  int total;                 // tiles over all problems
+  GemmProblem p[MAX_PROBLEMS];
   int alpha_pow;             // alpha = s^alpha_pow
   float eps;
   float c0, c1;              // POLY: b, c.  UPDATE: a.
   int* err;                  // device error flags
   const int* skip;           // non-null and set: do nothing (non-finite gradient)
+};
+
+// Per problem: A operand rows (box 64 x 128), B operand (K-major box 64 x 128
+// rows, or MN-major box 64 x 64), epilogue input (box 64 x 32), output (box
+// 64 x 32).
+struct GemmMaps {
+  CUtensorMap a[MAX_PROBLEMS], b[MAX_PROBLEMS], aux[MAX_PROBLEMS], out[MAX_PROBLEMS];
 };
 
 // Number of 256x256 pair tiles per matrix that the GEMM kind computes.
@@ -91,18 +116,22 @@ __host__ __device__ inline int gemm_tiles_per_mat(int kind, int tiles_m, int til
   return tiles_m * (tiles_m + 1) / 2;     // upper triangle of 256-blocks (tiles_n == tiles_m)
 }
 
-__device__ __forceinline__ void decode_tile(int kind, const GemmArgs& a, int t, int& bidx, int& ti,
+__device__ __forceinline__ void decode_tile(int kind, const GemmArgs& a, int t, int& pi, int& bidx, int& ti,
                                             int& tj) {
-  bidx = t / a.tiles_per_mat;
-  t -= bidx * a.tiles_per_mat;
+  pi = 0;
+  while (pi + 1 < a.nprob && a.p[pi + 1].tile_start <= t) ++pi;
+  const GemmProblem& P = a.p[pi];
+  t -= P.tile_start;
+  bidx = t / P.tiles_per_mat;
+  t -= bidx * P.tiles_per_mat;
   if (kind == EPI_UPDATE) {
-    ti = t % a.tiles_m;          // row tiles fastest: pairs in flight share X columns
-    tj = t / a.tiles_m;
+    ti = t % P.tiles_m;          // row tiles fastest: pairs in flight share X columns
+    tj = t / P.tiles_m;
     return;
   }
   ti = 0;
   while (true) {
-    const int cnt = a.tiles_n - ti;
+    const int cnt = P.tiles_n - ti;
     if (t < cnt) { tj = ti + t; return; }
     t -= cnt;
     ++ti;
@@ -130,15 +159,12 @@ __device__ __forceinline__ void store_staged(const uint8_t* stg, __nv_bfloat16* 
   }
 }
 
-// tmA: A operand rows (box 64 x 128), tmB: B operand (K-major box 64 x 128
-// rows, or MN-major box 64 x 64), tmAux: epilogue input (box 64 x 32),
-// tmOut: output (box 64 x 32).  Launched in clusters of two CTAs.
+// Launched in clusters of two CTAs.
 template <int KIND, bool B_MN_MAJOR>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1)
-    ns_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ CUtensorMap tmAux, const __grid_constant__ CUtensorMap tmOut,
-                   const GemmArgs args) {
+    ns_gemm_kernel(const __grid_constant__ GemmMaps maps, const __grid_constant__ GemmArgs args) {
   using namespace gemm_cfg;
+  constexpr int STAGES = stages_for(KIND);
   extern __shared__ uint8_t smem_raw[];
   if (args.skip != nullptr && *args.skip) return;   // uniform over the grid
 
@@ -146,7 +172,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* smem_epi = smem + STAGES * STAGE_BYTES;             // 1024-aligned slices
   uint8_t* smem_stg = smem_epi + EPI_WARPS * EPI_BYTES;
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem_stg + EPI_WARPS * STG_BYTES);
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem_stg + (mirrors(KIND) ? EPI_WARPS * STG_BYTES : 0));
   uint64_t* empty_bar = full_bar + STAGES;
   uint64_t* tfull_bar = empty_bar + STAGES;     // accumulator ready   (leader MMA -> both epilogues)
   uint64_t* tempty_bar = tfull_bar + 2;         // accumulator drained (both epilogues -> leader MMA)
@@ -161,8 +187,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
   const bool leader = rank == 0;
   const int pair = blockIdx.x >> 1;
   const int npairs = gridDim.x >> 1;
-  const int total = args.batch * args.tiles_per_mat;
-  const int nk = (args.K + BK - 1) / BK;
+  const int total = args.total;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -183,10 +208,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
     tmem_relinquish_pair();
   }
   if (warp == 0 && lane == 0) {
-    prefetch_tensormap(&tmA);
-    prefetch_tensormap(&tmB);
-    prefetch_tensormap(&tmOut);
-    if (KIND != EPI_GRAM) prefetch_tensormap(&tmAux);
+    for (int p = 0; p < args.nprob; ++p) {
+      prefetch_tensormap(&maps.a[p]);
+      prefetch_tensormap(&maps.b[p]);
+      prefetch_tensormap(&maps.out[p]);
+      if (KIND != EPI_GRAM) prefetch_tensormap(&maps.aux[p]);
+    }
   }
   tc_fence_before();
   cluster_sync();              // both CTAs' barriers exist before any remote use
@@ -199,8 +226,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
       const uint32_t full0 = map_to_cta(smem_u32(full_bar), 0);   // leader's full_bar[0]
       int it = 0;
       for (int t = pair; t < total && !*abort_flag; t += npairs) {
-        int bidx, ti, tj;
-        decode_tile(KIND, args, t, bidx, ti, tj);
+        int pi, bidx, ti, tj;
+        decode_tile(KIND, args, t, pi, bidx, ti, tj);
+        const CUtensorMap* tmA = &maps.a[pi];
+        const CUtensorMap* tmB = &maps.b[pi];
+        const int nk = (args.p[pi].K + BK - 1) / BK;
         for (int kb = 0; kb < nk; ++kb) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
@@ -209,13 +239,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
           uint8_t* b_dst = a_dst + A_BYTES;
           const uint32_t fb = full0 + s * 8;
           if (leader) mbar_arrive_expect_tx(&full_bar[s], 2 * STAGE_BYTES);
-          tma_load_3d_pair(a_dst, &tmA, fb, kb * BK, ti * TM + rank * HM, bidx);
+          tma_load_3d_pair(a_dst, tmA, fb, kb * BK, ti * TM + rank * HM, bidx);
           if (B_MN_MAJOR) {
 #pragma unroll
             for (int c = 0; c < HN / 64; ++c)
-              tma_load_3d_pair(b_dst + c * MN_CHUNK_BYTES, &tmB, fb, tj * TN + rank * HN + c * 64, kb * BK, bidx);
+              tma_load_3d_pair(b_dst + c * MN_CHUNK_BYTES, tmB, fb, tj * TN + rank * HN + c * 64, kb * BK, bidx);
           } else {
-            tma_load_3d_pair(b_dst, &tmB, fb, kb * BK, tj * TN + rank * HN, bidx);
+            tma_load_3d_pair(b_dst, tmB, fb, kb * BK, tj * TN + rank * HN, bidx);
           }
           ++it;
         }
@@ -234,6 +264,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
       int it = 0, lt = 0;
       bool ok = true;
       for (int t = pair; t < total && ok; t += npairs, ++lt) {
+        int pi, bidx, ti, tj;
+        decode_tile(KIND, args, t, pi, bidx, ti, tj);
+        const int nk = (args.p[pi].K + BK - 1) / BK;
         const int acc = lt & 1;
         if (!mbar_wait(&tempty_bar[acc], ((lt >> 1) & 1) ^ 1, args.err, abort_flag)) break;
         tc_fence_after();
@@ -277,28 +310,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
     bool aux_pending = false;
     int lt = 0;
     for (int t = pair; t < total; t += npairs, ++lt) {
-      int bidx, ti, tj;
-      decode_tile(KIND, args, t, bidx, ti, tj);
+      int pi, bidx, ti, tj;
+      decode_tile(KIND, args, t, pi, bidx, ti, tj);
+      const GemmProblem& P = args.p[pi];
+      const CUtensorMap* tmAux = &maps.aux[pi];
+      const CUtensorMap* tmOut = &maps.out[pi];
       const int acc = lt & 1;
       const int rb = ti * 2 + static_cast<int>(rank);   // 128-row block index of this CTA
       const int rbase = rb * HM + q * 32;
       const int cb = tj * 2 + half;          // 128-column block index
       const int col0 = cb * 128;
-      bool active = col0 < args.N && rbase < args.M;
+      bool active = col0 < P.N && rbase < P.M;
       bool mirror = false;
       if (KIND != EPI_UPDATE) {
         if (cb < rb) active = false;         // below the diagonal: mirrored by another tile
         mirror = cb > rb;
       }
-      const bool two_boxes = col0 + 64 < args.N;
+      const bool two_boxes = col0 + 64 < P.N;
       // the slice is free once the previous tile's TMA store has read it;
       // then fetch this tile's epilogue input into it
       if (lane == 0) {
         bulk_wait_group_read0();
         if (KIND != EPI_GRAM && active) {
           mbar_arrive_expect_tx(&aux_bar[ew], EPI_BYTES);
-          tma_load_3d(slice, &tmAux, &aux_bar[ew], col0, rbase, bidx);
-          tma_load_3d(slice + EPI_BOX_BYTES, &tmAux, &aux_bar[ew], col0 + 64, rbase, bidx);
+          tma_load_3d(slice, tmAux, &aux_bar[ew], col0, rbase, bidx);
+          tma_load_3d(slice + EPI_BOX_BYTES, tmAux, &aux_bar[ew], col0 + 64, rbase, bidx);
         }
       }
       if (KIND != EPI_GRAM && active) aux_pending = true;
@@ -315,15 +351,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
       }
       if (active) {
         float alpha = 1.0f;
-        if (args.norm2 != nullptr) {
-          const float sc = 1.0f / (sqrtf(args.norm2[bidx]) + args.eps);
+        if (P.norm2 != nullptr) {
+          const float sc = 1.0f / (sqrtf(P.norm2[bidx]) + args.eps);
           alpha = (args.alpha_pow == 2) ? sc * sc : sc;
         }
-        __nv_bfloat16* out = args.out + static_cast<int64_t>(bidx) * args.out_bs;
+        __nv_bfloat16* out = P.out + static_cast<int64_t>(bidx) * P.out_bs;
 #pragma unroll 1
         for (int c32 = 0; c32 < 4; ++c32) {
           const int cbase = col0 + c32 * 32;
-          if (cbase >= args.N) break;
+          if (cbase >= P.N) break;
           uint32_t raw[32];
           tmem_ld_32x32b_x32(tmem + acc * ACC_COLS + (static_cast<uint32_t>(q * 32) << 16) + half * 128 + c32 * 32,
                              raw);
@@ -373,7 +409,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
             for (int k = 0; k < 32; ++k)
               reinterpret_cast<__nv_bfloat16*>(stg + k * STG_PITCH)[lane] = __float2bfloat16_rn(v[k]);
             __syncwarp();
-            store_staged(stg, out, args.out_ld, cbase, rbase, args.N, args.M, lane);
+            store_staged(stg, out, P.out_ld, cbase, rbase, P.N, P.M, lane);
             __syncwarp();
           }
         }
@@ -381,8 +417,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
         fence_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_store_3d(&tmOut, slice, col0, rbase, bidx);
-          if (two_boxes) tma_store_3d(&tmOut, slice + EPI_BOX_BYTES, col0 + 64, rbase, bidx);
+          tma_store_3d(tmOut, slice, col0, rbase, bidx);
+          if (two_boxes) tma_store_3d(tmOut, slice + EPI_BOX_BYTES, col0 + 64, rbase, bidx);
           bulk_commit_group();
         }
       }
