@@ -104,7 +104,8 @@ def step_work(w, aux, ns_steps=5):
         "apply": ("byte", elems * (2 + 4 + 4)),
         # adamw: read bf16 grad, read+write param, m, v
         "adamw": ("byte", aux_el * (2 + 3 * 8)),
-        "precondition": ("fflop", pre),
+        # tensor cores: G [S_hi; S_lo] executes twice the algorithmic 2 rows cols d
+        "precondition": ("flop", pre),
         "newton_refresh": ("fflop", refresh / max(1, w.refresh_every)),
     }, elems, aux_el
 
@@ -470,8 +471,9 @@ def main():
                                                else " HBM copy")}
     ns_flops = work["gram"][1] + work["poly"][1] + work["update"][1]
     ns_ms = sum(kernels.get(k, {"ms_per_step": 0})["ms_per_step"] for k in ("gram", "poly", "update"))
-    ew_bytes = work["momentum"][1] + work["apply"][1] + (work["adamw"][1] if aux else 0)
-    ew_ms = sum(kernels.get(k, {"ms_per_step": 0})["ms_per_step"] for k in ("momentum", "apply", "adamw"))
+    ew_kinds = [k for k in ("momentum", "apply", "adamw") if k in kernels]
+    ew_bytes = sum(work[k][1] for k in ew_kinds)
+    ew_ms = sum(kernels[k]["ms_per_step"] for k in ew_kinds)
 
     # ---- end to end through the public API with host buffers ----
     e2e = None

@@ -191,9 +191,20 @@ struct Chunk {
   size_t off_norm;               // count floats, then count counters, then per-tile partials
   size_t off_partials;
   size_t off_pgrad;              // preconditioned gradients (fp32), if any
+  bool tc_pre;                   // preconditioning on the tensor-core engine
+  size_t off_gc, off_sst;        // its bf16 gradient copies and S^-1 hi/lo stacks
   std::vector<Run> runs;
   size_t bytes;
 };
+
+// Tensor-core preconditioning needs block widths that are whole 64-wide
+// K blocks (the hi/lo halves of K must not share one).
+inline bool tc_precond_ok(const Item& it) { return (it.cols / it.precond_blocks) % 64 == 0; }
+inline size_t gc_bytes(const Item& it) { return size_t(it.rows) * round_up(it.cols, 8) * 2; }
+inline size_t sst_bytes(const Item& it) {
+  const size_t d = size_t(it.cols / it.precond_blocks);
+  return size_t(it.precond_blocks) * 2 * d * d * 2;
+}
 
 constexpr size_t kAlign = 256;
 
@@ -208,8 +219,28 @@ size_t layout_chunk(Chunk& c, const std::vector<Item>& items) {
     tiles += cdiv(items[i].rows, EW_TILE) * cdiv(items[i].cols, EW_TILE);
   off += round_up(size_t(tiles) * sizeof(float), kAlign);
   c.off_pgrad = off;
+  bool any_pre = false;
+  c.tc_pre = true;
   for (int i = c.first; i < c.first + c.count; ++i)
-    if (items[i].precond) off += round_up(size_t(items[i].rows) * items[i].cols * 4, kAlign);
+    if (items[i].precond) {
+      off += round_up(size_t(items[i].rows) * items[i].cols * 4, kAlign);
+      any_pre = true;
+      c.tc_pre = c.tc_pre && tc_precond_ok(items[i]);
+    }
+  c.tc_pre = c.tc_pre && any_pre;
+  c.off_gc = c.off_sst = off;
+  if (c.tc_pre) {
+    size_t g = 0, t = 0;
+    for (int i = c.first; i < c.first + c.count; ++i)
+      if (items[i].precond) {
+        g += gc_bytes(items[i]);
+        t += sst_bytes(items[i]);
+      }
+    c.off_gc = off;
+    off += round_up(g, kAlign);
+    c.off_sst = off;
+    off += round_up(t, kAlign);
+  }
   c.runs.clear();
   int i = c.first;
   while (i < c.first + c.count) {
@@ -492,6 +523,56 @@ muon_status run_newton_schulz(muon_ctx* ctx, uint8_t* ws, const Run* runs, int n
   return MUON_OK;
 }
 
+// Matrices of one shape preconditioned on the tensor cores as one batched
+// problem: consecutive bf16 copies in gc, S^-1 hi/lo stacks in sst, fp32
+// results in pg.
+struct PreProblem {
+  int64_t rows, cols, ldc;
+  int nb, d, count, last;
+  __nv_bfloat16* gc;
+  __nv_bfloat16* sst;
+  float* pg;
+  int64_t pg_stride;
+};
+
+// G' = G [S_hi; S_lo] for every problem, up to MAX_PROBLEMS per launch.
+muon_status run_precondition(muon_ctx* ctx, const std::vector<PreProblem>& probs, const int* skip,
+                             cudaStream_t st) {
+  for (size_t b0 = 0; b0 < probs.size(); b0 += MAX_PROBLEMS) {
+    const int nb = int(std::min<size_t>(MAX_PROBLEMS, probs.size() - b0));
+    GemmMaps maps;
+    GemmArgs g{};
+    g.nprob = nb;
+    g.err = ctx->dflags;
+    g.skip = skip;
+    int tile = 0;
+    for (int j = 0; j < nb; ++j) {
+      const PreProblem& q = probs[b0 + j];
+      bool ok = encode_bf16_3d(&maps.a[j], q.gc, q.cols, q.rows, q.count, q.ldc, 64, 128);
+      ok &= encode_bf16_3d(&maps.b[j], q.sst, q.d, 2 * q.d, int64_t(q.count) * q.nb, q.d, 64, 64);
+      if (!ok) return fail(ctx, MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed (precondition)");
+      maps.aux[j] = maps.a[j];
+      maps.out[j] = maps.a[j];
+      GemmProblem& P = g.p[j];
+      P.M = int(q.rows); P.N = q.d; P.K = 2 * q.d;
+      P.batch = q.count * q.nb;
+      P.tiles_m = int(cdiv(q.rows, gemm_cfg::TM));
+      P.tiles_n = int(cdiv(q.d, gemm_cfg::TN));
+      P.tiles_per_mat = gemm_tiles_per_mat(EPI_PRECOND, P.tiles_m, P.tiles_n);
+      P.tile_start = tile;
+      P.out32 = q.pg; P.out32_ld = q.cols; P.out32_bs = q.pg_stride;
+      P.nblocks = q.nb;
+      P.scale = 1.0f;
+      const int64_t tt = int64_t(tile) + int64_t(P.batch) * P.tiles_per_mat;
+      if (tt > INT32_MAX) return fail(ctx, MUON_ERR_UNSUPPORTED, "too many tiles in one launch");
+      tile = int(tt);
+    }
+    g.total = tile;
+    CUDA_TRY(ctx, (launch_gemm<EPI_PRECOND, true>(ctx, maps, g, st)));
+  }
+  return MUON_OK;
+}
+
 muon_status check_hparams(muon_ctx* ctx, const muon_hparams* hp) {
   if (!hp) return fail(ctx, MUON_ERR_INVALID_ARG, "hparams is NULL");
   if (hp->ns_steps < 0 || hp->ns_steps > 100)
@@ -590,12 +671,18 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
   std::vector<int64_t> chunk_tiles(chunks.size(), 0);
   std::vector<int> chunk_pbegin(chunks.size(), 0), chunk_pcount(chunks.size(), 0);
   std::vector<int64_t> chunk_ptiles(chunks.size(), 0);
+  // tensor-core preconditioning: staging descriptors and batched problems
+  std::vector<PrepDesc> prep;
+  std::vector<int> chunk_prep_begin(chunks.size(), 0), chunk_prep_count(chunks.size(), 0);
+  std::vector<std::vector<PreProblem>> chunk_pprob(chunks.size());
   const bool check = mode == 0 && hp->check_finite;
   for (size_t ci = 0; ci < chunks.size(); ++ci) {
     Chunk& c = chunks[ci];
     int64_t tiles = 0;
     size_t pg_off = c.off_pgrad;
+    size_t gc_off = c.off_gc, sst_off = c.off_sst;
     chunk_pbegin[ci] = int(pdescs.size());
+    chunk_prep_begin[ci] = int(prep.size());
     int64_t ptiles = 0;
     for (const Run& r : c.runs) {
       for (int k = 0; k < r.count; ++k) {
@@ -604,7 +691,37 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
         MatDesc& d = descs[idx];
         d.grad = it.grad;
         d.grad_dtype = it.grad_dtype;
-        if (it.precond) {
+        if (it.precond && c.tc_pre) {
+          float* pg = reinterpret_cast<float*>(ws + pg_off);
+          const size_t pg_bytes = round_up(size_t(it.rows) * it.cols * 4, kAlign);
+          pg_off += pg_bytes;
+          PrepDesc pd{};
+          pd.g = static_cast<const __nv_bfloat16*>(it.grad);
+          pd.gc = reinterpret_cast<__nv_bfloat16*>(ws + gc_off);
+          pd.s_inv = it.precond;
+          pd.sst = reinterpret_cast<__nv_bfloat16*>(ws + sst_off);
+          pd.rows = it.rows;
+          pd.cols = it.cols;
+          pd.ldc = round_up(it.cols, 8);
+          pd.nb = it.precond_blocks;
+          pd.d = int(it.cols / it.precond_blocks);
+          gc_off += gc_bytes(it);
+          sst_off += sst_bytes(it);
+          prep.push_back(pd);
+          std::vector<PreProblem>& pp = chunk_pprob[ci];
+          if (!pp.empty() && pp.back().rows == it.rows && pp.back().cols == it.cols && pp.back().nb == pd.nb &&
+              pp.back().last == idx - 1) {
+            pp.back().count++;
+            pp.back().last = idx;
+          } else {
+            PreProblem q{};
+            q.rows = it.rows; q.cols = it.cols; q.nb = pd.nb; q.d = pd.d; q.count = 1; q.last = idx;
+            q.ldc = pd.ldc; q.gc = pd.gc; q.sst = pd.sst; q.pg = pg; q.pg_stride = int64_t(pg_bytes / 4);
+            pp.push_back(q);
+          }
+          d.grad = pg;
+          d.grad_dtype = MUON_F32;
+        } else if (it.precond) {
           float* pg = reinterpret_cast<float*>(ws + pg_off);
           pg_off += round_up(size_t(it.rows) * it.cols * 4, kAlign);
           PrecondDesc p{};
@@ -647,16 +764,20 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
     chunk_tiles[ci] = tiles;
     chunk_pcount[ci] = int(pdescs.size()) - chunk_pbegin[ci];
     chunk_ptiles[ci] = ptiles;
+    chunk_prep_count[ci] = int(prep.size()) - chunk_prep_begin[ci];
   }
   const size_t mat_bytes = round_up(descs.size() * sizeof(MatDesc), kAlign);
-  std::vector<uint8_t> table(mat_bytes + pdescs.size() * sizeof(PrecondDesc));
+  const size_t pd_bytes = round_up(pdescs.size() * sizeof(PrecondDesc), kAlign);
+  std::vector<uint8_t> table(mat_bytes + pd_bytes + prep.size() * sizeof(PrepDesc));
   std::memcpy(table.data(), descs.data(), descs.size() * sizeof(MatDesc));
   if (!pdescs.empty()) std::memcpy(table.data() + mat_bytes, pdescs.data(), pdescs.size() * sizeof(PrecondDesc));
+  if (!prep.empty()) std::memcpy(table.data() + mat_bytes + pd_bytes, prep.data(), prep.size() * sizeof(PrepDesc));
   void* dtab = nullptr;
   s = upload_table(ctx, table.data(), table.size(), st, &dtab);
   if (s != MUON_OK) return s;
   const MatDesc* ddesc = static_cast<const MatDesc*>(dtab);
   const PrecondDesc* dpdesc = reinterpret_cast<const PrecondDesc*>(static_cast<uint8_t*>(dtab) + mat_bytes);
+  const PrepDesc* dprep = reinterpret_cast<const PrepDesc*>(static_cast<uint8_t*>(dtab) + mat_bytes + pd_bytes);
 
   const int* skip = nullptr;
   if (check) {
@@ -681,6 +802,7 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
     if (s != MUON_OK) return s;
     ddesc = static_cast<const MatDesc*>(dtab);
     dpdesc = reinterpret_cast<const PrecondDesc*>(static_cast<uint8_t*>(dtab) + mat_bytes);
+    dprep = reinterpret_cast<const PrepDesc*>(static_cast<uint8_t*>(dtab) + mat_bytes + pd_bytes);
     const MatDesc* draw = reinterpret_cast<const MatDesc*>(static_cast<uint8_t*>(dtab) + off);
     {
       ProfScope ps(ctx, MUON_K_OTHER, st);
@@ -697,6 +819,20 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
     const Chunk& c = chunks[ci];
     float* norm2 = reinterpret_cast<float*>(ws + c.off_norm);
     CUDA_TRY(ctx, cudaMemsetAsync(norm2, 0, c.count * (sizeof(float) + sizeof(unsigned)), st));
+    if (chunk_prep_count[ci] > 0) {
+      ProfScope ps(ctx, MUON_K_PRECONDITION, st);
+      int64_t most = 0;
+      for (int k = 0; k < chunk_prep_count[ci]; ++k) {
+        const PrepDesc& pd = prep[chunk_prep_begin[ci] + k];
+        most = std::max<int64_t>(most, std::max<int64_t>(pd.rows * pd.cols, int64_t(pd.nb) * pd.d * pd.d));
+      }
+      const dim3 grid(unsigned(std::min<int64_t>(cdiv(most, 256), 512)), unsigned(chunk_prep_count[ci]));
+      precond_prep_kernel<<<grid, 256, 0, st>>>(dprep + chunk_prep_begin[ci]);
+      ctx->launches++;
+      CUDA_TRY(ctx, cudaGetLastError());
+      s = run_precondition(ctx, chunk_pprob[ci], skip, st);
+      if (s != MUON_OK) return s;
+    }
     if (chunk_pcount[ci] > 0) {
       ProfScope ps(ctx, MUON_K_PRECONDITION, st);
       precond_kernel<<<unsigned(chunk_ptiles[ci]), PRE_THREADS, 0, st>>>(dpdesc + chunk_pbegin[ci],
@@ -991,11 +1127,19 @@ muon_status muon_newton_refresh(muon_ctx* ctx, const muon_act_desc* acts, int32_
   if (!ctx) return MUON_ERR_INVALID_ARG;
   if (n < 0 || (n > 0 && !acts)) return fail(ctx, MUON_ERR_INVALID_ARG, "bad activation list");
   if (!(damping >= 0.f) || !std::isfinite(damping)) return fail(ctx, MUON_ERR_INVALID_ARG, "damping must be >= 0");
-  std::vector<GramDesc> gd;
+  // Per d-wide activation block: a transposed bf16 copy (d x tokens), the
+  // fp32 second moment S (then its Cholesky factor) and the output S^-1.
+  struct GramProb {
+    int64_t tokens, d, ldt;
+    int count;
+    size_t xt_off, s_off;
+  };
+  std::vector<ActBlock> ab;
   std::vector<CholDesc> cd;
-  int64_t gtiles = 0;
-  size_t scratch = 0;
+  std::vector<GramProb> gp;
+  size_t s_total = 0, xt_total = 0;
   int max_d = 0;
+  int64_t max_tiles = 0;
   for (int i = 0; i < n; ++i) {
     const muon_act_desc& a = acts[i];
     if (!a.acts || !a.s_inv) return fail(ctx, MUON_ERR_INVALID_ARG, "activation %d: NULL pointer", i);
@@ -1007,52 +1151,108 @@ muon_status muon_newton_refresh(muon_ctx* ctx, const muon_act_desc* acts, int32_
       return fail(ctx, MUON_ERR_UNSUPPORTED, "activation %d: block width %lld > %d", i, (long long)d, CHOL_MAX_D);
     if (!aligned16(a.acts) || !aligned16(a.s_inv))
       return fail(ctx, MUON_ERR_INVALID_ARG, "activation %d: not 16-byte aligned", i);
+    const int64_t ldt = round_up(a.tokens, 8);
     for (int b = 0; b < a.nblocks; ++b) {
-      GramDesc g{};
-      g.acts = static_cast<const __nv_bfloat16*>(a.acts);
-      g.tokens = a.tokens;
-      g.width = a.width;
-      g.col0 = b * d;
-      g.d = d;
-      g.tiles = int(cdiv(d, GRAM_T));
-      g.tile_start = gtiles;
-      g.s_out = reinterpret_cast<float*>(scratch);          // offset, rebased below
-      gtiles += int64_t(g.tiles) * g.tiles;
-      gd.push_back(g);
+      ActBlock x{};
+      x.acts = static_cast<const __nv_bfloat16*>(a.acts);
+      x.xt = reinterpret_cast<__nv_bfloat16*>(xt_total);    // offset, rebased below
+      x.tokens = a.tokens;
+      x.width = a.width;
+      x.col0 = b * d;
+      x.d = d;
+      x.ldt = ldt;
+      ab.push_back(x);
       CholDesc c{};
-      c.a = reinterpret_cast<float*>(scratch);
+      c.a = reinterpret_cast<float*>(s_total);               // offset, rebased below
       c.inv = a.s_inv + size_t(b) * d * d;
       c.d = int(d);
       cd.push_back(c);
-      scratch += round_up(size_t(d) * d * 4, kAlign);
+      if (!gp.empty() && gp.back().tokens == a.tokens && gp.back().d == d) {
+        gp.back().count++;
+      } else {
+        gp.push_back(GramProb{a.tokens, d, ldt, 1, xt_total, s_total});
+      }
+      xt_total += size_t(d) * ldt * 2;
+      s_total += size_t(d) * d * 4;
       max_d = std::max(max_d, int(d));
+      max_tiles = std::max<int64_t>(max_tiles, cdiv(a.tokens, TPOSE_T) * cdiv(d, TPOSE_T));
     }
   }
-  if (gd.empty()) return MUON_OK;
+  if (ab.empty()) return MUON_OK;
+  if (ab.size() > 65535) return fail(ctx, MUON_ERR_UNSUPPORTED, "more than 65535 activation blocks");
   muon_status s = set_device(ctx);
   if (s != MUON_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   ctx->last_stream = st;
   CUDA_TRY(ctx, cudaGetLastError());
+  const size_t s_region = round_up(s_total, kAlign);
   void* wsv = nullptr;
-  s = ensure_workspace(ctx, scratch, &wsv);
+  s = ensure_workspace(ctx, s_region + xt_total, &wsv);
   if (s != MUON_OK) return s;
   uint8_t* ws = static_cast<uint8_t*>(wsv);
-  for (auto& g : gd) g.s_out = reinterpret_cast<float*>(ws + reinterpret_cast<size_t>(g.s_out));
+  for (auto& x : ab) x.xt = reinterpret_cast<__nv_bfloat16*>(ws + s_region + reinterpret_cast<size_t>(x.xt));
   for (auto& c : cd) c.a = reinterpret_cast<float*>(ws + reinterpret_cast<size_t>(c.a));
-  const size_t gbytes = round_up(gd.size() * sizeof(GramDesc), kAlign);
-  std::vector<uint8_t> table(gbytes + cd.size() * sizeof(CholDesc));
-  std::memcpy(table.data(), gd.data(), gd.size() * sizeof(GramDesc));
-  std::memcpy(table.data() + gbytes, cd.data(), cd.size() * sizeof(CholDesc));
+  const size_t ab_bytes = round_up(ab.size() * sizeof(ActBlock), kAlign);
+  std::vector<uint8_t> table(ab_bytes + cd.size() * sizeof(CholDesc));
+  std::memcpy(table.data(), ab.data(), ab.size() * sizeof(ActBlock));
+  std::memcpy(table.data() + ab_bytes, cd.data(), cd.size() * sizeof(CholDesc));
   void* dtab = nullptr;
   s = upload_table(ctx, table.data(), table.size(), st, &dtab);
   if (s != MUON_OK) return s;
-  const GramDesc* dg = static_cast<const GramDesc*>(dtab);
-  const CholDesc* dc = reinterpret_cast<const CholDesc*>(static_cast<uint8_t*>(dtab) + gbytes);
+  const ActBlock* dab = static_cast<const ActBlock*>(dtab);
+  const CholDesc* dc = reinterpret_cast<const CholDesc*>(static_cast<uint8_t*>(dtab) + ab_bytes);
   ProfScope ps(ctx, MUON_K_NEWTON_REFRESH, st);
-  act_gram_kernel<<<unsigned(gtiles), GRAM_THREADS, 0, st>>>(dg, int(gd.size()));
+  act_transpose_kernel<<<dim3(unsigned(max_tiles), unsigned(ab.size())), 256, 0, st>>>(dab);
   ctx->launches++;
   CUDA_TRY(ctx, cudaGetLastError());
+  // S = Xt Xt^T / tokens on the tensor cores, up to MAX_PROBLEMS shapes per launch
+  for (size_t b0 = 0; b0 < gp.size(); b0 += MAX_PROBLEMS) {
+    const int nb = int(std::min<size_t>(MAX_PROBLEMS, gp.size() - b0));
+    GemmMaps maps;
+    GemmArgs g{};
+    g.nprob = nb;
+    g.err = ctx->dflags;
+    int tile = 0;
+    for (int j = 0; j < nb; ++j) {
+      const GramProb& q = gp[b0 + j];
+      if (!encode_bf16_3d(&maps.a[j], ws + s_region + q.xt_off, q.tokens, q.d, q.count, q.ldt, 64, 128))
+        return fail(ctx, MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed (second moment)");
+      maps.b[j] = maps.a[j];
+      maps.aux[j] = maps.a[j];
+      maps.out[j] = maps.a[j];
+      GemmProblem& P = g.p[j];
+      P.M = int(q.d); P.N = int(q.d); P.K = int(q.tokens);
+      P.batch = q.count;
+      P.tiles_m = P.tiles_n = int(cdiv(q.d, gemm_cfg::TM));
+      P.tiles_per_mat = gemm_tiles_per_mat(EPI_GRAM32, P.tiles_m, P.tiles_n);
+      P.tile_start = tile;
+      P.out32 = reinterpret_cast<float*>(ws + q.s_off);
+      P.out32_ld = q.d;
+      P.out32_bs = q.d * q.d;
+      P.nblocks = 1;
+      P.scale = 1.0f / float(q.tokens);
+      const int64_t tt = int64_t(tile) + int64_t(P.batch) * P.tiles_per_mat;
+      if (tt > INT32_MAX) return fail(ctx, MUON_ERR_UNSUPPORTED, "too many tiles in one launch");
+      tile = int(tt);
+    }
+    g.total = tile;
+    CUDA_TRY(ctx, (launch_gemm<EPI_GRAM32, false>(ctx, maps, g, st)));
+  }
+  if (max_d <= CHOL_BLOCKED_MAX_D) {
+    // blocked factorisation and inverse, panels of 32 in shared memory
+    const int smem = cholb_smem_bytes(max_d);
+    CUDA_TRY(ctx, cudaFuncSetAttribute(cholesky_blocked_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    CUDA_TRY(ctx, cudaFuncSetAttribute(chol_inverse_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       cinv_smem_bytes(max_d)));
+    cholesky_blocked_kernel<<<unsigned(cd.size()), CHOLB_THREADS, smem, st>>>(dc, damping, ctx->dflags);
+    ctx->launches++;
+    CUDA_TRY(ctx, cudaGetLastError());
+    const int parts = int(cdiv(max_d, CB));
+    chol_inverse_kernel<<<unsigned(cd.size() * parts), CINV_THREADS, cinv_smem_bytes(max_d), st>>>(dc, parts);
+    ctx->launches++;
+    CUDA_TRY(ctx, cudaGetLastError());
+    return MUON_OK;
+  }
   cholesky_kernel<<<unsigned(cd.size()), CHOL_THREADS, 0, st>>>(dc, damping, ctx->dflags);
   ctx->launches++;
   CUDA_TRY(ctx, cudaGetLastError());

@@ -4,38 +4,25 @@
 // S = X^T X / N before the standard Muon step; the MLP contraction uses a
 // four-block diagonal S, one d x d inverse per block of d gradient columns.
 //
-//   act_gram_kernel     S_b = X_b^T X_b / N, fp32 accumulation of bf16
-//                       activations (products of bf16 values are exact in
-//                       fp32), one 64x64 tile of S per block.
-//   cholesky_kernel     S = L L^T in place (fp32), one block per matrix;
-//                       L^T is mirrored into the upper triangle so every
-//                       later read is along a row.
-//   chol_solve_kernel   S^-1 row by row: L y = e_j, then L^T x = y; one warp
-//                       per row, blocks split the rows of each matrix.
-//   precond_kernel      G' = G blockdiag(S_b^-1), bf16 G, fp32 S^-1 and
-//                       output, 64x64 tiles with 4x4 outputs per thread.
+//   act_transpose_kernel  a d-wide activation block, transposed to bf16
+//                         d x tokens: the K-major operand of S = Xt Xt^T / N,
+//                         which the tensor-core engine computes (GRAM32).
+//   cholesky_blocked_kernel  S = L L^T in place (fp32), panels of 32, one
+//                         block per matrix (d <= 1536).
+//   chol_inverse_kernel   S^-1 = L^-T L^-1, 32 columns per block, blocked
+//                         forward and backward substitution.
+//   cholesky_kernel, chol_solve_kernel  unblocked versions for larger d.
+//   precond_prep_kernel   bf16 copies of the gradients and S^-1 split into
+//                         bf16 hi + lo, the operands of G' = G [S_hi; S_lo]
+//                         on the tensor-core engine (PRECOND).
+//   precond_kernel        G' = G blockdiag(S_b^-1) with fp32 FMAs, for block
+//                         widths that are not a multiple of 64.
 #pragma once
 
 #include <cstdint>
 #include <cuda_bf16.h>
 
 namespace muon {
-
-// ---------------------------------------------------------------------------
-// second moment
-// ---------------------------------------------------------------------------
-constexpr int GRAM_T = 64;
-constexpr int GRAM_K = 32;
-constexpr int GRAM_THREADS = 256;
-
-struct GramDesc {
-  const __nv_bfloat16* acts;   // tokens x width
-  float* s_out;                // d x d
-  int64_t tokens, width, col0, d;
-  int64_t tile_start;
-  int32_t tiles;               // ceil(d / 64)
-  int32_t pad;
-};
 
 template <typename D>
 __device__ __forceinline__ int find_tile_desc(const D* __restrict__ d, int n, int64_t tile) {
@@ -45,52 +32,6 @@ __device__ __forceinline__ int find_tile_desc(const D* __restrict__ d, int n, in
     if (d[mid].tile_start <= tile) lo = mid; else hi = mid - 1;
   }
   return lo;
-}
-
-__global__ void __launch_bounds__(GRAM_THREADS)
-    act_gram_kernel(const GramDesc* __restrict__ descs, int n) {
-  __shared__ float xi[GRAM_K][GRAM_T + 4];
-  __shared__ float xj[GRAM_K][GRAM_T + 4];
-  const int64_t gt = blockIdx.x;
-  const GramDesc& g = descs[find_tile_desc(descs, n, gt)];
-  const int64_t lt = gt - g.tile_start;
-  const int64_t i0 = (lt / g.tiles) * GRAM_T, j0 = (lt % g.tiles) * GRAM_T;
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;   // 16 x 16 threads, 4x4 outputs each
-  float acc[4][4] = {};
-  for (int64_t t0 = 0; t0 < g.tokens; t0 += GRAM_K) {
-    // stage 32 tokens x 64 columns of both column blocks
-    for (int e = threadIdx.x; e < GRAM_K * GRAM_T; e += GRAM_THREADS) {
-      const int tk = e / GRAM_T, c = e % GRAM_T;
-      const int64_t t = t0 + tk;
-      const bool tok = t < g.tokens;
-      const int64_t ci = i0 + c, cj = j0 + c;
-      xi[tk][c] = (tok && ci < g.d) ? __bfloat162float(g.acts[t * g.width + g.col0 + ci]) : 0.f;
-      xj[tk][c] = (tok && cj < g.d) ? __bfloat162float(g.acts[t * g.width + g.col0 + cj]) : 0.f;
-    }
-    __syncthreads();
-#pragma unroll 4
-    for (int tk = 0; tk < GRAM_K; ++tk) {
-      float a[4], b[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) { a[u] = xi[tk][ty * 4 + u]; b[u] = xj[tk][tx * 4 + u]; }
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-#pragma unroll
-        for (int v = 0; v < 4; ++v) acc[u][v] += a[u] * b[v];
-    }
-    __syncthreads();
-  }
-  const float inv_n = 1.0f / float(g.tokens);
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const int64_t i = i0 + ty * 4 + u;
-    if (i >= g.d) continue;
-#pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      const int64_t j = j0 + tx * 4 + v;
-      if (j < g.d) g.s_out[i * g.d + j] = acc[u][v] * inv_n;
-    }
-  }
 }
 
 // ---------------------------------------------------------------------------
@@ -147,6 +88,210 @@ __global__ void __launch_bounds__(CHOL_THREADS)
     __syncthreads();
   }
   if (threadIdx.x == 0 && s_bad) atomicOr(err, kDevErrNotSPD);
+}
+
+// ---------------------------------------------------------------------------
+// Blocked versions (panel width 32), used when d <= CHOL_BLOCKED_MAX_D.
+// ---------------------------------------------------------------------------
+constexpr int CB = 32;                      // panel width
+constexpr int CBP = CB + 1;                 // padded row of a panel in smem
+constexpr int CHOLB_THREADS = 512;
+constexpr int CHOL_BLOCKED_MAX_D = 1536;    // panel of d x 33 floats fits in smem
+
+__host__ __device__ inline int cholb_smem_bytes(int d) { return d * CBP * 4; }
+
+// Right-looking Cholesky S = L L^T in place (lower triangle), one block per
+// matrix: factor the 32x32 diagonal block (one warp), solve the panel below it
+// row by row, subtract the panel's rank-32 product from the trailing lower
+// triangle in 4x4 register tiles.  The panel lives in shared memory.
+__global__ void __launch_bounds__(CHOLB_THREADS)
+    cholesky_blocked_kernel(const CholDesc* __restrict__ descs, float damping, int* err) {
+  extern __shared__ float pan[];            // [d][CBP]: rows below the diagonal block
+  __shared__ float dg[CB][CBP];
+  __shared__ int bad;
+  const CholDesc& c = descs[blockIdx.x];
+  float* a = c.a;
+  const int d = c.d;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) bad = 0;
+  if (damping != 0.f)
+    for (int i = tid; i < d; i += CHOLB_THREADS) a[int64_t(i) * d + i] += damping;
+  __syncthreads();
+  for (int p0 = 0; p0 < d; p0 += CB) {
+    const int nb = min(CB, d - p0);
+    for (int e = tid; e < CB * CB; e += CHOLB_THREADS) {
+      const int i = e / CB, j = e % CB;
+      dg[i][j] = (i < nb && j <= i) ? a[int64_t(p0 + i) * d + p0 + j] : 0.f;
+    }
+    __syncthreads();
+    if (warp == 0) {                        // unblocked Cholesky of the diagonal block
+      for (int k = 0; k < nb; ++k) {
+        if (lane == 0) {
+          float dkk = dg[k][k];
+          if (!(dkk > 0.f)) { bad = 1; dkk = 1.f; }
+          dg[k][k] = sqrtf(dkk);
+        }
+        __syncwarp();
+        const float lkk = dg[k][k];
+        if (lane > k && lane < nb) dg[lane][k] /= lkk;
+        __syncwarp();
+        if (lane > k && lane < nb)
+          for (int j = k + 1; j <= lane; ++j) dg[lane][j] -= dg[lane][k] * dg[j][k];
+        __syncwarp();
+      }
+    }
+    __syncthreads();
+    for (int e = tid; e < nb * nb; e += CHOLB_THREADS) {
+      const int i = e / nb, j = e % nb;
+      if (j <= i) a[int64_t(p0 + i) * d + p0 + j] = dg[i][j];
+    }
+    // panel: row i below solves x L11^T = a_i (forward substitution)
+    const int r0 = p0 + nb, nrows = d - r0;
+    for (int ii = tid; ii < nrows; ii += CHOLB_THREADS) {
+      float x[CB];
+      float* arow = a + int64_t(r0 + ii) * d + p0;
+#pragma unroll
+      for (int j = 0; j < CB; ++j) x[j] = j < nb ? arow[j] : 0.f;
+#pragma unroll
+      for (int j = 0; j < CB; ++j) {
+        if (j < nb) {
+          float sum = x[j];
+#pragma unroll
+          for (int k = 0; k < j; ++k) sum -= x[k] * dg[j][k];
+          x[j] = sum / dg[j][j];
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < CB; ++j)
+        if (j < nb) {
+          arow[j] = x[j];
+          pan[ii * CBP + j] = x[j];
+        }
+    }
+    __syncthreads();
+    // trailing lower triangle: A[i][j] -= sum_k P[i][k] P[j][k], 4x4 tiles
+    const int t4 = (nrows + 3) / 4;
+    const int ntiles = t4 * (t4 + 1) / 2;
+    for (int t = tid; t < ntiles; t += CHOLB_THREADS) {
+      int ti = int((sqrtf(8.f * t + 1.f) - 1.f) * 0.5f);
+      while (ti * (ti + 1) / 2 > t) --ti;
+      while ((ti + 1) * (ti + 2) / 2 <= t) ++ti;
+      const int tj = t - ti * (ti + 1) / 2;
+      float acc[4][4] = {};
+      for (int k = 0; k < nb; ++k) {
+        float pi[4], pj[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int ri = 4 * ti + u, rj = 4 * tj + u;
+          pi[u] = ri < nrows ? pan[ri * CBP + k] : 0.f;
+          pj[u] = rj < nrows ? pan[rj * CBP + k] : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int v = 0; v < 4; ++v) acc[u][v] += pi[u] * pj[v];
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = 4 * ti + u;
+        if (i >= nrows) continue;
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const int j = 4 * tj + v;
+          if (j <= i) a[int64_t(r0 + i) * d + r0 + j] -= acc[u][v];
+        }
+      }
+    }
+    __syncthreads();
+  }
+  if (tid == 0 && bad) atomicOr(err, kDevErrNotSPD);
+}
+
+constexpr int CINV_THREADS = 256;
+__host__ __device__ inline int cinv_smem_bytes(int d) { return d * CBP * 4; }
+
+// S^-1 = L^-T L^-1, 32 columns per block: forward L Y = E (E = columns
+// c0 .. c0+31 of I; rows of Y above c0 are zero), then L^T X = Y, row blocks
+// of 32 at a time, Y and X resident in shared memory; X^T is written as rows
+// c0 .. c0+31 of the (symmetric) S^-1.  L is read from the lower triangle.
+__global__ void __launch_bounds__(CINV_THREADS)
+    chol_inverse_kernel(const CholDesc* __restrict__ descs, int blocks_per_mat) {
+  extern __shared__ float y[];              // [d][CBP]
+  __shared__ float acc_s[CB][CBP];
+  const CholDesc& c = descs[blockIdx.x / blocks_per_mat];
+  const int d = c.d;
+  const int c0 = (blockIdx.x % blocks_per_mat) * CB;
+  if (c0 >= d) return;
+  const float* L = c.a;
+  const int tid = threadIdx.x;
+  const int orow = tid >> 3, ocol = (tid & 7) * 4;     // this thread's 4 outputs in a 32x32 block
+  const int nrb = (d + CB - 1) / CB;
+  const int rb0 = c0 / CB;
+  // ---- forward ----
+  for (int rb = rb0; rb < nrb; ++rb) {
+    const int rbase = rb * CB;
+    float acc[4];
+    const int r = rbase + orow;
+#pragma unroll
+    for (int v = 0; v < 4; ++v) acc[v] = (r == c0 + ocol + v) ? 1.f : 0.f;
+    if (r < d) {
+      const float* lrow = L + int64_t(r) * d;
+      for (int k = c0; k < rbase; ++k) {
+        const float l = lrow[k];
+#pragma unroll
+        for (int v = 0; v < 4; ++v) acc[v] -= l * y[k * CBP + ocol + v];
+      }
+    }
+#pragma unroll
+    for (int v = 0; v < 4; ++v) acc_s[orow][ocol + v] = acc[v];
+    __syncthreads();
+    // within the block: column j of the RHS by thread j (forward substitution)
+    if (tid < CB) {
+      const int j = tid;
+      for (int i = 0; i < CB && rbase + i < d; ++i) {
+        const float* lrow = L + int64_t(rbase + i) * d + rbase;
+        float sum = acc_s[i][j];
+        for (int k = 0; k < i; ++k) sum -= lrow[k] * y[(rbase + k) * CBP + j];
+        y[(rbase + i) * CBP + j] = sum / lrow[i];
+      }
+    }
+    __syncthreads();
+  }
+  // ---- backward: L^T X = Y, bottom row block first; X overwrites Y ----
+  for (int rb = nrb - 1; rb >= 0; --rb) {
+    const int rbase = rb * CB;
+    const int r = rbase + orow;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    if (r < d) {
+      if (r >= c0 || rb >= rb0) {
+#pragma unroll
+        for (int v = 0; v < 4; ++v) acc[v] = y[r * CBP + ocol + v];
+      }
+      for (int k = rbase + CB; k < d; ++k) {
+        const float l = L[int64_t(k) * d + r];     // L^T[r][k]
+#pragma unroll
+        for (int v = 0; v < 4; ++v) acc[v] -= l * y[k * CBP + ocol + v];
+      }
+    }
+#pragma unroll
+    for (int v = 0; v < 4; ++v) acc_s[orow][ocol + v] = acc[v];
+    __syncthreads();
+    if (tid < CB) {
+      const int j = tid;
+      const int nb = min(CB, d - rbase);
+      for (int i = nb - 1; i >= 0; --i) {
+        float sum = acc_s[i][j];
+        for (int k = i + 1; k < nb; ++k) sum -= L[int64_t(rbase + k) * d + rbase + i] * y[(rbase + k) * CBP + j];
+        y[(rbase + i) * CBP + j] = sum / L[int64_t(rbase + i) * d + rbase + i];
+      }
+    }
+    __syncthreads();
+  }
+  // ---- rows c0 .. c0+31 of S^-1 = columns of X ----
+  for (int e = tid; e < CB * d; e += CINV_THREADS) {
+    const int j = e / d, i = e % d;
+    if (c0 + j < d) c.inv[int64_t(c0 + j) * d + i] = y[i * CBP + j];
+  }
 }
 
 // Row j of S^-1 (= column j, S^-1 symmetric): forward L y = e_j, backward
@@ -250,6 +395,76 @@ __global__ void __launch_bounds__(PRE_THREADS)
     for (int v = 0; v < 4; ++v) {
       const int64_t cidx = c0 + tx * 4 + v;
       if (cidx < p.d) p.out[r * p.cols + gcol0 + cidx] = acc[u][v];
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Staging for the tensor-core Newton-Muon products
+// ---------------------------------------------------------------------------
+constexpr int TPOSE_T = 64;
+
+// One d-wide column block of a tokens x width activation matrix, to be
+// written transposed (d rows of `tokens`, leading dimension ldt) as the
+// K-major operand of the second-moment product.
+struct ActBlock {
+  const __nv_bfloat16* acts;
+  __nv_bfloat16* xt;
+  int64_t tokens, width, col0, d, ldt;
+};
+
+// grid.y = block, grid.x = 64x64 tiles of (tokens x d)
+__global__ void __launch_bounds__(256) act_transpose_kernel(const ActBlock* __restrict__ blocks) {
+  __shared__ __nv_bfloat16 t[TPOSE_T][TPOSE_T + 2];
+  const ActBlock& b = blocks[blockIdx.y];
+  const int64_t tiles_j = (b.d + TPOSE_T - 1) / TPOSE_T;
+  const int64_t t0 = (blockIdx.x / tiles_j) * TPOSE_T, j0 = (blockIdx.x % tiles_j) * TPOSE_T;
+  if (t0 >= b.tokens) return;
+  for (int e = threadIdx.x; e < TPOSE_T * TPOSE_T; e += 256) {
+    const int tt = e / TPOSE_T, jj = e % TPOSE_T;
+    const int64_t tok = t0 + tt, j = j0 + jj;
+    t[tt][jj] = (tok < b.tokens && j < b.d) ? b.acts[tok * b.width + b.col0 + j] : __float2bfloat16_rn(0.f);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < TPOSE_T * TPOSE_T; e += 256) {
+    const int jj = e / TPOSE_T, tt = e % TPOSE_T;
+    const int64_t tok = t0 + tt, j = j0 + jj;
+    if (tok < b.tokens && j < b.d) b.xt[j * b.ldt + tok] = t[tt][jj];
+  }
+}
+
+// One preconditioned matrix: its bf16 gradient copied to a batched layout
+// (rows x ldc) and its nb fp32 inverses split into bf16 hi/lo stacks
+// (2d x d each: rows 0..d-1 = hi, d..2d-1 = lo, with hi + lo ~ S^-1).
+struct PrepDesc {
+  const __nv_bfloat16* g;
+  __nv_bfloat16* gc;
+  const float* s_inv;
+  __nv_bfloat16* sst;
+  int64_t rows, cols, ldc;
+  int32_t nb, d;
+};
+
+// grid.y = matrix, grid.x strides over max(rows*cols, nb*d*d) elements
+__global__ void __launch_bounds__(256) precond_prep_kernel(const PrepDesc* __restrict__ descs) {
+  const PrepDesc& p = descs[blockIdx.y];
+  const int64_t ng = p.rows * p.cols;
+  const int64_t dd = static_cast<int64_t>(p.d) * p.d;
+  const int64_t ns = p.nb * dd;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * 256;
+  for (int64_t e = blockIdx.x * 256 + threadIdx.x; e < ng || e < ns; e += stride) {
+    if (e < ng) {
+      const int64_t r = e / p.cols, c = e - r * p.cols;
+      p.gc[r * p.ldc + c] = p.g[e];
+    }
+    if (e < ns) {
+      const int64_t b = e / dd, rem = e - b * dd;
+      const float v = p.s_inv[e];
+      const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
+      __nv_bfloat16* st = p.sst + b * 2 * dd;
+      st[rem] = hi;
+      st[dd + rem] = lo;
     }
   }
 }

@@ -37,13 +37,24 @@
 // place (the swizzle keeps both conflict-free), then one lane stores the
 // slice with TMA.  Mirrored blocks of the symmetric products leave through a
 // small staging buffer as 64-byte row segments.
+//
+// Two more products serve Newton-Muon ("The Newton-Muon Optimizer", "What Is
+// Newton-Muon?") and write fp32 directly from registers:
+//
+//   GRAM32   S = (1/N) Xt Xt^T          M = N = d, K = N tokens  symmetric
+//            (Xt: bf16 activation block, transposed; bf16 products are exact
+//            in fp32)
+//   PRECOND  G' = G [S_hi; S_lo]         M = rows, N = d, K = 2d
+//            (S^-1 = S_hi + S_lo split into two bf16 matrices stacked along
+//            K, G's column block read twice, so the product keeps close to
+//            fp32 precision)
 #pragma once
 
 #include "sm100_ptx.cuh"
 
 namespace muon {
 
-enum EpiKind : int { EPI_GRAM = 0, EPI_POLY = 1, EPI_UPDATE = 2 };
+enum EpiKind : int { EPI_GRAM = 0, EPI_POLY = 1, EPI_UPDATE = 2, EPI_GRAM32 = 3, EPI_PRECOND = 4 };
 
 namespace gemm_cfg {
 constexpr int TM = 256;                              // pair tile rows (128 per CTA)
@@ -53,8 +64,8 @@ constexpr int HN = 128;                              // B rows (N side) per CTA
 constexpr int BK = 64;
 // Pipeline depth per product: the update product has no mirrored blocks and
 // spends the mirror staging space on a fifth stage.
-__host__ __device__ constexpr int stages_for(int kind) { return kind == 2 ? 5 : 4; }
-__host__ __device__ constexpr bool mirrors(int kind) { return kind != 2; }
+__host__ __device__ constexpr int stages_for(int kind) { return (kind == 0 || kind == 1) ? 4 : 5; }
+__host__ __device__ constexpr bool mirrors(int kind) { return kind == 0 || kind == 1; }
 constexpr int A_BYTES = HM * BK * 2;                 // 16 KB
 constexpr int B_BYTES = HN * BK * 2;                 // 16 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;       // 32 KB per CTA
@@ -86,6 +97,13 @@ struct GemmProblem {
   __nv_bfloat16* out;        // output, ld out_ld, batch stride out_bs (elements)
   int64_t out_ld, out_bs;
   const float* norm2;        // per-matrix ||U||_F^2 (nullptr: alpha = 1)
+  // fp32 output (GRAM32, PRECOND): element (r, c) of matrix z at
+  // out32[z * out32_bs + r * out32_ld + c]; PRECOND: z = bidx / nblocks and
+  // c is offset by (bidx % nblocks) * N
+  float* out32;
+  int64_t out32_ld, out32_bs;
+  int nblocks;
+  float scale;               // GRAM32 / PRECOND: result = scale * sum
 };
 
 // A launch covers up to MAX_PROBLEMS problems of one product kind (the shape
@@ -110,9 +128,13 @@ struct GemmMaps {
   CUtensorMap a[MAX_PROBLEMS], b[MAX_PROBLEMS], aux[MAX_PROBLEMS], out[MAX_PROBLEMS];
 };
 
+__host__ __device__ constexpr bool symmetric_kind(int kind) {
+  return kind == EPI_GRAM || kind == EPI_POLY || kind == EPI_GRAM32;
+}
+
 // Number of 256x256 pair tiles per matrix that the GEMM kind computes.
 __host__ __device__ inline int gemm_tiles_per_mat(int kind, int tiles_m, int tiles_n) {
-  if (kind == EPI_UPDATE) return tiles_m * tiles_n;
+  if (!symmetric_kind(kind)) return tiles_m * tiles_n;
   return tiles_m * (tiles_m + 1) / 2;     // upper triangle of 256-blocks (tiles_n == tiles_m)
 }
 
@@ -124,7 +146,7 @@ __device__ __forceinline__ void decode_tile(int kind, const GemmArgs& a, int t, 
   t -= P.tile_start;
   bidx = t / P.tiles_per_mat;
   t -= bidx * P.tiles_per_mat;
-  if (kind == EPI_UPDATE) {
+  if (!symmetric_kind(kind)) {
     ti = t % P.tiles_m;          // row tiles fastest: pairs in flight share X columns
     tj = t / P.tiles_m;
     return;
@@ -212,7 +234,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
       prefetch_tensormap(&maps.a[p]);
       prefetch_tensormap(&maps.b[p]);
       prefetch_tensormap(&maps.out[p]);
-      if (KIND != EPI_GRAM) prefetch_tensormap(&maps.aux[p]);
+      if (KIND == EPI_POLY || KIND == EPI_UPDATE) prefetch_tensormap(&maps.aux[p]);
     }
   }
   tc_fence_before();
@@ -239,7 +261,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
           uint8_t* b_dst = a_dst + A_BYTES;
           const uint32_t fb = full0 + s * 8;
           if (leader) mbar_arrive_expect_tx(&full_bar[s], 2 * STAGE_BYTES);
-          tma_load_3d_pair(a_dst, tmA, fb, kb * BK, ti * TM + rank * HM, bidx);
+          if (KIND == EPI_PRECOND) {
+            // A: column block (bidx % nblocks) of matrix bidx / nblocks, read
+            // twice along K (against S_hi, then S_lo)
+            const int nbk = args.p[pi].nblocks, d = args.p[pi].N;
+            const int blk = bidx % nbk, mat = bidx / nbk;
+            int kx = kb * BK;
+            if (kx >= d) kx -= d;
+            tma_load_3d_pair(a_dst, tmA, fb, blk * d + kx, ti * TM + rank * HM, mat);
+          } else {
+            tma_load_3d_pair(a_dst, tmA, fb, kb * BK, ti * TM + rank * HM, bidx);
+          }
           if (B_MN_MAJOR) {
 #pragma unroll
             for (int c = 0; c < HN / 64; ++c)
@@ -322,7 +354,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
       const int col0 = cb * 128;
       bool active = col0 < P.N && rbase < P.M;
       bool mirror = false;
-      if (KIND != EPI_UPDATE) {
+      if (symmetric_kind(KIND)) {
         if (cb < rb) active = false;         // below the diagonal: mirrored by another tile
         mirror = cb > rb;
       }
@@ -331,19 +363,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
       // then fetch this tile's epilogue input into it
       if (lane == 0) {
         bulk_wait_group_read0();
-        if (KIND != EPI_GRAM && active) {
+        if ((KIND == EPI_POLY || KIND == EPI_UPDATE) && active) {
           mbar_arrive_expect_tx(&aux_bar[ew], EPI_BYTES);
           tma_load_3d(slice, tmAux, &aux_bar[ew], col0, rbase, bidx);
           tma_load_3d(slice + EPI_BOX_BYTES, tmAux, &aux_bar[ew], col0 + 64, rbase, bidx);
         }
       }
-      if (KIND != EPI_GRAM && active) aux_pending = true;
+      if ((KIND == EPI_POLY || KIND == EPI_UPDATE) && active) aux_pending = true;
       __syncwarp();
       // warp-uniform decision: tcgen05.ld below is warp-collective
       const bool got = mbar_wait(&tfull_bar[acc], (lt >> 1) & 1, args.err, abort_flag);
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
-      if (active && KIND != EPI_GRAM) {
+      if (active && (KIND == EPI_POLY || KIND == EPI_UPDATE)) {
         const bool ok = mbar_wait(&aux_bar[ew], aux_phase, args.err, abort_flag);
         if (!__all_sync(0xffffffffu, ok)) break;
         aux_phase ^= 1;
@@ -364,6 +396,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
           tmem_ld_32x32b_x32(tmem + acc * ACC_COLS + (static_cast<uint32_t>(q * 32) << 16) + half * 128 + c32 * 32,
                              raw);
           tmem_ld_wait();
+          if constexpr (KIND == EPI_GRAM32 || KIND == EPI_PRECOND) {
+            // fp32 result straight to global memory
+            const int r = rbase + lane;
+            int64_t zoff = static_cast<int64_t>(bidx) * P.out32_bs;
+            int coff = 0;
+            if (KIND == EPI_PRECOND) {
+              zoff = static_cast<int64_t>(bidx / P.nblocks) * P.out32_bs;
+              coff = (bidx % P.nblocks) * P.N;
+            }
+            float v[32];
+#pragma unroll
+            for (int k = 0; k < 32; ++k) v[k] = P.scale * __uint_as_float(raw[k]);
+            if (r < P.M) {
+              float* dst = P.out32 + zoff + static_cast<int64_t>(r) * P.out32_ld + coff + cbase;
+              if (cbase + 32 <= P.N && ((P.out32_ld | coff) & 3) == 0) {
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                  reinterpret_cast<float4*>(dst)[u] = make_float4(v[u * 4], v[u * 4 + 1], v[u * 4 + 2], v[u * 4 + 3]);
+              } else {
+                for (int k = 0; k < 32 && cbase + k < P.N; ++k) dst[k] = v[k];
+              }
+              if (KIND == EPI_GRAM32 && mirror) {
+                // (r, c) also goes to (c, r): lanes write consecutive r
+#pragma unroll
+                for (int k = 0; k < 32; ++k)
+                  if (cbase + k < P.N) P.out32[zoff + static_cast<int64_t>(cbase + k) * P.out32_ld + r] = v[k];
+              }
+            }
+          } else {
           // this thread's row `lane`, 4 x 16 B at columns c32*32 + u*8 of the slice
           uint4* cell[4];
 #pragma unroll
@@ -412,11 +473,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
             store_staged(stg, out, P.out_ld, cbase, rbase, P.N, P.M, lane);
             __syncwarp();
           }
+          }
         }
         // the slice now holds the output: make it visible to the TMA unit, store it
         fence_async_smem();
         __syncwarp();
-        if (lane == 0) {
+        if (lane == 0 && (KIND == EPI_GRAM || KIND == EPI_POLY || KIND == EPI_UPDATE)) {
           tma_store_3d(tmOut, slice, col0, rbase, bidx);
           if (two_boxes) tma_store_3d(tmOut, slice + EPI_BOX_BYTES, col0 + 64, rbase, bidx);
           bulk_commit_group();

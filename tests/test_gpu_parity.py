@@ -252,11 +252,14 @@ def test_adamw_vs_oracle(ctx, mx):
 
 
 def test_newton_refresh_vs_oracle(ctx, mx):
-    """S^-1 of the activation second moment, one block and four blocks."""
+    """S^-1 of the activation second moment: one block, four blocks, a
+    ragged block width (partial panel) and the GPT-2 width 768."""
     tokens = 2048
     acts = [wl.bf16_round_np(wl.np_normal((tokens, 192), 1.0, seed=12, index=0, role=wl.ROLE_ACT)),
-            wl.bf16_round_np(wl.np_normal((tokens, 4 * 96), 1.0, seed=12, index=1, role=wl.ROLE_ACT))]
-    nblocks = [1, 4]
+            wl.bf16_round_np(wl.np_normal((tokens, 4 * 96), 1.0, seed=12, index=1, role=wl.ROLE_ACT)),
+            wl.bf16_round_np(wl.np_normal((tokens, 104), 1.0, seed=12, index=2, role=wl.ROLE_ACT)),
+            wl.bf16_round_np(wl.np_normal((8192, 768), 1.0, seed=12, index=3, role=wl.ROLE_ACT))]
+    nblocks = [1, 4, 1, 1]
     at = [dev(a, torch.bfloat16) for a in acts]
     si = [torch.empty((nb, a.shape[1] // nb, a.shape[1] // nb), device="cuda") for a, nb in zip(acts, nblocks)]
     ctx.newton_refresh(at, si, nblocks)
