@@ -223,6 +223,20 @@ MUON_API muon_status muon_check_device(muon_ctx* ctx);
 /* Number of kernels this context has launched since creation. */
 MUON_API uint64_t muon_launch_count(const muon_ctx* ctx);
 
+/* Owner-computes sharding across `world` ranks (host only, no GPU needed):
+ * every matrix i of shape rows[i] x cols[i] is an independent unit of the
+ * step, so each goes to one owner rank, which alone keeps its momentum and
+ * runs its Muon step; owners then send the updated weights to the other
+ * ranks (the caller's collective).  Assignment: longest-processing-time
+ * first on the nominal cost 5 (4 m^2 n + 2 m^3) + 5600 rows cols (Newton-
+ * Schulz FLOPs plus elementwise bytes weighted by the B200 FLOP/byte
+ * ratio), largest unit to the least-loaded rank, ties to the lower index
+ * and the lower rank; deterministic, so every rank computes the same
+ * owners.  owner[i] receives the rank of matrix i.  Errors: n < 0,
+ * world < 1, NULL arrays or non-positive shapes -> MUON_ERR_INVALID_ARG. */
+MUON_API muon_status muon_partition(const int64_t* rows, const int64_t* cols, int32_t n, int32_t world,
+                                    int32_t* owner);
+
 /* Kernel classes timed by the context's profiler. */
 typedef enum {
   MUON_K_MOMENTUM = 0,   /* momentum + cast + Frobenius partial sums      */

@@ -34,7 +34,7 @@ EXPORTED = [
     "muon_last_error", "muon_status_string", "muon_query_workspace", "muon_set_workspace",
     "muon_step", "muon_orthogonalize", "muon_adamw_step", "muon_newton_refresh",
     "muon_check_device", "muon_launch_count", "muon_profile_enable", "muon_profile_read",
-    "muon_orthogonalize_noalloc",
+    "muon_orthogonalize_noalloc", "muon_partition",
 ]
 
 KERNEL_KINDS = ["momentum", "gram", "poly", "update", "apply", "adamw", "newton_refresh",
@@ -124,6 +124,8 @@ def load_library() -> ctypes.CDLL:
         "muon_profile_enable": (st, [vp, ctypes.c_int]),
         "muon_profile_read": (st, [vp, ctypes.POINTER(KernelTimes)]),
         "muon_orthogonalize_noalloc": (st, [vp, i32, i64, i64, vp, ctypes.POINTER(Hparams), vp]),
+        "muon_partition": (st, [ctypes.POINTER(i64), ctypes.POINTER(i64), i32, i32,
+                                ctypes.POINTER(i32)]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -156,6 +158,19 @@ def default_adamw_hparams(**over) -> AdamwHparams:
 # ---------------------------------------------------------------------------
 # marshalling helpers
 # ---------------------------------------------------------------------------
+
+def partition(shapes: Sequence, world: int) -> list:
+    """Owner rank of every (rows, cols) matrix (muon_partition, host only)."""
+    lib = load_library()
+    n = len(shapes)
+    rows = (ctypes.c_int64 * max(1, n))(*[int(s[0]) for s in shapes])
+    cols = (ctypes.c_int64 * max(1, n))(*[int(s[1]) for s in shapes])
+    own = (ctypes.c_int32 * max(1, n))()
+    st = lib.muon_partition(rows, cols, n, int(world), own)
+    if st != MUON_OK:
+        raise MuonError(st, f"muon_partition: {lib.muon_status_string(st).decode()}")
+    return [int(own[i]) for i in range(n)]
+
 
 def orthogonalize_noalloc(x, out, hp: Optional[Hparams] = None, stream=None):
     """out (fp32) = Newton-Schulz of x, without a context and without any

@@ -1282,6 +1282,28 @@ muon_status muon_check_device(muon_ctx* ctx) {
 
 uint64_t muon_launch_count(const muon_ctx* ctx) { return ctx ? ctx->launches : 0; }
 
+muon_status muon_partition(const int64_t* rows, const int64_t* cols, int32_t n, int32_t world, int32_t* owner) {
+  if (n < 0 || world < 1 || (n > 0 && (!rows || !cols || !owner))) return MUON_ERR_INVALID_ARG;
+  std::vector<std::pair<double, int>> cost(n);
+  for (int i = 0; i < n; ++i) {
+    if (rows[i] < 1 || cols[i] < 1) return MUON_ERR_INVALID_ARG;
+    const double m = double(std::min(rows[i], cols[i])), nn = double(std::max(rows[i], cols[i]));
+    cost[i] = {5.0 * (4.0 * m * m * nn + 2.0 * m * m * m) + 5600.0 * double(rows[i]) * double(cols[i]), i};
+  }
+  std::stable_sort(cost.begin(), cost.end(), [](const std::pair<double, int>& a, const std::pair<double, int>& b) {
+    return a.first > b.first;
+  });
+  std::vector<double> load(world, 0.0);
+  for (const auto& c : cost) {
+    int best = 0;
+    for (int r = 1; r < world; ++r)
+      if (load[r] < load[best]) best = r;
+    load[best] += c.first;
+    owner[c.second] = best;
+  }
+  return MUON_OK;
+}
+
 muon_status muon_profile_enable(muon_ctx* ctx, int enable) {
   if (!ctx) return MUON_ERR_INVALID_ARG;
   ctx->prof = enable != 0;

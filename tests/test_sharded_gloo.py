@@ -1,0 +1,68 @@
+"""Owner-computes sharding on CPU ranks (gloo, world size 2): owners from
+muon_partition are consistent and complete, the sharded step reproduces
+the single-process result exactly, and a rank that leaves before the
+exchange makes the other fail within its timeout instead of hanging."""
+
+import os
+import socket
+
+import numpy as np
+import pytest
+
+import dist_workers as dw
+import oracle
+
+
+def free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def test_partition_is_complete_balanced_and_deterministic():
+    from matrix_aware_optimizer_step_b200.binding import partition
+    import workloads as wl
+    shapes = [(m.rows, m.cols) for m in wl.gpt2_small_mats()]
+    for world in (1, 2, 3, 4, 8):
+        own = partition(shapes, world)
+        assert own == partition(shapes, world)
+        assert sorted(set(own)) == list(range(min(world, len(shapes))))
+        cost = [5 * (4 * min(r, c) ** 2 * max(r, c) + 2 * min(r, c) ** 3) + 5600 * r * c for r, c in shapes]
+        loads = [sum(x for x, o in zip(cost, own) if o == k) for k in range(world)]
+        # LPT is within 4/3 of the optimum, which is at least the mean load
+        assert max(loads) <= 4 / 3 * sum(loads) / world + max(cost)
+    with pytest.raises(Exception):
+        partition([(0, 3)], 2)
+
+
+def test_sharded_step_matches_single_process(tmp_path):
+    import torch.multiprocessing as mp
+    mp.spawn(dw.sharded_step_worker, args=(2, free_port(), str(tmp_path)), nprocs=2, join=True)
+    ws, gs = dw._inputs()
+    bufs = [np.zeros(s) for s in dw.SHAPES]
+    for k in range(3):
+        for i in range(len(ws)):
+            ws[i], bufs[i], _ = oracle.muon_step(ws[i], gs[k][i], bufs[i])
+    r0 = np.load(tmp_path / "rank0.npz")
+    r1 = np.load(tmp_path / "rank1.npz")
+    assert np.array_equal(r0["owner"], r1["owner"])
+    assert set(r0["owner"].tolist()) == {0, 1}
+    for i in range(len(ws)):
+        assert np.array_equal(r0[f"arr_{i}"], r1[f"arr_{i}"])
+        assert np.array_equal(r0[f"arr_{i}"], ws[i])
+
+
+def test_dead_rank_is_detected_by_timeout(tmp_path):
+    import multiprocessing as mpl
+    ctx = mpl.get_context("spawn")
+    port = free_port()
+    procs = [ctx.Process(target=dw.dying_rank_worker, args=(r, 2, port, str(tmp_path))) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert not p.is_alive()
+    status = (tmp_path / "rank0.txt").read_text()
+    assert status.startswith("error:"), status
