@@ -313,6 +313,8 @@ def main():
     ap.add_argument("--workload", default="gpt2-small", choices=sorted(wl.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--serial-adamw", action="store_true",
+                    help="run the aux AdamW on the Muon stream instead of a second stream")
     args = ap.parse_args()
     w, aux = workload_def(args.workload)
     if args.impl == "reference":
@@ -379,16 +381,28 @@ def main():
     hp = mx.default_hparams()
     ahp = mx.default_adamw_hparams()
     stream = torch.cuda.current_stream()
+    # The aux AdamW touches none of the Muon tensors: it runs on a second
+    # stream, forked from and joined back into the Muon stream every step,
+    # so its HBM traffic overlaps the tensor-core Newton-Schulz products.
+    aux_stream = stream if args.serial_adamw else torch.cuda.Stream()
+    fork_ev = [torch.cuda.Event() for _ in range(2)]
+    join_ev = [torch.cuda.Event() for _ in range(2)]
+    ctx_aux = ctx if args.serial_adamw else mx.MuonContext(local)
     pre_groups = [groups_for(s) for s in range(n_cycle)]
     adam_step = [0]
 
     def one_step(k):
+        if aux:
+            fork_ev[k & 1].record(stream)
+            aux_stream.wait_event(fork_ev[k & 1])
+            adam_step[0] += 1
+            ctx_aux.adamw_step(Ps, AGs[k % n_cycle], Ms, Vs, adam_step[0], ahp, aux_stream)
+            join_ev[k & 1].record(aux_stream)
         if newton and k % w.refresh_every == 0:
             ctx.newton_refresh(Acts, Sinv, nblk, 0.0, stream)
         ctx.step(pre_groups[k % n_cycle], hp, stream)
         if aux:
-            adam_step[0] += 1
-            ctx.adamw_step(Ps, AGs[k % n_cycle], Ms, Vs, adam_step[0], ahp, stream)
+            stream.wait_event(join_ev[k & 1])
 
     def barrier():
         if dist is not None:
@@ -421,11 +435,11 @@ def main():
     # ---- headline: device-resident inputs ----
     clocks = ClockSampler(local)
     clocks.start()
-    l0 = ctx.launch_count
+    l0 = ctx.launch_count + (ctx_aux.launch_count if ctx_aux is not ctx else 0)
     clocks.mark(0)
     ms = timed(args.steps, lambda k: one_step(args.warmup + k))
     clocks.mark(1)
-    launches = ctx.launch_count - l0
+    launches = ctx.launch_count + (ctx_aux.launch_count if ctx_aux is not ctx else 0) - l0
     clk = clocks.stop()
     ctx.check_device()
     ms_per_step = ms / args.steps
@@ -433,9 +447,17 @@ def main():
 
     # ---- per-kernel device times (events on the launching stream) ----
     ctx.profile(True)
+    if ctx_aux is not ctx:
+        ctx_aux.profile(True)
     timed(args.steps, lambda k: one_step(args.warmup + args.steps + k))
     kt = ctx.profile_read()
     ctx.profile(False)
+    if ctx_aux is not ctx:
+        ka = ctx_aux.profile_read()
+        ctx_aux.profile(False)
+        for kind, (t_ms, nl) in ka.items():
+            if nl:
+                kt[kind] = (kt[kind][0] + t_ms, kt[kind][1] + nl)
     work, elems, aux_el = step_work(w, aux, hp.ns_steps)
     pk = peaks()
     kernels = {}
@@ -515,6 +537,7 @@ def main():
         "config": {"workload": w.name, "matrices": len(w.mats), "hidden_params": elems,
                    "aux_params": aux_el, "grad_dtype": w.grad_dtype, "ns_steps": hp.ns_steps,
                    "grad_sets_cycled": n_cycle, "l2": "inputs larger than L2 (no flush)",
+                   "aux_adamw": "same stream" if args.serial_adamw else "second stream, joined every step",
                    "parallelism": f"replicas x{world}" if world > 1 else "single"},
         "ns_tflops": ns_flops / (ns_ms * 1e-3) / 1e12 if ns_ms else None,
         "ns_tflops_of_step": ns_flops / (ms_per_step * 1e-3) / 1e12,
@@ -525,6 +548,8 @@ def main():
         "launches_per_step": launches / args.steps,
         "clocks": clk, "e2e": e2e, "cpu_baseline": cpu,
     }
+    if ctx_aux is not ctx:
+        ctx_aux.close()
     ctx.close()
     if dist is not None:
         dist.destroy_process_group()
