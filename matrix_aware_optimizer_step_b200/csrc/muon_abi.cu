@@ -96,7 +96,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // bf16 tensor [batch][rows][ld] viewed as (cols, rows, batch), 128-byte swizzle.
 bool encode_bf16_3d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, uint64_t batch,
-                    uint64_t ld, uint32_t box_cols, uint32_t box_rows) {
+                    uint64_t ld, uint32_t box_cols, uint32_t box_rows,
+                    CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[3] = {cols, rows, batch};
@@ -104,7 +105,7 @@ bool encode_bf16_3d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t 
   cuuint32_t box[3] = {box_cols, box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -425,6 +426,7 @@ cudaError_t launch_gemm(muon_ctx* ctx, const GemmMaps& maps, const GemmArgs& g, 
 struct RunMaps {
   __nv_bfloat16 *x[2], *A, *B;
   CUtensorMap x_r128[2], x_mn[2], x_r32[2], a_r128, a_r32, b_r128, b_r32;
+  CUtensorMap x_c32[2], a_c32;   // 32 x 32 output chunks, 64-byte swizzle
 };
 
 bool encode_run(uint8_t* ws, const Run& r, RunMaps& mp) {
@@ -437,7 +439,9 @@ bool encode_run(uint8_t* ws, const Run& r, RunMaps& mp) {
     ok &= encode_bf16_3d(&mp.x_r128[k], mp.x[k], r.n, r.m, r.count, r.ld_n, 64, 128);
     ok &= encode_bf16_3d(&mp.x_mn[k], mp.x[k], r.n, r.m, r.count, r.ld_n, 64, 64);
     ok &= encode_bf16_3d(&mp.x_r32[k], mp.x[k], r.n, r.m, r.count, r.ld_n, 64, 32);
+    ok &= encode_bf16_3d(&mp.x_c32[k], mp.x[k], r.n, r.m, r.count, r.ld_n, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
   }
+  ok &= encode_bf16_3d(&mp.a_c32, mp.A, r.m, r.m, r.count, r.ld_m, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
   ok &= encode_bf16_3d(&mp.a_r128, mp.A, r.m, r.m, r.count, r.ld_m, 64, 128);
   ok &= encode_bf16_3d(&mp.a_r32, mp.A, r.m, r.m, r.count, r.ld_m, 64, 32);
   ok &= encode_bf16_3d(&mp.b_r128, mp.B, r.m, r.m, r.count, r.ld_m, 64, 128);
@@ -457,6 +461,10 @@ muon_status run_newton_schulz(muon_ctx* ctx, uint8_t* ws, const Run* runs, int n
     if (!encode_run(ws, runs[j], mp[j]))
       return fail(ctx, MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed (run %lldx%lld)", (long long)runs[j].m,
                   (long long)runs[j].n);
+  // Successive products walk their tile lists in opposite directions, so
+  // each launch starts on the matrices the previous one wrote last, which
+  // are still in L2 (the first Gram starts where the momentum pass ended).
+  int launch_no = 0;
   for (int b0 = 0; b0 < nruns; b0 += MAX_PROBLEMS) {
     const int nb = std::min(MAX_PROBLEMS, nruns - b0);
     int cur = 0;
@@ -470,8 +478,10 @@ muon_status run_newton_schulz(muon_ctx* ctx, uint8_t* ws, const Run* runs, int n
         g.err = ctx->dflags;
         g.skip = skip;
         g.alpha_pow = kind == EPI_GRAM ? 2 : 1;
-        g.c0 = kind == EPI_POLY ? hp->ns_b : hp->ns_a;
+        g.c0 = hp->ns_b;
         g.c1 = hp->ns_c;
+        g.c2 = hp->ns_a;
+        g.reverse = (launch_no++ & 1) ^ 1;
         int tile = 0;
         for (int j = 0; j < nb; ++j) {
           const Run& r = runs[b0 + j];
@@ -486,19 +496,19 @@ muon_status run_newton_schulz(muon_ctx* ctx, uint8_t* ws, const Run* runs, int n
             P.tiles_n = tm;
             P.out = m.A; P.out_ld = r.ld_m; P.out_bs = r.m * r.ld_m;
             P.norm2 = first ? norm2s[b0 + j] : nullptr;
-            maps.a[j] = m.x_r128[cur]; maps.b[j] = m.x_r128[cur]; maps.aux[j] = m.a_r32; maps.out[j] = m.a_r32;
-          } else if (kind == EPI_POLY) {   // B = b A + c A A
+            maps.a[j] = m.x_r128[cur]; maps.b[j] = m.x_r128[cur]; maps.aux[j] = m.a_r32; maps.out[j] = m.a_c32;
+          } else if (kind == EPI_POLY) {   // B' = b A + c A A + a I
             P.M = int(r.m); P.N = int(r.m); P.K = int(r.m);
             P.tiles_n = tm;
             P.out = m.B; P.out_ld = r.ld_m; P.out_bs = r.m * r.ld_m;
             P.norm2 = nullptr;
             maps.a[j] = m.a_r128; maps.b[j] = m.a_r128; maps.aux[j] = m.a_r32; maps.out[j] = m.b_r32;
-          } else {                         // X' = alpha (a X + B X)
+          } else {                         // X' = alpha B' X  (= alpha (a X + B X))
             P.M = int(r.m); P.N = int(r.n); P.K = int(r.m);
             P.tiles_n = int(cdiv(r.n, gemm_cfg::TN));
             P.out = m.x[cur ^ 1]; P.out_ld = r.ld_n; P.out_bs = r.m * r.ld_n;
             P.norm2 = first ? norm2s[b0 + j] : nullptr;
-            maps.a[j] = m.b_r128; maps.b[j] = m.x_mn[cur]; maps.aux[j] = m.x_r32[cur]; maps.out[j] = m.x_r32[cur ^ 1];
+            maps.a[j] = m.b_r128; maps.b[j] = m.x_mn[cur]; maps.aux[j] = m.x_r32[cur ^ 1]; maps.out[j] = m.x_c32[cur ^ 1];
           }
           P.tiles_per_mat = gemm_tiles_per_mat(kind, P.tiles_m, P.tiles_n);
           const int64_t tt = int64_t(tile) + int64_t(P.batch) * P.tiles_per_mat;

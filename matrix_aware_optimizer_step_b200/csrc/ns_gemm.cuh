@@ -6,8 +6,14 @@
 // section 3, X <- a X + b (X X^T) X + c (X X^T)^2 X):
 //
 //   GRAM    A  = alpha * X X^T           M = N = m, K = n   symmetric
-//   POLY    B  = b A + c A A             M = N = K = m      symmetric
-//   UPDATE  X' = alpha * (a X + B X)     M = m, N = n, K = m
+//   POLY    B' = b A + c A A + a I       M = N = K = m      symmetric
+//   UPDATE  X' = alpha * B' X            M = m, N = n, K = m
+//
+// a X + B X is computed as (a I + B) X: the same product, but the update
+// needs no second read of X.  Rounding a I + B to bf16 instead of B costs no
+// accuracy: late in the iteration B's diagonal is near -a + 0.7, so B' has
+// the smaller entries (bf16 emulation over 3x5 ... 4096x1024 matrices: equal
+// or lower error than rounding B).
 //
 // The symmetric products compute only the tiles that touch the upper
 // triangle and write each strictly-upper 128x128 block twice (direct and
@@ -31,11 +37,11 @@
 // 128x256 fp32 accumulators per CTA (512 TMEM columns) let eight epilogue
 // warps drain one tile while the next is computed.  Epilogue warp w reads
 // TMEM lanes 32*(w%4) .. +31 and one 128-column half of the CTA's 128x256
-// accumulator.  Its 32x128 slice of the epilogue input (A for the poly, X for
-// the update) arrives by TMA into a 128-byte-swizzled shared region before
+// accumulator.  For the poly, its 32x128 slice of the epilogue input A
+// arrives by TMA into a 128-byte-swizzled shared region before
 // the accumulator is ready; the warp reads it and writes its output back in
-// place (the swizzle keeps both conflict-free), then one lane stores the
-// slice with TMA.  Mirrored blocks of the symmetric products leave through a
+// place (the swizzle keeps both conflict-free); the other products write
+// the slice without reading it.  One lane then stores the slice with TMA.  Mirrored blocks of the symmetric products leave through a
 // small staging buffer as 64-byte row segments.
 //
 // Two more products serve Newton-Muon ("The Newton-Muon Optimizer", "What Is
@@ -62,10 +68,15 @@ constexpr int TN = 256;                              // pair tile columns
 constexpr int HM = 128;                              // rows per CTA
 constexpr int HN = 128;                              // B rows (N side) per CTA
 constexpr int BK = 64;
-// Pipeline depth per product: the update product has no mirrored blocks and
-// spends the mirror staging space on a fifth stage.
-__host__ __device__ constexpr int stages_for(int kind) { return (kind == 0 || kind == 1) ? 4 : 5; }
+// Pipeline depth per product.  GRAM and UPDATE stage their output in 2 KB
+// chunks (below) and spend the space saved on a fifth / sixth stage; the
+// update also has no mirrored blocks.
+__host__ __device__ constexpr int stages_for(int kind) { return kind == 0 ? 5 : kind == 1 ? 4 : kind == 2 ? 6 : 5; }
 __host__ __device__ constexpr bool mirrors(int kind) { return kind == 0 || kind == 1; }
+// Output leaves through two alternating 32x32 chunk buffers per warp
+// (GRAM, UPDATE) instead of a whole 32x128 slice (POLY reads its input A
+// into the slice and overwrites it in place).
+__host__ __device__ constexpr bool chunked_out(int kind) { return kind == 0 || kind == 2; }
 constexpr int A_BYTES = HM * BK * 2;                 // 16 KB
 constexpr int B_BYTES = HN * BK * 2;                 // 16 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;       // 32 KB per CTA
@@ -76,9 +87,12 @@ constexpr int EPI_BOX_BYTES = 32 * 128;              // 32 rows x 64 bf16, 128-b
 constexpr int EPI_BYTES = 2 * EPI_BOX_BYTES;         // a warp's 32x128 slice
 constexpr int STG_PITCH = 64;                        // mirror staging: 32 rows x 64 B
 constexpr int STG_BYTES = 32 * STG_PITCH;
+constexpr int CH_BYTES = 32 * 64;                    // 32 rows x 32 bf16, 64-byte swizzle
+constexpr int CH_BUFS = 2;
 constexpr int BAR_BYTES = 256;
 __host__ __device__ constexpr int smem_bytes(int kind) {
-  return stages_for(kind) * STAGE_BYTES + EPI_WARPS * (EPI_BYTES + (mirrors(kind) ? STG_BYTES : 0)) + BAR_BYTES +
+  return stages_for(kind) * STAGE_BYTES +
+         EPI_WARPS * ((chunked_out(kind) ? CH_BUFS * CH_BYTES : EPI_BYTES) + (mirrors(kind) ? STG_BYTES : 0)) + BAR_BYTES +
          1024;   // + alignment slack
 }
 constexpr int ACC_COLS = 256;                        // one fp32 128x256 accumulator per CTA
@@ -116,9 +130,10 @@ struct GemmArgs {
   GemmProblem p[MAX_PROBLEMS];
   int alpha_pow;             // alpha = s^alpha_pow
   float eps;
-  float c0, c1;              // POLY: b, c.  UPDATE: a.
+  float c0, c1, c2;          // POLY: b, c, and a (added on the diagonal)
   int* err;                  // device error flags
   const int* skip;           // non-null and set: do nothing (non-finite gradient)
+  int reverse;               // walk the tile list from its end (see run_newton_schulz)
 };
 
 // Per problem: A operand rows (box 64 x 128), B operand (K-major box 64 x 128
@@ -140,6 +155,7 @@ __host__ __device__ inline int gemm_tiles_per_mat(int kind, int tiles_m, int til
 
 __device__ __forceinline__ void decode_tile(int kind, const GemmArgs& a, int t, int& pi, int& bidx, int& ti,
                                             int& tj) {
+  if (a.reverse) t = a.total - 1 - t;
   pi = 0;
   while (pi + 1 < a.nprob && a.p[pi + 1].tile_start <= t) ++pi;
   const GemmProblem& P = a.p[pi];
@@ -193,7 +209,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* smem_epi = smem + STAGES * STAGE_BYTES;             // 1024-aligned slices
-  uint8_t* smem_stg = smem_epi + EPI_WARPS * EPI_BYTES;
+  uint8_t* smem_stg = smem_epi + EPI_WARPS * (chunked_out(KIND) ? CH_BUFS * CH_BYTES : EPI_BYTES);
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem_stg + (mirrors(KIND) ? EPI_WARPS * STG_BYTES : 0));
   uint64_t* empty_bar = full_bar + STAGES;
   uint64_t* tfull_bar = empty_bar + STAGES;     // accumulator ready   (leader MMA -> both epilogues)
@@ -234,7 +250,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
       prefetch_tensormap(&maps.a[p]);
       prefetch_tensormap(&maps.b[p]);
       prefetch_tensormap(&maps.out[p]);
-      if (KIND == EPI_POLY || KIND == EPI_UPDATE) prefetch_tensormap(&maps.aux[p]);
+      if (KIND == EPI_POLY) prefetch_tensormap(&maps.aux[p]);
     }
   }
   tc_fence_before();
@@ -253,6 +269,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
         const CUtensorMap* tmA = &maps.a[pi];
         const CUtensorMap* tmB = &maps.b[pi];
         const int nk = (args.p[pi].K + BK - 1) / BK;
+        // diagonal tile of a symmetric product: each CTA's B rows are its A
+        // rows, so only A is loaded and the MMA reads it for both operands
+        const bool diag = symmetric_kind(KIND) && ti == tj;
         for (int kb = 0; kb < nk; ++kb) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
@@ -260,7 +279,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
           uint8_t* a_dst = smem + s * STAGE_BYTES;
           uint8_t* b_dst = a_dst + A_BYTES;
           const uint32_t fb = full0 + s * 8;
-          if (leader) mbar_arrive_expect_tx(&full_bar[s], 2 * STAGE_BYTES);
+          if (leader) mbar_arrive_expect_tx(&full_bar[s], diag ? 2 * A_BYTES : 2 * STAGE_BYTES);
           if (KIND == EPI_PRECOND) {
             // A: column block (bidx % nblocks) of matrix bidx / nblocks, read
             // twice along K (against S_hi, then S_lo)
@@ -276,7 +295,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
 #pragma unroll
             for (int c = 0; c < HN / 64; ++c)
               tma_load_3d_pair(b_dst + c * MN_CHUNK_BYTES, tmB, fb, tj * TN + rank * HN + c * 64, kb * BK, bidx);
-          } else {
+          } else if (!diag) {
             tma_load_3d_pair(b_dst, tmB, fb, kb * BK, tj * TN + rank * HN, bidx);
           }
           ++it;
@@ -299,6 +318,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
         int pi, bidx, ti, tj;
         decode_tile(KIND, args, t, pi, bidx, ti, tj);
         const int nk = (args.p[pi].K + BK - 1) / BK;
+        const bool diag = symmetric_kind(KIND) && ti == tj;
         const int acc = lt & 1;
         if (!mbar_wait(&tempty_bar[acc], ((lt >> 1) & 1) ^ 1, args.err, abort_flag)) break;
         tc_fence_after();
@@ -309,7 +329,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
           if (!mbar_wait(&full_bar[s], ph, args.err, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_base = smem_u32(smem + s * STAGE_BYTES);
-          const uint32_t b_base = a_base + A_BYTES;
+          const uint32_t b_base = diag ? a_base : a_base + A_BYTES;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint64_t adesc = sdesc_kmajor_sw128(a_base + kk * 32);
@@ -335,7 +355,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
     const int ew = warp - 2;
     const int q = warp & 3;                 // TMEM lane quarter this warp may read
     const int half = ew >> 2;               // 128-column half of the tile
-    uint8_t* slice = smem_epi + ew * EPI_BYTES;
+    uint8_t* slice = smem_epi + ew * (chunked_out(KIND) ? CH_BUFS * CH_BYTES : EPI_BYTES);
+    uint32_t nch = 0;                       // output chunks stored so far (buffer = nch & 1)
     uint8_t* stg = smem_stg + ew * STG_BYTES;
     const uint32_t tempty0 = map_to_cta(smem_u32(tempty_bar), 0);
     uint32_t aux_phase = 0;
@@ -361,21 +382,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
       const bool two_boxes = col0 + 64 < P.N;
       // the slice is free once the previous tile's TMA store has read it;
       // then fetch this tile's epilogue input into it
-      if (lane == 0) {
+      if (lane == 0 && KIND == EPI_POLY) {
         bulk_wait_group_read0();
-        if ((KIND == EPI_POLY || KIND == EPI_UPDATE) && active) {
+        if (active) {
           mbar_arrive_expect_tx(&aux_bar[ew], EPI_BYTES);
           tma_load_3d(slice, tmAux, &aux_bar[ew], col0, rbase, bidx);
           tma_load_3d(slice + EPI_BOX_BYTES, tmAux, &aux_bar[ew], col0 + 64, rbase, bidx);
         }
       }
-      if ((KIND == EPI_POLY || KIND == EPI_UPDATE) && active) aux_pending = true;
+      if (KIND == EPI_POLY && active) aux_pending = true;
       __syncwarp();
       // warp-uniform decision: tcgen05.ld below is warp-collective
       const bool got = mbar_wait(&tfull_bar[acc], (lt >> 1) & 1, args.err, abort_flag);
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
-      if (active && (KIND == EPI_POLY || KIND == EPI_UPDATE)) {
+      if (active && KIND == EPI_POLY) {
         const bool ok = mbar_wait(&aux_bar[ew], aux_phase, args.err, abort_flag);
         if (!__all_sync(0xffffffffu, ok)) break;
         aux_phase ^= 1;
@@ -424,6 +445,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
                   if (cbase + k < P.N) P.out32[zoff + static_cast<int64_t>(cbase + k) * P.out32_ld + r] = v[k];
               }
             }
+          } else if constexpr (chunked_out(KIND)) {
+            float v[32];
+#pragma unroll
+            for (int k = 0; k < 32; ++k) v[k] = alpha * __uint_as_float(raw[k]);
+            // the store that last read this buffer (two chunks ago) is done with it
+            uint8_t* buf = slice + (nch & 1) * CH_BYTES;
+            if (lane == 0) bulk_wait_group_read1();
+            __syncwarp();
+            // row `lane`: 16-byte unit u at unit u ^ ((lane / 2) % 4) (64-byte swizzle)
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              uint4 w;
+              w.x = pack_bf16x2(v[u * 8 + 0], v[u * 8 + 1]);
+              w.y = pack_bf16x2(v[u * 8 + 2], v[u * 8 + 3]);
+              w.z = pack_bf16x2(v[u * 8 + 4], v[u * 8 + 5]);
+              w.w = pack_bf16x2(v[u * 8 + 6], v[u * 8 + 7]);
+              *reinterpret_cast<uint4*>(buf + lane * 64 + ((u ^ ((lane >> 1) & 3)) << 4)) = w;
+            }
+            if (mirror) {
+#pragma unroll
+              for (int k = 0; k < 32; ++k)
+                reinterpret_cast<__nv_bfloat16*>(stg + k * STG_PITCH)[lane] = __float2bfloat16_rn(v[k]);
+              __syncwarp();
+              store_staged(stg, out, P.out_ld, cbase, rbase, P.N, P.M, lane);
+            }
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_3d(tmOut, buf, cbase, rbase, bidx);
+              bulk_commit_group();
+            }
+            ++nch;
           } else {
           // this thread's row `lane`, 4 x 16 B at columns c32*32 + u*8 of the slice
           uint4* cell[4];
@@ -435,10 +488,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
                                                ((j ^ (lane & 7)) << 4));
           }
           float v[32];
-          if (KIND == EPI_GRAM) {
+          if (KIND != EPI_POLY) {
 #pragma unroll
             for (int k = 0; k < 32; ++k) v[k] = alpha * __uint_as_float(raw[k]);
           } else {
+            // B' = b A + c A^2 + a I: the diagonal element of this row, if it
+            // falls in this chunk, is column rbase + lane
+            const int dk = rbase + lane - cbase;
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
               const uint4 w = *cell[u];
@@ -451,7 +507,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
 #pragma unroll
               for (int e = 0; e < 8; ++e) {
                 const float a = __uint_as_float(raw[u * 8 + e]);
-                v[u * 8 + e] = (KIND == EPI_POLY) ? args.c0 * in[e] + args.c1 * a : alpha * (args.c0 * in[e] + a);
+                v[u * 8 + e] = args.c0 * in[e] + args.c1 * a + (u * 8 + e == dk ? args.c2 : 0.0f);
               }
             }
           }
@@ -478,15 +534,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
         // the slice now holds the output: make it visible to the TMA unit, store it
         fence_async_smem();
         __syncwarp();
-        if (lane == 0 && (KIND == EPI_GRAM || KIND == EPI_POLY || KIND == EPI_UPDATE)) {
+        if (lane == 0 && KIND == EPI_POLY) {
           tma_store_3d(tmOut, slice, col0, rbase, bidx);
           if (two_boxes) tma_store_3d(tmOut, slice + EPI_BOX_BYTES, col0 + 64, rbase, bidx);
           bulk_commit_group();
         }
       }
+      // this warp's tcgen05.ld reads of the accumulator have completed
+      // (tcgen05.wait::ld); the MMA may overwrite it
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(tempty0 + acc * 8);   // leader's tempty_bar[acc]
+      if (lane == 0) mbar_arrive_cluster_relaxed(tempty0 + acc * 8);   // leader's tempty_bar[acc]
     }
     if (lane == 0) {
       if (aux_pending) {
