@@ -29,6 +29,12 @@ namespace muon {
 constexpr int EW_TILE = 64;        // 64 x 64 element tiles
 constexpr int EW_THREADS = 256;
 
+// Transposing tile: element (c, r) of a 64 x 64 bf16 tile sits in row c at
+// 16-byte unit (r / 8) ^ (c / 8 % 8).  Writing one column (8 rows c apart,
+// 4 consecutive r per warp) and reading 8-element row units are both free of
+// bank conflicts.
+__device__ __forceinline__ int tsw(int c, int r) { return ((((r >> 3) ^ (c >> 3)) & 7) << 3) | (r & 7); }
+
 // One matrix as the elementwise kernels see it.  Lives in a device table.
 struct MatDesc {
   const void* grad;          // rows x cols, grad_dtype (momentum) / input (export)
@@ -112,7 +118,7 @@ __global__ void __launch_bounds__(EW_THREADS)
     momentum_kernel(const MatDesc* __restrict__ descs, const __grid_constant__ SegTable segs, int64_t tile_base,
                     float beta, int nesterov, const int* skip) {
   if (skip != nullptr && *skip) return;
-  __shared__ __align__(16) __nv_bfloat16 tile[EW_TILE][EW_TILE + 8];
+  __shared__ __align__(16) __nv_bfloat16 tile[EW_TILE][EW_TILE];
   __shared__ float red[EW_THREADS / 32];
   const int64_t gt = tile_base + blockIdx.x;
   const MatDesc& d = descs[seg_find(segs, gt)];
@@ -157,7 +163,7 @@ __global__ void __launch_bounds__(EW_THREADS)
         *reinterpret_cast<uint4*>(d.x_in + r * d.ld + c) = w;
       } else {
 #pragma unroll
-        for (int k = 0; k < 8; ++k) tile[cl + k][rl] = __float2bfloat16_rn(u[k]);
+        for (int k = 0; k < 8; ++k) tile[cl + k][tsw(cl + k, rl)] = __float2bfloat16_rn(u[k]);
       }
     } else {
       for (int k = 0; k < 8; ++k) {
@@ -175,7 +181,7 @@ __global__ void __launch_bounds__(EW_THREADS)
         }
         ss += uk * uk;
         if (!d.transposed) d.x_in[r * d.ld + cc] = __float2bfloat16_rn(uk);
-        else tile[cl + k][rl] = __float2bfloat16_rn(uk);
+        else tile[cl + k][tsw(cl + k, rl)] = __float2bfloat16_rn(uk);
       }
     }
   }
@@ -190,9 +196,9 @@ __global__ void __launch_bounds__(EW_THREADS)
       if (wr >= d.cols) continue;
       __nv_bfloat16* dst = d.x_in + wr * d.ld + wc;
       if (wc + 8 <= d.rows && (d.ld % 8 == 0)) {
-        *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(&tile[cl][rl]);
+        *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(&tile[cl][tsw(cl, rl)]);
       } else {
-        for (int k = 0; k < 8 && wc + k < d.rows; ++k) dst[k] = tile[cl][rl + k];
+        for (int k = 0; k < 8 && wc + k < d.rows; ++k) dst[k] = tile[cl][tsw(cl, rl + k)];
       }
     }
   }
@@ -229,7 +235,7 @@ __global__ void __launch_bounds__(EW_THREADS)
     apply_kernel(const MatDesc* __restrict__ descs, const __grid_constant__ SegTable segs, int64_t tile_base,
                  int normalise, float eps, const int* skip) {
   if (skip != nullptr && *skip) return;
-  __shared__ __align__(16) __nv_bfloat16 tile[EW_TILE][EW_TILE + 8];
+  __shared__ __align__(16) __nv_bfloat16 tile[EW_TILE][EW_TILE];
   const int64_t gt = tile_base + blockIdx.x;
   const MatDesc& d = descs[seg_find(segs, gt)];
   const int64_t lt = gt - d.tile_start;
@@ -246,9 +252,9 @@ __global__ void __launch_bounds__(EW_THREADS)
       if (wr >= d.cols) continue;
       const __nv_bfloat16* src = d.x_out + wr * d.ld + wc;
       if (wc + 8 <= d.rows && (d.ld % 8 == 0)) {
-        *reinterpret_cast<uint4*>(&tile[cl][rl]) = *reinterpret_cast<const uint4*>(src);
+        *reinterpret_cast<uint4*>(&tile[cl][tsw(cl, rl)]) = *reinterpret_cast<const uint4*>(src);
       } else {
-        for (int k = 0; k < 8 && wc + k < d.rows; ++k) tile[cl][rl + k] = src[k];
+        for (int k = 0; k < 8 && wc + k < d.rows; ++k) tile[cl][tsw(cl, rl + k)] = src[k];
       }
     }
     __syncthreads();
@@ -271,7 +277,7 @@ __global__ void __launch_bounds__(EW_THREADS)
         f = unpack_bf16x2(w.w); o[6] = f.x; o[7] = f.y;
       } else {
 #pragma unroll
-        for (int k = 0; k < 8; ++k) o[k] = __bfloat162float(tile[cl + k][rl]);
+        for (int k = 0; k < 8; ++k) o[k] = __bfloat162float(tile[cl + k][tsw(cl + k, rl)]);
       }
 #pragma unroll
       for (int k = 0; k < 8; ++k) o[k] *= s;
@@ -294,7 +300,7 @@ __global__ void __launch_bounds__(EW_THREADS)
       for (int k = 0; k < 8; ++k) {
         const int64_t cc = c + k;
         if (cc >= d.cols) break;
-        const float ok = s * (d.transposed ? __bfloat162float(tile[cl + k][rl])
+        const float ok = s * (d.transposed ? __bfloat162float(tile[cl + k][tsw(cl + k, rl)])
                                            : __bfloat162float(d.x_out[r * d.ld + cc]));
         const int64_t idx = r * d.cols + cc;
         if (MODE == 0) d.weight[idx] = d.weight[idx] * d.decay - d.lr_scale * ok;

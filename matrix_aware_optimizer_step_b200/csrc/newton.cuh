@@ -44,7 +44,9 @@ constexpr int SOLVE_THREADS = 512;
 constexpr int kDevErrNotSPD = 2;
 
 struct CholDesc {
-  float* a;          // d x d scratch: S in, L (lower) + L^T (strict upper) out
+  float* a;          // d x d scratch: S in, L (lower) out; strict upper: L^T
+                     // (unblocked path) or, in each 32x32 diagonal block,
+                     // the transpose of that block's inverse (blocked path)
   float* inv;        // d x d output S^-1
   int32_t d;
   int32_t pad;
@@ -103,7 +105,10 @@ __host__ __device__ inline int cholb_smem_bytes(int d) { return d * CBP * 4; }
 // Right-looking Cholesky S = L L^T in place (lower triangle), one block per
 // matrix: factor the 32x32 diagonal block (one warp), solve the panel below it
 // row by row, subtract the panel's rank-32 product from the trailing lower
-// triangle in 4x4 register tiles.  The panel lives in shared memory.
+// triangle in 4x4 register tiles.  The panel lives in shared memory.  Warp 0
+// also inverts each factored diagonal block D (column j of D^-1 by lane j) and
+// stores D^-1 transposed in the block's strict upper triangle, where the
+// inverse kernel turns its in-block substitutions into products.
 __global__ void __launch_bounds__(CHOLB_THREADS)
     cholesky_blocked_kernel(const CholDesc* __restrict__ descs, float damping, int* err) {
   extern __shared__ float pan[];            // [d][CBP]: rows below the diagonal block
@@ -144,6 +149,21 @@ __global__ void __launch_bounds__(CHOLB_THREADS)
     for (int e = tid; e < nb * nb; e += CHOLB_THREADS) {
       const int i = e / nb, j = e % nb;
       if (j <= i) a[int64_t(p0 + i) * d + p0 + j] = dg[i][j];
+    }
+    if (warp == 0) {
+      // D x = e_lane by forward substitution; x = column `lane` of D^-1
+      float x[CB];
+#pragma unroll
+      for (int i = 0; i < CB; ++i) {
+        float sum = (i == lane) ? 1.f : 0.f;
+#pragma unroll
+        for (int k = 0; k < i; ++k) sum -= dg[i][k] * x[k];
+        x[i] = (i < nb) ? sum / dg[i][i] : 0.f;
+      }
+      // D^-1[i][lane] (i > lane) goes to row p0 + lane, column p0 + i
+#pragma unroll
+      for (int i = 0; i < CB; ++i)
+        if (i > lane && i < nb) a[int64_t(p0 + lane) * d + p0 + i] = x[i];
     }
     // panel: row i below solves x L11^T = a_i (forward substitution)
     const int r0 = p0 + nb, nrows = d - r0;
@@ -208,16 +228,35 @@ __global__ void __launch_bounds__(CHOLB_THREADS)
 }
 
 constexpr int CINV_THREADS = 256;
+
+// dv = D^-1 for the diagonal block at rbase (zero outside the matrix):
+// D^-1[i][k] for k < i sits at (rbase + k, rbase + i) of the factor's
+// storage, the diagonal is 1 / L[i][i].
+__device__ __forceinline__ void load_diag_inverse(const float* L, int d, int rbase, float (*dv)[CBP], int tid) {
+  for (int e = tid; e < CB * CB; e += CINV_THREADS) {
+    const int i = e / CB, k = e % CB;
+    const int gi = rbase + i, gk = rbase + k;
+    float v = 0.f;
+    if (gi < d && gk < d) {
+      if (k < i) v = L[int64_t(gk) * d + gi];
+      else if (k == i) v = 1.f / L[int64_t(gi) * d + gi];
+    }
+    dv[i][k] = v;
+  }
+}
 __host__ __device__ inline int cinv_smem_bytes(int d) { return d * CBP * 4; }
 
 // S^-1 = L^-T L^-1, 32 columns per block: forward L Y = E (E = columns
 // c0 .. c0+31 of I; rows of Y above c0 are zero), then L^T X = Y, row blocks
 // of 32 at a time, Y and X resident in shared memory; X^T is written as rows
 // c0 .. c0+31 of the (symmetric) S^-1.  L is read from the lower triangle.
+// Within a row block the substitution is a product with the diagonal
+// block's inverse (D^-1 forward, D^-T backward), spread over all threads.
 __global__ void __launch_bounds__(CINV_THREADS)
     chol_inverse_kernel(const CholDesc* __restrict__ descs, int blocks_per_mat) {
   extern __shared__ float y[];              // [d][CBP]
   __shared__ float acc_s[CB][CBP];
+  __shared__ float dv[CB][CBP];             // inverse of the current diagonal block
   const CholDesc& c = descs[blockIdx.x / blocks_per_mat];
   const int d = c.d;
   const int c0 = (blockIdx.x % blocks_per_mat) * CB;
@@ -244,15 +283,19 @@ __global__ void __launch_bounds__(CINV_THREADS)
     }
 #pragma unroll
     for (int v = 0; v < 4; ++v) acc_s[orow][ocol + v] = acc[v];
+    load_diag_inverse(L, d, rbase, dv, tid);
     __syncthreads();
-    // within the block: column j of the RHS by thread j (forward substitution)
-    if (tid < CB) {
-      const int j = tid;
-      for (int i = 0; i < CB && rbase + i < d; ++i) {
-        const float* lrow = L + int64_t(rbase + i) * d + rbase;
-        float sum = acc_s[i][j];
-        for (int k = 0; k < i; ++k) sum -= lrow[k] * y[(rbase + k) * CBP + j];
-        y[(rbase + i) * CBP + j] = sum / lrow[i];
+    // Y_block = D^-1 * acc
+    {
+      float out[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int k = 0; k <= orow; ++k) {
+        const float dk = dv[orow][k];
+#pragma unroll
+        for (int v = 0; v < 4; ++v) out[v] += dk * acc_s[k][ocol + v];
+      }
+      if (r < d) {
+#pragma unroll
+        for (int v = 0; v < 4; ++v) y[r * CBP + ocol + v] = out[v];
       }
     }
     __syncthreads();
@@ -275,14 +318,19 @@ __global__ void __launch_bounds__(CINV_THREADS)
     }
 #pragma unroll
     for (int v = 0; v < 4; ++v) acc_s[orow][ocol + v] = acc[v];
+    load_diag_inverse(L, d, rbase, dv, tid);
     __syncthreads();
-    if (tid < CB) {
-      const int j = tid;
-      const int nb = min(CB, d - rbase);
-      for (int i = nb - 1; i >= 0; --i) {
-        float sum = acc_s[i][j];
-        for (int k = i + 1; k < nb; ++k) sum -= L[int64_t(rbase + k) * d + rbase + i] * y[(rbase + k) * CBP + j];
-        y[(rbase + i) * CBP + j] = sum / L[int64_t(rbase + i) * d + rbase + i];
+    // X_block = D^-T * acc
+    {
+      float out[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int k = orow; k < CB; ++k) {
+        const float dk = dv[k][orow];
+#pragma unroll
+        for (int v = 0; v < 4; ++v) out[v] += dk * acc_s[k][ocol + v];
+      }
+      if (r < d) {
+#pragma unroll
+        for (int v = 0; v < 4; ++v) y[r * CBP + ocol + v] = out[v];
       }
     }
     __syncthreads();
