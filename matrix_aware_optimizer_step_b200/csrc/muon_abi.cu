@@ -836,7 +836,8 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
         const PrepDesc& pd = prep[chunk_prep_begin[ci] + k];
         most = std::max<int64_t>(most, std::max<int64_t>(pd.rows * pd.cols, int64_t(pd.nb) * pd.d * pd.d));
       }
-      const dim3 grid(unsigned(std::min<int64_t>(cdiv(most, 256), 512)), unsigned(chunk_prep_count[ci]));
+      const dim3 grid(unsigned(std::max<int64_t>(1, std::min<int64_t>(cdiv(most, 256 * 8), 512))),
+                      unsigned(chunk_prep_count[ci]));
       precond_prep_kernel<<<grid, 256, 0, st>>>(dprep + chunk_prep_begin[ci]);
       ctx->launches++;
       CUDA_TRY(ctx, cudaGetLastError());
@@ -1252,13 +1253,24 @@ muon_status muon_newton_refresh(muon_ctx* ctx, const muon_act_desc* acts, int32_
     // blocked factorisation and inverse, panels of 32 in shared memory
     const int smem = cholb_smem_bytes(max_d);
     CUDA_TRY(ctx, cudaFuncSetAttribute(cholesky_blocked_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-    CUDA_TRY(ctx, cudaFuncSetAttribute(chol_inverse_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    CUDA_TRY(ctx, cudaFuncSetAttribute(chol_linv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        cinv_smem_bytes(max_d)));
     cholesky_blocked_kernel<<<unsigned(cd.size()), CHOLB_THREADS, smem, st>>>(dc, damping, ctx->dflags);
     ctx->launches++;
     CUDA_TRY(ctx, cudaGetLastError());
+    // L^-1 into the output buffers, then S^-1 = L^-T L^-1 into the scratch
+    // that held L, then copied out
     const int parts = int(cdiv(max_d, CB));
-    chol_inverse_kernel<<<unsigned(cd.size() * parts), CINV_THREADS, cinv_smem_bytes(max_d), st>>>(dc, parts);
+    chol_linv_kernel<<<unsigned(cd.size() * parts), CINV_THREADS, cinv_smem_bytes(max_d), st>>>(dc, parts);
+    ctx->launches++;
+    CUDA_TRY(ctx, cudaGetLastError());
+    const int nt = int(cdiv(max_d, SIP_T));
+    spd_inverse_product_kernel<<<dim3(unsigned(nt * (nt + 1) / 2), unsigned(cd.size())), SIP_THREADS, 0, st>>>(dc);
+    ctx->launches++;
+    CUDA_TRY(ctx, cudaGetLastError());
+    const int64_t most = int64_t(max_d) * max_d;
+    copy_inverse_kernel<<<dim3(unsigned(std::min<int64_t>(cdiv(most, 4 * 256), 1024)), unsigned(cd.size())), 256, 0,
+                          st>>>(dc);
     ctx->launches++;
     CUDA_TRY(ctx, cudaGetLastError());
     return MUON_OK;

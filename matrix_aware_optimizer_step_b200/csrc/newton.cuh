@@ -9,8 +9,10 @@
 //                         which the tensor-core engine computes (GRAM32).
 //   cholesky_blocked_kernel  S = L L^T in place (fp32), panels of 32, one
 //                         block per matrix (d <= 1536).
-//   chol_inverse_kernel   S^-1 = L^-T L^-1, 32 columns per block, blocked
-//                         forward and backward substitution.
+//   chol_linv_kernel      L^-1, 32 columns per block, blocked forward
+//                         substitution with the diagonal blocks' inverses.
+//   spd_inverse_product_kernel  S^-1 = L^-T L^-1 in 64x64 tiles of the lower
+//                         triangle (mirrored), then copy_inverse_kernel.
 //   cholesky_kernel, chol_solve_kernel  unblocked versions for larger d.
 //   precond_prep_kernel   bf16 copies of the gradients and S^-1 split into
 //                         bf16 hi + lo, the operands of G' = G [S_hi; S_lo]
@@ -21,6 +23,8 @@
 
 #include <cstdint>
 #include <cuda_bf16.h>
+
+#include "elementwise.cuh"   // tsw: the swizzled transposing tile
 
 namespace muon {
 
@@ -246,14 +250,14 @@ __device__ __forceinline__ void load_diag_inverse(const float* L, int d, int rba
 }
 __host__ __device__ inline int cinv_smem_bytes(int d) { return d * CBP * 4; }
 
-// S^-1 = L^-T L^-1, 32 columns per block: forward L Y = E (E = columns
-// c0 .. c0+31 of I; rows of Y above c0 are zero), then L^T X = Y, row blocks
-// of 32 at a time, Y and X resident in shared memory; X^T is written as rows
-// c0 .. c0+31 of the (symmetric) S^-1.  L is read from the lower triangle.
-// Within a row block the substitution is a product with the diagonal
-// block's inverse (D^-1 forward, D^-T backward), spread over all threads.
+// L^-1, 32 columns per block: forward L Y = E (E = columns c0 .. c0+31 of
+// I; rows of Y above c0 are zero), row blocks of 32 at a time, Y resident in
+// shared memory.  Within a row block the substitution is a product with the
+// diagonal block's inverse D^-1, spread over all threads.  Y is written to
+// c.inv (rows from c0 rounded down to 64, zeros above c0), the operand of
+// spd_inverse_product_kernel.  L is read from the lower triangle of c.a.
 __global__ void __launch_bounds__(CINV_THREADS)
-    chol_inverse_kernel(const CholDesc* __restrict__ descs, int blocks_per_mat) {
+    chol_linv_kernel(const CholDesc* __restrict__ descs, int blocks_per_mat) {
   extern __shared__ float y[];              // [d][CBP]
   __shared__ float acc_s[CB][CBP];
   __shared__ float dv[CB][CBP];             // inverse of the current diagonal block
@@ -300,45 +304,102 @@ __global__ void __launch_bounds__(CINV_THREADS)
     }
     __syncthreads();
   }
-  // ---- backward: L^T X = Y, bottom row block first; X overwrites Y ----
-  for (int rb = nrb - 1; rb >= 0; --rb) {
-    const int rbase = rb * CB;
-    const int r = rbase + orow;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    if (r < d) {
-      if (r >= c0 || rb >= rb0) {
-#pragma unroll
-        for (int v = 0; v < 4; ++v) acc[v] = y[r * CBP + ocol + v];
+  // ---- columns c0 .. c0+31 of L^-1 ----
+  const int rw = c0 & ~63;
+  for (int e = tid; e < (d - rw) * CB; e += CINV_THREADS) {
+    const int i = rw + e / CB, j = e % CB;
+    if (c0 + j < d) c.inv[int64_t(i) * d + c0 + j] = i < c0 ? 0.f : y[i * CBP + j];
+  }
+}
+
+// S^-1 = L^-T L^-1: S^-1[i][j] = sum over k >= max(i, j) of L^-1[k][i] L^-1[k][j].
+// One 64x64 tile of the lower triangle per block (grid.x: tile, grid.y:
+// matrix), K in chunks of 32 rows of L^-1 staged in shared memory, 4x4
+// register tiles; the tile and its mirror are written to c.a.
+constexpr int SIP_T = 64, SIP_K = 32, SIP_THREADS = 256;
+__global__ void __launch_bounds__(SIP_THREADS) spd_inverse_product_kernel(const CholDesc* __restrict__ descs) {
+  const CholDesc& c = descs[blockIdx.y];
+  const int d = c.d;
+  const int nt = (d + SIP_T - 1) / SIP_T;
+  const int t = blockIdx.x;
+  if (t >= nt * (nt + 1) / 2) return;
+  int ti = int((sqrtf(8.f * t + 1.f) - 1.f) * 0.5f);
+  while (ti * (ti + 1) / 2 > t) --ti;
+  while ((ti + 1) * (ti + 2) / 2 <= t) ++ti;
+  const int tj = t - ti * (ti + 1) / 2;
+  const int i0 = ti * SIP_T, j0 = tj * SIP_T;
+  const float* li = c.inv;
+  __shared__ __align__(16) float as[SIP_K][SIP_T];
+  __shared__ __align__(16) float bs[SIP_K][SIP_T];
+  __shared__ float cs[SIP_T][SIP_T + 1];
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  const bool vec = (d % 4) == 0;
+  float acc[4][4] = {};
+  for (int k0 = i0; k0 < d; k0 += SIP_K) {
+    for (int e = tid; e < SIP_K * SIP_T / 4; e += SIP_THREADS) {
+      const int kr = e >> 4, c4 = (e & 15) * 4;
+      const int k = k0 + kr;
+      float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+      if (k < d) {
+        const float* row = li + int64_t(k) * d;
+        if (vec && i0 + c4 + 4 <= d) {
+          a = *reinterpret_cast<const float4*>(row + i0 + c4);
+        } else {
+          float* pa = reinterpret_cast<float*>(&a);
+          for (int u = 0; u < 4; ++u) pa[u] = i0 + c4 + u < d ? row[i0 + c4 + u] : 0.f;
+        }
+        if (vec && j0 + c4 + 4 <= d) {
+          b = *reinterpret_cast<const float4*>(row + j0 + c4);
+        } else {
+          float* pb = reinterpret_cast<float*>(&b);
+          for (int u = 0; u < 4; ++u) pb[u] = j0 + c4 + u < d ? row[j0 + c4 + u] : 0.f;
+        }
       }
-      for (int k = rbase + CB; k < d; ++k) {
-        const float l = L[int64_t(k) * d + r];     // L^T[r][k]
-#pragma unroll
-        for (int v = 0; v < 4; ++v) acc[v] -= l * y[k * CBP + ocol + v];
-      }
+      *reinterpret_cast<float4*>(&as[kr][c4]) = a;
+      *reinterpret_cast<float4*>(&bs[kr][c4]) = b;
     }
-#pragma unroll
-    for (int v = 0; v < 4; ++v) acc_s[orow][ocol + v] = acc[v];
-    load_diag_inverse(L, d, rbase, dv, tid);
     __syncthreads();
-    // X_block = D^-T * acc
-    {
-      float out[4] = {0.f, 0.f, 0.f, 0.f};
-      for (int k = orow; k < CB; ++k) {
-        const float dk = dv[k][orow];
+#pragma unroll 8
+    for (int kk = 0; kk < SIP_K; ++kk) {
+      const float4 a = *reinterpret_cast<const float4*>(&as[kk][ty * 4]);
+      const float4 b = *reinterpret_cast<const float4*>(&bs[kk][tx * 4]);
+      const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-        for (int v = 0; v < 4; ++v) out[v] += dk * acc_s[k][ocol + v];
-      }
-      if (r < d) {
+      for (int u = 0; u < 4; ++u)
 #pragma unroll
-        for (int v = 0; v < 4; ++v) y[r * CBP + ocol + v] = out[v];
-      }
+        for (int v = 0; v < 4; ++v) acc[u][v] += av[u] * bv[v];
     }
     __syncthreads();
   }
-  // ---- rows c0 .. c0+31 of S^-1 = columns of X ----
-  for (int e = tid; e < CB * d; e += CINV_THREADS) {
-    const int j = e / d, i = e % d;
-    if (c0 + j < d) c.inv[int64_t(c0 + j) * d + i] = y[i * CBP + j];
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+#pragma unroll
+    for (int v = 0; v < 4; ++v) cs[ty * 4 + u][tx * 4 + v] = acc[u][v];
+  __syncthreads();
+  float* out = c.a;
+  for (int e = tid; e < SIP_T * SIP_T; e += SIP_THREADS) {
+    const int r = e >> 6, q = e & 63;
+    if (i0 + r < d && j0 + q < d) out[int64_t(i0 + r) * d + j0 + q] = cs[r][q];
+  }
+  if (ti != tj) {
+    for (int e = tid; e < SIP_T * SIP_T; e += SIP_THREADS) {
+      const int q = e >> 6, r = e & 63;      // output row j0 + q, column i0 + r
+      if (i0 + r < d && j0 + q < d) out[int64_t(j0 + q) * d + i0 + r] = cs[r][q];
+    }
+  }
+}
+
+// c.inv = c.a (d x d), grid.y = matrix.
+__global__ void __launch_bounds__(256) copy_inverse_kernel(const CholDesc* __restrict__ descs) {
+  const CholDesc& c = descs[blockIdx.y];
+  const int64_t n = int64_t(c.d) * c.d;
+  const int64_t stride = int64_t(gridDim.x) * 256;
+  if (n % 4 == 0) {
+    const float4* src = reinterpret_cast<const float4*>(c.a);
+    float4* dst = reinterpret_cast<float4*>(c.inv);
+    for (int64_t e = blockIdx.x * 256 + threadIdx.x; e < n / 4; e += stride) dst[e] = src[e];
+  } else {
+    for (int64_t e = blockIdx.x * 256 + threadIdx.x; e < n; e += stride) c.inv[e] = c.a[e];
   }
 }
 
@@ -461,23 +522,48 @@ struct ActBlock {
   int64_t tokens, width, col0, d, ldt;
 };
 
-// grid.y = block, grid.x = 64x64 tiles of (tokens x d)
+// grid.y = block, grid.x = 64x64 tiles of (tokens x d).  16-byte loads and
+// stores through a swizzled 64x64 tile (tsw, conflict-free in both
+// directions) when the widths allow, elementwise at ragged edges.
 __global__ void __launch_bounds__(256) act_transpose_kernel(const ActBlock* __restrict__ blocks) {
-  __shared__ __nv_bfloat16 t[TPOSE_T][TPOSE_T + 2];
+  __shared__ __align__(16) __nv_bfloat16 t[TPOSE_T][TPOSE_T];   // t[j][tsw(j, tok)]
   const ActBlock& b = blocks[blockIdx.y];
   const int64_t tiles_j = (b.d + TPOSE_T - 1) / TPOSE_T;
   const int64_t t0 = (blockIdx.x / tiles_j) * TPOSE_T, j0 = (blockIdx.x % tiles_j) * TPOSE_T;
   if (t0 >= b.tokens) return;
-  for (int e = threadIdx.x; e < TPOSE_T * TPOSE_T; e += 256) {
-    const int tt = e / TPOSE_T, jj = e % TPOSE_T;
-    const int64_t tok = t0 + tt, j = j0 + jj;
-    t[tt][jj] = (tok < b.tokens && j < b.d) ? b.acts[tok * b.width + b.col0 + j] : __float2bfloat16_rn(0.f);
+  const bool vec = (b.width % 8 == 0) && (b.col0 % 8 == 0) && (b.ldt % 8 == 0);
+#pragma unroll
+  for (int it = 0; it < 2; ++it) {
+    const int v = threadIdx.x + it * 256;
+    const int tt = v >> 3, jv = (v & 7) * 8;
+    const int64_t tok = t0 + tt, j = j0 + jv;
+    __nv_bfloat16 x[8];
+    if (vec && tok < b.tokens && j + 8 <= b.d) {
+      const uint4 w = *reinterpret_cast<const uint4*>(b.acts + tok * b.width + b.col0 + j);
+      const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&w);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) x[k] = e[k];
+    } else {
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        x[k] = (tok < b.tokens && j + k < b.d) ? b.acts[tok * b.width + b.col0 + j + k] : __float2bfloat16_rn(0.f);
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) t[jv + k][tsw(jv + k, tt)] = x[k];
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < TPOSE_T * TPOSE_T; e += 256) {
-    const int jj = e / TPOSE_T, tt = e % TPOSE_T;
-    const int64_t tok = t0 + tt, j = j0 + jj;
-    if (tok < b.tokens && j < b.d) b.xt[j * b.ldt + tok] = t[tt][jj];
+#pragma unroll
+  for (int it = 0; it < 2; ++it) {
+    const int v = threadIdx.x + it * 256;
+    const int jj = v >> 3, tv = (v & 7) * 8;
+    const int64_t j = j0 + jj, tok = t0 + tv;
+    if (j >= b.d) continue;
+    __nv_bfloat16* dst = b.xt + j * b.ldt + tok;
+    if (vec && tok + 8 <= b.tokens) {
+      *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(&t[jj][tsw(jj, tv)]);
+    } else {
+      for (int k = 0; k < 8 && tok + k < b.tokens; ++k) dst[k] = t[jj][tsw(jj, tv + k)];
+    }
   }
 }
 
@@ -493,26 +579,56 @@ struct PrepDesc {
   int32_t nb, d;
 };
 
-// grid.y = matrix, grid.x strides over max(rows*cols, nb*d*d) elements
+// grid.y = matrix, grid.x strides over max(rows*cols, nb*d*d) elements, 8
+// per thread and step (16-byte loads and stores) when the gradient width and
+// d*d are multiples of 8, one otherwise.  Pointers are 16-byte aligned.
 __global__ void __launch_bounds__(256) precond_prep_kernel(const PrepDesc* __restrict__ descs) {
   const PrepDesc& p = descs[blockIdx.y];
   const int64_t ng = p.rows * p.cols;
   const int64_t dd = static_cast<int64_t>(p.d) * p.d;
   const int64_t ns = p.nb * dd;
+  const bool gvec = (p.cols % 8) == 0;       // then ldc == cols: a flat copy
+  const bool svec = (dd % 8) == 0;
+  const int64_t ngu = gvec ? ng / 8 : ng;
+  const int64_t nsu = svec ? ns / 8 : ns;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * 256;
-  for (int64_t e = blockIdx.x * 256 + threadIdx.x; e < ng || e < ns; e += stride) {
-    if (e < ng) {
-      const int64_t r = e / p.cols, c = e - r * p.cols;
-      p.gc[r * p.ldc + c] = p.g[e];
+  for (int64_t e = blockIdx.x * 256 + threadIdx.x; e < ngu || e < nsu; e += stride) {
+    if (e < ngu) {
+      if (gvec) {
+        reinterpret_cast<uint4*>(p.gc)[e] = reinterpret_cast<const uint4*>(p.g)[e];
+      } else {
+        const int64_t r = e / p.cols, c = e - r * p.cols;
+        p.gc[r * p.ldc + c] = p.g[e];
+      }
     }
-    if (e < ns) {
-      const int64_t b = e / dd, rem = e - b * dd;
-      const float v = p.s_inv[e];
-      const __nv_bfloat16 hi = __float2bfloat16_rn(v);
-      const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
-      __nv_bfloat16* st = p.sst + b * 2 * dd;
-      st[rem] = hi;
-      st[dd + rem] = lo;
+    if (e < nsu) {
+      if (svec) {
+        const int64_t e8 = e * 8;
+        const int64_t b = e8 / dd, rem = e8 - b * dd;
+        const float4* src = reinterpret_cast<const float4*>(p.s_inv + e8);
+        const float4 v0 = src[0], v1 = src[1];
+        const float v[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        uint32_t hw[4], lw[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const __nv_bfloat16 h0 = __float2bfloat16_rn(v[2 * k]), h1 = __float2bfloat16_rn(v[2 * k + 1]);
+          const __nv_bfloat16 l0 = __float2bfloat16_rn(v[2 * k] - __bfloat162float(h0));
+          const __nv_bfloat16 l1 = __float2bfloat16_rn(v[2 * k + 1] - __bfloat162float(h1));
+          hw[k] = uint32_t(__bfloat16_as_ushort(h0)) | (uint32_t(__bfloat16_as_ushort(h1)) << 16);
+          lw[k] = uint32_t(__bfloat16_as_ushort(l0)) | (uint32_t(__bfloat16_as_ushort(l1)) << 16);
+        }
+        __nv_bfloat16* st = p.sst + b * 2 * dd;
+        *reinterpret_cast<uint4*>(st + rem) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        *reinterpret_cast<uint4*>(st + dd + rem) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+      } else {
+        const int64_t b = e / dd, rem = e - b * dd;
+        const float v = p.s_inv[e];
+        const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+        const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
+        __nv_bfloat16* st = p.sst + b * 2 * dd;
+        st[rem] = hi;
+        st[dd + rem] = lo;
+      }
     }
   }
 }
