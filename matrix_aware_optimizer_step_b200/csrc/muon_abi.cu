@@ -1250,14 +1250,22 @@ muon_status muon_newton_refresh(muon_ctx* ctx, const muon_act_desc* acts, int32_
     CUDA_TRY(ctx, (launch_gemm<EPI_GRAM32, false>(ctx, maps, g, st)));
   }
   if (max_d <= CHOL_BLOCKED_MAX_D) {
-    // blocked factorisation and inverse, panels of 32 in shared memory
-    const int smem = cholb_smem_bytes(max_d);
-    CUDA_TRY(ctx, cudaFuncSetAttribute(cholesky_blocked_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    // blocked factorisation, panels of 32: panel, then trailing update
     CUDA_TRY(ctx, cudaFuncSetAttribute(chol_linv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        cinv_smem_bytes(max_d)));
-    cholesky_blocked_kernel<<<unsigned(cd.size()), CHOLB_THREADS, smem, st>>>(dc, damping, ctx->dflags);
-    ctx->launches++;
-    CUDA_TRY(ctx, cudaGetLastError());
+    for (int p0 = 0; p0 < max_d; p0 += CB) {
+      const int rest = max_d - p0 - CB;                   // trailing rows of the largest matrix
+      const unsigned chunks = unsigned(std::max<int64_t>(1, cdiv(std::max(rest, 0), CPR)));
+      chol_panel_kernel<<<dim3(chunks, unsigned(cd.size())), CP_THREADS, 0, st>>>(dc, p0, damping, ctx->dflags);
+      ctx->launches++;
+      CUDA_TRY(ctx, cudaGetLastError());
+      if (rest > 0) {
+        const int nt = int(cdiv(rest, CU_T));
+        chol_update_kernel<<<dim3(unsigned(nt * (nt + 1) / 2), unsigned(cd.size())), CP_THREADS, 0, st>>>(dc, p0);
+        ctx->launches++;
+        CUDA_TRY(ctx, cudaGetLastError());
+      }
+    }
     // L^-1 into the output buffers, then S^-1 = L^-T L^-1 into the scratch
     // that held L, then copied out
     const int parts = int(cdiv(max_d, CB));

@@ -7,8 +7,9 @@
 //   act_transpose_kernel  a d-wide activation block, transposed to bf16
 //                         d x tokens: the K-major operand of S = Xt Xt^T / N,
 //                         which the tensor-core engine computes (GRAM32).
-//   cholesky_blocked_kernel  S = L L^T in place (fp32), panels of 32, one
-//                         block per matrix (d <= 1536).
+//   chol_panel_kernel, chol_update_kernel  S = L L^T in place (fp32),
+//                         panels of 32, two batched launches per panel
+//                         (d <= 1536).
 //   chol_linv_kernel      L^-1, 32 columns per block, blocked forward
 //                         substitution with the diagonal blocks' inverses.
 //   spd_inverse_product_kernel  S^-1 = L^-T L^-1 in 64x64 tiles of the lower
@@ -101,154 +102,165 @@ __global__ void __launch_bounds__(CHOL_THREADS)
 // ---------------------------------------------------------------------------
 constexpr int CB = 32;                      // panel width
 constexpr int CBP = CB + 1;                 // padded row of a panel in smem
-constexpr int CHOLB_THREADS = 512;
-constexpr int CHOL_BLOCKED_MAX_D = 1536;    // panel of d x 33 floats fits in smem
+constexpr int CHOL_BLOCKED_MAX_D = 1536;    // chol_linv_kernel keeps d x 32 floats in smem
+constexpr int CP_THREADS = 256;
+constexpr int CPR = 64;                     // panel rows per chol_panel_kernel block
 
-__host__ __device__ inline int cholb_smem_bytes(int d) { return d * CBP * 4; }
-
-// Right-looking Cholesky S = L L^T in place (lower triangle), one block per
-// matrix: factor the 32x32 diagonal block (one warp), solve the panel below it
-// row by row, subtract the panel's rank-32 product from the trailing lower
-// triangle in 4x4 register tiles.  The panel lives in shared memory.  Warp 0
-// also inverts each factored diagonal block D (column j of D^-1 by lane j) and
-// stores D^-1 transposed in the block's strict upper triangle, where the
-// inverse kernel turns its in-block substitutions into products.
-__global__ void __launch_bounds__(CHOLB_THREADS)
-    cholesky_blocked_kernel(const CholDesc* __restrict__ descs, float damping, int* err) {
-  extern __shared__ float pan[];            // [d][CBP]: rows below the diagonal block
-  __shared__ float dg[CB][CBP];
-  __shared__ int bad;
-  const CholDesc& c = descs[blockIdx.x];
-  float* a = c.a;
+// Right-looking blocked Cholesky S = L L^T in place (lower triangle), batched
+// over matrices, two launches per 32-wide panel at p0:
+//
+//   chol_panel_kernel   every block factors the panel's 32x32 diagonal block
+//                       D (one warp, in shared memory) and inverts it (lane j
+//                       solves for column j of D^-1); block 0 writes D to the
+//                       lower triangle and D^-1 transposed to the block's
+//                       strict upper triangle (read back by chol_linv_kernel);
+//                       each block then forms CPR rows of the panel below D,
+//                       P = A_panel D^-T, as a product over all threads.
+//   chol_update_kernel  the trailing lower triangle minus P P^T, in 64x64
+//                       tiles with 4x4 register tiles (grid.x: tile).
+//
+// Damping (added to the diagonal) is applied to each diagonal block as it is
+// loaded for factoring: every trailing update only subtracts, so the order
+// does not matter.  A non-positive pivot raises kDevErrNotSPD and continues
+// with pivot 1 so the launch sequence stays well defined.
+__global__ void __launch_bounds__(CP_THREADS)
+    chol_panel_kernel(const CholDesc* __restrict__ descs, int p0, float damping, int* err) {
+  const CholDesc& c = descs[blockIdx.y];
   const int d = c.d;
+  if (p0 >= d) return;
+  float* a = c.a;
+  const int nb = min(CB, d - p0);
+  const int r0 = p0 + nb + blockIdx.x * CPR;           // first panel row of this block
+  if (blockIdx.x > 0 && r0 >= d) return;
+  __shared__ float dg[CB][CBP];
+  __shared__ float dinv[CB][CBP];
+  __shared__ float ap[CPR][CBP];
+  __shared__ int bad;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid == 0) bad = 0;
-  if (damping != 0.f)
-    for (int i = tid; i < d; i += CHOLB_THREADS) a[int64_t(i) * d + i] += damping;
+  for (int e = tid; e < CB * CB; e += CP_THREADS) {
+    const int i = e / CB, j = e % CB;
+    float v = (i < nb && j <= i) ? a[int64_t(p0 + i) * d + p0 + j] : 0.f;
+    if (i == j && i < nb) v += damping;
+    dg[i][j] = v;
+  }
+  for (int e = tid; e < CPR * CB; e += CP_THREADS) {
+    const int rr = e / CB, j = e % CB;
+    ap[rr][j] = (r0 + rr < d && j < nb) ? a[int64_t(r0 + rr) * d + p0 + j] : 0.f;
+  }
   __syncthreads();
-  for (int p0 = 0; p0 < d; p0 += CB) {
-    const int nb = min(CB, d - p0);
-    for (int e = tid; e < CB * CB; e += CHOLB_THREADS) {
-      const int i = e / CB, j = e % CB;
-      dg[i][j] = (i < nb && j <= i) ? a[int64_t(p0 + i) * d + p0 + j] : 0.f;
-    }
-    __syncthreads();
-    if (warp == 0) {                        // unblocked Cholesky of the diagonal block
-      for (int k = 0; k < nb; ++k) {
-        if (lane == 0) {
-          float dkk = dg[k][k];
-          if (!(dkk > 0.f)) { bad = 1; dkk = 1.f; }
-          dg[k][k] = sqrtf(dkk);
-        }
-        __syncwarp();
-        const float lkk = dg[k][k];
-        if (lane > k && lane < nb) dg[lane][k] /= lkk;
-        __syncwarp();
-        if (lane > k && lane < nb)
-          for (int j = k + 1; j <= lane; ++j) dg[lane][j] -= dg[lane][k] * dg[j][k];
-        __syncwarp();
+  if (warp == 0) {
+    // unblocked Cholesky of D
+    for (int k = 0; k < nb; ++k) {
+      if (lane == 0) {
+        float dkk = dg[k][k];
+        if (!(dkk > 0.f)) { bad = 1; dkk = 1.f; }
+        dg[k][k] = sqrtf(dkk);
       }
+      __syncwarp();
+      const float lkk = dg[k][k];
+      if (lane > k && lane < nb) dg[lane][k] /= lkk;
+      __syncwarp();
+      if (lane > k && lane < nb)
+        for (int j = k + 1; j <= lane; ++j) dg[lane][j] -= dg[lane][k] * dg[j][k];
+      __syncwarp();
     }
-    __syncthreads();
-    for (int e = tid; e < nb * nb; e += CHOLB_THREADS) {
+    // D x = e_lane: x = column `lane` of D^-1
+    float x[CB];
+#pragma unroll
+    for (int i = 0; i < CB; ++i) {
+      float sum = (i == lane) ? 1.f : 0.f;
+#pragma unroll
+      for (int k = 0; k < i; ++k) sum -= dg[i][k] * x[k];
+      x[i] = (i < nb) ? sum / dg[i][i] : 0.f;
+    }
+#pragma unroll
+    for (int i = 0; i < CB; ++i) dinv[i][lane] = x[i];
+  }
+  __syncthreads();
+  if (blockIdx.x == 0) {
+    for (int e = tid; e < nb * nb; e += CP_THREADS) {
       const int i = e / nb, j = e % nb;
       if (j <= i) a[int64_t(p0 + i) * d + p0 + j] = dg[i][j];
+      else a[int64_t(p0 + i) * d + p0 + j] = dinv[j][i];     // D^-1[j][i], j > i, at (p0 + i, p0 + j)
     }
-    if (warp == 0) {
-      // D x = e_lane by forward substitution; x = column `lane` of D^-1
-      float x[CB];
-#pragma unroll
-      for (int i = 0; i < CB; ++i) {
-        float sum = (i == lane) ? 1.f : 0.f;
-#pragma unroll
-        for (int k = 0; k < i; ++k) sum -= dg[i][k] * x[k];
-        x[i] = (i < nb) ? sum / dg[i][i] : 0.f;
-      }
-      // D^-1[i][lane] (i > lane) goes to row p0 + lane, column p0 + i
-#pragma unroll
-      for (int i = 0; i < CB; ++i)
-        if (i > lane && i < nb) a[int64_t(p0 + lane) * d + p0 + i] = x[i];
-    }
-    // panel: row i below solves x L11^T = a_i (forward substitution)
-    const int r0 = p0 + nb, nrows = d - r0;
-    for (int ii = tid; ii < nrows; ii += CHOLB_THREADS) {
-      float x[CB];
-      float* arow = a + int64_t(r0 + ii) * d + p0;
-#pragma unroll
-      for (int j = 0; j < CB; ++j) x[j] = j < nb ? arow[j] : 0.f;
-#pragma unroll
-      for (int j = 0; j < CB; ++j) {
-        if (j < nb) {
-          float sum = x[j];
-#pragma unroll
-          for (int k = 0; k < j; ++k) sum -= x[k] * dg[j][k];
-          x[j] = sum / dg[j][j];
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < CB; ++j)
-        if (j < nb) {
-          arow[j] = x[j];
-          pan[ii * CBP + j] = x[j];
-        }
-    }
-    __syncthreads();
-    // trailing lower triangle: A[i][j] -= sum_k P[i][k] P[j][k], 4x4 tiles
-    const int t4 = (nrows + 3) / 4;
-    const int ntiles = t4 * (t4 + 1) / 2;
-    for (int t = tid; t < ntiles; t += CHOLB_THREADS) {
-      int ti = int((sqrtf(8.f * t + 1.f) - 1.f) * 0.5f);
-      while (ti * (ti + 1) / 2 > t) --ti;
-      while ((ti + 1) * (ti + 2) / 2 <= t) ++ti;
-      const int tj = t - ti * (ti + 1) / 2;
-      float acc[4][4] = {};
-      for (int k = 0; k < nb; ++k) {
-        float pi[4], pj[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int ri = 4 * ti + u, rj = 4 * tj + u;
-          pi[u] = ri < nrows ? pan[ri * CBP + k] : 0.f;
-          pj[u] = rj < nrows ? pan[rj * CBP + k] : 0.f;
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-#pragma unroll
-          for (int v = 0; v < 4; ++v) acc[u][v] += pi[u] * pj[v];
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int i = 4 * ti + u;
-        if (i >= nrows) continue;
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          const int j = 4 * tj + v;
-          if (j <= i) a[int64_t(r0 + i) * d + r0 + j] -= acc[u][v];
-        }
-      }
-    }
-    __syncthreads();
+    if (tid == 0 && bad) atomicOr(err, kDevErrNotSPD);
   }
-  if (tid == 0 && bad) atomicOr(err, kDevErrNotSPD);
+  // P[rr][j] = sum over k <= j of A[rr][k] D^-1[j][k]; 8 outputs per thread
+  const int rr = tid >> 2, jb = (tid & 3) * 8;
+  float out[8] = {};
+#pragma unroll 4
+  for (int k = 0; k < CB; ++k) {
+    const float av = ap[rr][k];
+#pragma unroll
+    for (int v = 0; v < 8; ++v) out[v] += av * dinv[jb + v][k];   // zero for k > jb + v
+  }
+  if (r0 + rr < d) {
+#pragma unroll
+    for (int v = 0; v < 8; ++v)
+      if (jb + v < nb) a[int64_t(r0 + rr) * d + p0 + jb + v] = out[v];
+  }
+}
+
+// Trailing update after the panel at p0: A[i][j] -= sum over k < 32 of
+// P[i][k] P[j][k] for p0 + 32 <= j <= i < d, one 64x64 lower tile per block.
+constexpr int CU_T = 64;
+constexpr int CU_P = CU_T + 4;              // padded row of the transposed panel slices (16-byte rows)
+__global__ void __launch_bounds__(CP_THREADS) chol_update_kernel(const CholDesc* __restrict__ descs, int p0) {
+  const CholDesc& c = descs[blockIdx.y];
+  const int d = c.d;
+  const int q0 = p0 + CB;
+  if (q0 >= d) return;
+  const int nt = (d - q0 + CU_T - 1) / CU_T;
+  const int t = blockIdx.x;
+  if (t >= nt * (nt + 1) / 2) return;
+  int ti = int((sqrtf(8.f * t + 1.f) - 1.f) * 0.5f);
+  while (ti * (ti + 1) / 2 > t) --ti;
+  while ((ti + 1) * (ti + 2) / 2 <= t) ++ti;
+  const int tj = t - ti * (ti + 1) / 2;
+  const int i0 = q0 + ti * CU_T, j0 = q0 + tj * CU_T;
+  float* a = c.a;
+  __shared__ __align__(16) float pi_s[CB][CU_P];   // pi_s[k][r] = P[i0 + r][k]
+  __shared__ __align__(16) float pj_s[CB][CU_P];
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  for (int e = tid; e < CU_T * CB; e += CP_THREADS) {
+    const int r = e / CB, k = e % CB;
+    pi_s[k][r] = (i0 + r < d) ? a[int64_t(i0 + r) * d + p0 + k] : 0.f;
+    pj_s[k][r] = (j0 + r < d) ? a[int64_t(j0 + r) * d + p0 + k] : 0.f;
+  }
+  __syncthreads();
+  float acc[4][4] = {};
+#pragma unroll 8
+  for (int k = 0; k < CB; ++k) {
+    const float4 x = *reinterpret_cast<const float4*>(&pi_s[k][ty * 4]);
+    const float4 y = *reinterpret_cast<const float4*>(&pj_s[k][tx * 4]);
+    const float xv[4] = {x.x, x.y, x.z, x.w}, yv[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int v = 0; v < 4; ++v) acc[u][v] += xv[u] * yv[v];
+  }
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int i = i0 + ty * 4 + u;
+    if (i >= d) continue;
+    const int j = j0 + tx * 4;
+    float* row = a + int64_t(i) * d;
+    if (j + 3 <= i && j + 3 < d && (d % 4) == 0) {
+      float4 w = *reinterpret_cast<float4*>(row + j);
+      w.x -= acc[u][0]; w.y -= acc[u][1]; w.z -= acc[u][2]; w.w -= acc[u][3];
+      *reinterpret_cast<float4*>(row + j) = w;
+    } else {
+#pragma unroll
+      for (int v = 0; v < 4; ++v)
+        if (j + v <= i && j + v < d) row[j + v] -= acc[u][v];
+    }
+  }
 }
 
 constexpr int CINV_THREADS = 256;
 
-// dv = D^-1 for the diagonal block at rbase (zero outside the matrix):
-// D^-1[i][k] for k < i sits at (rbase + k, rbase + i) of the factor's
-// storage, the diagonal is 1 / L[i][i].
-__device__ __forceinline__ void load_diag_inverse(const float* L, int d, int rbase, float (*dv)[CBP], int tid) {
-  for (int e = tid; e < CB * CB; e += CINV_THREADS) {
-    const int i = e / CB, k = e % CB;
-    const int gi = rbase + i, gk = rbase + k;
-    float v = 0.f;
-    if (gi < d && gk < d) {
-      if (k < i) v = L[int64_t(gk) * d + gi];
-      else if (k == i) v = 1.f / L[int64_t(gi) * d + gi];
-    }
-    dv[i][k] = v;
-  }
-}
-__host__ __device__ inline int cinv_smem_bytes(int d) { return d * CBP * 4; }
+__host__ __device__ inline int cinv_smem_bytes(int d) { return d * CB * 4; }
 
 // L^-1, 32 columns per block: forward L Y = E (E = columns c0 .. c0+31 of
 // I; rows of Y above c0 are zero), row blocks of 32 at a time, Y resident in
@@ -258,9 +270,10 @@ __host__ __device__ inline int cinv_smem_bytes(int d) { return d * CBP * 4; }
 // spd_inverse_product_kernel.  L is read from the lower triangle of c.a.
 __global__ void __launch_bounds__(CINV_THREADS)
     chol_linv_kernel(const CholDesc* __restrict__ descs, int blocks_per_mat) {
-  extern __shared__ float y[];              // [d][CBP]
+  extern __shared__ float4 y4[];           // Y: [d][CB] floats, 16-byte rows units
+  float* y = reinterpret_cast<float*>(y4);
   __shared__ float acc_s[CB][CBP];
-  __shared__ float dv[CB][CBP];             // inverse of the current diagonal block
+  __shared__ float ls[2][CB][CBP];          // 32x32 chunks of L's row block, double-buffered
   const CholDesc& c = descs[blockIdx.x / blocks_per_mat];
   const int d = c.d;
   const int c0 = (blockIdx.x % blocks_per_mat) * CB;
@@ -277,17 +290,57 @@ __global__ void __launch_bounds__(CINV_THREADS)
     const int r = rbase + orow;
 #pragma unroll
     for (int v = 0; v < 4; ++v) acc[v] = (r == c0 + ocol + v) ? 1.f : 0.f;
-    if (r < d) {
-      const float* lrow = L + int64_t(r) * d;
-      for (int k = c0; k < rbase; ++k) {
-        const float l = lrow[k];
+    // acc -= L[rbase.., c0..rbase) Y[c0..rbase), L staged in 32x32 chunks;
+    // the next chunk and this row block's D^-1 are loaded into registers
+    // while the current chunk is used
+    const int nch = (rbase - c0) / CB;
+    float lreg[4], dreg[4];
+    auto load_chunk = [&](int k0) {
 #pragma unroll
-        for (int v = 0; v < 4; ++v) acc[v] -= l * y[k * CBP + ocol + v];
+      for (int q = 0; q < 4; ++q) {
+        const int e = tid + q * CINV_THREADS, i = e >> 5, kk = e & 31;
+        lreg[q] = (rbase + i < d) ? L[int64_t(rbase + i) * d + k0 + kk] : 0.f;
+      }
+    };
+    if (nch > 0) load_chunk(c0);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int e = tid + q * CINV_THREADS, i = e >> 5, k = e & 31;
+      const int gi = rbase + i, gk = rbase + k;
+      float v = 0.f;
+      if (gi < d && gk < d) {
+        if (k < i) v = L[int64_t(gk) * d + gi];
+        else if (k == i) v = 1.f / L[int64_t(gi) * d + gi];
+      }
+      dreg[q] = v;
+    }
+    for (int ch = 0; ch < nch; ++ch) {
+      float (*lb)[CBP] = ls[ch & 1];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int e = tid + q * CINV_THREADS;
+        lb[e >> 5][e & 31] = lreg[q];
+      }
+      __syncthreads();
+      const int k0 = c0 + ch * CB;
+      if (ch + 1 < nch) load_chunk(k0 + CB);
+#pragma unroll 8
+      for (int kk = 0; kk < CB; ++kk) {
+        const float l = lb[orow][kk];
+        const float4 yv = *reinterpret_cast<const float4*>(&y[(k0 + kk) * CB + ocol]);
+        acc[0] -= l * yv.x; acc[1] -= l * yv.y; acc[2] -= l * yv.z; acc[3] -= l * yv.w;
       }
     }
 #pragma unroll
     for (int v = 0; v < 4; ++v) acc_s[orow][ocol + v] = acc[v];
-    load_diag_inverse(L, d, rbase, dv, tid);
+    // D^-1 goes to the chunk buffer the last chunk did not use (keeps two
+    // blocks per SM within shared memory)
+    float (*dv)[CBP] = ls[nch & 1];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int e = tid + q * CINV_THREADS;
+      dv[e >> 5][e & 31] = dreg[q];
+    }
     __syncthreads();
     // Y_block = D^-1 * acc
     {
@@ -297,10 +350,7 @@ __global__ void __launch_bounds__(CINV_THREADS)
 #pragma unroll
         for (int v = 0; v < 4; ++v) out[v] += dk * acc_s[k][ocol + v];
       }
-      if (r < d) {
-#pragma unroll
-        for (int v = 0; v < 4; ++v) y[r * CBP + ocol + v] = out[v];
-      }
+      if (r < d) *reinterpret_cast<float4*>(&y[r * CB + ocol]) = make_float4(out[0], out[1], out[2], out[3]);
     }
     __syncthreads();
   }
@@ -308,7 +358,7 @@ __global__ void __launch_bounds__(CINV_THREADS)
   const int rw = c0 & ~63;
   for (int e = tid; e < (d - rw) * CB; e += CINV_THREADS) {
     const int i = rw + e / CB, j = e % CB;
-    if (c0 + j < d) c.inv[int64_t(i) * d + c0 + j] = i < c0 ? 0.f : y[i * CBP + j];
+    if (c0 + j < d) c.inv[int64_t(i) * d + c0 + j] = i < c0 ? 0.f : y[i * CB + j];
   }
 }
 
