@@ -4,8 +4,9 @@
 //                     look-ahead U cast to bf16 and written in the wide
 //                     (rows <= cols) layout the Newton-Schulz engine reads,
 //                     transposing through shared memory for tall matrices,
-//                     and the per-matrix sum of U^2 (block reduction + one
-//                     atomic per block).  12 B/element with bf16 gradients.
+//                     and one partial sum of U^2 per tile (block reduction).
+//                     12 B/element with bf16 gradients.
+//   norm_reduce_kernel  ||U||^2 per matrix from its tiles' partials.
 //   apply_kernel      W <- W (1 - lr wd) - lr scale O, O read from the final
 //                     wide bf16 X (transposed back through shared memory for
 //                     tall matrices); optionally O to an fp32 output.
@@ -45,7 +46,6 @@ struct MatDesc {
   const __nv_bfloat16* x_out;  // wide layout, final Newton-Schulz output
   float* norm2;              // this matrix's ||U||^2 slot
   float* partials;           // one partial sum per tile of the launch (indexed by tile)
-  unsigned int* counter;     // tiles of this matrix finished so far (starts at 0)
   int64_t rows, cols;
   int64_t ld;                // leading dimension of the wide layout
   int64_t tile_start;        // first 64x64 tile of this matrix in the launch
@@ -117,6 +117,7 @@ template <int MODE>
 __global__ void __launch_bounds__(EW_THREADS)
     momentum_kernel(const MatDesc* __restrict__ descs, const __grid_constant__ SegTable segs, int64_t tile_base,
                     float beta, int nesterov, const int* skip) {
+  pdl_wait();      // previous kernel's results visible (no-op without PDL)
   if (skip != nullptr && *skip) return;
   __shared__ __align__(16) __nv_bfloat16 tile[EW_TILE][EW_TILE];
   __shared__ float red[EW_THREADS / 32];
@@ -202,29 +203,25 @@ __global__ void __launch_bounds__(EW_THREADS)
       }
     }
   }
-  // Deterministic sum of U^2: every block stores its partial; the last block
-  // of the matrix to finish adds all partials in tile order.
-  __shared__ bool is_last;
+  // this tile's share of sum(U^2); norm_reduce_kernel adds the partials of
+  // each matrix in tile order (deterministic, no atomics or fences here)
   const float tot = block_sum(ss, red);
-  if (threadIdx.x == 0) {
-    d.partials[gt] = tot;
-    __threadfence();
-    const unsigned ntiles = static_cast<unsigned>(((d.rows + EW_TILE - 1) / EW_TILE) * d.tiles_c);
-    is_last = atomicAdd(d.counter, 1u) == ntiles - 1;
-  }
-  __syncthreads();
-  if (is_last) {
-    __threadfence();
-    const int64_t ntiles = ((d.rows + EW_TILE - 1) / EW_TILE) * d.tiles_c;
-    float acc = 0.f;
-    for (int64_t t = threadIdx.x; t < ntiles; t += EW_THREADS)
-      acc += *reinterpret_cast<volatile float*>(&d.partials[d.tile_start + t]);
-    const float all = block_sum(acc, red);
-    if (threadIdx.x == 0) {
-      *d.norm2 = all;
-      *d.counter = 0u;     // ready for the next call
-    }
-  }
+  if (threadIdx.x == 0) d.partials[gt] = tot;
+}
+
+// ||U||^2 of matrix descs[blockIdx.x]: its tiles' partials summed in a fixed
+// order (thread t takes tiles t, t + 256, ...; then a fixed tree), so the
+// result is the same run to run.
+__global__ void __launch_bounds__(EW_THREADS) norm_reduce_kernel(const MatDesc* __restrict__ descs, const int* skip) {
+  pdl_wait();      // previous kernel's results visible (no-op without PDL)
+  if (skip != nullptr && *skip) return;
+  __shared__ float red[EW_THREADS / 32];
+  const MatDesc& d = descs[blockIdx.x];
+  const int64_t ntiles = ((d.rows + EW_TILE - 1) / EW_TILE) * d.tiles_c;
+  float acc = 0.f;
+  for (int64_t t = threadIdx.x; t < ntiles; t += EW_THREADS) acc += d.partials[d.tile_start + t];
+  const float all = block_sum(acc, red);
+  if (threadIdx.x == 0) *d.norm2 = all;
 }
 
 // mode 0: apply update to W (and optionally write O)
@@ -234,6 +231,7 @@ template <int MODE>
 __global__ void __launch_bounds__(EW_THREADS)
     apply_kernel(const MatDesc* __restrict__ descs, const __grid_constant__ SegTable segs, int64_t tile_base,
                  int normalise, float eps, const int* skip) {
+  pdl_wait();      // previous kernel's results visible (no-op without PDL)
   if (skip != nullptr && *skip) return;
   __shared__ __align__(16) __nv_bfloat16 tile[EW_TILE][EW_TILE];
   const int64_t gt = tile_base + blockIdx.x;
@@ -315,6 +313,7 @@ __global__ void __launch_bounds__(EW_THREADS)
 __global__ void __launch_bounds__(EW_THREADS)
     finite_kernel(const MatDesc* __restrict__ descs, const __grid_constant__ SegTable segs, int64_t tile_base,
                   int* flag) {
+  pdl_wait();      // previous kernel's results visible (no-op without PDL)
   const int64_t gt = tile_base + blockIdx.x;
   const MatDesc& d = descs[seg_find(segs, gt)];
   const int64_t lt = gt - d.tile_start;
@@ -367,6 +366,7 @@ __device__ __forceinline__ void adam_one(float& p, float g, float& m, float& v, 
 
 __global__ void __launch_bounds__(EW_THREADS)
     adamw_kernel(const AdamDesc* __restrict__ descs, int n, AdamScalars s) {
+  pdl_wait();      // previous kernel's results visible (no-op without PDL)
   const int64_t ch = blockIdx.x;
   const AdamDesc& d = descs[find_adam(descs, n, ch)];
   const int64_t base = (ch - d.chunk_start) * ADAM_CHUNK;

@@ -189,7 +189,7 @@ struct Run {
 
 struct Chunk {
   int first, count;              // item range
-  size_t off_norm;               // count floats, then count counters, then per-tile partials
+  size_t off_norm;               // count floats, then per-tile partials
   size_t off_partials;
   size_t off_pgrad;              // preconditioned gradients (fp32), if any
   bool tc_pre;                   // preconditioning on the tensor-core engine
@@ -213,7 +213,7 @@ constexpr size_t kAlign = 256;
 size_t layout_chunk(Chunk& c, const std::vector<Item>& items) {
   size_t off = 0;
   c.off_norm = off;
-  off += round_up(c.count * (sizeof(float) + sizeof(unsigned)), kAlign);
+  off += round_up(c.count * sizeof(float), kAlign);
   c.off_partials = off;
   int64_t tiles = 0;
   for (int i = c.first; i < c.first + c.count; ++i)
@@ -393,6 +393,25 @@ muon_status set_device(muon_ctx* ctx) {
 // ---------------------------------------------------------------------------
 // launches
 // ---------------------------------------------------------------------------
+// Launch with programmatic stream serialization: the kernel may be scheduled
+// while the previous kernel in the stream drains; every kernel launched this
+// way calls pdl_wait() before its first global-memory access.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 template <int KIND, bool BMN>
 cudaError_t launch_gemm(muon_ctx* ctx, const GemmMaps& maps, const GemmArgs& g, cudaStream_t st) {
   static bool attr_done[64] = {};
@@ -417,9 +436,10 @@ cudaError_t launch_gemm(muon_ctx* ctx, const GemmMaps& maps, const GemmArgs& g, 
   }
   if (g.total <= 0) return cudaSuccess;
   const int pairs = std::min(g.total, max_pairs[dev]);   // persistent pairs
-  ns_gemm_kernel<KIND, BMN><<<unsigned(2 * pairs), gemm_cfg::THREADS, gemm_cfg::smem_bytes(KIND), st>>>(maps, g);
+  const cudaError_t e = launch_pdl(ns_gemm_kernel<KIND, BMN>, dim3(unsigned(2 * pairs)), dim3(gemm_cfg::THREADS),
+                                   size_t(gemm_cfg::smem_bytes(KIND)), st, maps, g);
   ctx->launches++;
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 // Device buffers and tensor maps of one shape run.
@@ -757,7 +777,6 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
         d.x_out = reinterpret_cast<__nv_bfloat16*>(ws + (final_buf ? r.off_x1 : r.off_x0)) +
                   int64_t(k) * r.m * r.ld_n;
         d.norm2 = reinterpret_cast<float*>(ws + c.off_norm) + (idx - c.first);
-        d.counter = reinterpret_cast<unsigned*>(ws + c.off_norm + c.count * sizeof(float)) + (idx - c.first);
         d.partials = reinterpret_cast<float*>(ws + c.off_partials);
         d.rows = it.rows;
         d.cols = it.cols;
@@ -817,7 +836,8 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
     {
       ProfScope ps(ctx, MUON_K_OTHER, st);
       for (const SegLaunch& L : build_seg_launches(raw.data(), int(raw.size()))) {
-      finite_kernel<<<unsigned(L.tiles), EW_THREADS, 0, st>>>(draw, L.t, L.tile_base, ctx->dflags + 1);
+      launch_pdl(finite_kernel, dim3(unsigned(L.tiles)), dim3(EW_THREADS), size_t(0), st,
+                 draw, L.t, L.tile_base, ctx->dflags + 1);
       ctx->launches++;
     }
     }
@@ -828,7 +848,6 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
   for (size_t ci = 0; ci < chunks.size(); ++ci) {
     const Chunk& c = chunks[ci];
     float* norm2 = reinterpret_cast<float*>(ws + c.off_norm);
-    CUDA_TRY(ctx, cudaMemsetAsync(norm2, 0, c.count * (sizeof(float) + sizeof(unsigned)), st));
     if (chunk_prep_count[ci] > 0) {
       ProfScope ps(ctx, MUON_K_PRECONDITION, st);
       int64_t most = 0;
@@ -838,7 +857,7 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
       }
       const dim3 grid(unsigned(std::max<int64_t>(1, std::min<int64_t>(cdiv(most, 256 * 8), 512))),
                       unsigned(chunk_prep_count[ci]));
-      precond_prep_kernel<<<grid, 256, 0, st>>>(dprep + chunk_prep_begin[ci]);
+      launch_pdl(precond_prep_kernel, grid, dim3(256), size_t(0), st, dprep + chunk_prep_begin[ci]);
       ctx->launches++;
       CUDA_TRY(ctx, cudaGetLastError());
       s = run_precondition(ctx, chunk_pprob[ci], skip, st);
@@ -846,8 +865,8 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
     }
     if (chunk_pcount[ci] > 0) {
       ProfScope ps(ctx, MUON_K_PRECONDITION, st);
-      precond_kernel<<<unsigned(chunk_ptiles[ci]), PRE_THREADS, 0, st>>>(dpdesc + chunk_pbegin[ci],
-                                                                        chunk_pcount[ci], skip);
+      launch_pdl(precond_kernel, dim3(unsigned(chunk_ptiles[ci])), dim3(PRE_THREADS), size_t(0), st,
+          dpdesc + chunk_pbegin[ci], chunk_pcount[ci], skip);
       ctx->launches++;
       CUDA_TRY(ctx, cudaGetLastError());
     }
@@ -856,14 +875,15 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
       ProfScope ps(ctx, MUON_K_MOMENTUM, st);
       for (const SegLaunch& L : segl) {
         if (mode == 0)
-          momentum_kernel<0><<<unsigned(L.tiles), EW_THREADS, 0, st>>>(ddesc + c.first, L.t, L.tile_base,
-                                                                       hp->momentum, hp->nesterov, skip);
+          launch_pdl(momentum_kernel<0>, dim3(unsigned(L.tiles)), dim3(EW_THREADS), size_t(0), st,
+              ddesc + c.first, L.t, L.tile_base, hp->momentum, hp->nesterov, skip);
         else
-          momentum_kernel<1><<<unsigned(L.tiles), EW_THREADS, 0, st>>>(ddesc + c.first, L.t, L.tile_base, 0.f,
-                                                                       0, skip);
+          launch_pdl(momentum_kernel<1>, dim3(unsigned(L.tiles)), dim3(EW_THREADS), size_t(0), st,
+              ddesc + c.first, L.t, L.tile_base, 0.f, 0, skip);
       }
+      launch_pdl(norm_reduce_kernel, dim3(unsigned(c.count)), dim3(EW_THREADS), size_t(0), st, ddesc + c.first, skip);
     }
-    ctx->launches += segl.size();
+    ctx->launches += segl.size() + 1;
     CUDA_TRY(ctx, cudaGetLastError());
     {
       std::vector<const float*> n2(c.runs.size());
@@ -875,11 +895,11 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
       ProfScope ps(ctx, MUON_K_APPLY, st);
       for (const SegLaunch& L : segl) {
         if (mode == 0)
-          apply_kernel<0><<<unsigned(L.tiles), EW_THREADS, 0, st>>>(ddesc + c.first, L.t, L.tile_base,
-                                                                    hp->ns_steps == 0, hp->eps, skip);
+          launch_pdl(apply_kernel<0>, dim3(unsigned(L.tiles)), dim3(EW_THREADS), size_t(0), st,
+              ddesc + c.first, L.t, L.tile_base, hp->ns_steps == 0, hp->eps, skip);
         else
-          apply_kernel<1><<<unsigned(L.tiles), EW_THREADS, 0, st>>>(ddesc + c.first, L.t, L.tile_base,
-                                                                    hp->ns_steps == 0, hp->eps, skip);
+          launch_pdl(apply_kernel<1>, dim3(unsigned(L.tiles)), dim3(EW_THREADS), size_t(0), st,
+              ddesc + c.first, L.t, L.tile_base, hp->ns_steps == 0, hp->eps, skip);
       }
     }
     ctx->launches += segl.size();
@@ -1125,8 +1145,8 @@ muon_status muon_adamw_step(muon_ctx* ctx, const muon_adamw_tensor* tensors, int
   sc.bc2_sqrt = float(std::sqrt(1.0 - std::pow(double(hp->beta2), double(step))));
   {
     ProfScope ps(ctx, MUON_K_ADAMW, st);
-    adamw_kernel<<<unsigned(chunks), EW_THREADS, 0, st>>>(static_cast<const AdamDesc*>(dtab), int(descs.size()),
-                                                          sc);
+    launch_pdl(adamw_kernel, dim3(unsigned(chunks)), dim3(EW_THREADS), size_t(0), st,
+        static_cast<const AdamDesc*>(dtab), int(descs.size()), sc);
   }
   ctx->launches++;
   CUDA_TRY(ctx, cudaGetLastError());
@@ -1213,7 +1233,7 @@ muon_status muon_newton_refresh(muon_ctx* ctx, const muon_act_desc* acts, int32_
   const ActBlock* dab = static_cast<const ActBlock*>(dtab);
   const CholDesc* dc = reinterpret_cast<const CholDesc*>(static_cast<uint8_t*>(dtab) + ab_bytes);
   ProfScope ps(ctx, MUON_K_NEWTON_REFRESH, st);
-  act_transpose_kernel<<<dim3(unsigned(max_tiles), unsigned(ab.size())), 256, 0, st>>>(dab);
+  launch_pdl(act_transpose_kernel, dim3(unsigned(max_tiles), unsigned(ab.size())), dim3(256), size_t(0), st, dab);
   ctx->launches++;
   CUDA_TRY(ctx, cudaGetLastError());
   // S = Xt Xt^T / tokens on the tensor cores, up to MAX_PROBLEMS shapes per launch
@@ -1256,12 +1276,14 @@ muon_status muon_newton_refresh(muon_ctx* ctx, const muon_act_desc* acts, int32_
     for (int p0 = 0; p0 < max_d; p0 += CB) {
       const int rest = max_d - p0 - CB;                   // trailing rows of the largest matrix
       const unsigned chunks = unsigned(std::max<int64_t>(1, cdiv(std::max(rest, 0), CPR)));
-      chol_panel_kernel<<<dim3(chunks, unsigned(cd.size())), CP_THREADS, 0, st>>>(dc, p0, damping, ctx->dflags);
+      launch_pdl(chol_panel_kernel, dim3(chunks, unsigned(cd.size())), dim3(CP_THREADS), size_t(0), st,
+          dc, p0, damping, ctx->dflags);
       ctx->launches++;
       CUDA_TRY(ctx, cudaGetLastError());
       if (rest > 0) {
         const int nt = int(cdiv(rest, CU_T));
-        chol_update_kernel<<<dim3(unsigned(nt * (nt + 1) / 2), unsigned(cd.size())), CP_THREADS, 0, st>>>(dc, p0);
+        launch_pdl(chol_update_kernel, dim3(unsigned(nt * (nt + 1) / 2), unsigned(cd.size())), dim3(CP_THREADS),
+                   size_t(0), st, dc, p0);
         ctx->launches++;
         CUDA_TRY(ctx, cudaGetLastError());
       }
@@ -1269,16 +1291,18 @@ muon_status muon_newton_refresh(muon_ctx* ctx, const muon_act_desc* acts, int32_
     // L^-1 into the output buffers, then S^-1 = L^-T L^-1 into the scratch
     // that held L, then copied out
     const int parts = int(cdiv(max_d, CB));
-    chol_linv_kernel<<<unsigned(cd.size() * parts), CINV_THREADS, cinv_smem_bytes(max_d), st>>>(dc, parts);
+    launch_pdl(chol_linv_kernel, dim3(unsigned(cd.size() * parts)), dim3(CINV_THREADS),
+               size_t(cinv_smem_bytes(max_d)), st, dc, parts);
     ctx->launches++;
     CUDA_TRY(ctx, cudaGetLastError());
     const int nt = int(cdiv(max_d, SIP_T));
-    spd_inverse_product_kernel<<<dim3(unsigned(nt * (nt + 1) / 2), unsigned(cd.size())), SIP_THREADS, 0, st>>>(dc);
+    launch_pdl(spd_inverse_product_kernel, dim3(unsigned(nt * (nt + 1) / 2), unsigned(cd.size())),
+               dim3(SIP_THREADS), size_t(0), st, dc);
     ctx->launches++;
     CUDA_TRY(ctx, cudaGetLastError());
     const int64_t most = int64_t(max_d) * max_d;
-    copy_inverse_kernel<<<dim3(unsigned(std::min<int64_t>(cdiv(most, 4 * 256), 1024)), unsigned(cd.size())), 256, 0,
-                          st>>>(dc);
+    launch_pdl(copy_inverse_kernel, dim3(unsigned(std::min<int64_t>(cdiv(most, 4 * 256), 1024)), unsigned(cd.size())),
+               dim3(256), size_t(0), st, dc);
     ctx->launches++;
     CUDA_TRY(ctx, cudaGetLastError());
     return MUON_OK;
@@ -1381,7 +1405,7 @@ muon_status muon_orthogonalize_noalloc(const void* input, int32_t in_dtype, int6
   if (s != MUON_OK) return s;
   tmp.device = device;
 
-  // Layout: flags | descriptor | norm + counter | partials | X0 | X1 | A | B
+  // Layout: flags | descriptor | norm | partials | X0 | X1 | A | B
   Item it{};
   it.rows = rows;
   it.cols = cols;
@@ -1410,7 +1434,6 @@ muon_status muon_orthogonalize_noalloc(const void* input, int32_t in_dtype, int6
   d.x_in = reinterpret_cast<__nv_bfloat16*>(ws + r.off_x0);
   d.x_out = reinterpret_cast<__nv_bfloat16*>(ws + ((hp->ns_steps % 2) ? r.off_x1 : r.off_x0));
   d.norm2 = reinterpret_cast<float*>(ws + c.off_norm);
-  d.counter = reinterpret_cast<unsigned*>(ws + c.off_norm + sizeof(float));
   d.partials = reinterpret_cast<float*>(ws + c.off_partials);
   d.rows = rows;
   d.cols = cols;
@@ -1424,12 +1447,12 @@ muon_status muon_orthogonalize_noalloc(const void* input, int32_t in_dtype, int6
   // The descriptor is copied from this stack frame; the runtime stages a
   // pageable source before the call returns.
   if (cudaMemcpyAsync(ddesc, &d, sizeof(MatDesc), cudaMemcpyHostToDevice, st) != cudaSuccess) return MUON_ERR_CUDA;
-  // Previous calls leave their values behind: zero the flags, the norm and
-  // the tile counter (everything else is fully overwritten before it is read).
+  // Previous calls leave their values behind: zero the flags (everything
+  // else is fully overwritten before it is read).
   if (cudaMemsetAsync(flags, 0, sizeof(int) * 4, st) != cudaSuccess) return MUON_ERR_CUDA;
-  if (cudaMemsetAsync(ws + c.off_norm, 0, sizeof(float) + sizeof(unsigned), st) != cudaSuccess) return MUON_ERR_CUDA;
   const std::vector<SegLaunch> segl = build_seg_launches(&d, 1);
   momentum_kernel<1><<<unsigned(tiles), EW_THREADS, 0, st>>>(ddesc, segl[0].t, 0, 0.f, 0, nullptr);
+  norm_reduce_kernel<<<1, EW_THREADS, 0, st>>>(ddesc, nullptr);
   if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;
   tmp.dflags = flags;
   const float* n2 = d.norm2;

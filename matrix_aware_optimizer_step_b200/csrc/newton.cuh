@@ -125,6 +125,7 @@ constexpr int CPR = 64;                     // panel rows per chol_panel_kernel 
 // with pivot 1 so the launch sequence stays well defined.
 __global__ void __launch_bounds__(CP_THREADS)
     chol_panel_kernel(const CholDesc* __restrict__ descs, int p0, float damping, int* err) {
+  pdl_wait();      // previous kernel's results visible (no-op without PDL)
   const CholDesc& c = descs[blockIdx.y];
   const int d = c.d;
   if (p0 >= d) return;
@@ -207,6 +208,7 @@ __global__ void __launch_bounds__(CP_THREADS)
 constexpr int CU_T = 64;
 constexpr int CU_P = CU_T + 4;              // padded row of the transposed panel slices (16-byte rows)
 __global__ void __launch_bounds__(CP_THREADS) chol_update_kernel(const CholDesc* __restrict__ descs, int p0) {
+  pdl_wait();      // previous kernel's results visible (no-op without PDL)
   const CholDesc& c = descs[blockIdx.y];
   const int d = c.d;
   const int q0 = p0 + CB;
@@ -270,6 +272,7 @@ __host__ __device__ inline int cinv_smem_bytes(int d) { return d * CB * 4; }
 // spd_inverse_product_kernel.  L is read from the lower triangle of c.a.
 __global__ void __launch_bounds__(CINV_THREADS)
     chol_linv_kernel(const CholDesc* __restrict__ descs, int blocks_per_mat) {
+  pdl_wait();      // previous kernel's results visible (no-op without PDL)
   extern __shared__ float4 y4[];           // Y: [d][CB] floats, 16-byte rows units
   float* y = reinterpret_cast<float*>(y4);
   __shared__ float acc_s[CB][CBP];
@@ -368,6 +371,7 @@ __global__ void __launch_bounds__(CINV_THREADS)
 // register tiles; the tile and its mirror are written to c.a.
 constexpr int SIP_T = 64, SIP_K = 32, SIP_THREADS = 256;
 __global__ void __launch_bounds__(SIP_THREADS) spd_inverse_product_kernel(const CholDesc* __restrict__ descs) {
+  pdl_wait();      // previous kernel's results visible (no-op without PDL)
   const CholDesc& c = descs[blockIdx.y];
   const int d = c.d;
   const int nt = (d + SIP_T - 1) / SIP_T;
@@ -441,6 +445,7 @@ __global__ void __launch_bounds__(SIP_THREADS) spd_inverse_product_kernel(const 
 
 // c.inv = c.a (d x d), grid.y = matrix.
 __global__ void __launch_bounds__(256) copy_inverse_kernel(const CholDesc* __restrict__ descs) {
+  pdl_wait();      // previous kernel's results visible (no-op without PDL)
   const CholDesc& c = descs[blockIdx.y];
   const int64_t n = int64_t(c.d) * c.d;
   const int64_t stride = int64_t(gridDim.x) * 256;
@@ -508,6 +513,7 @@ struct PrecondDesc {
 
 __global__ void __launch_bounds__(PRE_THREADS)
     precond_kernel(const PrecondDesc* __restrict__ descs, int n, const int* skip) {
+  pdl_wait();      // previous kernel's results visible (no-op without PDL)
   if (skip != nullptr && *skip) return;
   __shared__ float gs[PRE_BK][PRE_BM + 4];   // G tile, transposed (k, row)
   __shared__ float ss[PRE_BK][PRE_BN + 4];   // S^-1 tile (k, col)
@@ -576,6 +582,7 @@ struct ActBlock {
 // stores through a swizzled 64x64 tile (tsw, conflict-free in both
 // directions) when the widths allow, elementwise at ragged edges.
 __global__ void __launch_bounds__(256) act_transpose_kernel(const ActBlock* __restrict__ blocks) {
+  pdl_wait();      // previous kernel's results visible (no-op without PDL)
   __shared__ __align__(16) __nv_bfloat16 t[TPOSE_T][TPOSE_T];   // t[j][tsw(j, tok)]
   const ActBlock& b = blocks[blockIdx.y];
   const int64_t tiles_j = (b.d + TPOSE_T - 1) / TPOSE_T;
@@ -633,6 +640,7 @@ struct PrepDesc {
 // per thread and step (16-byte loads and stores) when the gradient width and
 // d*d are multiples of 8, one otherwise.  Pointers are 16-byte aligned.
 __global__ void __launch_bounds__(256) precond_prep_kernel(const PrepDesc* __restrict__ descs) {
+  pdl_wait();      // previous kernel's results visible (no-op without PDL)
   const PrepDesc& p = descs[blockIdx.y];
   const int64_t ng = p.rows * p.cols;
   const int64_t dd = static_cast<int64_t>(p.d) * p.d;

@@ -208,7 +208,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
   using namespace gemm_cfg;
   constexpr int STAGES = stages_for(KIND);
   extern __shared__ uint8_t smem_raw[];
-  if (args.skip != nullptr && *args.skip) return;   // uniform over the grid
 
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -229,7 +228,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
   const bool leader = rank == 0;
   const int pair = blockIdx.x >> 1;
   const int npairs = gridDim.x >> 1;
-  const int total = args.total;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -261,6 +259,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
   cluster_sync();              // both CTAs' barriers exist before any remote use
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // everything above touches only shared memory, TMEM and the parameter
+  // space, so it runs before the wait for the previous kernel
+  pdl_wait();
+  // a non-finite gradient flag (uniform over the grid) leaves an empty tile list
+  const int total = (args.skip != nullptr && *args.skip) ? 0 : args.total;
 
   if (warp == 0) {
     // ---------------- TMA producer (both CTAs load their halves) ----------------

@@ -74,8 +74,8 @@ def _group(mx, rows, cols, count, dtype=1, keep=None):
 
 def test_query_workspace_plans_wide_layout(mx):
     """Workspace = per shape run: two wide bf16 X buffers (m x ld_n) and the
-    symmetric A, B (m x ld_m); plus one fp32 norm and one counter per matrix
-    and one fp32 partial per 64x64 tile; 256-byte aligned regions.  Tall
+    symmetric A, B (m x ld_m); plus one fp32 norm per matrix and one fp32
+    partial per 64x64 tile; 256-byte aligned regions.  Tall
     matrices share the run of their transpose."""
     lib = mx.load_library()
     keep = []
@@ -89,7 +89,7 @@ def test_query_workspace_plans_wide_layout(mx):
     def r256(x):
         return (x + 255) // 256 * 256
     tiles = 24 * 576 + 48 * 144           # 64x64 tiles: one fp32 partial norm each
-    want = r256(72 * 8) + r256(tiles * 4)
+    want = r256(72 * 4) + r256(tiles * 4)
     want += 2 * r256(24 * 768 * 3072 * 2) + 2 * r256(24 * 768 * 768 * 2)
     want += 2 * r256(48 * 768 * 768 * 2) + 2 * r256(48 * 768 * 768 * 2)
     assert n.value == want
@@ -97,7 +97,7 @@ def test_query_workspace_plans_wide_layout(mx):
     arr1 = (mx.binding.Group * 1)()
     arr1[0] = _group(mx, 5, 3, 1, keep=keep)
     assert lib.muon_query_workspace(arr1, 1, ctypes.byref(n)) == 0
-    assert n.value == r256(8) + r256(4) + 2 * r256(3 * 8 * 2) + 2 * r256(3 * 8 * 2)
+    assert n.value == r256(4) + r256(4) + 2 * r256(3 * 8 * 2) + 2 * r256(3 * 8 * 2)
 
 
 def test_query_workspace_rejects_bad_groups(mx):
