@@ -126,8 +126,46 @@ __global__ void __launch_bounds__(EW_THREADS)
   const int64_t lt = gt - d.tile_start;
   const int64_t r0 = (lt / d.tiles_c) * EW_TILE;
   const int64_t c0 = (lt % d.tiles_c) * EW_TILE;
-  const bool vec_ok = (d.cols % 8 == 0) && (d.ld % 8 == 0);
   float ss = 0.f;
+  if (!d.transposed && d.ld == d.cols && (d.cols % 8) == 0) {
+    // Rows are contiguous in both layouts: block lt takes elements
+    // [4096 lt, 4096 lt + 4096) of the flattened matrix, so each warp moves
+    // 256 consecutive elements (the matrix has at least as many 64x64 tiles
+    // as 4096-element runs; the blocks past its end store a zero partial).
+    const int64_t n = d.rows * d.cols;
+#pragma unroll
+    for (int it = 0; it < 2; ++it) {
+      const int64_t e = lt * (EW_TILE * EW_TILE) + (threadIdx.x + it * EW_THREADS) * 8;
+      if (e >= n) continue;
+      float g[8], u[8];
+      load8_grad(d.grad, d.grad_dtype, e, g);
+      if (MODE == 0) {
+        float4* bp = reinterpret_cast<float4*>(d.momentum + e);
+        const float4 b0 = bp[0], b1 = bp[1];
+        float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          b[k] = beta * b[k] + (1.f - beta) * g[k];
+          u[k] = nesterov ? (1.f - beta) * g[k] + beta * b[k] : b[k];
+        }
+        bp[0] = make_float4(b[0], b[1], b[2], b[3]);
+        bp[1] = make_float4(b[4], b[5], b[6], b[7]);
+      } else {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) u[k] = g[k];
+      }
+#pragma unroll
+      for (int k = 0; k < 8; ++k) ss += u[k] * u[k];
+      uint4 w;
+      w.x = pack_bf16x2(u[0], u[1]); w.y = pack_bf16x2(u[2], u[3]);
+      w.z = pack_bf16x2(u[4], u[5]); w.w = pack_bf16x2(u[6], u[7]);
+      *reinterpret_cast<uint4*>(d.x_in + e) = w;
+    }
+    const float tot = block_sum(ss, red);
+    if (threadIdx.x == 0) d.partials[gt] = tot;
+    return;
+  }
+  const bool vec_ok = (d.cols % 8 == 0) && (d.ld % 8 == 0);
   // 64 rows x 8 vectors of 8 columns = 512 vectors, 2 per thread
 #pragma unroll
   for (int it = 0; it < 2; ++it) {
@@ -224,6 +262,25 @@ __global__ void __launch_bounds__(EW_THREADS) norm_reduce_kernel(const MatDesc* 
   if (threadIdx.x == 0) *d.norm2 = all;
 }
 
+// W[0..8) <- W (1 - lr wd) - lr scale O, W already loaded into w.
+__device__ __forceinline__ void store_weight8(float* dst, const float4 (&w)[2], const float (&o)[8], float decay,
+                                              float lr_scale) {
+  float4 w0 = w[0], w1 = w[1];
+  w0.x = w0.x * decay - lr_scale * o[0]; w0.y = w0.y * decay - lr_scale * o[1];
+  w0.z = w0.z * decay - lr_scale * o[2]; w0.w = w0.w * decay - lr_scale * o[3];
+  w1.x = w1.x * decay - lr_scale * o[4]; w1.y = w1.y * decay - lr_scale * o[5];
+  w1.z = w1.z * decay - lr_scale * o[6]; w1.w = w1.w * decay - lr_scale * o[7];
+  float4* wp = reinterpret_cast<float4*>(dst);
+  wp[0] = w0;
+  wp[1] = w1;
+}
+
+__device__ __forceinline__ void store_f32x8(float* dst, const float (&o)[8]) {
+  float4* op = reinterpret_cast<float4*>(dst);
+  op[0] = make_float4(o[0], o[1], o[2], o[3]);
+  op[1] = make_float4(o[4], o[5], o[6], o[7]);
+}
+
 // mode 0: apply update to W (and optionally write O)
 // mode 1: export O only (Newton-Schulz only path)
 // norm_scale: when no iteration ran, O = U / (||U|| + eps) is formed here.
@@ -240,6 +297,56 @@ __global__ void __launch_bounds__(EW_THREADS)
   const int64_t r0 = (lt / d.tiles_c) * EW_TILE;
   const int64_t c0 = (lt % d.tiles_c) * EW_TILE;
   const float s = normalise ? 1.0f / (sqrtf(*d.norm2) + eps) : 1.0f;
+  if (!d.transposed && d.ld == d.cols && (d.cols % 8) == 0) {
+    // contiguous rows: the flat element run of momentum_kernel, loads of both
+    // vectors issued before any store
+    const int64_t n = d.rows * d.cols;
+    float o[2][8];
+    float4 w[2][2];
+#pragma unroll
+    for (int it = 0; it < 2; ++it) {
+      const int64_t e = lt * (EW_TILE * EW_TILE) + (threadIdx.x + it * EW_THREADS) * 8;
+      if (e < n) {
+        const uint4 x = *reinterpret_cast<const uint4*>(d.x_out + e);
+        float2 f;
+        f = unpack_bf16x2(x.x); o[it][0] = f.x; o[it][1] = f.y;
+        f = unpack_bf16x2(x.y); o[it][2] = f.x; o[it][3] = f.y;
+        f = unpack_bf16x2(x.z); o[it][4] = f.x; o[it][5] = f.y;
+        f = unpack_bf16x2(x.w); o[it][6] = f.x; o[it][7] = f.y;
+        if (MODE == 0) {
+          const float4* wp = reinterpret_cast<const float4*>(d.weight + e);
+          w[it][0] = wp[0];
+          w[it][1] = wp[1];
+        }
+      }
+    }
+#pragma unroll
+    for (int it = 0; it < 2; ++it) {
+      const int64_t e = lt * (EW_TILE * EW_TILE) + (threadIdx.x + it * EW_THREADS) * 8;
+      if (e >= n) continue;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) o[it][k] *= s;
+      if (MODE == 0) store_weight8(d.weight + e, w[it], o[it], d.decay, d.lr_scale);
+      if (d.update_out != nullptr) store_f32x8(d.update_out + e, o[it]);
+    }
+    return;
+  }
+  // 64x64 tile: W loads first (independent of O), then O (through shared
+  // memory for tall matrices), then the stores
+  const bool vec_ok = (d.cols % 8 == 0) && (d.ld % 8 == 0);
+  float4 w[2][2];
+  bool full[2];
+#pragma unroll
+  for (int it = 0; it < 2; ++it) {
+    const int v = threadIdx.x + it * EW_THREADS;
+    const int64_t r = r0 + (v >> 3), c = c0 + (v & 7) * 8;
+    full[it] = r < d.rows && vec_ok && c + 8 <= d.cols;
+    if (full[it] && MODE == 0) {
+      const float4* wp = reinterpret_cast<const float4*>(d.weight + r * d.cols + c);
+      w[it][0] = wp[0];
+      w[it][1] = wp[1];
+    }
+  }
   if (d.transposed) {
     // stage the 64x64 block of the wide X (rows c0.., cols r0..) in smem
 #pragma unroll
@@ -257,22 +364,21 @@ __global__ void __launch_bounds__(EW_THREADS)
     }
     __syncthreads();
   }
-  const bool vec_ok = (d.cols % 8 == 0) && (d.ld % 8 == 0);
 #pragma unroll
   for (int it = 0; it < 2; ++it) {
     const int v = threadIdx.x + it * EW_THREADS;
     const int rl = v >> 3, cl = (v & 7) * 8;
     const int64_t r = r0 + rl, c = c0 + cl;
     if (r >= d.rows) continue;
-    if (vec_ok && c + 8 <= d.cols) {
+    if (full[it]) {
       float o[8];
       if (!d.transposed) {
-        const uint4 w = *reinterpret_cast<const uint4*>(d.x_out + r * d.ld + c);
+        const uint4 x = *reinterpret_cast<const uint4*>(d.x_out + r * d.ld + c);
         float2 f;
-        f = unpack_bf16x2(w.x); o[0] = f.x; o[1] = f.y;
-        f = unpack_bf16x2(w.y); o[2] = f.x; o[3] = f.y;
-        f = unpack_bf16x2(w.z); o[4] = f.x; o[5] = f.y;
-        f = unpack_bf16x2(w.w); o[6] = f.x; o[7] = f.y;
+        f = unpack_bf16x2(x.x); o[0] = f.x; o[1] = f.y;
+        f = unpack_bf16x2(x.y); o[2] = f.x; o[3] = f.y;
+        f = unpack_bf16x2(x.z); o[4] = f.x; o[5] = f.y;
+        f = unpack_bf16x2(x.w); o[6] = f.x; o[7] = f.y;
       } else {
 #pragma unroll
         for (int k = 0; k < 8; ++k) o[k] = __bfloat162float(tile[cl + k][tsw(cl + k, rl)]);
@@ -280,20 +386,8 @@ __global__ void __launch_bounds__(EW_THREADS)
 #pragma unroll
       for (int k = 0; k < 8; ++k) o[k] *= s;
       const int64_t idx = r * d.cols + c;
-      if (MODE == 0) {
-        float4* wp = reinterpret_cast<float4*>(d.weight + idx);
-        float4 w0 = wp[0], w1 = wp[1];
-        w0.x = w0.x * d.decay - d.lr_scale * o[0]; w0.y = w0.y * d.decay - d.lr_scale * o[1];
-        w0.z = w0.z * d.decay - d.lr_scale * o[2]; w0.w = w0.w * d.decay - d.lr_scale * o[3];
-        w1.x = w1.x * d.decay - d.lr_scale * o[4]; w1.y = w1.y * d.decay - d.lr_scale * o[5];
-        w1.z = w1.z * d.decay - d.lr_scale * o[6]; w1.w = w1.w * d.decay - d.lr_scale * o[7];
-        wp[0] = w0; wp[1] = w1;
-      }
-      if (d.update_out != nullptr) {
-        float4* op = reinterpret_cast<float4*>(d.update_out + idx);
-        op[0] = make_float4(o[0], o[1], o[2], o[3]);
-        op[1] = make_float4(o[4], o[5], o[6], o[7]);
-      }
+      if (MODE == 0) store_weight8(d.weight + idx, w[it], o, d.decay, d.lr_scale);
+      if (d.update_out != nullptr) store_f32x8(d.update_out + idx, o);
     } else {
       for (int k = 0; k < 8; ++k) {
         const int64_t cc = c + k;
