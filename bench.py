@@ -343,13 +343,35 @@ def main():
           for i, m in enumerate(w.mats)]
     Bs = [torch.zeros((m.rows, m.cols), device=dev) for m in w.mats]
     n_cycle = min(GRAD_CYCLE, max(1, w.steps)) if args.workload != "llama3-8b" else 1
-    Gs = [[wl.torch_normal((m.rows, m.cols), w.grad_std, seed, s, i, wl.ROLE_GRAD, dtype=tdt, device=dev)
-           for i, m in enumerate(w.mats)] for s in range(n_cycle)]
+    def flat_set(shapes, dtype):
+        # one contiguous buffer per set (every tensor starts on a 16-byte
+        # boundary), so a set moves between host and device in one copy
+        sizes = [math.prod(sh) for sh in shapes]
+        pads = [(n + 7) // 8 * 8 for n in sizes]
+        flat = torch.empty(sum(pads), dtype=dtype, device=dev)
+        views, off = [], 0
+        for sh, n, pn in zip(shapes, sizes, pads):
+            views.append(flat[off:off + n].view(sh))
+            off += pn
+        return flat, views
+
+    G_flat, Gs = [], []
+    for s in range(n_cycle):
+        f, vs = flat_set([(m.rows, m.cols) for m in w.mats], tdt)
+        for i, (m, v) in enumerate(zip(w.mats, vs)):
+            wl.torch_normal((m.rows, m.cols), w.grad_std, seed, s, i, wl.ROLE_GRAD, out=v)
+        G_flat.append(f)
+        Gs.append(vs)
     Ps = [wl.torch_normal((n,), 0.02, seed, 0, 10000 + i, wl.ROLE_WEIGHT, device=dev) for i, (_, n) in enumerate(aux)]
     Ms = [torch.zeros(n, device=dev) for _, n in aux]
     Vs = [torch.zeros(n, device=dev) for _, n in aux]
-    AGs = [[wl.torch_normal((n,), 1e-3, seed, s, 10000 + i, wl.ROLE_AUX, dtype=torch.bfloat16, device=dev)
-            for i, (_, n) in enumerate(aux)] for s in range(n_cycle)]
+    AG_flat, AGs = [], []
+    for s in range(n_cycle):
+        f, vs = flat_set([(n,) for _, n in aux], torch.bfloat16)
+        for i, ((_, n), v) in enumerate(zip(aux, vs)):
+            wl.torch_normal((n,), 1e-3, seed, s, 10000 + i, wl.ROLE_AUX, out=v)
+        AG_flat.append(f)
+        AGs.append(vs)
 
     by_shape = {}
     for i, m in enumerate(w.mats):
@@ -415,13 +437,15 @@ def main():
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
 
-    def timed(k_steps, body):
+    def timed(k_steps, body, finish=None):
         barrier()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for k in range(k_steps):
             body(k)
+        if finish is not None:
+            finish()          # join side streams into `stream` before the end event
         e1.record(stream)
         torch.cuda.synchronize()
         barrier()
@@ -500,30 +524,71 @@ def main():
     # ---- end to end through the public API with host buffers ----
     e2e = None
     if not args.no_e2e:
-        hG = [[t.cpu().pin_memory() for t in Gs[s]] for s in range(n_cycle)]
-        hAG = [[t.cpu().pin_memory() for t in AGs[s]] for s in range(n_cycle)]
-        hW = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in Ws]
-        hP = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in Ps]
-        h2d = sum(t.numel() * t.element_size() for t in hG[0]) + sum(t.numel() * t.element_size() for t in hAG[0])
-        d2h = sum(t.numel() * t.element_size() for t in hW) + sum(t.numel() * t.element_size() for t in hP)
+        hG = [G_flat[s].cpu().pin_memory() for s in range(n_cycle)]
+        hAG = [AG_flat[s].cpu().pin_memory() for s in range(n_cycle)] if aux else [None] * n_cycle
+        dev_w = Ws + Ps
+        w_elems = sum(t.numel() for t in dev_w)
+        h_w = torch.empty(w_elems, dtype=torch.float32, pin_memory=True)   # every weight, concatenated
+        h2d = G_flat[0].numel() * G_flat[0].element_size() + (AG_flat[0].numel() * 2 if aux else 0)
+        d2h = w_elems * 4
         k_e2e = max(3, min(args.steps, 50))
+        # Pipelined like a training loop that streams gradients in and weights
+        # out: step k's gradients arrive on a copy-in stream (into the device
+        # set the step reads; the set is reused every n_cycle steps), the
+        # updated weights are copied on the device into one of two staging
+        # buffers and leave for the host on a copy-out stream, so PCIe in
+        # both directions overlaps the next step's kernels.
+        s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+        staging = w_elems * 4 <= (8 << 30)          # large sets copy out of the weights directly
+        stage = [torch.empty(w_elems, dtype=torch.float32, device=dev) for _ in range(2)] if staging else None
+        h_views, off = [], 0
+        for t in dev_w:
+            h_views.append(h_w[off:off + t.numel()].view(t.shape))
+            off += t.numel()
+        in_done = [torch.cuda.Event() for _ in range(n_cycle)]
+        used = [torch.cuda.Event() for _ in range(n_cycle)]
+        staged = [torch.cuda.Event() for _ in range(2)]
+        out_done = [torch.cuda.Event() for _ in range(2)]
 
         def e2e_step(k):
-            s = k % n_cycle
-            for dst, src in zip(Gs[s], hG[s]):
-                dst.copy_(src, non_blocking=True)
-            for dst, src in zip(AGs[s], hAG[s]):
-                dst.copy_(src, non_blocking=True)
+            s, b = k % n_cycle, k & 1
+            with torch.cuda.stream(s_in):
+                if k >= n_cycle:
+                    s_in.wait_event(used[s])          # the step that last read this set is done
+                G_flat[s].copy_(hG[s], non_blocking=True)
+                if aux:
+                    AG_flat[s].copy_(hAG[s], non_blocking=True)
+                in_done[s].record(s_in)
+            stream.wait_event(in_done[s])
+            if not staging and k >= 1:
+                stream.wait_event(out_done[b ^ 1])    # the previous weights have left before they change
             one_step(k)
-            for dst, src in zip(hW, Ws):
-                dst.copy_(src, non_blocking=True)
-            for dst, src in zip(hP, Ps):
-                dst.copy_(src, non_blocking=True)
+            used[s].record(stream)
+            if staging:
+                if k >= 2:
+                    stream.wait_event(out_done[b])    # staging buffer b (two steps ago) has left
+                torch.cat([t.view(-1) for t in dev_w], out=stage[b])   # one device kernel
+            staged[b].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(staged[b])
+                if staging:
+                    h_w.copy_(stage[b], non_blocking=True)
+                else:
+                    for dst, src in zip(h_views, dev_w):
+                        dst.copy_(src, non_blocking=True)
+                out_done[b].record(s_out)
 
-        ms_e2e = timed(k_e2e, e2e_step)
+        def e2e_finish():
+            stream.wait_event(out_done[(k_e2e - 1) & 1])
+
+        ms_e2e = timed(k_e2e, e2e_step, e2e_finish)
+        # the host holds the last step's weights
+        if not torch.equal(h_w, torch.cat([t.view(-1) for t in dev_w]).cpu()):
+            raise RuntimeError("e2e: host weights differ from the device weights")
         e2e = {"value": world * 1e3 * k_e2e / ms_e2e, "unit": "Muon step/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h,
-               "note": "gradients copied host->device and updated weights device->host every step"}
+               "note": "every step: gradients host->device (copy-in stream), updated fp32 weights device->device->host "
+                       "(copy-out stream), overlapped with the next step's kernels"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
