@@ -151,21 +151,32 @@ __global__ void __launch_bounds__(CP_THREADS)
   }
   __syncthreads();
   if (warp == 0) {
-    // unblocked Cholesky of D
-    for (int k = 0; k < nb; ++k) {
-      if (lane == 0) {
-        float dkk = dg[k][k];
-        if (!(dkk > 0.f)) { bad = 1; dkk = 1.f; }
-        dg[k][k] = sqrtf(dkk);
+    // unblocked Cholesky of D in registers: lane i holds row i (zero above
+    // the diagonal and past nb); column k travels by shuffle
+    float a[CB];
+#pragma unroll
+    for (int j = 0; j < CB; ++j) a[j] = dg[lane][j];
+    bool neg = false;
+#pragma unroll
+    for (int k = 0; k < CB; ++k) {
+      if (k < nb) {
+        float akk = __shfl_sync(0xffffffffu, a[k], k);
+        if (!(akk > 0.f)) { neg = true; akk = 1.f; }
+        const float lkk = sqrtf(akk);
+        if (lane == k) a[k] = lkk;
+        else if (lane > k) a[k] = a[k] / lkk;
+        const float lik = a[k];
+#pragma unroll
+        for (int j = k + 1; j < CB; ++j) {
+          const float ljk = __shfl_sync(0xffffffffu, a[k], j);
+          if (lane >= j) a[j] -= lik * ljk;
+        }
       }
-      __syncwarp();
-      const float lkk = dg[k][k];
-      if (lane > k && lane < nb) dg[lane][k] /= lkk;
-      __syncwarp();
-      if (lane > k && lane < nb)
-        for (int j = k + 1; j <= lane; ++j) dg[lane][j] -= dg[lane][k] * dg[j][k];
-      __syncwarp();
     }
+    if (lane == 0 && neg) bad = 1;
+#pragma unroll
+    for (int j = 0; j < CB; ++j) dg[lane][j] = a[j];
+    __syncwarp();
     // D x = e_lane: x = column `lane` of D^-1
     float x[CB];
 #pragma unroll
