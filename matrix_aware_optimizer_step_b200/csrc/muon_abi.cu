@@ -109,6 +109,20 @@ bool encode_bf16_3d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t 
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// fp32 matrix rows x cols (row pitch cols) viewed as (cols, rows, 1): 32 x 32
+// boxes, 128-byte swizzle (a box row is 128 bytes).
+bool encode_f32_matrix(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {cols, rows, 1};
+  cuuint64_t strides[2] = {cols * 4, rows * cols * 4};
+  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ---------------------------------------------------------------------------
 // small helpers
 // ---------------------------------------------------------------------------
@@ -475,7 +489,7 @@ bool encode_run(uint8_t* ws, const Run& r, RunMaps& mp) {
 // MAX_PROBLEMS runs.
 muon_status run_newton_schulz(muon_ctx* ctx, uint8_t* ws, const Run* runs, int nruns,
                               const float* const* norm2s, const muon_hparams* hp, const int* skip,
-                              cudaStream_t st) {
+                              cudaStream_t st, const ApplyDesc* const* run_apply = nullptr) {
   std::vector<RunMaps> mp(nruns);
   for (int j = 0; j < nruns; ++j)
     if (!encode_run(ws, runs[j], mp[j]))
@@ -502,6 +516,11 @@ muon_status run_newton_schulz(muon_ctx* ctx, uint8_t* ws, const Run* runs, int n
         g.c1 = hp->ns_c;
         g.c2 = hp->ns_a;
         g.reverse = (launch_no++ & 1) ^ 1;
+        // the last update applies the weight step itself when every run of
+        // the launch has its per-matrix weight descriptors
+        bool fuse = kind == EPI_UPDATE && it == hp->ns_steps - 1 && run_apply != nullptr;
+        for (int j = 0; fuse && j < nb; ++j) fuse = run_apply[b0 + j] != nullptr;
+        if (fuse) g.apply = run_apply[b0];
         int tile = 0;
         for (int j = 0; j < nb; ++j) {
           const Run& r = runs[b0 + j];
@@ -529,6 +548,7 @@ muon_status run_newton_schulz(muon_ctx* ctx, uint8_t* ws, const Run* runs, int n
             P.out = m.x[cur ^ 1]; P.out_ld = r.ld_n; P.out_bs = r.m * r.ld_n;
             P.norm2 = first ? norm2s[b0 + j] : nullptr;
             maps.a[j] = m.b_r128; maps.b[j] = m.x_mn[cur]; maps.aux[j] = m.x_r32[cur ^ 1]; maps.out[j] = m.x_c32[cur ^ 1];
+            if (fuse) P.apply_base = int(run_apply[b0 + j] - run_apply[b0]);
           }
           P.tiles_per_mat = gemm_tiles_per_mat(kind, P.tiles_m, P.tiles_n);
           const int64_t tt = int64_t(tile) + int64_t(P.batch) * P.tiles_per_mat;
@@ -542,6 +562,9 @@ muon_status run_newton_schulz(muon_ctx* ctx, uint8_t* ws, const Run* runs, int n
         } else if (kind == EPI_POLY) {
           ProfScope ps(ctx, MUON_K_POLY, st);
           CUDA_TRY(ctx, (launch_gemm<EPI_POLY, false>(ctx, maps, g, st)));
+        } else if (fuse) {
+          ProfScope ps(ctx, MUON_K_UPDATE, st);
+          CUDA_TRY(ctx, (launch_gemm<EPI_UPDATE_APPLY, true>(ctx, maps, g, st)));
         } else {
           ProfScope ps(ctx, MUON_K_UPDATE, st);
           CUDA_TRY(ctx, (launch_gemm<EPI_UPDATE, true>(ctx, maps, g, st)));
@@ -795,12 +818,50 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
     chunk_ptiles[ci] = ptiles;
     chunk_prep_count[ci] = int(prep.size()) - chunk_prep_begin[ci];
   }
+  // The last Newton-Schulz product applies the weight step itself (no apply
+  // pass, O never reaches memory) for every chunk whose matrices TMA can
+  // reach as fp32 rows x cols (row pitch a multiple of 16 bytes) and that
+  // asks for no update_out.  One ApplyDesc per matrix, in run order.
+  std::vector<ApplyDesc> adescs;
+  std::vector<std::vector<int64_t>> run_apply_idx(chunks.size());
+  std::vector<char> chunk_fused(chunks.size(), 0);
+  if (mode == 0 && hp->ns_steps >= 1) {
+    for (size_t ci = 0; ci < chunks.size(); ++ci) {
+      const Chunk& c = chunks[ci];
+      bool ok = true;
+      for (int i = c.first; i < c.first + c.count && ok; ++i)
+        ok = items[i].update_out == nullptr && items[i].cols % 4 == 0;
+      const size_t a0 = adescs.size();
+      std::vector<int64_t> idx;
+      for (size_t j = 0; ok && j < c.runs.size(); ++j) {
+        const Run& r = c.runs[j];
+        idx.push_back(int64_t(adescs.size()));
+        for (int k = 0; ok && k < r.count; ++k) {
+          const Item& it = items[r.first + k];
+          ApplyDesc ad{};
+          ok = encode_f32_matrix(&ad.w, it.weight, uint64_t(it.cols), uint64_t(it.rows));
+          ad.lr_scale = hp->lr * shape_scale(it.rows, it.cols, hp->scale_mode);
+          ad.decay = 1.0f - hp->lr * hp->weight_decay;
+          ad.transposed = it.transposed ? 1 : 0;
+          adescs.push_back(ad);
+        }
+      }
+      if (!ok) {
+        adescs.resize(a0);
+        continue;
+      }
+      run_apply_idx[ci] = idx;
+      chunk_fused[ci] = 1;
+    }
+  }
   const size_t mat_bytes = round_up(descs.size() * sizeof(MatDesc), kAlign);
   const size_t pd_bytes = round_up(pdescs.size() * sizeof(PrecondDesc), kAlign);
-  std::vector<uint8_t> table(mat_bytes + pd_bytes + prep.size() * sizeof(PrepDesc));
+  const size_t ap_off = round_up(mat_bytes + pd_bytes + prep.size() * sizeof(PrepDesc), kAlign);
+  std::vector<uint8_t> table(ap_off + adescs.size() * sizeof(ApplyDesc));
   std::memcpy(table.data(), descs.data(), descs.size() * sizeof(MatDesc));
   if (!pdescs.empty()) std::memcpy(table.data() + mat_bytes, pdescs.data(), pdescs.size() * sizeof(PrecondDesc));
   if (!prep.empty()) std::memcpy(table.data() + mat_bytes + pd_bytes, prep.data(), prep.size() * sizeof(PrepDesc));
+  if (!adescs.empty()) std::memcpy(table.data() + ap_off, adescs.data(), adescs.size() * sizeof(ApplyDesc));
   void* dtab = nullptr;
   s = upload_table(ctx, table.data(), table.size(), st, &dtab);
   if (s != MUON_OK) return s;
@@ -888,10 +949,16 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
     {
       std::vector<const float*> n2(c.runs.size());
       for (size_t j = 0; j < c.runs.size(); ++j) n2[j] = norm2 + (c.runs[j].first - c.first);
-      s = run_newton_schulz(ctx, ws, c.runs.data(), int(c.runs.size()), n2.data(), hp, skip, st);
+      std::vector<const ApplyDesc*> ra;
+      if (chunk_fused[ci]) {
+        const ApplyDesc* dapply = reinterpret_cast<const ApplyDesc*>(static_cast<uint8_t*>(dtab) + ap_off);
+        for (int64_t k : run_apply_idx[ci]) ra.push_back(dapply + k);
+      }
+      s = run_newton_schulz(ctx, ws, c.runs.data(), int(c.runs.size()), n2.data(), hp, skip, st,
+                            chunk_fused[ci] ? ra.data() : nullptr);
       if (s != MUON_OK) return s;
     }
-    {
+    if (!chunk_fused[ci]) {
       ProfScope ps(ctx, MUON_K_APPLY, st);
       for (const SegLaunch& L : segl) {
         if (mode == 0)
@@ -901,8 +968,8 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
           launch_pdl(apply_kernel<1>, dim3(unsigned(L.tiles)), dim3(EW_THREADS), size_t(0), st,
               ddesc + c.first, L.t, L.tile_base, hp->ns_steps == 0, hp->eps, skip);
       }
+      ctx->launches += segl.size();
     }
-    ctx->launches += segl.size();
     CUDA_TRY(ctx, cudaGetLastError());
   }
 

@@ -64,7 +64,7 @@
 
 namespace muon {
 
-enum EpiKind : int { EPI_GRAM = 0, EPI_POLY = 1, EPI_UPDATE = 2, EPI_GRAM32 = 3, EPI_PRECOND = 4 };
+enum EpiKind : int { EPI_GRAM = 0, EPI_POLY = 1, EPI_UPDATE = 2, EPI_GRAM32 = 3, EPI_PRECOND = 4, EPI_UPDATE_APPLY = 5 };
 
 namespace gemm_cfg {
 constexpr int TM = 256;                              // pair tile rows (128 per CTA)
@@ -76,6 +76,10 @@ constexpr int BK = 64;
 // chunks (below) and spend the space saved on a fifth / sixth stage; the
 // update also has no mirrored blocks.
 __host__ __device__ constexpr int stages_for(int kind) { return kind == 0 ? 5 : kind == 1 ? 4 : kind == 2 ? 6 : 5; }
+// The last update of an optimizer step may apply W <- W (1 - lr wd) - lr
+// scale O in its epilogue (EPI_UPDATE_APPLY): W moves through two 4 KB
+// 32x32 fp32 chunk buffers per warp by TMA, and O never reaches memory.
+__host__ __device__ constexpr bool apply_out(int kind) { return kind == 5; }
 __host__ __device__ constexpr bool mirrors(int kind) { return kind == 0 || kind == 1; }
 // Output leaves through two alternating 32x32 chunk buffers per warp
 // (GRAM, UPDATE) instead of a whole 32x128 slice (POLY reads its input A
@@ -93,15 +97,18 @@ constexpr int STG_PITCH = 64;                        // mirror staging: 32 rows 
 constexpr int STG_BYTES = 32 * STG_PITCH;
 constexpr int CH_BYTES = 32 * 64;                    // 32 rows x 32 bf16, 64-byte swizzle
 constexpr int CH_BUFS = 2;
-constexpr int BAR_BYTES = 256;
+constexpr int WCH_BYTES = 32 * 128;                  // 32 x 32 fp32 weight chunk, 128-byte swizzle
+constexpr int BAR_BYTES = 384;
 __host__ __device__ constexpr int smem_bytes(int kind) {
   return stages_for(kind) * STAGE_BYTES +
-         EPI_WARPS * ((chunked_out(kind) ? CH_BUFS * CH_BYTES : EPI_BYTES) + (mirrors(kind) ? STG_BYTES : 0)) + BAR_BYTES +
-         1024;   // + alignment slack
+         EPI_WARPS * ((apply_out(kind) ? 2 * WCH_BYTES : chunked_out(kind) ? CH_BUFS * CH_BYTES : EPI_BYTES) +
+                      (mirrors(kind) ? STG_BYTES : 0)) +
+         BAR_BYTES + 1024;   // + alignment slack
 }
 constexpr int ACC_COLS = 256;                        // one fp32 128x256 accumulator per CTA
 constexpr int TMEM_COLS = 2 * ACC_COLS;              // double-buffered
-static_assert(smem_bytes(0) <= 232448 && smem_bytes(1) <= 232448 && smem_bytes(2) <= 232448,
+static_assert(smem_bytes(0) <= 232448 && smem_bytes(1) <= 232448 && smem_bytes(2) <= 232448 &&
+                  smem_bytes(5) <= 232448,
               "shared memory per block");
 }  // namespace gemm_cfg
 
@@ -122,6 +129,18 @@ struct GemmProblem {
   int64_t out32_ld, out32_bs;
   int nblocks;
   float scale;               // GRAM32 / PRECOND: result = scale * sum
+  int apply_base;            // UPDATE_APPLY: first ApplyDesc of this problem's matrices
+};
+
+// Per matrix of a fused update + apply: the fp32 weight as a TMA tensor
+// (rows x cols, box 32 x 32, 128-byte swizzle), its step scalars and its
+// orientation (transposed: rows > cols, so the wide X' is W's transpose).
+struct alignas(64) ApplyDesc {
+  CUtensorMap w;
+  float lr_scale;            // lr * shape scale
+  float decay;               // 1 - lr * wd
+  int transposed;
+  int pad;
 };
 
 // A launch covers up to MAX_PROBLEMS problems of one product kind (the shape
@@ -138,6 +157,7 @@ struct GemmArgs {
   int* err;                  // device error flags
   const int* skip;           // non-null and set: do nothing (non-finite gradient)
   int reverse;               // walk the tile list from its end (see run_newton_schulz)
+  const ApplyDesc* apply;    // UPDATE_APPLY: per-matrix weights (device memory)
 };
 
 // Per problem: A operand rows (box 64 x 128), B operand (K-major box 64 x 128
@@ -212,14 +232,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* smem_epi = smem + STAGES * STAGE_BYTES;             // 1024-aligned slices
-  uint8_t* smem_stg = smem_epi + EPI_WARPS * (chunked_out(KIND) ? CH_BUFS * CH_BYTES : EPI_BYTES);
+  constexpr int SLICE = apply_out(KIND) ? 2 * WCH_BYTES : chunked_out(KIND) ? CH_BUFS * CH_BYTES : EPI_BYTES;
+  uint8_t* smem_stg = smem_epi + EPI_WARPS * SLICE;
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem_stg + (mirrors(KIND) ? EPI_WARPS * STG_BYTES : 0));
   uint64_t* empty_bar = full_bar + STAGES;
   uint64_t* tfull_bar = empty_bar + STAGES;     // accumulator ready   (leader MMA -> both epilogues)
   uint64_t* tempty_bar = tfull_bar + 2;         // accumulator drained (both epilogues -> leader MMA)
   uint64_t* drain_bar = tempty_bar + 2;
-  uint64_t* aux_bar = drain_bar + 1;            // one per epilogue warp
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(aux_bar + EPI_WARPS);
+  uint64_t* aux_bar = drain_bar + 1;            // two per epilogue warp (POLY uses the first)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(aux_bar + 2 * EPI_WARPS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -239,7 +260,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
       mbar_init(&tempty_bar[a], 2 * EPI_WARPS);
     }
     mbar_init(drain_bar, 1);
-    for (int w = 0; w < EPI_WARPS; ++w) mbar_init(&aux_bar[w], 1);
+    for (int w = 0; w < 2 * EPI_WARPS; ++w) mbar_init(&aux_bar[w], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -362,7 +383,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
     const int ew = warp - 2;
     const int q = warp & 3;                 // TMEM lane quarter this warp may read
     const int half = ew >> 2;               // 128-column half of the tile
-    uint8_t* slice = smem_epi + ew * (chunked_out(KIND) ? CH_BUFS * CH_BYTES : EPI_BYTES);
+    uint8_t* slice = smem_epi + ew * SLICE;
+    uint32_t wph = 0;                       // UPDATE_APPLY: phase bit per weight buffer (bits 0, 1)
+    uint32_t wpend = 0;                     // UPDATE_APPLY: weight loads in flight per buffer
     uint32_t nch = 0;                       // output chunks stored so far (buffer = nch & 1)
     uint8_t* stg = smem_stg + ew * STG_BYTES;
     const uint32_t tempty0 = map_to_cta(smem_u32(tempty_bar), 0);
@@ -389,6 +412,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
       const bool two_boxes = col0 + 64 < P.N;
       // the slice is free once the previous tile's TMA store has read it;
       // then fetch this tile's epilogue input into it
+      if constexpr (apply_out(KIND)) {
+        // weight chunks 0 and 1 of this tile into the two buffers, once the
+        // previous tile's stores have read them
+        if (lane == 0 && active) {
+          bulk_wait_group_read0();
+          const ApplyDesc& ad = args.apply[P.apply_base + bidx];
+          for (int c = 0; c < 2 && col0 + c * 32 < P.N; ++c) {
+            const int cb = col0 + c * 32;
+            mbar_arrive_expect_tx(&aux_bar[2 * ew + c], WCH_BYTES);
+            if (ad.transposed) tma_load_3d(slice + c * WCH_BYTES, &ad.w, &aux_bar[2 * ew + c], rbase, cb, 0);
+            else tma_load_3d(slice + c * WCH_BYTES, &ad.w, &aux_bar[2 * ew + c], cb, rbase, 0);
+            wpend |= 1u << c;
+          }
+        }
+      }
       if (lane == 0 && KIND == EPI_POLY) {
         bulk_wait_group_read0();
         if (active) {
@@ -452,6 +490,54 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
                   if (cbase + k < P.N) P.out32[zoff + static_cast<int64_t>(cbase + k) * P.out32_ld + r] = v[k];
               }
             }
+          } else if constexpr (apply_out(KIND)) {
+            const ApplyDesc& ad = args.apply[P.apply_base + bidx];
+            const int wb = c32 & 1;
+            uint8_t* wbuf = slice + wb * WCH_BYTES;
+            // lane 0 issued the load; all lanes wait on its barrier
+            const bool okw = mbar_wait(&aux_bar[2 * ew + wb], (wph >> wb) & 1u, args.err, abort_flag);
+            if (!__all_sync(0xffffffffu, okw)) break;
+            wph ^= 1u << wb;
+            wpend &= ~(1u << wb);
+            const float dec = ad.decay, lrs = ad.lr_scale;
+            if (!ad.transposed) {
+              // row `lane` of the chunk: 16-byte unit u at unit u ^ (lane % 8)
+#pragma unroll
+              for (int u = 0; u < 8; ++u) {
+                float4* pw = reinterpret_cast<float4*>(wbuf + lane * 128 + ((u ^ (lane & 7)) << 4));
+                float4 w = *pw;
+                w.x = w.x * dec - lrs * (alpha * __uint_as_float(raw[u * 4 + 0]));
+                w.y = w.y * dec - lrs * (alpha * __uint_as_float(raw[u * 4 + 1]));
+                w.z = w.z * dec - lrs * (alpha * __uint_as_float(raw[u * 4 + 2]));
+                w.w = w.w * dec - lrs * (alpha * __uint_as_float(raw[u * 4 + 3]));
+                *pw = w;
+              }
+            } else {
+              // W is X'^T: element k of this lane's row is W[cbase + k][rbase + lane],
+              // row k of the chunk, column `lane`
+#pragma unroll
+              for (int k = 0; k < 32; ++k) {
+                float* pw = reinterpret_cast<float*>(wbuf + k * 128 + ((((lane >> 2) ^ k) & 7) << 4) + (lane & 3) * 4);
+                *pw = *pw * dec - lrs * (alpha * __uint_as_float(raw[k]));
+              }
+            }
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              if (ad.transposed) tma_store_3d(&ad.w, wbuf, rbase, cbase, 0);
+              else tma_store_3d(&ad.w, wbuf, cbase, rbase, 0);
+              bulk_commit_group();
+              // chunk c32 + 2 into this buffer once the store has read it
+              const int cn = cbase + 64;
+              if (c32 + 2 < 4 && cn < P.N) {
+                bulk_wait_group_read0();
+                mbar_arrive_expect_tx(&aux_bar[2 * ew + wb], WCH_BYTES);
+                if (ad.transposed) tma_load_3d(wbuf, &ad.w, &aux_bar[2 * ew + wb], rbase, cn, 0);
+                else tma_load_3d(wbuf, &ad.w, &aux_bar[2 * ew + wb], cn, rbase, 0);
+                wpend |= 1u << wb;
+              }
+            }
+            wpend = __shfl_sync(0xffffffffu, wpend, 0);
           } else if constexpr (chunked_out(KIND)) {
             float v[32];
 #pragma unroll
@@ -558,6 +644,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
         volatile int no_abort = 0;
         mbar_wait(&aux_bar[ew], aux_phase, args.err, &no_abort);   // let the copy land
       }
+      for (int b = 0; b < 2; ++b)
+        if (wpend & (1u << b)) {
+          volatile int no_abort = 0;
+          mbar_wait(&aux_bar[2 * ew + b], (wph >> b) & 1u, args.err, &no_abort);
+        }
       bulk_wait_group0();
     }
     __syncwarp();

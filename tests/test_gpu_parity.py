@@ -123,6 +123,47 @@ def _step_case(ctx, mx, shapes, steps, grad_dtype, hp_over=None, seed=0, grad_st
     return wt, bt
 
 
+def test_step_fused_apply_vs_oracle_and_unfused(ctx, mx):
+    """Without update_out the last Newton-Schulz product applies the weight
+    step in its epilogue (O stays in fp32 and never reaches memory).  Three
+    steps on square, wide, tall and ragged shapes (widths a multiple of 4):
+    momentum matches the oracle, the applied update (W_prev (1 - lr wd) -
+    W_new) / (lr scale) matches the oracle's Newton-Schulz output, and on the
+    first step it matches the unfused path's update_out up to bf16 rounding.
+    A set holding a width that is not a multiple of 4 takes the unfused path."""
+    hp = mx.default_hparams()
+    decay = 1 - hp.lr * hp.weight_decay
+    for shapes in ([(256, 256), (768, 3072), (3072, 768), (1000, 336), (520, 1028), (72, 8)],
+                   [(130, 34), (96, 200)]):
+        w = [wl.np_normal(s, 0.02, seed=21, index=i, role=wl.ROLE_WEIGHT) for i, s in enumerate(shapes)]
+        wa = [dev(x) for x in w]
+        wb = [dev(x) for x in w]
+        ba = [torch.zeros(s, device="cuda") for s in shapes]
+        bb = [torch.zeros(s, device="cuda") for s in shapes]
+        ob = [torch.empty(s, device="cuda") for s in shapes]
+        buf = [np.zeros(s) for s in shapes]
+        for step in range(3):
+            g = [wl.bf16_round_np(wl.np_normal(s, 1e-3, seed=21, step=step, index=i)) for i, s in enumerate(shapes)]
+            gt = [dev(x, torch.bfloat16) for x in g]
+            prev_a = [to_np(t) for t in wa]
+            ctx.step([dict(weights=[wa[i]], grads=[gt[i]], momentum=[ba[i]]) for i in range(len(shapes))], hp)
+            if step == 0:
+                ctx.step([dict(weights=[wb[i]], grads=[gt[i]], momentum=[bb[i]], update_out=[ob[i]])
+                          for i in range(len(shapes))], hp)
+            torch.cuda.synchronize()
+            ctx.check_device()
+            for i, s in enumerate(shapes):
+                nb, u = oracle.nesterov_momentum(g[i], buf[i])
+                assert rel_fro(to_np(ba[i]), nb) < EW_TOL, (s, step)
+                buf[i] = nb
+                scale = oracle.shape_scale(s[0], s[1])
+                upd = (prev_a[i] * decay - to_np(wa[i])) / (hp.lr * scale)
+                assert rel_fro(upd, oracle.newton_schulz(u, 5)) < ns_tol(s), (s, step)
+                if step == 0:
+                    assert rel_fro(upd, to_np(ob[i])) < 5e-3, s
+                    assert torch.equal(ba[i], bb[i]), s
+
+
 def test_step_single_256_f32(ctx, mx):
     """One 256x256 fp32 gradient N(0,1), weights N(0,0.02), zero momentum,
     one step with the defaults."""
