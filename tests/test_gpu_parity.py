@@ -79,6 +79,20 @@ def test_orthogonalize_ns_steps(ctx, mx, steps):
     assert rel_fro(to_np(out), oracle.newton_schulz(x, steps)) < NS_TOL
 
 
+@pytest.mark.parametrize("coeffs", [(1.5, -0.5, 0.0), (2.0, -1.5, 0.5)], ids=["cubic_c0", "quintic_alt"])
+def test_orthogonalize_custom_coefficients(ctx, mx, coeffs):
+    """Other coefficient sets through the ABI, including c = 0 (the cubic
+    iteration), against the oracle with the same coefficients."""
+    a, b, c = coeffs
+    hp = mx.default_hparams(ns_a=a, ns_b=b, ns_c=c, ns_steps=8)
+    x = wl.np_normal((256, 384), 1.0, seed=31)
+    out = torch.empty((256, 384), device="cuda")
+    ctx.orthogonalize([dev(x, torch.bfloat16)], [out], hp)
+    torch.cuda.synchronize()
+    want = oracle.newton_schulz(wl.bf16_round_np(x), 8, a=a, b=b, c=c)
+    assert rel_fro(to_np(out), want) < NS_TOL
+
+
 def _step_case(ctx, mx, shapes, steps, grad_dtype, hp_over=None, seed=0, grad_std=1e-3):
     """Run `steps` Muon steps on GPU and oracle side by side; check momentum
     and staged apply every step, and the update against the oracle's."""
