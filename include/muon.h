@@ -197,7 +197,18 @@ MUON_API muon_status muon_set_workspace(muon_ctx* ctx, void* ptr, size_t bytes);
 /* One Muon step over ngroups groups: for every matrix, Nesterov momentum,
  * Frobenius normalisation, hp->ns_steps quintic Newton-Schulz iterations in
  * bf16 with fp32 accumulation (on the transpose when rows > cols), then
- * W <- W (1 - lr wd) - lr scale O. */
+ * W <- W (1 - lr wd) - lr scale O.
+ *
+ * When no group asks for update_out and every width is a multiple of 4, the
+ * weight step is applied inside the last Newton-Schulz product, with O in
+ * fp32 (never rounded to bf16 or written out); otherwise O is the bf16
+ * result of the last product, written to update_out when requested and
+ * applied by a separate pass.  Both agree to bf16 rounding of O.
+ *
+ * The kernels are enqueued on `stream` (NULL: the legacy default stream)
+ * with programmatic stream serialization: each may be scheduled while its
+ * predecessor drains and waits for it (griddepcontrol.wait) before touching
+ * global memory, so stream order holds as for ordinary launches. */
 MUON_API muon_status muon_step(muon_ctx* ctx, const muon_group* groups, int32_t ngroups,
                       const muon_hparams* hp, void* stream);
 
