@@ -75,7 +75,12 @@ constexpr int BK = 64;
 // Pipeline depth per product.  GRAM and UPDATE stage their output in 2 KB
 // chunks (below) and spend the space saved on a fifth / sixth stage; the
 // update also has no mirrored blocks.
-__host__ __device__ constexpr int stages_for(int kind) { return kind == 0 ? 5 : kind == 1 ? 4 : kind == 2 ? 6 : 5; }
+__host__ __device__ constexpr int stages_for(int kind) {
+  return kind == 0 ? 5 : kind == 1 ? 4 : kind == 2 ? 6 : kind == 5 ? 5 : 7;
+}
+// GRAM32 and PRECOND write fp32 straight from registers: no epilogue buffers,
+// so their pipelines take the shared memory.
+__host__ __device__ constexpr bool fp32_out(int kind) { return kind == 3 || kind == 4; }
 // The last update of an optimizer step may apply W <- W (1 - lr wd) - lr
 // scale O in its epilogue (EPI_UPDATE_APPLY): W moves through two 4 KB
 // 32x32 fp32 chunk buffers per warp by TMA, and O never reaches memory.
@@ -101,14 +106,17 @@ constexpr int WCH_BYTES = 32 * 128;                  // 32 x 32 fp32 weight chun
 constexpr int BAR_BYTES = 384;
 __host__ __device__ constexpr int smem_bytes(int kind) {
   return stages_for(kind) * STAGE_BYTES +
-         EPI_WARPS * ((apply_out(kind) ? 2 * WCH_BYTES : chunked_out(kind) ? CH_BUFS * CH_BYTES : EPI_BYTES) +
+         EPI_WARPS * ((apply_out(kind)     ? 2 * WCH_BYTES
+                       : chunked_out(kind) ? CH_BUFS * CH_BYTES
+                       : fp32_out(kind)    ? 0
+                                           : EPI_BYTES) +
                       (mirrors(kind) ? STG_BYTES : 0)) +
          BAR_BYTES + 1024;   // + alignment slack
 }
 constexpr int ACC_COLS = 256;                        // one fp32 128x256 accumulator per CTA
 constexpr int TMEM_COLS = 2 * ACC_COLS;              // double-buffered
 static_assert(smem_bytes(0) <= 232448 && smem_bytes(1) <= 232448 && smem_bytes(2) <= 232448 &&
-                  smem_bytes(5) <= 232448,
+                  smem_bytes(3) <= 232448 && smem_bytes(4) <= 232448 && smem_bytes(5) <= 232448,
               "shared memory per block");
 }  // namespace gemm_cfg
 
@@ -232,7 +240,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* smem_epi = smem + STAGES * STAGE_BYTES;             // 1024-aligned slices
-  constexpr int SLICE = apply_out(KIND) ? 2 * WCH_BYTES : chunked_out(KIND) ? CH_BUFS * CH_BYTES : EPI_BYTES;
+  constexpr int SLICE = apply_out(KIND) ? 2 * WCH_BYTES : chunked_out(KIND) ? CH_BUFS * CH_BYTES
+                        : fp32_out(KIND)  ? 0 : EPI_BYTES;
   uint8_t* smem_stg = smem_epi + EPI_WARPS * SLICE;
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem_stg + (mirrors(KIND) ? EPI_WARPS * STG_BYTES : 0));
   uint64_t* empty_bar = full_bar + STAGES;

@@ -283,6 +283,32 @@ def test_workspace_cap_and_caller_workspace(ctx, mx):
         assert torch.equal(a, b)
 
 
+def test_fused_step_chunked_matches_unchunked(ctx, mx):
+    """The fused weight step under a bounded workspace (several chunks, each
+    with its own descriptor table and last-product launch) leaves the same
+    weights and momentum, bit for bit, as one unbounded call."""
+    shapes = [(256, 512)] * 6 + [(512, 256)] * 3 + [(128, 128)] * 4
+    w0 = [wl.np_normal(s, 0.02, seed=11, index=i, role=wl.ROLE_WEIGHT) for i, s in enumerate(shapes)]
+    g = [dev(wl.bf16_round_np(wl.np_normal(s, 1e-3, seed=11, index=i)), torch.bfloat16)
+         for i, s in enumerate(shapes)]
+    per = 2 * 256 * 512 * 2 + 2 * 256 * 256 * 2 + 4096 + 256 * 512 * 4
+    small = mx.MuonContext(0, workspace_bytes=3 * per)
+    results = []
+    for c in (ctx, small):
+        w = [dev(x) for x in w0]
+        b = [torch.zeros(s, device="cuda") for s in shapes]
+        for _ in range(2):
+            c.step([dict(weights=[w[i]], grads=[g[i]], momentum=[b[i]]) for i in range(len(shapes))])
+        torch.cuda.synchronize()
+        results.append((w, b))
+    small.close()
+    for (wa, ba), (wb, bb) in [(results[0], results[1])]:
+        for x, y in zip(wa, wb):
+            assert torch.equal(x, y)
+        for x, y in zip(ba, bb):
+            assert torch.equal(x, y)
+
+
 def test_adamw_vs_oracle(ctx, mx):
     sizes = [1, 3, 768, 1000, 50257 * 8 + 3, 12345]
     ps = [wl.np_normal((n,), 0.02, seed=11, index=i, role=wl.ROLE_WEIGHT) for i, n in enumerate(sizes)]
