@@ -44,7 +44,10 @@ def _band_ok(o, rows, cols):
 
 def test_llama3_8b_step_full_size(mx):
     """One Llama-3-8B-shaped step (224 matrices, bf16 grads N(0,1e-3), fp32
-    weights N(0,0.02), zero momentum), run in three calls of whole layers."""
+    weights N(0,0.02), zero momentum), run in three calls of whole layers.
+    Every matrix: momentum and staged apply on 4096 sampled elements,
+    finiteness, the singular-value band; the seven matrices of layers 0 and
+    31: the whole Newton-Schulz output against the fp64 oracle."""
     dev = torch.device("cuda")
     mats = wl.llama3_8b_mats()
     hp = mx.default_hparams()
@@ -60,7 +63,9 @@ def test_llama3_8b_step_full_size(mx):
                 O[i] = torch.empty((m.rows, m.cols), device=dev)
                 idx = _sample_idx(m.rows * m.cols, 4096, seed=i)
                 samp[i] = (idx, W[i].view(-1)[idx].double().cpu().numpy(), G[i].view(-1)[idx].double().cpu().numpy())
-            full = {i: (W[i].double().cpu().numpy(), G[i].double().cpu().numpy()) for i in ids if i < 7}
+            # every matrix of the first and the last layer against the full oracle
+            full = {i: (W[i].double().cpu().numpy(), G[i].double().cpu().numpy()) for i in ids
+                    if i < 7 or i >= len(mats) - 7}
             groups = {}
             for i in ids:
                 groups.setdefault((mats[i].rows, mats[i].cols), []).append(i)
