@@ -10,7 +10,10 @@
 //   apply_kernel      W <- W (1 - lr wd) - lr scale O, O read from the final
 //                     wide bf16 X (transposed back through shared memory for
 //                     tall matrices); optionally O to an fp32 output.
-//                     10 B/element.
+//                     10 B/element.  Used when the weight step cannot be
+//                     fused into the last Newton-Schulz product (an update_out
+//                     was requested, a width is not a multiple of 4, or no
+//                     iteration runs) and for the Newton-Schulz-only export.
 //   finite_kernel     read-only NaN/Inf scan of the gradients.
 //   adamw_kernel      fused AdamW over a list of tensors, bias-corrected.
 //

@@ -8,12 +8,16 @@
 //   GRAM    A  = alpha * X X^T           M = N = m, K = n   symmetric
 //   POLY    B' = b A + c A A + a I       M = N = K = m      symmetric
 //   UPDATE  X' = alpha * B' X            M = m, N = n, K = m
+//   UPDATE_APPLY (the last update of an optimizer step)
+//           W <- W (1 - lr wd) - lr scale * alpha * B' X, with W read and
+//           written in 32x32 fp32 chunks by TMA; X' is not stored
 //
 // a X + B X is computed as (a I + B) X: the same product, but the update
 // needs no second read of X.  Rounding a I + B to bf16 instead of B costs no
-// accuracy on matrices of 16 or more: late in the iteration B's diagonal is near -a + 0.7, so B' has
-// the smaller entries (bf16 emulation, 16x16 ... 1024x4096: lower error than
-// rounding B; only a 5x3 matrix came out higher, 3.0e-2 against 2.4e-2).
+// accuracy on matrices of 16 or more: late in the iteration B's diagonal is
+// near -a + 0.7, so B' has the smaller entries (bf16 emulation, 16x16 ...
+// 1024x4096: lower error than rounding B; only a 5x3 matrix came out higher,
+// 3.0e-2 against 2.4e-2).
 //
 // The symmetric products compute only the tiles that touch the upper
 // triangle and write each strictly-upper 128x128 block twice (direct and
