@@ -83,11 +83,14 @@ def step_work(w, aux, ns_steps=5):
             nb = w.precond[m.name][1]
             d = m.cols // nb
             pre += 2 * m.rows * m.cols * d
-    refresh = 0
+    refresh_tc = refresh_alu = 0
     for _, tokens, width in w.acts:
         nb = 4 if width > 768 else 1
         d = width // nb
-        refresh += nb * (2 * tokens * d * d + d ** 3 // 3 * 2 + 2 * d ** 3)
+        # second moment on the tensor cores; Cholesky (d^3/3 FMA), L^-1 (d^3/6)
+        # and L^-T L^-1 (d^3/6) on the fp32 ALUs
+        refresh_tc += nb * 2 * tokens * d * d
+        refresh_alu += nb * 2 * (d ** 3 // 3 + d ** 3 // 3)
     for m in w.mats:
         a, b = min(m.rows, m.cols), max(m.rows, m.cols)
         gram += 2 * a * a * b * ns_steps
@@ -96,8 +99,13 @@ def step_work(w, aux, ns_steps=5):
         elems += m.rows * m.cols
     gbytes = 2 if w.grad_dtype == "bf16" else 4
     aux_el = sum(n for _, n in aux)
+    per_iter = upd // max(1, ns_steps)
     return {
         "gram": ("flop", gram), "poly": ("flop", poly), "update": ("flop", upd),
+        # the last update with the weight step fused: one iteration's FLOPs
+        # and the fp32 weights read and written (8 B/element); the update
+        # class then holds the other ns_steps - 1 iterations
+        "update_apply": ("mixed", (per_iter, elems * 8)),
         # momentum: read grad + buf, write buf + bf16 U
         "momentum": ("byte", elems * (gbytes + 4 + 4 + 2)),
         # apply: read bf16 O + W, write W
@@ -106,7 +114,7 @@ def step_work(w, aux, ns_steps=5):
         "adamw": ("byte", aux_el * (2 + 3 * 8)),
         # tensor cores: G [S_hi; S_lo] executes twice the algorithmic 2 rows cols d
         "precondition": ("flop", pre),
-        "newton_refresh": ("fflop", refresh / max(1, w.refresh_every)),
+        "newton_refresh": ("seq", (refresh_tc / max(1, w.refresh_every), refresh_alu / max(1, w.refresh_every))),
     }, elems, aux_el
 
 
@@ -269,7 +277,7 @@ def run_reference(args, w, aux):
 # the CUDA path
 # ---------------------------------------------------------------------------
 
-SOURCE_GROUPS = {"gram": "ns_gemm", "poly": "ns_gemm", "update": "ns_gemm",
+SOURCE_GROUPS = {"gram": "ns_gemm", "poly": "ns_gemm", "update": "ns_gemm", "update_apply": "ns_gemm",
                  "momentum": "elementwise", "apply": "elementwise", "adamw": "elementwise"}
 
 
@@ -483,6 +491,8 @@ def main():
             if nl:
                 kt[kind] = (kt[kind][0] + t_ms, kt[kind][1] + nl)
     work, elems, aux_el = step_work(w, aux, hp.ns_steps)
+    if kt.get("update_apply", (0, 0))[1] > 0:
+        work["update"] = ("flop", work["update"][1] - work["update_apply"][1][0])
     pk = peaks()
     kernels = {}
     for kind, (t_ms, nl) in kt.items():
@@ -499,6 +509,25 @@ def main():
             ach = tot / (t_ms * 1e-3) / 1e12
             kernels[kind] = {"ms_per_step": t_ms / args.steps, "launches": nl, "achieved": ach,
                              "unit": "TFLOP/s", "bound": "alu", "frac": ach / FP32_PEAK_TFLOPS}
+        elif unit == "seq":
+            # tensor-core FLOPs then fp32 ALU FLOPs in separate launches: the
+            # roofline time is the sum of the two lower bounds
+            tc, alu = per_step[0] * args.steps, per_step[1] * args.steps
+            t_s = t_ms * 1e-3
+            bound_s = tc / (pk["bf16"] * 1e12) + alu / (FP32_PEAK_TFLOPS * 1e12)
+            kernels[kind] = {"ms_per_step": t_ms / args.steps, "launches": nl,
+                             "achieved": (tc + alu) / t_s / 1e12, "unit": "TFLOP/s",
+                             "frac": bound_s / t_s, "bound": "tensor+alu"}
+        elif unit == "mixed":
+            # tensor-core FLOPs and HBM bytes in one launch: the roofline time
+            # is the larger of the two lower bounds
+            fl, by = per_step[0] * args.steps, per_step[1] * args.steps
+            t_s = t_ms * 1e-3
+            bound_s = max(fl / (pk["bf16"] * 1e12), by / (pk["hbm"] * 1e9))
+            kernels[kind] = {"ms_per_step": t_ms / args.steps, "launches": nl,
+                             "achieved": fl / t_s / 1e12, "unit": "TFLOP/s",
+                             "achieved_gbs": by / t_s / 1e9, "frac": bound_s / t_s,
+                             "bound": "hbm" if by / (pk["hbm"] * 1e9) > fl / (pk["bf16"] * 1e12) else "tensor"}
         else:
             ach = tot / (t_ms * 1e-3) / 1e9
             kernels[kind] = {"ms_per_step": t_ms / args.steps, "launches": nl, "achieved": ach,
@@ -509,14 +538,20 @@ def main():
     dom = max(kernels, key=lambda k: kernels[k]["ms_per_step"])
     d = kernels[dom]
     traffic = read_traffic(dom, args.workload)
-    roofline = {"bound": "tensor" if d["unit"] == "TFLOP/s" else "hbm", "kernel": dom,
-                "achieved": d["achieved"], "peak": pk["bf16"] if d["unit"] == "TFLOP/s" else pk["hbm"],
+    bound = d.get("bound", "tensor" if d["unit"] == "TFLOP/s" else "hbm")
+    peak = {"alu": FP32_PEAK_TFLOPS, "hbm": pk["hbm"]}.get(bound, pk["bf16"])
+    roofline = {"bound": bound, "kernel": dom,
+                "achieved": d["achieved"], "peak": peak,
                 "unit": d["unit"], "frac": d["frac"],
                 "traffic": (traffic / d["launches"] * args.steps) if traffic is not None else None,
-                "peak_source": pk["source"] + (" burst bf16 (torch.matmul 8192^3)" if d["unit"] == "TFLOP/s"
-                                               else " HBM copy")}
-    ns_flops = work["gram"][1] + work["poly"][1] + work["update"][1]
-    ns_ms = sum(kernels.get(k, {"ms_per_step": 0})["ms_per_step"] for k in ("gram", "poly", "update"))
+                "peak_source": {"hbm": pk["source"] + " HBM copy",
+                                "alu": "derived: 148 SMs x 128 fp32 lanes x 2 FLOP x 1.965 GHz",
+                                "tensor+alu": pk["source"] + " burst bf16 for the tensor-core part, derived fp32 "
+                                              "peak for the ALU part; frac = summed lower bounds / time"
+                                }.get(bound, pk["source"] + " burst bf16 (torch.matmul 8192^3)")}
+    ns_flops = work["gram"][1] + work["poly"][1] + work["update"][1] + \
+        (work["update_apply"][1][0] if "update_apply" in kernels else 0)
+    ns_ms = sum(kernels.get(k, {"ms_per_step": 0})["ms_per_step"] for k in ("gram", "poly", "update", "update_apply"))
     ew_kinds = [k for k in ("momentum", "apply", "adamw") if k in kernels]
     ew_bytes = sum(work[k][1] for k in ew_kinds)
     ew_ms = sum(kernels[k]["ms_per_step"] for k in ew_kinds)

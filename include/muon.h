@@ -259,7 +259,8 @@ typedef enum {
   MUON_K_NEWTON_REFRESH = 6,
   MUON_K_PRECONDITION = 7,
   MUON_K_OTHER = 8,      /* finite scan                                    */
-  MUON_K_COUNT = 9
+  MUON_K_UPDATE_APPLY = 9, /* last update with the weight step in its epilogue */
+  MUON_K_COUNT = 10
 } muon_kernel_kind;
 
 typedef struct {

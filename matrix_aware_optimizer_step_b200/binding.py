@@ -38,7 +38,7 @@ EXPORTED = [
 ]
 
 KERNEL_KINDS = ["momentum", "gram", "poly", "update", "apply", "adamw", "newton_refresh",
-                "precondition", "other"]
+                "precondition", "other", "update_apply"]
 
 
 class MuonError(RuntimeError):
@@ -88,7 +88,7 @@ class ActDesc(ctypes.Structure):
 
 
 class KernelTimes(ctypes.Structure):
-    _fields_ = [("ms", ctypes.c_double * 9), ("launches", ctypes.c_uint64 * 9)]
+    _fields_ = [("ms", ctypes.c_double * len(KERNEL_KINDS)), ("launches", ctypes.c_uint64 * len(KERNEL_KINDS))]
 
 
 _lib = None

@@ -563,7 +563,7 @@ muon_status run_newton_schulz(muon_ctx* ctx, uint8_t* ws, const Run* runs, int n
           ProfScope ps(ctx, MUON_K_POLY, st);
           CUDA_TRY(ctx, (launch_gemm<EPI_POLY, false>(ctx, maps, g, st)));
         } else if (fuse) {
-          ProfScope ps(ctx, MUON_K_UPDATE, st);
+          ProfScope ps(ctx, MUON_K_UPDATE_APPLY, st);
           CUDA_TRY(ctx, (launch_gemm<EPI_UPDATE_APPLY, true>(ctx, maps, g, st)));
         } else {
           ProfScope ps(ctx, MUON_K_UPDATE, st);
