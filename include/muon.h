@@ -226,6 +226,25 @@ MUON_API muon_status muon_adamw_step(muon_ctx* ctx, const muon_adamw_tensor* ten
 MUON_API muon_status muon_newton_refresh(muon_ctx* ctx, const muon_act_desc* acts, int32_t n,
                                 float damping, void* stream);
 
+/* Newton-Muon right-preconditioning on its own ("What Is Newton-Muon?",
+ * the update rule with the gradient replaced by G S^-1, block-diagonal over
+ * precond_blocks column blocks): for every matrix of every group,
+ *   update_out[i] (fp32 rows x cols) = grads[i] [S_1^-1, ..., S_nb^-1]
+ * with S_b^-1 = precond[i] + b d d (fp32 d x d, row-major, d = cols / nb).
+ * Each group needs grads (MUON_BF16), precond, precond_blocks and
+ * update_out; weights and momentum are ignored and may be NULL.  muon_step
+ * does the same product internally when a group carries precond; this call
+ * exposes it for callers that precondition and orthogonalise in separate
+ * stages.  Block widths that are multiples of 64 run on the tensor cores
+ * (S^-1 split into bf16 hi + lo, G in bf16, fp32 accumulation); others on an
+ * fp32 tile kernel.  Tensor-core matrices stage a bf16 copy of G and the
+ * S^-1 hi/lo stacks in workspace (rows x round_up(cols, 8) x 2 +
+ * nb x 2 d^2 x 2 bytes each, 256-byte aligned), in batches that fit a
+ * capped or caller-owned workspace; MUON_ERR_WORKSPACE if one matrix does
+ * not fit.  Argument errors are reported before any launch. */
+MUON_API muon_status muon_newton_precondition(muon_ctx* ctx, const muon_group* groups, int32_t ngroups,
+                                     void* stream);
+
 /* Synchronise the context's last stream and report device-side flags:
  * MUON_ERR_TIMEOUT if a bounded wait gave up since the last check (the flag
  * is cleared), MUON_ERR_CUDA on an asynchronous CUDA error, else MUON_OK. */

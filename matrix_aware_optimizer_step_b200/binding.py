@@ -33,6 +33,7 @@ EXPORTED = [
     "muon_default_hparams", "muon_default_adamw_hparams", "muon_init", "muon_destroy",
     "muon_last_error", "muon_status_string", "muon_query_workspace", "muon_set_workspace",
     "muon_step", "muon_orthogonalize", "muon_adamw_step", "muon_newton_refresh",
+    "muon_newton_precondition",
     "muon_check_device", "muon_launch_count", "muon_profile_enable", "muon_profile_read",
     "muon_orthogonalize_noalloc", "muon_partition",
 ]
@@ -119,6 +120,7 @@ def load_library() -> ctypes.CDLL:
         "muon_adamw_step": (st, [vp, ctypes.POINTER(AdamwTensor), i32, ctypes.POINTER(AdamwHparams),
                                  i64, vp]),
         "muon_newton_refresh": (st, [vp, ctypes.POINTER(ActDesc), i32, ctypes.c_float, vp]),
+        "muon_newton_precondition": (st, [vp, ctypes.POINTER(Group), i32, vp]),
         "muon_check_device": (st, [vp]),
         "muon_launch_count": (ctypes.c_uint64, [vp]),
         "muon_profile_enable": (st, [vp, ctypes.c_int]),
@@ -372,6 +374,19 @@ class MuonContext:
             arr[i].s_inv = s_invs[i].data_ptr()
         self._check(self._lib.muon_newton_refresh(self._ctx, arr, n, float(damping),
                                                   _stream_ptr(stream)), "muon_newton_refresh")
+
+    def newton_precondition(self, grads: Sequence, s_invs: Sequence, nblocks: int, outputs: Sequence,
+                            stream=None):
+        """outputs[i] (fp32) = grads[i] (bf16 rows x cols) right-multiplied
+        block-diagonally by s_invs[i] (fp32, nblocks x d x d, d = cols /
+        nblocks).  All grads share one shape."""
+        grads = list(grads)
+        if not grads:
+            return
+        arr, keep = self.make_groups([{"grads": grads, "update_out": list(outputs),
+                                       "precond": list(s_invs), "precond_blocks": int(nblocks)}])
+        self._check(self._lib.muon_newton_precondition(self._ctx, arr, 1, _stream_ptr(stream)),
+                    "muon_newton_precondition")
 
     def check_device(self):
         self._check(self._lib.muon_check_device(self._ctx), "muon_check_device")

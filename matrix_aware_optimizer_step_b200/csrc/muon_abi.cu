@@ -626,6 +626,110 @@ muon_status run_precondition(muon_ctx* ctx, const std::vector<PreProblem>& probs
   return MUON_OK;
 }
 
+// Newton-Muon preconditioning on its own: update_out[i] = G_i S^-1 in fp32.
+// Matrices whose block width is a multiple of 64 go through the tensor-core
+// engine (bf16 gradient copy and S^-1 hi/lo stacks staged in workspace, in
+// batches that fit it); the rest through the plain fp32 tile kernel, which
+// writes the caller's buffers directly.
+muon_status run_precondition_items(muon_ctx* ctx, const std::vector<Item>& items, cudaStream_t st) {
+  if (items.empty()) return MUON_OK;
+  const size_t limit = ws_limit(ctx);
+  std::vector<PrepDesc> prep;
+  std::vector<PreProblem> probs;
+  std::vector<int> batch_begin;             // first prep (= problem) index of each batch
+  std::vector<PrecondDesc> pdescs;
+  int64_t ptiles = 0;
+  size_t cur = 0, need = 0;
+  for (const Item& it : items) {
+    if (tc_precond_ok(it)) {
+      const size_t gb = round_up(gc_bytes(it), kAlign), sb = round_up(sst_bytes(it), kAlign);
+      if (limit != 0 && gb + sb > limit)
+        return fail(ctx, MUON_ERR_WORKSPACE, "one matrix needs %zu bytes of workspace, %zu available", gb + sb,
+                    limit);
+      if (batch_begin.empty() || (limit != 0 && cur + gb + sb > limit)) {
+        batch_begin.push_back(int(prep.size()));
+        cur = 0;
+      }
+      // workspace offsets for now; rebased once the workspace is known
+      PrepDesc pd{};
+      pd.g = static_cast<const __nv_bfloat16*>(it.grad);
+      pd.gc = reinterpret_cast<__nv_bfloat16*>(cur);
+      pd.s_inv = it.precond;
+      pd.sst = reinterpret_cast<__nv_bfloat16*>(cur + gb);
+      pd.rows = it.rows;
+      pd.cols = it.cols;
+      pd.ldc = round_up(it.cols, 8);
+      pd.nb = it.precond_blocks;
+      pd.d = int(it.cols / it.precond_blocks);
+      prep.push_back(pd);
+      PreProblem q{};
+      q.rows = it.rows; q.cols = it.cols; q.nb = pd.nb; q.d = pd.d; q.count = 1; q.last = 0;
+      q.ldc = pd.ldc; q.pg = it.update_out; q.pg_stride = it.rows * it.cols;
+      probs.push_back(q);
+      cur += gb + sb;
+      need = std::max(need, cur);
+    } else {
+      PrecondDesc p{};
+      p.grad = static_cast<const __nv_bfloat16*>(it.grad);
+      p.s_inv = it.precond;
+      p.out = it.update_out;
+      p.rows = it.rows;
+      p.cols = it.cols;
+      p.d = it.cols / it.precond_blocks;
+      p.tiles_r = int(cdiv(it.rows, PRE_BM));
+      p.tiles_c = int(cdiv(p.d, PRE_BN));
+      p.tile_start = ptiles;
+      ptiles += int64_t(p.tiles_r) * p.tiles_c * it.precond_blocks;
+      pdescs.push_back(p);
+    }
+  }
+  if (ptiles > INT32_MAX) return fail(ctx, MUON_ERR_UNSUPPORTED, "too many precondition tiles in one launch");
+  uint8_t* ws = nullptr;
+  if (need > 0) {
+    void* wsv = nullptr;
+    muon_status s = ensure_workspace(ctx, need, &wsv);
+    if (s != MUON_OK) return s;
+    ws = static_cast<uint8_t*>(wsv);
+  }
+  for (size_t i = 0; i < prep.size(); ++i) {
+    prep[i].gc = reinterpret_cast<__nv_bfloat16*>(ws + reinterpret_cast<uintptr_t>(prep[i].gc));
+    prep[i].sst = reinterpret_cast<__nv_bfloat16*>(ws + reinterpret_cast<uintptr_t>(prep[i].sst));
+    probs[i].gc = prep[i].gc;
+    probs[i].sst = prep[i].sst;
+  }
+  const size_t prep_bytes = round_up(prep.size() * sizeof(PrepDesc), kAlign);
+  std::vector<uint8_t> table(prep_bytes + pdescs.size() * sizeof(PrecondDesc));
+  if (!prep.empty()) std::memcpy(table.data(), prep.data(), prep.size() * sizeof(PrepDesc));
+  if (!pdescs.empty()) std::memcpy(table.data() + prep_bytes, pdescs.data(), pdescs.size() * sizeof(PrecondDesc));
+  void* dtab = nullptr;
+  muon_status s = upload_table(ctx, table.data(), table.size(), st, &dtab);
+  if (s != MUON_OK) return s;
+  const PrepDesc* dprep = static_cast<const PrepDesc*>(dtab);
+  const PrecondDesc* dpdesc = reinterpret_cast<const PrecondDesc*>(static_cast<uint8_t*>(dtab) + prep_bytes);
+  ProfScope ps(ctx, MUON_K_PRECONDITION, st);
+  for (size_t b = 0; b < batch_begin.size(); ++b) {
+    const int b0 = batch_begin[b];
+    const int b1 = b + 1 < batch_begin.size() ? batch_begin[b + 1] : int(prep.size());
+    int64_t most = 0;
+    for (int k = b0; k < b1; ++k)
+      most = std::max<int64_t>(most, std::max<int64_t>(prep[k].rows * prep[k].cols,
+                                                       int64_t(prep[k].nb) * prep[k].d * prep[k].d));
+    const dim3 grid(unsigned(std::max<int64_t>(1, std::min<int64_t>(cdiv(most, 256 * 8), 512))), unsigned(b1 - b0));
+    launch_pdl(precond_prep_kernel, grid, dim3(256), size_t(0), st, dprep + b0);
+    ctx->launches++;
+    CUDA_TRY(ctx, cudaGetLastError());
+    s = run_precondition(ctx, std::vector<PreProblem>(probs.begin() + b0, probs.begin() + b1), nullptr, st);
+    if (s != MUON_OK) return s;
+  }
+  if (!pdescs.empty()) {
+    launch_pdl(precond_kernel, dim3(unsigned(ptiles)), dim3(PRE_THREADS), size_t(0), st, dpdesc,
+               int(pdescs.size()), static_cast<const int*>(nullptr));
+    ctx->launches++;
+    CUDA_TRY(ctx, cudaGetLastError());
+  }
+  return MUON_OK;
+}
+
 muon_status check_hparams(muon_ctx* ctx, const muon_hparams* hp) {
   if (!hp) return fail(ctx, MUON_ERR_INVALID_ARG, "hparams is NULL");
   if (hp->ns_steps < 0 || hp->ns_steps > 100)
@@ -1162,6 +1266,25 @@ muon_status muon_orthogonalize(muon_ctx* ctx, const muon_ns_group* groups, int32
   ctx->last_stream = st;
   CUDA_TRY(ctx, cudaGetLastError());
   return run_items(ctx, items, hp, 1, st);
+}
+
+muon_status muon_newton_precondition(muon_ctx* ctx, const muon_group* groups, int32_t ngroups, void* stream) {
+  if (!ctx) return MUON_ERR_INVALID_ARG;
+  if (ngroups < 0 || (ngroups > 0 && !groups)) return fail(ctx, MUON_ERR_INVALID_ARG, "bad groups");
+  for (int i = 0; i < ngroups; ++i) {
+    if (groups[i].count <= 0) continue;
+    if (!groups[i].precond) return fail(ctx, MUON_ERR_INVALID_ARG, "group %d: precond is NULL", i);
+    if (!groups[i].update_out) return fail(ctx, MUON_ERR_INVALID_ARG, "group %d: update_out is NULL", i);
+  }
+  std::vector<Item> items;
+  muon_status s = collect_items(ctx, groups, ngroups, items, false);
+  if (s != MUON_OK) return s;
+  s = set_device(ctx);
+  if (s != MUON_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  ctx->last_stream = st;
+  CUDA_TRY(ctx, cudaGetLastError());
+  return run_precondition_items(ctx, items, st);
 }
 
 muon_status muon_adamw_step(muon_ctx* ctx, const muon_adamw_tensor* tensors, int32_t n,

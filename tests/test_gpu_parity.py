@@ -353,6 +353,75 @@ def test_newton_refresh_vs_oracle(ctx, mx):
             assert rel_fro(to_np(s[b]), want) < 1e-4
 
 
+def _s_inv_blocks(tokens, d, nb, seed, index):
+    a = wl.bf16_round_np(wl.np_normal((tokens, nb * d), 1.0, seed=seed, index=index, role=wl.ROLE_ACT))
+    return [oracle.spd_inverse(oracle.second_moment(a[:, b * d:(b + 1) * d])) for b in range(nb)]
+
+
+# (rows, d, nb): tensor-core block widths (multiples of 64) with ragged row
+# counts, then widths the fp32 tile kernel takes (multiples of 8 only).
+PRECOND_CASES = [(200, 128, 1), (96, 64, 4), (300, 192, 2), (77, 104, 1), (130, 40, 2), (1, 8, 3)]
+
+
+@pytest.mark.parametrize("case", PRECOND_CASES, ids=lambda c: f"{c[0]}x{c[1]}x{c[2]}")
+def test_newton_precondition_vs_oracle(ctx, mx, case):
+    """The stand-alone right-preconditioning G S^-1 against the oracle's
+    block-diagonal product, three gradients sharing one S^-1."""
+    rows, d, nb = case
+    blocks = _s_inv_blocks(512, d, nb, seed=14, index=d + nb)
+    st = dev(np.stack(blocks))
+    gs = [wl.bf16_round_np(wl.np_normal((rows, nb * d), 1e-3, seed=14, index=i)) for i in range(3)]
+    out = [torch.full((rows, nb * d), float("nan"), device="cuda") for _ in gs]
+    ctx.newton_precondition([dev(g, torch.bfloat16) for g in gs], [st] * 3, nb, out)
+    torch.cuda.synchronize()
+    ctx.check_device()
+    for g, o in zip(gs, out):
+        assert rel_fro(to_np(o), oracle.right_precondition(g, blocks)) < 1e-4
+
+
+def test_newton_precondition_matches_step_and_batches(ctx, mx):
+    """The stand-alone product equals the preconditioned gradient the step
+    folds into its momentum (momentum starts at zero, beta = 0), and a
+    workspace that holds one matrix at a time gives the same bits."""
+    d, nb, rows = 128, 2, 256
+    blocks = _s_inv_blocks(1024, d, nb, seed=15, index=0)
+    st = dev(np.stack(blocks))
+    shape = (rows, nb * d)
+    gt = [dev(wl.bf16_round_np(wl.np_normal(shape, 1e-3, seed=15, index=i)), torch.bfloat16) for i in range(4)]
+    ref = [torch.empty(shape, device="cuda") for _ in gt]
+    ctx.newton_precondition(gt, [st] * 4, nb, ref)
+    wt = [torch.zeros(shape, device="cuda") for _ in gt]
+    bt = [torch.zeros(shape, device="cuda") for _ in gt]
+    ctx.step([dict(weights=wt, grads=gt, momentum=bt, precond=[st] * 4, precond_blocks=nb)],
+             mx.default_hparams(momentum=0.0, nesterov=0, lr=0.0))
+    torch.cuda.synchronize()
+    for a, b in zip(ref, bt):
+        assert torch.equal(a, b)
+    per = rows * nb * d * 2 + nb * 2 * d * d * 2
+    wst = torch.empty(per + 4096, dtype=torch.uint8, device="cuda")
+    ctx.set_workspace(wst)
+    out = [torch.empty(shape, device="cuda") for _ in gt]
+    ctx.newton_precondition(gt, [st] * 4, nb, out)
+    torch.cuda.synchronize()
+    ctx.set_workspace(None)
+    for a, b in zip(ref, out):
+        assert torch.equal(a, b)
+
+
+def test_newton_precondition_rejects_bad_arguments(ctx, mx):
+    g = torch.zeros((64, 128), device="cuda", dtype=torch.bfloat16)
+    s = torch.eye(128, device="cuda")[None].contiguous()
+    o = torch.full((64, 128), 7.0, device="cuda")
+    with pytest.raises(mx.MuonError):      # fp32 gradient
+        ctx.newton_precondition([g.float()], [s], 1, [o])
+    with pytest.raises(mx.MuonError):      # block width 128 / 3 not whole
+        ctx.newton_precondition([g], [torch.zeros(3 * 42 * 42, device="cuda")], 3, [o])
+    arr, keep = ctx.make_groups([dict(grads=[g], precond=[s], precond_blocks=1)])
+    assert ctx._lib.muon_newton_precondition(ctx._ctx, arr, 1, None) == mx.binding.MUON_ERR_INVALID_ARG
+    torch.cuda.synchronize()
+    assert torch.all(o == 7.0)
+
+
 def test_newton_muon_step_vs_oracle(ctx, mx):
     """Right-preconditioned step: shared S^-1 for Q/K/V-like matrices and a
     four-block S^-1 for the contraction."""
