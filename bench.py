@@ -321,8 +321,9 @@ def main():
     ap.add_argument("--workload", default="gpt2-small", choices=sorted(wl.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--serial-adamw", action="store_true",
-                    help="run the aux AdamW on the Muon stream instead of a second stream")
+    ap.add_argument("--overlap-adamw", action="store_true",
+                    help="run the aux AdamW on a second stream, forked from and joined into the Muon "
+                         "stream every step (per-kernel times are then taken under contention)")
     args = ap.parse_args()
     w, aux = workload_def(args.workload)
     if args.impl == "reference":
@@ -411,13 +412,16 @@ def main():
     hp = mx.default_hparams()
     ahp = mx.default_adamw_hparams()
     stream = torch.cuda.current_stream()
-    # The aux AdamW touches none of the Muon tensors: it runs on a second
-    # stream, forked from and joined back into the Muon stream every step,
-    # so its HBM traffic overlaps the tensor-core Newton-Schulz products.
-    aux_stream = stream if args.serial_adamw else torch.cuda.Stream()
+    # The aux AdamW runs on the Muon stream, ahead of the Muon step.  It touches
+    # none of the Muon tensors, so --overlap-adamw may run it on a second
+    # stream, forked from and joined back into the Muon stream every step; on
+    # GPT-2-small that gives the same step time (its HBM traffic competes with
+    # the momentum pass), and the per-kernel times get mixed up.
+    serial = not args.overlap_adamw
+    aux_stream = stream if serial else torch.cuda.Stream()
     fork_ev = [torch.cuda.Event() for _ in range(2)]
     join_ev = [torch.cuda.Event() for _ in range(2)]
-    ctx_aux = ctx if args.serial_adamw else mx.MuonContext(local)
+    ctx_aux = ctx if serial else mx.MuonContext(local)
     pre_groups = [groups_for(s) for s in range(n_cycle)]
     adam_step = [0]
 
@@ -637,7 +641,7 @@ def main():
         "config": {"workload": w.name, "matrices": len(w.mats), "hidden_params": elems,
                    "aux_params": aux_el, "grad_dtype": w.grad_dtype, "ns_steps": hp.ns_steps,
                    "grad_sets_cycled": n_cycle, "l2": "inputs larger than L2 (no flush)",
-                   "aux_adamw": "same stream" if args.serial_adamw else "second stream, joined every step",
+                   "aux_adamw": "same stream" if serial else "second stream, joined every step",
                    "parallelism": f"replicas x{world}" if world > 1 else "single"},
         "ns_tflops": ns_flops / (ns_ms * 1e-3) / 1e12 if ns_ms else None,
         "ns_tflops_of_step": ns_flops / (ms_per_step * 1e-3) / 1e12,
