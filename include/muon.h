@@ -237,11 +237,11 @@ MUON_API muon_status muon_newton_refresh(muon_ctx* ctx, const muon_act_desc* act
  * exposes it for callers that precondition and orthogonalise in separate
  * stages.  Block widths that are multiples of 64 run on the tensor cores
  * (S^-1 split into bf16 hi + lo, G in bf16, fp32 accumulation); others on an
- * fp32 tile kernel.  Tensor-core matrices stage a bf16 copy of G and the
- * S^-1 hi/lo stacks in workspace (rows x round_up(cols, 8) x 2 +
- * nb x 2 d^2 x 2 bytes each, 256-byte aligned), in batches that fit a
- * capped or caller-owned workspace; MUON_ERR_WORKSPACE if one matrix does
- * not fit.  Argument errors are reported before any launch. */
+ * fp32 tile kernel.  The tensor cores read G in place; each distinct S^-1
+ * is split once into bf16 hi/lo stacks in workspace (nb x 2 d^2 x 2 bytes,
+ * 256-byte aligned), in batches that fit a capped or caller-owned
+ * workspace; MUON_ERR_WORKSPACE if one S^-1 does not fit.  Argument errors
+ * are reported before any launch. */
 MUON_API muon_status muon_newton_precondition(muon_ctx* ctx, const muon_group* groups, int32_t ngroups,
                                      void* stream);
 

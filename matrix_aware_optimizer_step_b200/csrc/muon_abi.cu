@@ -18,6 +18,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <map>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -207,7 +208,7 @@ struct Chunk {
   size_t off_partials;
   size_t off_pgrad;              // preconditioned gradients (fp32), if any
   bool tc_pre;                   // preconditioning on the tensor-core engine
-  size_t off_gc, off_sst;        // its bf16 gradient copies and S^-1 hi/lo stacks
+  size_t off_sst;                // S^-1 hi/lo stacks (tensor-core preconditioning)
   std::vector<Run> runs;
   size_t bytes;
 };
@@ -215,7 +216,6 @@ struct Chunk {
 // Tensor-core preconditioning needs block widths that are whole 64-wide
 // K blocks (the hi/lo halves of K must not share one).
 inline bool tc_precond_ok(const Item& it) { return (it.cols / it.precond_blocks) % 64 == 0; }
-inline size_t gc_bytes(const Item& it) { return size_t(it.rows) * round_up(it.cols, 8) * 2; }
 inline size_t sst_bytes(const Item& it) {
   const size_t d = size_t(it.cols / it.precond_blocks);
   return size_t(it.precond_blocks) * 2 * d * d * 2;
@@ -243,18 +243,12 @@ size_t layout_chunk(Chunk& c, const std::vector<Item>& items) {
       c.tc_pre = c.tc_pre && tc_precond_ok(items[i]);
     }
   c.tc_pre = c.tc_pre && any_pre;
-  c.off_gc = c.off_sst = off;
+  c.off_sst = off;
   if (c.tc_pre) {
-    size_t g = 0, t = 0;
+    size_t t = 0;
     for (int i = c.first; i < c.first + c.count; ++i)
-      if (items[i].precond) {
-        g += gc_bytes(items[i]);
-        t += sst_bytes(items[i]);
-      }
-    c.off_gc = off;
-    off += round_up(g, kAlign);
-    c.off_sst = off;
-    off += round_up(t, kAlign);
+      if (items[i].precond) t += round_up(sst_bytes(items[i]), kAlign);
+    off += t;
   }
   c.runs.clear();
   int i = c.first;
@@ -577,35 +571,41 @@ muon_status run_newton_schulz(muon_ctx* ctx, uint8_t* ws, const Run* runs, int n
 }
 
 // Matrices of one shape preconditioned on the tensor cores as one batched
-// problem: consecutive bf16 copies in gc, S^-1 hi/lo stacks in sst, fp32
-// results in pg.
+// problem: `count` matrices whose operand maps are consecutive PrecondMaps
+// from pmap_base on, fp32 results consecutive in pg (pg_stride floats
+// apart).
 struct PreProblem {
-  int64_t rows, cols, ldc;
+  int64_t rows, cols;
   int nb, d, count, last;
-  __nv_bfloat16* gc;
-  __nv_bfloat16* sst;
+  int pmap_base;
   float* pg;
   int64_t pg_stride;
 };
 
-// G' = G [S_hi; S_lo] for every problem, up to MAX_PROBLEMS per launch.
-muon_status run_precondition(muon_ctx* ctx, const std::vector<PreProblem>& probs, const int* skip,
-                             cudaStream_t st) {
+// Operand maps of one preconditioned matrix: its gradient in place and the
+// hi/lo stacks of its S^-1 at sst.
+bool encode_precond_maps(PrecondMaps* pm, const void* grad, int64_t rows, int64_t cols, int nb, int d,
+                         const __nv_bfloat16* sst) {
+  bool ok = encode_bf16_3d(&pm->a, grad, cols, rows, 1, cols, 64, 128);
+  ok &= encode_bf16_3d(&pm->b, sst, d, 2 * int64_t(d), nb, d, 64, 64);
+  return ok;
+}
+
+// G' = G [S_hi; S_lo] for every problem, up to MAX_PROBLEMS per launch;
+// pmaps is the device copy of the PrecondMaps table.
+muon_status run_precondition(muon_ctx* ctx, const std::vector<PreProblem>& probs, const PrecondMaps* pmaps,
+                             const int* skip, cudaStream_t st) {
   for (size_t b0 = 0; b0 < probs.size(); b0 += MAX_PROBLEMS) {
     const int nb = int(std::min<size_t>(MAX_PROBLEMS, probs.size() - b0));
-    GemmMaps maps;
+    GemmMaps maps{};           // unused: the operands' maps are in pmaps
     GemmArgs g{};
     g.nprob = nb;
     g.err = ctx->dflags;
     g.skip = skip;
+    g.pmaps = pmaps;
     int tile = 0;
     for (int j = 0; j < nb; ++j) {
       const PreProblem& q = probs[b0 + j];
-      bool ok = encode_bf16_3d(&maps.a[j], q.gc, q.cols, q.rows, q.count, q.ldc, 64, 128);
-      ok &= encode_bf16_3d(&maps.b[j], q.sst, q.d, 2 * q.d, int64_t(q.count) * q.nb, q.d, 64, 64);
-      if (!ok) return fail(ctx, MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed (precondition)");
-      maps.aux[j] = maps.a[j];
-      maps.out[j] = maps.a[j];
       GemmProblem& P = g.p[j];
       P.M = int(q.rows); P.N = q.d; P.K = 2 * q.d;
       P.batch = q.count * q.nb;
@@ -616,6 +616,7 @@ muon_status run_precondition(muon_ctx* ctx, const std::vector<PreProblem>& probs
       P.out32 = q.pg; P.out32_ld = q.cols; P.out32_bs = q.pg_stride;
       P.nblocks = q.nb;
       P.scale = 1.0f;
+      P.pmap_base = q.pmap_base;
       const int64_t tt = int64_t(tile) + int64_t(P.batch) * P.tiles_per_mat;
       if (tt > INT32_MAX) return fail(ctx, MUON_ERR_UNSUPPORTED, "too many tiles in one launch");
       tile = int(tt);
@@ -626,48 +627,67 @@ muon_status run_precondition(muon_ctx* ctx, const std::vector<PreProblem>& probs
   return MUON_OK;
 }
 
+// The S^-1 hi/lo stacks of a launch, one per distinct (S^-1, nb, d): the
+// staging pass splits each once, however many matrices share it.
+struct StackKey {
+  const float* s_inv;
+  int nb, d;
+  bool operator<(const StackKey& o) const {
+    return s_inv != o.s_inv ? s_inv < o.s_inv : nb != o.nb ? nb < o.nb : d < o.d;
+  }
+};
+
 // Newton-Muon preconditioning on its own: update_out[i] = G_i S^-1 in fp32.
 // Matrices whose block width is a multiple of 64 go through the tensor-core
-// engine (bf16 gradient copy and S^-1 hi/lo stacks staged in workspace, in
-// batches that fit it); the rest through the plain fp32 tile kernel, which
-// writes the caller's buffers directly.
+// engine (S^-1 hi/lo stacks staged in workspace, in batches that fit it;
+// each matrix its own problem, since the outputs are the caller's); the rest
+// through the plain fp32 tile kernel, which writes the caller's buffers
+// directly.
 muon_status run_precondition_items(muon_ctx* ctx, const std::vector<Item>& items, cudaStream_t st) {
   if (items.empty()) return MUON_OK;
   const size_t limit = ws_limit(ctx);
-  std::vector<PrepDesc> prep;
+  std::vector<PrepDesc> prep;               // one per distinct stack of a batch
+  std::vector<PrecondMaps> pmaps;           // one per tensor-core matrix
+  std::vector<size_t> pm_sst;               // workspace offset of its stacks
   std::vector<PreProblem> probs;
-  std::vector<int> batch_begin;             // first prep (= problem) index of each batch
+  std::vector<int> batch_prep, batch_prob;  // first prep / problem index of each batch
   std::vector<PrecondDesc> pdescs;
+  std::map<StackKey, size_t> stacks;        // this batch's stacks
   int64_t ptiles = 0;
   size_t cur = 0, need = 0;
   for (const Item& it : items) {
     if (tc_precond_ok(it)) {
-      const size_t gb = round_up(gc_bytes(it), kAlign), sb = round_up(sst_bytes(it), kAlign);
-      if (limit != 0 && gb + sb > limit)
-        return fail(ctx, MUON_ERR_WORKSPACE, "one matrix needs %zu bytes of workspace, %zu available", gb + sb,
-                    limit);
-      if (batch_begin.empty() || (limit != 0 && cur + gb + sb > limit)) {
-        batch_begin.push_back(int(prep.size()));
+      const int d = int(it.cols / it.precond_blocks);
+      const StackKey key{it.precond, it.precond_blocks, d};
+      const size_t sb = round_up(sst_bytes(it), kAlign);
+      if (limit != 0 && sb > limit)
+        return fail(ctx, MUON_ERR_WORKSPACE, "one matrix needs %zu bytes of workspace, %zu available", sb, limit);
+      const bool have = !batch_prep.empty() && stacks.count(key) != 0;
+      if (batch_prep.empty() || (!have && limit != 0 && cur + sb > limit)) {
+        batch_prep.push_back(int(prep.size()));
+        batch_prob.push_back(int(probs.size()));
+        stacks.clear();
         cur = 0;
       }
-      // workspace offsets for now; rebased once the workspace is known
-      PrepDesc pd{};
-      pd.g = static_cast<const __nv_bfloat16*>(it.grad);
-      pd.gc = reinterpret_cast<__nv_bfloat16*>(cur);
-      pd.s_inv = it.precond;
-      pd.sst = reinterpret_cast<__nv_bfloat16*>(cur + gb);
-      pd.rows = it.rows;
-      pd.cols = it.cols;
-      pd.ldc = round_up(it.cols, 8);
-      pd.nb = it.precond_blocks;
-      pd.d = int(it.cols / it.precond_blocks);
-      prep.push_back(pd);
+      auto f = stacks.find(key);
+      if (f == stacks.end()) {
+        f = stacks.emplace(key, cur).first;
+        PrepDesc pd{};
+        pd.s_inv = it.precond;
+        pd.sst = reinterpret_cast<__nv_bfloat16*>(cur);     // offset; rebased below
+        pd.nb = it.precond_blocks;
+        pd.d = d;
+        prep.push_back(pd);
+        cur += sb;
+        need = std::max(need, cur);
+      }
       PreProblem q{};
-      q.rows = it.rows; q.cols = it.cols; q.nb = pd.nb; q.d = pd.d; q.count = 1; q.last = 0;
-      q.ldc = pd.ldc; q.pg = it.update_out; q.pg_stride = it.rows * it.cols;
+      q.rows = it.rows; q.cols = it.cols; q.nb = it.precond_blocks; q.d = d; q.count = 1;
+      q.pmap_base = int(pmaps.size());
+      q.pg = it.update_out; q.pg_stride = it.rows * it.cols;
       probs.push_back(q);
-      cur += gb + sb;
-      need = std::max(need, cur);
+      pmaps.push_back(PrecondMaps{});
+      pm_sst.push_back(f->second);
     } else {
       PrecondDesc p{};
       p.grad = static_cast<const __nv_bfloat16*>(it.grad);
@@ -691,34 +711,45 @@ muon_status run_precondition_items(muon_ctx* ctx, const std::vector<Item>& items
     if (s != MUON_OK) return s;
     ws = static_cast<uint8_t*>(wsv);
   }
-  for (size_t i = 0; i < prep.size(); ++i) {
-    prep[i].gc = reinterpret_cast<__nv_bfloat16*>(ws + reinterpret_cast<uintptr_t>(prep[i].gc));
-    prep[i].sst = reinterpret_cast<__nv_bfloat16*>(ws + reinterpret_cast<uintptr_t>(prep[i].sst));
-    probs[i].gc = prep[i].gc;
-    probs[i].sst = prep[i].sst;
+  for (PrepDesc& pd : prep) pd.sst = reinterpret_cast<__nv_bfloat16*>(ws + reinterpret_cast<uintptr_t>(pd.sst));
+  {
+    size_t k = 0;
+    for (const Item& it : items) {
+      if (!tc_precond_ok(it)) continue;
+      if (!encode_precond_maps(&pmaps[k], it.grad, it.rows, it.cols, it.precond_blocks,
+                               int(it.cols / it.precond_blocks),
+                               reinterpret_cast<const __nv_bfloat16*>(ws + pm_sst[k])))
+        return fail(ctx, MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed (precondition)");
+      ++k;
+    }
   }
   const size_t prep_bytes = round_up(prep.size() * sizeof(PrepDesc), kAlign);
-  std::vector<uint8_t> table(prep_bytes + pdescs.size() * sizeof(PrecondDesc));
+  const size_t pm_off = prep_bytes;
+  const size_t pm_bytes = round_up(pmaps.size() * sizeof(PrecondMaps), kAlign);
+  std::vector<uint8_t> table(pm_off + pm_bytes + pdescs.size() * sizeof(PrecondDesc));
   if (!prep.empty()) std::memcpy(table.data(), prep.data(), prep.size() * sizeof(PrepDesc));
-  if (!pdescs.empty()) std::memcpy(table.data() + prep_bytes, pdescs.data(), pdescs.size() * sizeof(PrecondDesc));
+  if (!pmaps.empty()) std::memcpy(table.data() + pm_off, pmaps.data(), pmaps.size() * sizeof(PrecondMaps));
+  if (!pdescs.empty())
+    std::memcpy(table.data() + pm_off + pm_bytes, pdescs.data(), pdescs.size() * sizeof(PrecondDesc));
   void* dtab = nullptr;
   muon_status s = upload_table(ctx, table.data(), table.size(), st, &dtab);
   if (s != MUON_OK) return s;
   const PrepDesc* dprep = static_cast<const PrepDesc*>(dtab);
-  const PrecondDesc* dpdesc = reinterpret_cast<const PrecondDesc*>(static_cast<uint8_t*>(dtab) + prep_bytes);
+  const PrecondMaps* dpm = reinterpret_cast<const PrecondMaps*>(static_cast<uint8_t*>(dtab) + pm_off);
+  const PrecondDesc* dpdesc = reinterpret_cast<const PrecondDesc*>(static_cast<uint8_t*>(dtab) + pm_off + pm_bytes);
   ProfScope ps(ctx, MUON_K_PRECONDITION, st);
-  for (size_t b = 0; b < batch_begin.size(); ++b) {
-    const int b0 = batch_begin[b];
-    const int b1 = b + 1 < batch_begin.size() ? batch_begin[b + 1] : int(prep.size());
+  for (size_t b = 0; b < batch_prep.size(); ++b) {
+    const int p0 = batch_prep[b];
+    const int p1 = b + 1 < batch_prep.size() ? batch_prep[b + 1] : int(prep.size());
+    const int q0 = batch_prob[b];
+    const int q1 = b + 1 < batch_prob.size() ? batch_prob[b + 1] : int(probs.size());
     int64_t most = 0;
-    for (int k = b0; k < b1; ++k)
-      most = std::max<int64_t>(most, std::max<int64_t>(prep[k].rows * prep[k].cols,
-                                                       int64_t(prep[k].nb) * prep[k].d * prep[k].d));
-    const dim3 grid(unsigned(std::max<int64_t>(1, std::min<int64_t>(cdiv(most, 256 * 8), 512))), unsigned(b1 - b0));
-    launch_pdl(precond_prep_kernel, grid, dim3(256), size_t(0), st, dprep + b0);
+    for (int k = p0; k < p1; ++k) most = std::max<int64_t>(most, int64_t(prep[k].nb) * prep[k].d * prep[k].d);
+    const dim3 grid(unsigned(std::max<int64_t>(1, std::min<int64_t>(cdiv(most, 256 * 8), 512))), unsigned(p1 - p0));
+    launch_pdl(precond_prep_kernel, grid, dim3(256), size_t(0), st, dprep + p0);
     ctx->launches++;
     CUDA_TRY(ctx, cudaGetLastError());
-    s = run_precondition(ctx, std::vector<PreProblem>(probs.begin() + b0, probs.begin() + b1), nullptr, st);
+    s = run_precondition(ctx, std::vector<PreProblem>(probs.begin() + q0, probs.begin() + q1), dpm, nullptr, st);
     if (s != MUON_OK) return s;
   }
   if (!pdescs.empty()) {
@@ -828,8 +859,10 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
   std::vector<int64_t> chunk_tiles(chunks.size(), 0);
   std::vector<int> chunk_pbegin(chunks.size(), 0), chunk_pcount(chunks.size(), 0);
   std::vector<int64_t> chunk_ptiles(chunks.size(), 0);
-  // tensor-core preconditioning: staging descriptors and batched problems
+  // tensor-core preconditioning: staging descriptors (one per distinct S^-1
+  // stack of a chunk), per-matrix operand maps and batched problems
   std::vector<PrepDesc> prep;
+  std::vector<PrecondMaps> pmaps;
   std::vector<int> chunk_prep_begin(chunks.size(), 0), chunk_prep_count(chunks.size(), 0);
   std::vector<std::vector<PreProblem>> chunk_pprob(chunks.size());
   const bool check = mode == 0 && hp->check_finite;
@@ -837,7 +870,8 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
     Chunk& c = chunks[ci];
     int64_t tiles = 0;
     size_t pg_off = c.off_pgrad;
-    size_t gc_off = c.off_gc, sst_off = c.off_sst;
+    size_t sst_off = c.off_sst;
+    std::map<StackKey, const __nv_bfloat16*> stacks;
     chunk_pbegin[ci] = int(pdescs.size());
     chunk_prep_begin[ci] = int(prep.size());
     int64_t ptiles = 0;
@@ -852,28 +886,33 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
           float* pg = reinterpret_cast<float*>(ws + pg_off);
           const size_t pg_bytes = round_up(size_t(it.rows) * it.cols * 4, kAlign);
           pg_off += pg_bytes;
-          PrepDesc pd{};
-          pd.g = static_cast<const __nv_bfloat16*>(it.grad);
-          pd.gc = reinterpret_cast<__nv_bfloat16*>(ws + gc_off);
-          pd.s_inv = it.precond;
-          pd.sst = reinterpret_cast<__nv_bfloat16*>(ws + sst_off);
-          pd.rows = it.rows;
-          pd.cols = it.cols;
-          pd.ldc = round_up(it.cols, 8);
-          pd.nb = it.precond_blocks;
-          pd.d = int(it.cols / it.precond_blocks);
-          gc_off += gc_bytes(it);
-          sst_off += sst_bytes(it);
-          prep.push_back(pd);
+          const int dd = int(it.cols / it.precond_blocks);
+          const StackKey key{it.precond, it.precond_blocks, dd};
+          auto f = stacks.find(key);
+          if (f == stacks.end()) {
+            PrepDesc pd{};
+            pd.s_inv = it.precond;
+            pd.sst = reinterpret_cast<__nv_bfloat16*>(ws + sst_off);
+            pd.nb = it.precond_blocks;
+            pd.d = dd;
+            sst_off += round_up(sst_bytes(it), kAlign);
+            prep.push_back(pd);
+            f = stacks.emplace(key, pd.sst).first;
+          }
+          PrecondMaps pm{};
+          if (!encode_precond_maps(&pm, it.grad, it.rows, it.cols, it.precond_blocks, dd, f->second))
+            return fail(ctx, MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed (precondition)");
+          pmaps.push_back(pm);
           std::vector<PreProblem>& pp = chunk_pprob[ci];
-          if (!pp.empty() && pp.back().rows == it.rows && pp.back().cols == it.cols && pp.back().nb == pd.nb &&
-              pp.back().last == idx - 1) {
+          if (!pp.empty() && pp.back().rows == it.rows && pp.back().cols == it.cols &&
+              pp.back().nb == it.precond_blocks && pp.back().last == idx - 1) {
             pp.back().count++;
             pp.back().last = idx;
           } else {
             PreProblem q{};
-            q.rows = it.rows; q.cols = it.cols; q.nb = pd.nb; q.d = pd.d; q.count = 1; q.last = idx;
-            q.ldc = pd.ldc; q.gc = pd.gc; q.sst = pd.sst; q.pg = pg; q.pg_stride = int64_t(pg_bytes / 4);
+            q.rows = it.rows; q.cols = it.cols; q.nb = it.precond_blocks; q.d = dd; q.count = 1; q.last = idx;
+            q.pmap_base = int(pmaps.size()) - 1;
+            q.pg = pg; q.pg_stride = int64_t(pg_bytes / 4);
             pp.push_back(q);
           }
           d.grad = pg;
@@ -961,11 +1000,13 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
   const size_t mat_bytes = round_up(descs.size() * sizeof(MatDesc), kAlign);
   const size_t pd_bytes = round_up(pdescs.size() * sizeof(PrecondDesc), kAlign);
   const size_t ap_off = round_up(mat_bytes + pd_bytes + prep.size() * sizeof(PrepDesc), kAlign);
-  std::vector<uint8_t> table(ap_off + adescs.size() * sizeof(ApplyDesc));
+  const size_t pm_off = round_up(ap_off + adescs.size() * sizeof(ApplyDesc), kAlign);
+  std::vector<uint8_t> table(pm_off + pmaps.size() * sizeof(PrecondMaps));
   std::memcpy(table.data(), descs.data(), descs.size() * sizeof(MatDesc));
   if (!pdescs.empty()) std::memcpy(table.data() + mat_bytes, pdescs.data(), pdescs.size() * sizeof(PrecondDesc));
   if (!prep.empty()) std::memcpy(table.data() + mat_bytes + pd_bytes, prep.data(), prep.size() * sizeof(PrepDesc));
   if (!adescs.empty()) std::memcpy(table.data() + ap_off, adescs.data(), adescs.size() * sizeof(ApplyDesc));
+  if (!pmaps.empty()) std::memcpy(table.data() + pm_off, pmaps.data(), pmaps.size() * sizeof(PrecondMaps));
   void* dtab = nullptr;
   s = upload_table(ctx, table.data(), table.size(), st, &dtab);
   if (s != MUON_OK) return s;
@@ -1018,14 +1059,15 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
       int64_t most = 0;
       for (int k = 0; k < chunk_prep_count[ci]; ++k) {
         const PrepDesc& pd = prep[chunk_prep_begin[ci] + k];
-        most = std::max<int64_t>(most, std::max<int64_t>(pd.rows * pd.cols, int64_t(pd.nb) * pd.d * pd.d));
+        most = std::max<int64_t>(most, int64_t(pd.nb) * pd.d * pd.d);
       }
       const dim3 grid(unsigned(std::max<int64_t>(1, std::min<int64_t>(cdiv(most, 256 * 8), 512))),
                       unsigned(chunk_prep_count[ci]));
       launch_pdl(precond_prep_kernel, grid, dim3(256), size_t(0), st, dprep + chunk_prep_begin[ci]);
       ctx->launches++;
       CUDA_TRY(ctx, cudaGetLastError());
-      s = run_precondition(ctx, chunk_pprob[ci], skip, st);
+      s = run_precondition(ctx, chunk_pprob[ci],
+                           reinterpret_cast<const PrecondMaps*>(static_cast<uint8_t*>(dtab) + pm_off), skip, st);
       if (s != MUON_OK) return s;
     }
     if (chunk_pcount[ci] > 0) {

@@ -15,9 +15,10 @@
 //   spd_inverse_product_kernel  S^-1 = L^-T L^-1 in 64x64 tiles of the lower
 //                         triangle (mirrored), then copy_inverse_kernel.
 //   cholesky_kernel, chol_solve_kernel  unblocked versions for larger d.
-//   precond_prep_kernel   bf16 copies of the gradients and S^-1 split into
-//                         bf16 hi + lo, the operands of G' = G [S_hi; S_lo]
-//                         on the tensor-core engine (PRECOND).
+//   precond_prep_kernel   S^-1 split into bf16 hi + lo, once per distinct
+//                         S^-1: the B operand of G' = G [S_hi; S_lo] on the
+//                         tensor-core engine (PRECOND), which reads G in
+//                         place.
 //   precond_kernel        G' = G blockdiag(S_b^-1) with fp32 FMAs, for block
 //                         widths that are not a multiple of 64.
 #pragma once
@@ -635,69 +636,53 @@ __global__ void __launch_bounds__(256) act_transpose_kernel(const ActBlock* __re
   }
 }
 
-// One preconditioned matrix: its bf16 gradient copied to a batched layout
-// (rows x ldc) and its nb fp32 inverses split into bf16 hi/lo stacks
-// (2d x d each: rows 0..d-1 = hi, d..2d-1 = lo, with hi + lo ~ S^-1).
+// One S^-1 of a preconditioning launch (nb fp32 d x d blocks) split into
+// bf16 hi/lo stacks, 2d x d per block: rows 0..d-1 = hi, d..2d-1 = lo, with
+// hi + lo ~ S^-1.  Matrices that share an S^-1 share its stacks.
 struct PrepDesc {
-  const __nv_bfloat16* g;
-  __nv_bfloat16* gc;
   const float* s_inv;
   __nv_bfloat16* sst;
-  int64_t rows, cols, ldc;
   int32_t nb, d;
 };
 
-// grid.y = matrix, grid.x strides over max(rows*cols, nb*d*d) elements, 8
-// per thread and step (16-byte loads and stores) when the gradient width and
-// d*d are multiples of 8, one otherwise.  Pointers are 16-byte aligned.
+// grid.y = stack, grid.x strides over its nb*d*d elements, 8 per thread and
+// step (16-byte loads and stores) when d*d is a multiple of 8, one
+// otherwise.  Pointers are 16-byte aligned.
 __global__ void __launch_bounds__(256) precond_prep_kernel(const PrepDesc* __restrict__ descs) {
   pdl_wait();      // previous kernel's results visible (no-op without PDL)
   const PrepDesc& p = descs[blockIdx.y];
-  const int64_t ng = p.rows * p.cols;
   const int64_t dd = static_cast<int64_t>(p.d) * p.d;
   const int64_t ns = p.nb * dd;
-  const bool gvec = (p.cols % 8) == 0;       // then ldc == cols: a flat copy
   const bool svec = (dd % 8) == 0;
-  const int64_t ngu = gvec ? ng / 8 : ng;
   const int64_t nsu = svec ? ns / 8 : ns;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * 256;
-  for (int64_t e = blockIdx.x * 256 + threadIdx.x; e < ngu || e < nsu; e += stride) {
-    if (e < ngu) {
-      if (gvec) {
-        reinterpret_cast<uint4*>(p.gc)[e] = reinterpret_cast<const uint4*>(p.g)[e];
-      } else {
-        const int64_t r = e / p.cols, c = e - r * p.cols;
-        p.gc[r * p.ldc + c] = p.g[e];
-      }
-    }
-    if (e < nsu) {
-      if (svec) {
-        const int64_t e8 = e * 8;
-        const int64_t b = e8 / dd, rem = e8 - b * dd;
-        const float4* src = reinterpret_cast<const float4*>(p.s_inv + e8);
-        const float4 v0 = src[0], v1 = src[1];
-        const float v[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-        uint32_t hw[4], lw[4];
+  for (int64_t e = blockIdx.x * 256 + threadIdx.x; e < nsu; e += stride) {
+    if (svec) {
+      const int64_t e8 = e * 8;
+      const int64_t b = e8 / dd, rem = e8 - b * dd;
+      const float4* src = reinterpret_cast<const float4*>(p.s_inv + e8);
+      const float4 v0 = src[0], v1 = src[1];
+      const float v[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+      uint32_t hw[4], lw[4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const __nv_bfloat16 h0 = __float2bfloat16_rn(v[2 * k]), h1 = __float2bfloat16_rn(v[2 * k + 1]);
-          const __nv_bfloat16 l0 = __float2bfloat16_rn(v[2 * k] - __bfloat162float(h0));
-          const __nv_bfloat16 l1 = __float2bfloat16_rn(v[2 * k + 1] - __bfloat162float(h1));
-          hw[k] = uint32_t(__bfloat16_as_ushort(h0)) | (uint32_t(__bfloat16_as_ushort(h1)) << 16);
-          lw[k] = uint32_t(__bfloat16_as_ushort(l0)) | (uint32_t(__bfloat16_as_ushort(l1)) << 16);
-        }
-        __nv_bfloat16* st = p.sst + b * 2 * dd;
-        *reinterpret_cast<uint4*>(st + rem) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-        *reinterpret_cast<uint4*>(st + dd + rem) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-      } else {
-        const int64_t b = e / dd, rem = e - b * dd;
-        const float v = p.s_inv[e];
-        const __nv_bfloat16 hi = __float2bfloat16_rn(v);
-        const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
-        __nv_bfloat16* st = p.sst + b * 2 * dd;
-        st[rem] = hi;
-        st[dd + rem] = lo;
+      for (int k = 0; k < 4; ++k) {
+        const __nv_bfloat16 h0 = __float2bfloat16_rn(v[2 * k]), h1 = __float2bfloat16_rn(v[2 * k + 1]);
+        const __nv_bfloat16 l0 = __float2bfloat16_rn(v[2 * k] - __bfloat162float(h0));
+        const __nv_bfloat16 l1 = __float2bfloat16_rn(v[2 * k + 1] - __bfloat162float(h1));
+        hw[k] = uint32_t(__bfloat16_as_ushort(h0)) | (uint32_t(__bfloat16_as_ushort(h1)) << 16);
+        lw[k] = uint32_t(__bfloat16_as_ushort(l0)) | (uint32_t(__bfloat16_as_ushort(l1)) << 16);
       }
+      __nv_bfloat16* st = p.sst + b * 2 * dd;
+      *reinterpret_cast<uint4*>(st + rem) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      *reinterpret_cast<uint4*>(st + dd + rem) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    } else {
+      const int64_t b = e / dd, rem = e - b * dd;
+      const float v = p.s_inv[e];
+      const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
+      __nv_bfloat16* st = p.sst + b * 2 * dd;
+      st[rem] = hi;
+      st[dd + rem] = lo;
     }
   }
 }

@@ -61,7 +61,8 @@
 //   PRECOND  G' = G [S_hi; S_lo]         M = rows, N = d, K = 2d
 //            (S^-1 = S_hi + S_lo split into two bf16 matrices stacked along
 //            K, G's column block read twice, so the product keeps close to
-//            fp32 precision)
+//            fp32 precision; G is read in place and each matrix's operands
+//            come from its own tensor maps in device memory)
 #pragma once
 
 #include "sm100_ptx.cuh"
@@ -142,6 +143,7 @@ struct GemmProblem {
   int nblocks;
   float scale;               // GRAM32 / PRECOND: result = scale * sum
   int apply_base;            // UPDATE_APPLY: first ApplyDesc of this problem's matrices
+  int pmap_base;             // PRECOND: first PrecondMaps of this problem's matrices
 };
 
 // Per matrix of a fused update + apply: the fp32 weight as a TMA tensor
@@ -153,6 +155,15 @@ struct alignas(64) ApplyDesc {
   float decay;               // 1 - lr * wd
   int transposed;
   int pad;
+};
+
+// Per matrix of a preconditioning product: its bf16 gradient read in place
+// (cols x rows, box 64 x 128) and the hi/lo stacks of its S^-1 (d x 2d x
+// nb, box 64 x 64, one stack per column block; matrices that share an S^-1
+// share the stacks).
+struct alignas(64) PrecondMaps {
+  CUtensorMap a;
+  CUtensorMap b;
 };
 
 // A launch covers up to MAX_PROBLEMS problems of one product kind (the shape
@@ -170,6 +181,7 @@ struct GemmArgs {
   const int* skip;           // non-null and set: do nothing (non-finite gradient)
   int reverse;               // walk the tile list from its end (see run_newton_schulz)
   const ApplyDesc* apply;    // UPDATE_APPLY: per-matrix weights (device memory)
+  const PrecondMaps* pmaps;  // PRECOND: per-matrix operand maps (device memory)
 };
 
 // Per problem: A operand rows (box 64 x 128), B operand (K-major box 64 x 128
@@ -281,7 +293,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
     tmem_alloc_pair(tmem_slot, TMEM_COLS);
     tmem_relinquish_pair();
   }
-  if (warp == 0 && lane == 0) {
+  if (warp == 0 && lane == 0 && KIND != EPI_PRECOND) {   // PRECOND's maps live in device memory
     for (int p = 0; p < args.nprob; ++p) {
       prefetch_tensormap(&maps.a[p]);
       prefetch_tensormap(&maps.b[p]);
@@ -309,6 +321,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
         decode_tile(KIND, args, t, pi, bidx, ti, tj);
         const CUtensorMap* tmA = &maps.a[pi];
         const CUtensorMap* tmB = &maps.b[pi];
+        int za = bidx, zb = bidx;              // depth coordinates of the A and B loads
+        if (KIND == EPI_PRECOND) {
+          // tile bidx: column block bidx % nblocks of matrix bidx / nblocks
+          const int nbk = args.p[pi].nblocks;
+          const PrecondMaps& pm = args.pmaps[args.p[pi].pmap_base + bidx / nbk];
+          tmA = &pm.a;
+          tmB = &pm.b;
+          za = 0;
+          zb = bidx % nbk;
+        }
         const int nk = (args.p[pi].K + BK - 1) / BK;
         // diagonal tile of a symmetric product: each CTA's B rows are its A
         // rows, so only A is loaded and the MMA reads it for both operands
@@ -322,22 +344,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
           const uint32_t fb = full0 + s * 8;
           if (leader) mbar_arrive_expect_tx(&full_bar[s], diag ? 2 * A_BYTES : 2 * STAGE_BYTES);
           if (KIND == EPI_PRECOND) {
-            // A: column block (bidx % nblocks) of matrix bidx / nblocks, read
-            // twice along K (against S_hi, then S_lo)
-            const int nbk = args.p[pi].nblocks, d = args.p[pi].N;
-            const int blk = bidx % nbk, mat = bidx / nbk;
+            // A: the gradient's column block zb, read twice along K (against
+            // S_hi, then S_lo)
+            const int d = args.p[pi].N;
             int kx = kb * BK;
             if (kx >= d) kx -= d;
-            tma_load_3d_pair(a_dst, tmA, fb, blk * d + kx, ti * TM + rank * HM, mat);
+            tma_load_3d_pair(a_dst, tmA, fb, zb * d + kx, ti * TM + rank * HM, za);
           } else {
-            tma_load_3d_pair(a_dst, tmA, fb, kb * BK, ti * TM + rank * HM, bidx);
+            tma_load_3d_pair(a_dst, tmA, fb, kb * BK, ti * TM + rank * HM, za);
           }
           if (B_MN_MAJOR) {
 #pragma unroll
             for (int c = 0; c < HN / 64; ++c)
-              tma_load_3d_pair(b_dst + c * MN_CHUNK_BYTES, tmB, fb, tj * TN + rank * HN + c * 64, kb * BK, bidx);
+              tma_load_3d_pair(b_dst + c * MN_CHUNK_BYTES, tmB, fb, tj * TN + rank * HN + c * 64, kb * BK, zb);
           } else if (!diag) {
-            tma_load_3d_pair(b_dst, tmB, fb, kb * BK, tj * TN + rank * HN, bidx);
+            tma_load_3d_pair(b_dst, tmB, fb, kb * BK, tj * TN + rank * HN, zb);
           }
           ++it;
         }

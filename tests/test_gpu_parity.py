@@ -381,27 +381,29 @@ def test_newton_precondition_vs_oracle(ctx, mx, case):
 
 def test_newton_precondition_matches_step_and_batches(ctx, mx):
     """The stand-alone product equals the preconditioned gradient the step
-    folds into its momentum (momentum starts at zero, beta = 0), and a
-    workspace that holds one matrix at a time gives the same bits."""
+    folds into its momentum (momentum starts at zero, beta = 0), for two
+    S^-1 each shared by two gradients; a workspace that holds one S^-1's
+    hi/lo stacks at a time (two staging batches) gives the same bits."""
     d, nb, rows = 128, 2, 256
-    blocks = _s_inv_blocks(1024, d, nb, seed=15, index=0)
-    st = dev(np.stack(blocks))
+    sa = dev(np.stack(_s_inv_blocks(1024, d, nb, seed=15, index=0)))
+    sb = dev(np.stack(_s_inv_blocks(1024, d, nb, seed=15, index=1)))
+    ss = [sa, sa, sb, sb]
     shape = (rows, nb * d)
     gt = [dev(wl.bf16_round_np(wl.np_normal(shape, 1e-3, seed=15, index=i)), torch.bfloat16) for i in range(4)]
     ref = [torch.empty(shape, device="cuda") for _ in gt]
-    ctx.newton_precondition(gt, [st] * 4, nb, ref)
+    ctx.newton_precondition(gt, ss, nb, ref)
     wt = [torch.zeros(shape, device="cuda") for _ in gt]
     bt = [torch.zeros(shape, device="cuda") for _ in gt]
-    ctx.step([dict(weights=wt, grads=gt, momentum=bt, precond=[st] * 4, precond_blocks=nb)],
+    ctx.step([dict(weights=wt, grads=gt, momentum=bt, precond=ss, precond_blocks=nb)],
              mx.default_hparams(momentum=0.0, nesterov=0, lr=0.0))
     torch.cuda.synchronize()
     for a, b in zip(ref, bt):
         assert torch.equal(a, b)
-    per = rows * nb * d * 2 + nb * 2 * d * d * 2
-    wst = torch.empty(per + 4096, dtype=torch.uint8, device="cuda")
+    stack = nb * 2 * d * d * 2
+    wst = torch.empty(stack + 1024, dtype=torch.uint8, device="cuda")
     ctx.set_workspace(wst)
     out = [torch.empty(shape, device="cuda") for _ in gt]
-    ctx.newton_precondition(gt, [st] * 4, nb, out)
+    ctx.newton_precondition(gt, ss, nb, out)
     torch.cuda.synchronize()
     ctx.set_workspace(None)
     for a, b in zip(ref, out):
