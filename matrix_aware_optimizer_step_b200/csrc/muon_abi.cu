@@ -1390,13 +1390,20 @@ muon_status muon_newton_refresh(muon_ctx* ctx, const muon_act_desc* acts, int32_
   if (!ctx) return MUON_ERR_INVALID_ARG;
   if (n < 0 || (n > 0 && !acts)) return fail(ctx, MUON_ERR_INVALID_ARG, "bad activation list");
   if (!(damping >= 0.f) || !std::isfinite(damping)) return fail(ctx, MUON_ERR_INVALID_ARG, "damping must be >= 0");
-  // Per d-wide activation block: a transposed bf16 copy (d x tokens), the
-  // fp32 second moment S (then its Cholesky factor) and the output S^-1.
+  // Per d-wide activation block: the fp32 second moment S (then its
+  // Cholesky factor) and the output S^-1.  When every width and block width
+  // is a multiple of 8 elements (16 bytes, the TMA coordinate granule) the
+  // second-moment product reads the activations in place; otherwise each
+  // block is first copied transposed (d x tokens bf16).
   struct GramProb {
     int64_t tokens, d, ldt;
-    int count;
+    int count, nb, pmap_base;
     size_t xt_off, s_off;
+    int64_t s_stride;          // floats between consecutive blocks' S
   };
+  bool direct = true;
+  for (int i = 0; i < n; ++i)
+    direct = direct && acts[i].nblocks >= 1 && acts[i].width % 8 == 0 && (acts[i].width / acts[i].nblocks) % 8 == 0;
   std::vector<ActBlock> ab;
   std::vector<CholDesc> cd;
   std::vector<GramProb> gp;
@@ -1415,6 +1422,9 @@ muon_status muon_newton_refresh(muon_ctx* ctx, const muon_act_desc* acts, int32_
     if (!aligned16(a.acts) || !aligned16(a.s_inv))
       return fail(ctx, MUON_ERR_INVALID_ARG, "activation %d: not 16-byte aligned", i);
     const int64_t ldt = round_up(a.tokens, 8);
+    // each block's S starts 256-byte aligned, whatever d is (the Cholesky
+    // kernels take 16-byte vector paths when d is a multiple of 4)
+    const size_t s_bytes = round_up(size_t(d) * d * 4, kAlign);
     for (int b = 0; b < a.nblocks; ++b) {
       ActBlock x{};
       x.acts = static_cast<const __nv_bfloat16*>(a.acts);
@@ -1430,13 +1440,13 @@ muon_status muon_newton_refresh(muon_ctx* ctx, const muon_act_desc* acts, int32_
       c.inv = a.s_inv + size_t(b) * d * d;
       c.d = int(d);
       cd.push_back(c);
-      if (!gp.empty() && gp.back().tokens == a.tokens && gp.back().d == d) {
+      if (!gp.empty() && gp.back().tokens == a.tokens && gp.back().d == d && (!direct || gp.back().nb == a.nblocks)) {
         gp.back().count++;
       } else {
-        gp.push_back(GramProb{a.tokens, d, ldt, 1, xt_total, s_total});
+        gp.push_back(GramProb{a.tokens, d, ldt, 1, a.nblocks, i, xt_total, s_total, int64_t(s_bytes / 4)});
       }
-      xt_total += size_t(d) * ldt * 2;
-      s_total += size_t(d) * d * 4;
+      if (!direct) xt_total += size_t(d) * ldt * 2;
+      s_total += s_bytes;
       max_d = std::max(max_d, int(d));
       max_tiles = std::max<int64_t>(max_tiles, cdiv(a.tokens, TPOSE_T) * cdiv(d, TPOSE_T));
     }
@@ -1455,34 +1465,46 @@ muon_status muon_newton_refresh(muon_ctx* ctx, const muon_act_desc* acts, int32_
   uint8_t* ws = static_cast<uint8_t*>(wsv);
   for (auto& x : ab) x.xt = reinterpret_cast<__nv_bfloat16*>(ws + s_region + reinterpret_cast<size_t>(x.xt));
   for (auto& c : cd) c.a = reinterpret_cast<float*>(ws + reinterpret_cast<size_t>(c.a));
+  // in place: one map per activation over its whole tokens x width matrix
+  std::vector<PrecondMaps> pmaps(direct ? n : 0);
+  for (int i = 0; direct && i < n; ++i)
+    if (!encode_bf16_3d(&pmaps[i].a, acts[i].acts, acts[i].width, acts[i].tokens, 1, acts[i].width, 64, 64))
+      return fail(ctx, MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed (second moment)");
   const size_t ab_bytes = round_up(ab.size() * sizeof(ActBlock), kAlign);
-  std::vector<uint8_t> table(ab_bytes + cd.size() * sizeof(CholDesc));
+  const size_t pm_off = round_up(ab_bytes + cd.size() * sizeof(CholDesc), kAlign);
+  std::vector<uint8_t> table(pm_off + pmaps.size() * sizeof(PrecondMaps));
   std::memcpy(table.data(), ab.data(), ab.size() * sizeof(ActBlock));
   std::memcpy(table.data() + ab_bytes, cd.data(), cd.size() * sizeof(CholDesc));
+  if (!pmaps.empty()) std::memcpy(table.data() + pm_off, pmaps.data(), pmaps.size() * sizeof(PrecondMaps));
   void* dtab = nullptr;
   s = upload_table(ctx, table.data(), table.size(), st, &dtab);
   if (s != MUON_OK) return s;
   const ActBlock* dab = static_cast<const ActBlock*>(dtab);
   const CholDesc* dc = reinterpret_cast<const CholDesc*>(static_cast<uint8_t*>(dtab) + ab_bytes);
   ProfScope ps(ctx, MUON_K_NEWTON_REFRESH, st);
-  launch_pdl(act_transpose_kernel, dim3(unsigned(max_tiles), unsigned(ab.size())), dim3(256), size_t(0), st, dab);
-  ctx->launches++;
-  CUDA_TRY(ctx, cudaGetLastError());
+  if (!direct) {
+    launch_pdl(act_transpose_kernel, dim3(unsigned(max_tiles), unsigned(ab.size())), dim3(256), size_t(0), st, dab);
+    ctx->launches++;
+    CUDA_TRY(ctx, cudaGetLastError());
+  }
   // S = Xt Xt^T / tokens on the tensor cores, up to MAX_PROBLEMS shapes per launch
   for (size_t b0 = 0; b0 < gp.size(); b0 += MAX_PROBLEMS) {
     const int nb = int(std::min<size_t>(MAX_PROBLEMS, gp.size() - b0));
-    GemmMaps maps;
+    GemmMaps maps{};
     GemmArgs g{};
     g.nprob = nb;
     g.err = ctx->dflags;
+    if (direct) g.pmaps = reinterpret_cast<const PrecondMaps*>(static_cast<uint8_t*>(dtab) + pm_off);
     int tile = 0;
     for (int j = 0; j < nb; ++j) {
       const GramProb& q = gp[b0 + j];
-      if (!encode_bf16_3d(&maps.a[j], ws + s_region + q.xt_off, q.tokens, q.d, q.count, q.ldt, 64, 128))
-        return fail(ctx, MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed (second moment)");
-      maps.b[j] = maps.a[j];
-      maps.aux[j] = maps.a[j];
-      maps.out[j] = maps.a[j];
+      if (!direct) {
+        if (!encode_bf16_3d(&maps.a[j], ws + s_region + q.xt_off, q.tokens, q.d, q.count, q.ldt, 64, 128))
+          return fail(ctx, MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed (second moment)");
+        maps.b[j] = maps.a[j];
+        maps.aux[j] = maps.a[j];
+        maps.out[j] = maps.a[j];
+      }
       GemmProblem& P = g.p[j];
       P.M = int(q.d); P.N = int(q.d); P.K = int(q.tokens);
       P.batch = q.count;
@@ -1491,15 +1513,17 @@ muon_status muon_newton_refresh(muon_ctx* ctx, const muon_act_desc* acts, int32_
       P.tile_start = tile;
       P.out32 = reinterpret_cast<float*>(ws + q.s_off);
       P.out32_ld = q.d;
-      P.out32_bs = q.d * q.d;
-      P.nblocks = 1;
+      P.out32_bs = q.s_stride;
+      P.nblocks = direct ? q.nb : 1;
+      P.pmap_base = q.pmap_base;
       P.scale = 1.0f / float(q.tokens);
       const int64_t tt = int64_t(tile) + int64_t(P.batch) * P.tiles_per_mat;
       if (tt > INT32_MAX) return fail(ctx, MUON_ERR_UNSUPPORTED, "too many tiles in one launch");
       tile = int(tt);
     }
     g.total = tile;
-    CUDA_TRY(ctx, (launch_gemm<EPI_GRAM32, false>(ctx, maps, g, st)));
+    if (direct) CUDA_TRY(ctx, (launch_gemm<EPI_GRAM32, true>(ctx, maps, g, st)));
+    else CUDA_TRY(ctx, (launch_gemm<EPI_GRAM32, false>(ctx, maps, g, st)));
   }
   if (max_d <= CHOL_BLOCKED_MAX_D) {
     // blocked factorisation, panels of 32: panel, then trailing update

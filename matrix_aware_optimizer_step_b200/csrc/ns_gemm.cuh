@@ -57,7 +57,10 @@
 //
 //   GRAM32   S = (1/N) Xt Xt^T          M = N = d, K = N tokens  symmetric
 //            (Xt: bf16 activation block, transposed; bf16 products are exact
-//            in fp32)
+//            in fp32).  Launched with MN-major operands it reads the tokens
+//            x width activation in place: A and B are both MN-major, with
+//            the block's column offset added to the MN coordinate, and the
+//            per-activation maps come from device memory.
 //   PRECOND  G' = G [S_hi; S_lo]         M = rows, N = d, K = 2d
 //            (S^-1 = S_hi + S_lo split into two bf16 matrices stacked along
 //            K, G's column block read twice, so the product keeps close to
@@ -191,6 +194,12 @@ struct GemmMaps {
   CUtensorMap a[MAX_PROBLEMS], b[MAX_PROBLEMS], aux[MAX_PROBLEMS], out[MAX_PROBLEMS];
 };
 
+// Launches whose operand tensor maps are per matrix in device memory
+// (args.pmaps) rather than per problem in parameter space.
+__host__ __device__ constexpr bool device_maps(int kind, bool b_mn_major) {
+  return kind == EPI_PRECOND || (kind == EPI_GRAM32 && b_mn_major);
+}
+
 __host__ __device__ constexpr bool symmetric_kind(int kind) {
   return kind == EPI_GRAM || kind == EPI_POLY || kind == EPI_GRAM32;
 }
@@ -251,6 +260,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
     ns_gemm_kernel(const __grid_constant__ GemmMaps maps, const __grid_constant__ GemmArgs args) {
   using namespace gemm_cfg;
   constexpr int STAGES = stages_for(KIND);
+  // GRAM32 with MN-major operands reads the activations in place: A is
+  // MN-major too, and both operands' maps come from args.pmaps
+  constexpr bool A_MN = KIND == EPI_GRAM32 && B_MN_MAJOR;
   extern __shared__ uint8_t smem_raw[];
 
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -293,7 +305,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
     tmem_alloc_pair(tmem_slot, TMEM_COLS);
     tmem_relinquish_pair();
   }
-  if (warp == 0 && lane == 0 && KIND != EPI_PRECOND) {   // PRECOND's maps live in device memory
+  if (warp == 0 && lane == 0 && !device_maps(KIND, B_MN_MAJOR)) {
     for (int p = 0; p < args.nprob; ++p) {
       prefetch_tensormap(&maps.a[p]);
       prefetch_tensormap(&maps.b[p]);
@@ -322,6 +334,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
         const CUtensorMap* tmA = &maps.a[pi];
         const CUtensorMap* tmB = &maps.b[pi];
         int za = bidx, zb = bidx;              // depth coordinates of the A and B loads
+        int xoff = 0;                          // MN offset of both operands (GRAM32 direct)
         if (KIND == EPI_PRECOND) {
           // tile bidx: column block bidx % nblocks of matrix bidx / nblocks
           const int nbk = args.p[pi].nblocks;
@@ -330,6 +343,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
           tmB = &pm.b;
           za = 0;
           zb = bidx % nbk;
+        } else if (A_MN) {
+          // tile bidx: column block bidx % nblocks of activation bidx / nblocks,
+          // both operands read from the tokens x width activation itself
+          const int nbk = args.p[pi].nblocks;
+          const PrecondMaps& pm = args.pmaps[args.p[pi].pmap_base + bidx / nbk];
+          tmA = tmB = &pm.a;
+          za = zb = 0;
+          xoff = (bidx % nbk) * args.p[pi].N;
         }
         const int nk = (args.p[pi].K + BK - 1) / BK;
         // diagonal tile of a symmetric product: each CTA's B rows are its A
@@ -350,13 +371,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
             int kx = kb * BK;
             if (kx >= d) kx -= d;
             tma_load_3d_pair(a_dst, tmA, fb, zb * d + kx, ti * TM + rank * HM, za);
+          } else if (A_MN) {
+#pragma unroll
+            for (int c = 0; c < HM / 64; ++c)
+              tma_load_3d_pair(a_dst + c * MN_CHUNK_BYTES, tmA, fb, xoff + ti * TM + rank * HM + c * 64, kb * BK, za);
           } else {
             tma_load_3d_pair(a_dst, tmA, fb, kb * BK, ti * TM + rank * HM, za);
           }
-          if (B_MN_MAJOR) {
+          // a diagonal tile's B is its A (expect_tx above counts A only)
+          if (B_MN_MAJOR && !diag) {
 #pragma unroll
             for (int c = 0; c < HN / 64; ++c)
-              tma_load_3d_pair(b_dst + c * MN_CHUNK_BYTES, tmB, fb, tj * TN + rank * HN + c * 64, kb * BK, zb);
+              tma_load_3d_pair(b_dst + c * MN_CHUNK_BYTES, tmB, fb, xoff + tj * TN + rank * HN + c * 64, kb * BK, zb);
           } else if (!diag) {
             tma_load_3d_pair(b_dst, tmB, fb, kb * BK, tj * TN + rank * HN, zb);
           }
@@ -373,7 +399,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
   } else if (warp == 1) {
     // ---------------- MMA issuer (leader CTA only) ----------------
     if (leader && lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(TM, TN, B_MN_MAJOR);
+      constexpr uint32_t idesc = idesc_bf16_f32(TM, TN, B_MN_MAJOR, A_MN);
       int it = 0, lt = 0;
       bool ok = true;
       for (int t = pair; t < total && ok; t += npairs, ++lt) {
@@ -394,7 +420,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
           const uint32_t b_base = diag ? a_base : a_base + A_BYTES;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t adesc = sdesc_kmajor_sw128(a_base + kk * 32);
+            const uint64_t adesc = A_MN ? sdesc_mnmajor_sw128(a_base + kk * 16 * 128, MN_CHUNK_BYTES)
+                                        : sdesc_kmajor_sw128(a_base + kk * 32);
             const uint64_t bdesc = B_MN_MAJOR ? sdesc_mnmajor_sw128(b_base + kk * 16 * 128, MN_CHUNK_BYTES)
                                               : sdesc_kmajor_sw128(b_base + kk * 32);
             mma_bf16_ss_pair(d_tmem, adesc, bdesc, idesc, (kb > 0 || kk > 0) ? 1u : 0u);

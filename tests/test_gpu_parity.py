@@ -424,6 +424,29 @@ def test_newton_precondition_rejects_bad_arguments(ctx, mx):
     assert torch.all(o == 7.0)
 
 
+@pytest.mark.parametrize("case", [[((1001, 256), 2)], [((1001, 100), 1)], [((640, 90), 2), ((512, 128), 1)]],
+                         ids=["in-place-ragged-tokens", "transposed-width-100", "transposed-odd-block-then-even"])
+def test_newton_refresh_paths(ctx, mx, case):
+    """The second moment read in place (widths multiples of 8, here with a
+    token count that is not) and through transposed copies (a width or block
+    width that is not a multiple of 8; an odd block width followed, in the
+    same call, by a block whose kernels take 16-byte vector paths) all match
+    the oracle."""
+    acts, outs = [], []
+    for k, (shape, nb) in enumerate(case):
+        a = wl.bf16_round_np(wl.np_normal(shape, 1.0, seed=16, index=shape[1] + k, role=wl.ROLE_ACT))
+        d = shape[1] // nb
+        acts.append((a, nb, d))
+        outs.append(torch.empty((nb, d, d), device="cuda"))
+    ctx.newton_refresh([dev(a, torch.bfloat16) for a, _, _ in acts], outs, [nb for _, nb, _ in acts])
+    torch.cuda.synchronize()
+    ctx.check_device()
+    for (a, nb, d), s in zip(acts, outs):
+        for b in range(nb):
+            want = oracle.spd_inverse(oracle.second_moment(a[:, b * d:(b + 1) * d]))
+            assert rel_fro(to_np(s[b]), want) < 1e-4
+
+
 def test_newton_muon_step_vs_oracle(ctx, mx):
     """Right-preconditioned step: shared S^-1 for Q/K/V-like matrices and a
     four-block S^-1 for the contraction."""
