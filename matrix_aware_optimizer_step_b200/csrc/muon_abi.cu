@@ -1460,11 +1460,16 @@ muon_status muon_newton_refresh(muon_ctx* ctx, const muon_act_desc* acts, int32_
   CUDA_TRY(ctx, cudaGetLastError());
   const size_t s_region = round_up(s_total, kAlign);
   void* wsv = nullptr;
-  s = ensure_workspace(ctx, s_region + xt_total, &wsv);
+  // S / L per block, then the recursive L^-1's T per block (same layout),
+  // then the transposed activation copies
+  s = ensure_workspace(ctx, 2 * s_region + xt_total, &wsv);
   if (s != MUON_OK) return s;
   uint8_t* ws = static_cast<uint8_t*>(wsv);
-  for (auto& x : ab) x.xt = reinterpret_cast<__nv_bfloat16*>(ws + s_region + reinterpret_cast<size_t>(x.xt));
-  for (auto& c : cd) c.a = reinterpret_cast<float*>(ws + reinterpret_cast<size_t>(c.a));
+  for (auto& x : ab) x.xt = reinterpret_cast<__nv_bfloat16*>(ws + 2 * s_region + reinterpret_cast<size_t>(x.xt));
+  for (auto& c : cd) {
+    c.t = reinterpret_cast<float*>(ws + s_region + reinterpret_cast<size_t>(c.a));
+    c.a = reinterpret_cast<float*>(ws + reinterpret_cast<size_t>(c.a));
+  }
   // in place: one map per activation over its whole tokens x width matrix
   std::vector<PrecondMaps> pmaps(direct ? n : 0);
   for (int i = 0; direct && i < n; ++i)
@@ -1499,7 +1504,7 @@ muon_status muon_newton_refresh(muon_ctx* ctx, const muon_act_desc* acts, int32_
     for (int j = 0; j < nb; ++j) {
       const GramProb& q = gp[b0 + j];
       if (!direct) {
-        if (!encode_bf16_3d(&maps.a[j], ws + s_region + q.xt_off, q.tokens, q.d, q.count, q.ldt, 64, 128))
+        if (!encode_bf16_3d(&maps.a[j], ws + 2 * s_region + q.xt_off, q.tokens, q.d, q.count, q.ldt, 64, 128))
           return fail(ctx, MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed (second moment)");
         maps.b[j] = maps.a[j];
         maps.aux[j] = maps.a[j];
@@ -1527,8 +1532,6 @@ muon_status muon_newton_refresh(muon_ctx* ctx, const muon_act_desc* acts, int32_
   }
   if (max_d <= CHOL_BLOCKED_MAX_D) {
     // blocked factorisation, panels of 32: panel, then trailing update
-    CUDA_TRY(ctx, cudaFuncSetAttribute(chol_linv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       cinv_smem_bytes(max_d)));
     for (int p0 = 0; p0 < max_d; p0 += CB) {
       const int rest = max_d - p0 - CB;                   // trailing rows of the largest matrix
       const unsigned chunks = unsigned(std::max<int64_t>(1, cdiv(std::max(rest, 0), CPR)));
@@ -1544,13 +1547,23 @@ muon_status muon_newton_refresh(muon_ctx* ctx, const muon_act_desc* acts, int32_
         CUDA_TRY(ctx, cudaGetLastError());
       }
     }
-    // L^-1 into the output buffers, then S^-1 = L^-T L^-1 into the scratch
+    // L^-1 into the output buffers (diagonal-block inverses, then doubling
+    // levels of two products each), then S^-1 = L^-T L^-1 into the scratch
     // that held L, then copied out
-    const int parts = int(cdiv(max_d, CB));
-    launch_pdl(chol_linv_kernel, dim3(unsigned(cd.size() * parts)), dim3(CINV_THREADS),
-               size_t(cinv_smem_bytes(max_d)), st, dc, parts);
+    launch_pdl(linv_init_kernel, dim3(unsigned(cdiv(max_d, 64)), unsigned(cd.size())), dim3(256), size_t(0), st,
+               dc);
     ctx->launches++;
     CUDA_TRY(ctx, cudaGetLastError());
+    for (int sl = CB; sl < max_d; sl *= 2) {
+      const int64_t tiles = cdiv(sl, LV_T);
+      const int64_t pairs = cdiv(max_d - sl, 2 * int64_t(sl));
+      for (int mode = 0; mode < 2; ++mode) {
+        launch_pdl(linv_level_kernel, dim3(unsigned(pairs * tiles * tiles), unsigned(cd.size())), dim3(LV_THREADS),
+                   size_t(0), st, dc, sl, mode);
+        ctx->launches++;
+        CUDA_TRY(ctx, cudaGetLastError());
+      }
+    }
     const int nt = int(cdiv(max_d, SIP_T));
     launch_pdl(spd_inverse_product_kernel, dim3(unsigned(nt * (nt + 1) / 2), unsigned(cd.size())),
                dim3(SIP_THREADS), size_t(0), st, dc);

@@ -10,8 +10,9 @@
 //   chol_panel_kernel, chol_update_kernel  S = L L^T in place (fp32),
 //                         panels of 32, two batched launches per panel
 //                         (d <= 1536).
-//   chol_linv_kernel      L^-1, 32 columns per block, blocked forward
-//                         substitution with the diagonal blocks' inverses.
+//   linv_init_kernel, linv_level_kernel  L^-1 from the diagonal blocks'
+//                         inverses by recursive doubling, two batched tile
+//                         products per level.
 //   spd_inverse_product_kernel  S^-1 = L^-T L^-1 in 64x64 tiles of the lower
 //                         triangle (mirrored), then copy_inverse_kernel.
 //   cholesky_kernel, chol_solve_kernel  unblocked versions for larger d.
@@ -54,6 +55,7 @@ struct CholDesc {
                      // (unblocked path) or, in each 32x32 diagonal block,
                      // the transpose of that block's inverse (blocked path)
   float* inv;        // d x d output S^-1
+  float* t;          // d x d scratch of the recursive L^-1 (blocked path)
   int32_t d;
   int32_t pad;
 };
@@ -103,7 +105,7 @@ __global__ void __launch_bounds__(CHOL_THREADS)
 // ---------------------------------------------------------------------------
 constexpr int CB = 32;                      // panel width
 constexpr int CBP = CB + 1;                 // padded row of a panel in smem
-constexpr int CHOL_BLOCKED_MAX_D = 1536;    // chol_linv_kernel keeps d x 32 floats in smem
+constexpr int CHOL_BLOCKED_MAX_D = 1536;    // widest block the blocked path takes (larger: unblocked kernels)
 constexpr int CP_THREADS = 256;
 constexpr int CPR = 64;                     // panel rows per chol_panel_kernel block
 
@@ -114,7 +116,7 @@ constexpr int CPR = 64;                     // panel rows per chol_panel_kernel 
 //                       D (one warp, in shared memory) and inverts it (lane j
 //                       solves for column j of D^-1); block 0 writes D to the
 //                       lower triangle and D^-1 transposed to the block's
-//                       strict upper triangle (read back by chol_linv_kernel);
+//                       strict upper triangle (read back by linv_init_kernel);
 //                       each block then forms CPR rows of the panel below D,
 //                       P = A_panel D^-T, as a product over all threads.
 //   chol_update_kernel  the trailing lower triangle minus P P^T, in 64x64
@@ -272,108 +274,111 @@ __global__ void __launch_bounds__(CP_THREADS) chol_update_kernel(const CholDesc*
   }
 }
 
-constexpr int CINV_THREADS = 256;
-
-__host__ __device__ inline int cinv_smem_bytes(int d) { return d * CB * 4; }
-
-// L^-1, 32 columns per block: forward L Y = E (E = columns c0 .. c0+31 of
-// I; rows of Y above c0 are zero), row blocks of 32 at a time, Y resident in
-// shared memory.  Within a row block the substitution is a product with the
-// diagonal block's inverse D^-1, spread over all threads.  Y is written to
-// c.inv (rows from c0 rounded down to 64, zeros above c0), the operand of
-// spd_inverse_product_kernel.  L is read from the lower triangle of c.a.
-__global__ void __launch_bounds__(CINV_THREADS)
-    chol_linv_kernel(const CholDesc* __restrict__ descs, int blocks_per_mat) {
+// L^-1 by recursive doubling of the 32x32 diagonal blocks: for a lower
+// triangular [[A, 0], [C, B]], the inverse is [[A^-1, 0], [-B^-1 C A^-1,
+// B^-1]].  Level l pairs consecutive blocks of s = 32 * 2^l rows: block p
+// of the level spans rows r0 = 2 s p .. r0 + s + s2 (s2 = min(s, d - r0 - s),
+// the second block may be short), and once A^-1 and B^-1 are in X its
+// off-diagonal block is two products,
+//   T   = C A^-1         (rows r0+s.., columns r0..; A^-1 lower: k >= j)
+//   X21 = -B^-1 T        (B^-1 lower: k <= i)
+// so the chain of dependent launches is 2 log2(d / 32) long instead of d /
+// 32 row blocks.  X is written to c.inv, T to c.t; C is read from L's lower
+// triangle in c.a.  Every output is an fp32 sum of products of fp32 values,
+// as in forward substitution, in a different order.
+//
+// linv_init_kernel: X's 64x64 diagonal tiles (grid.x: tile, grid.y: matrix)
+// hold the two 32x32 diagonal-block inverses and zeros above the diagonal
+// (the upper triangle of these tiles is read as zeros by the tile products
+// below and by spd_inverse_product_kernel); the lower-left 32x32 block is
+// left to level 0.
+__global__ void __launch_bounds__(256) linv_init_kernel(const CholDesc* __restrict__ descs) {
   pdl_wait();      // previous kernel's results visible (no-op without PDL)
-  extern __shared__ float4 y4[];           // Y: [d][CB] floats, 16-byte rows units
-  float* y = reinterpret_cast<float*>(y4);
-  __shared__ float acc_s[CB][CBP];
-  __shared__ float ls[2][CB][CBP];          // 32x32 chunks of L's row block, double-buffered
-  const CholDesc& c = descs[blockIdx.x / blocks_per_mat];
+  const CholDesc& c = descs[blockIdx.y];
   const int d = c.d;
-  const int c0 = (blockIdx.x % blocks_per_mat) * CB;
-  if (c0 >= d) return;
-  const float* L = c.a;
-  const int tid = threadIdx.x;
-  const int orow = tid >> 3, ocol = (tid & 7) * 4;     // this thread's 4 outputs in a 32x32 block
-  const int nrb = (d + CB - 1) / CB;
-  const int rb0 = c0 / CB;
-  // ---- forward ----
-  for (int rb = rb0; rb < nrb; ++rb) {
-    const int rbase = rb * CB;
-    float acc[4];
-    const int r = rbase + orow;
-#pragma unroll
-    for (int v = 0; v < 4; ++v) acc[v] = (r == c0 + ocol + v) ? 1.f : 0.f;
-    // acc -= L[rbase.., c0..rbase) Y[c0..rbase), L staged in 32x32 chunks;
-    // the next chunk and this row block's D^-1 are loaded into registers
-    // while the current chunk is used
-    const int nch = (rbase - c0) / CB;
-    float lreg[4], dreg[4];
-    auto load_chunk = [&](int k0) {
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int e = tid + q * CINV_THREADS, i = e >> 5, kk = e & 31;
-        lreg[q] = (rbase + i < d) ? L[int64_t(rbase + i) * d + k0 + kk] : 0.f;
-      }
-    };
-    if (nch > 0) load_chunk(c0);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int e = tid + q * CINV_THREADS, i = e >> 5, k = e & 31;
-      const int gi = rbase + i, gk = rbase + k;
-      float v = 0.f;
-      if (gi < d && gk < d) {
-        if (k < i) v = L[int64_t(gk) * d + gi];
-        else if (k == i) v = 1.f / L[int64_t(gi) * d + gi];
-      }
-      dreg[q] = v;
+  const int t0 = blockIdx.x * 64;
+  if (t0 >= d) return;
+  for (int e = threadIdx.x; e < 64 * 64; e += 256) {
+    const int r = t0 + (e >> 6), col = t0 + (e & 63);
+    if (r >= d || col >= d) continue;
+    const int br = r / CB, bc = col / CB;
+    float v;
+    if (bc > br || col > r) {
+      v = 0.f;
+    } else if (bc == br) {
+      // D^-1 of the 32-block starting at p0: strict lower part stored
+      // transposed above the diagonal of L's diagonal block, diagonal 1/L_ii
+      const int p0 = br * CB;
+      v = col == r ? 1.f / c.a[int64_t(r) * d + r] : c.a[int64_t(col) * d + p0 + (r - p0)];
+    } else {
+      continue;      // lower-left 32x32 block: level 0
     }
-    for (int ch = 0; ch < nch; ++ch) {
-      float (*lb)[CBP] = ls[ch & 1];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int e = tid + q * CINV_THREADS;
-        lb[e >> 5][e & 31] = lreg[q];
-      }
-      __syncthreads();
-      const int k0 = c0 + ch * CB;
-      if (ch + 1 < nch) load_chunk(k0 + CB);
-#pragma unroll 8
-      for (int kk = 0; kk < CB; ++kk) {
-        const float l = lb[orow][kk];
-        const float4 yv = *reinterpret_cast<const float4*>(&y[(k0 + kk) * CB + ocol]);
-        acc[0] -= l * yv.x; acc[1] -= l * yv.y; acc[2] -= l * yv.z; acc[3] -= l * yv.w;
-      }
-    }
-#pragma unroll
-    for (int v = 0; v < 4; ++v) acc_s[orow][ocol + v] = acc[v];
-    // D^-1 goes to the chunk buffer the last chunk did not use (keeps two
-    // blocks per SM within shared memory)
-    float (*dv)[CBP] = ls[nch & 1];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int e = tid + q * CINV_THREADS;
-      dv[e >> 5][e & 31] = dreg[q];
+    c.inv[int64_t(r) * d + col] = v;
+  }
+}
+
+// One product of a doubling level (grid.x: pair x output tile, grid.y:
+// matrix), 64x64 output tiles, 4x4 per thread, K staged 32 at a time.
+// mode 0: T = C A^-1, mode 1: X21 = -B^-1 T.
+constexpr int LV_T = 64, LV_K = 32, LV_THREADS = 256;
+__global__ void __launch_bounds__(LV_THREADS) linv_level_kernel(const CholDesc* __restrict__ descs, int s, int mode) {
+  pdl_wait();      // previous kernel's results visible (no-op without PDL)
+  const CholDesc& c = descs[blockIdx.y];
+  const int d = c.d;
+  if (d <= s) return;
+  const int tiles = (s + LV_T - 1) / LV_T;                // per side of a pair's output
+  const int pair = blockIdx.x / (tiles * tiles);
+  const int rem = blockIdx.x % (tiles * tiles);
+  const int r0 = 2 * s * pair;
+  if (r0 + s >= d) return;                                // no second block
+  const int s2 = min(s, d - r0 - s);
+  const int it = rem / tiles, jt = rem % tiles;
+  const int i0 = it * LV_T, j0 = jt * LV_T;               // output tile, relative to (r0 + s, r0)
+  if (i0 >= s2) return;
+  // K range: mode 0, k in [j0, s) (A^-1 lower); mode 1, k in [0, min(i0 + 64, s2)) (B^-1 lower)
+  const int klo = mode == 0 ? j0 : 0;
+  const int khi = mode == 0 ? s : min(i0 + LV_T, s2);
+  // P[i][k], Q[k][j] (relative indices) and the output, as row-major views
+  const float* P = mode == 0 ? c.a + int64_t(r0 + s) * d + r0 : c.inv + int64_t(r0 + s) * d + (r0 + s);
+  const float* Q = mode == 0 ? c.inv + int64_t(r0) * d + r0 : c.t + int64_t(r0 + s) * d + r0;
+  float* O = mode == 0 ? c.t + int64_t(r0 + s) * d + r0 : c.inv + int64_t(r0 + s) * d + r0;
+  const int kdim = mode == 0 ? s : s2;                    // valid k of the operands
+  __shared__ __align__(16) float ps[LV_K][LV_T + 4];     // P transposed: ps[k][i]
+  __shared__ __align__(16) float qs[LV_K][LV_T];
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  float acc[4][4] = {};
+  for (int k0 = klo; k0 < khi; k0 += LV_K) {
+    for (int e = tid; e < LV_T * LV_K; e += LV_THREADS) {
+      const int i = e >> 5, k = e & 31;                   // P: 32 consecutive k per row
+      const int gi = i0 + i, gk = k0 + k;
+      ps[k][i] = (gi < s2 && gk < khi && gk < kdim) ? P[int64_t(gi) * d + gk] : 0.f;
+      const int qk = e >> 6, qj = e & 63;                 // Q: 64 consecutive j per row
+      const int hk = k0 + qk, hj = j0 + qj;
+      qs[qk][qj] = (hk < khi && hk < kdim && hj < s) ? Q[int64_t(hk) * d + hj] : 0.f;
     }
     __syncthreads();
-    // Y_block = D^-1 * acc
-    {
-      float out[4] = {0.f, 0.f, 0.f, 0.f};
-      for (int k = 0; k <= orow; ++k) {
-        const float dk = dv[orow][k];
+#pragma unroll 8
+    for (int kk = 0; kk < LV_K; ++kk) {
+      const float4 a = *reinterpret_cast<const float4*>(&ps[kk][ty * 4]);
+      const float4 b = *reinterpret_cast<const float4*>(&qs[kk][tx * 4]);
+      const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-        for (int v = 0; v < 4; ++v) out[v] += dk * acc_s[k][ocol + v];
-      }
-      if (r < d) *reinterpret_cast<float4*>(&y[r * CB + ocol]) = make_float4(out[0], out[1], out[2], out[3]);
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) acc[u][v] += av[u] * bv[v];
     }
     __syncthreads();
   }
-  // ---- columns c0 .. c0+31 of L^-1 ----
-  const int rw = c0 & ~63;
-  for (int e = tid; e < (d - rw) * CB; e += CINV_THREADS) {
-    const int i = rw + e / CB, j = e % CB;
-    if (c0 + j < d) c.inv[int64_t(i) * d + c0 + j] = i < c0 ? 0.f : y[i * CB + j];
+  const float sign = mode == 0 ? 1.f : -1.f;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int i = i0 + ty * 4 + u;
+    if (i >= s2) continue;
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      const int j = j0 + tx * 4 + v;
+      if (j < s) O[int64_t(i) * d + j] = sign * acc[u][v];
+    }
   }
 }
 
