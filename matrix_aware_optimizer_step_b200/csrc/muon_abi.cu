@@ -21,6 +21,7 @@
 #include <map>
 #include <mutex>
 #include <string>
+#include <tuple>
 #include <vector>
 
 #include "../../include/muon.h"
@@ -1410,7 +1411,17 @@ muon_status muon_newton_refresh(muon_ctx* ctx, const muon_act_desc* acts, int32_
   size_t s_total = 0, xt_total = 0;
   int max_d = 0;
   int64_t max_tiles = 0;
-  for (int i = 0; i < n; ++i) {
+  // activations of one (tokens, d, nblocks) next to each other, so each
+  // shape is one batched problem of the second-moment product
+  std::vector<int> order(n);
+  for (int i = 0; i < n; ++i) order[i] = i;
+  auto key = [&](int i) {
+    const int64_t nb = acts[i].nblocks >= 1 ? acts[i].nblocks : 1;
+    return std::make_tuple(acts[i].tokens, acts[i].width / nb, acts[i].nblocks);
+  };
+  std::stable_sort(order.begin(), order.end(), [&](int x, int y) { return key(x) < key(y); });
+  for (int oi = 0; oi < n; ++oi) {
+    const int i = order[oi];
     const muon_act_desc& a = acts[i];
     if (!a.acts || !a.s_inv) return fail(ctx, MUON_ERR_INVALID_ARG, "activation %d: NULL pointer", i);
     if (a.act_dtype != MUON_BF16) return fail(ctx, MUON_ERR_UNSUPPORTED, "activation %d: bf16 only", i);
@@ -1443,7 +1454,7 @@ muon_status muon_newton_refresh(muon_ctx* ctx, const muon_act_desc* acts, int32_
       if (!gp.empty() && gp.back().tokens == a.tokens && gp.back().d == d && (!direct || gp.back().nb == a.nblocks)) {
         gp.back().count++;
       } else {
-        gp.push_back(GramProb{a.tokens, d, ldt, 1, a.nblocks, i, xt_total, s_total, int64_t(s_bytes / 4)});
+        gp.push_back(GramProb{a.tokens, d, ldt, 1, a.nblocks, oi, xt_total, s_total, int64_t(s_bytes / 4)});
       }
       if (!direct) xt_total += size_t(d) * ldt * 2;
       s_total += s_bytes;
@@ -1470,11 +1481,14 @@ muon_status muon_newton_refresh(muon_ctx* ctx, const muon_act_desc* acts, int32_
     c.t = reinterpret_cast<float*>(ws + s_region + reinterpret_cast<size_t>(c.a));
     c.a = reinterpret_cast<float*>(ws + reinterpret_cast<size_t>(c.a));
   }
-  // in place: one map per activation over its whole tokens x width matrix
+  // in place: one map per activation over its whole tokens x width matrix,
+  // in the sorted order
   std::vector<PrecondMaps> pmaps(direct ? n : 0);
-  for (int i = 0; direct && i < n; ++i)
-    if (!encode_bf16_3d(&pmaps[i].a, acts[i].acts, acts[i].width, acts[i].tokens, 1, acts[i].width, 64, 64))
+  for (int oi = 0; direct && oi < n; ++oi) {
+    const muon_act_desc& a = acts[order[oi]];
+    if (!encode_bf16_3d(&pmaps[oi].a, a.acts, a.width, a.tokens, 1, a.width, 64, 64))
       return fail(ctx, MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed (second moment)");
+  }
   const size_t ab_bytes = round_up(ab.size() * sizeof(ActBlock), kAlign);
   const size_t pm_off = round_up(ab_bytes + cd.size() * sizeof(CholDesc), kAlign);
   std::vector<uint8_t> table(pm_off + pmaps.size() * sizeof(PrecondMaps));
