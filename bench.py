@@ -87,10 +87,11 @@ def step_work(w, aux, ns_steps=5):
     for _, tokens, width in w.acts:
         nb = 4 if width > 768 else 1
         d = width // nb
-        # second moment on the tensor cores; Cholesky (d^3/3 FMA), L^-1 (d^3/6)
-        # and L^-T L^-1 (d^3/6) on the fp32 ALUs
+        # second moment on the tensor cores; Cholesky, L^-1 and L^-T L^-1 on
+        # the fp32 ALUs, d^3/3 FLOPs each (the LAPACK counts of potrf, trtri
+        # and lauum)
         refresh_tc += nb * 2 * tokens * d * d
-        refresh_alu += nb * 2 * (d ** 3 // 3 + d ** 3 // 3)
+        refresh_alu += nb * 3 * (d ** 3 // 3)
     for m in w.mats:
         a, b = min(m.rows, m.cols), max(m.rows, m.cols)
         gram += 2 * a * a * b * ns_steps
