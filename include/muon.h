@@ -245,6 +245,13 @@ MUON_API muon_status muon_newton_refresh(muon_ctx* ctx, const muon_act_desc* act
 MUON_API muon_status muon_newton_precondition(muon_ctx* ctx, const muon_group* groups, int32_t ngroups,
                                      void* stream);
 
+/* Failure-detection self test: enqueues one kernel whose single bounded
+ * wait (an mbarrier that nothing completes) runs out after its 2 s limit,
+ * records the timeout in the context's device flags and returns; nothing
+ * faults or hangs and the context stays usable.  The next
+ * muon_check_device() returns MUON_ERR_TIMEOUT and clears the flag. */
+MUON_API muon_status muon_selftest_wait(muon_ctx* ctx, void* stream);
+
 /* Synchronise the context's last stream and report device-side flags:
  * MUON_ERR_TIMEOUT if a bounded wait gave up since the last check (the flag
  * is cleared), MUON_ERR_CUDA on an asynchronous CUDA error, else MUON_OK. */

@@ -34,7 +34,7 @@ EXPORTED = [
     "muon_last_error", "muon_status_string", "muon_query_workspace", "muon_set_workspace",
     "muon_step", "muon_orthogonalize", "muon_adamw_step", "muon_newton_refresh",
     "muon_newton_precondition",
-    "muon_check_device", "muon_launch_count", "muon_profile_enable", "muon_profile_read",
+    "muon_check_device", "muon_selftest_wait", "muon_launch_count", "muon_profile_enable", "muon_profile_read",
     "muon_orthogonalize_noalloc", "muon_partition",
 ]
 
@@ -122,6 +122,7 @@ def load_library() -> ctypes.CDLL:
         "muon_newton_refresh": (st, [vp, ctypes.POINTER(ActDesc), i32, ctypes.c_float, vp]),
         "muon_newton_precondition": (st, [vp, ctypes.POINTER(Group), i32, vp]),
         "muon_check_device": (st, [vp]),
+        "muon_selftest_wait": (st, [vp, vp]),
         "muon_launch_count": (ctypes.c_uint64, [vp]),
         "muon_profile_enable": (st, [vp, ctypes.c_int]),
         "muon_profile_read": (st, [vp, ctypes.POINTER(KernelTimes)]),
@@ -390,6 +391,11 @@ class MuonContext:
 
     def check_device(self):
         self._check(self._lib.muon_check_device(self._ctx), "muon_check_device")
+
+    def selftest_wait(self, stream=None):
+        """Enqueue the failure-detection self test: a bounded device-side
+        wait that runs out (2 s); check_device() then raises MUON_ERR_TIMEOUT."""
+        self._check(self._lib.muon_selftest_wait(self._ctx, _stream_ptr(stream)), "muon_selftest_wait")
 
     @property
     def launch_count(self) -> int:

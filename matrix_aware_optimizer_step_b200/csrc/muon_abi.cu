@@ -1159,6 +1159,22 @@ muon_status noalloc_scratch_address(int device, uint8_t** out) {
 // ===========================================================================
 // extern "C"
 // ===========================================================================
+// Failure detection without a fault: one thread waits on an mbarrier that
+// nothing completes.  The bounded wait gives up after its limit (2 s of
+// %globaltimer), records kDevErrTimeout in the context's flags and the
+// kernel returns, leaving the context usable.
+__global__ void selftest_wait_kernel(int* err) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, err, &abort_flag);
+}
+
 extern "C" {
 
 void muon_default_hparams(muon_hparams* hp) {
@@ -1614,6 +1630,19 @@ muon_status muon_check_device(muon_ctx* ctx) {
       return fail(ctx, MUON_ERR_INVALID_ARG, "a second moment was not positive definite (flags 0x%x)", flags);
     return fail(ctx, MUON_ERR_CUDA, "device error flags 0x%x", flags);
   }
+  return MUON_OK;
+}
+
+muon_status muon_selftest_wait(muon_ctx* ctx, void* stream) {
+  if (!ctx) return MUON_ERR_INVALID_ARG;
+  muon_status s = set_device(ctx);
+  if (s != MUON_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  ctx->last_stream = st;
+  CUDA_TRY(ctx, cudaGetLastError());
+  selftest_wait_kernel<<<1, 32, 0, st>>>(ctx->dflags);
+  ctx->launches++;
+  CUDA_TRY(ctx, cudaGetLastError());
   return MUON_OK;
 }
 

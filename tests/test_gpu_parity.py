@@ -258,6 +258,25 @@ def test_nonfinite_gradient_is_rejected(ctx, mx):
     assert not torch.all(w == 1)
 
 
+def test_bounded_wait_reports_timeout_and_context_survives(ctx, mx):
+    """Failure detection without a fault: a kernel waits on an mbarrier that
+    nothing completes; its bounded wait gives up after 2 s, the timeout
+    surfaces as MUON_ERR_TIMEOUT from check_device, the flag is cleared, and
+    the context keeps computing correct results."""
+    ctx.check_device()
+    ctx.selftest_wait()
+    with pytest.raises(mx.MuonError) as e:
+        ctx.check_device()
+    assert e.value.status == mx.binding.MUON_ERR_TIMEOUT
+    ctx.check_device()
+    g = wl.np_normal((256, 256), 1.0, seed=17, index=0)
+    out = torch.empty((256, 256), device="cuda")
+    ctx.orthogonalize([dev(g)], [out])
+    torch.cuda.synchronize()
+    ctx.check_device()
+    assert rel_fro(to_np(out), oracle.newton_schulz(g, 5)) < NS_TOL
+
+
 def test_workspace_cap_and_caller_workspace(ctx, mx):
     """A bounded workspace (chunked execution) and a caller-owned workspace
     give the same result as the library's own."""
