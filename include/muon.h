@@ -153,7 +153,7 @@ typedef struct {
  * (X_b^T X_b / tokens + damping I)^-1. */
 typedef struct {
   const void* acts;
-  int32_t act_dtype;               /* muon_dtype; MUON_BF16 only in this build */
+  int32_t act_dtype;               /* muon_dtype: MUON_BF16 or MUON_F32 */
   int32_t nblocks;
   int64_t tokens;
   int64_t width;
@@ -162,39 +162,63 @@ typedef struct {
 
 typedef struct muon_ctx muon_ctx;
 
-/* Defaults of the first page ("Usage", "Hyperparameter tuning") and the
- * blog's coefficients: lr 0.02, momentum 0.95, weight decay 0.01, eps 1e-7,
- * a b c = 3.4445 -4.7750 2.0315, Nesterov on, 5 steps, ORIGINAL scale. */
+/* Source: "Muon: An optimizer for the hidden layers of neural networks",
+ * sections "Usage" and "Hyperparameter tuning" (lr 0.02, momentum 0.95,
+ * weight decay 0.01, Nesterov, 5 steps); "Muon: when the LLM optimizer
+ * treats weight matrices as matrices", section 3 (a b c = 3.4445 -4.7750
+ * 2.0315).  Fills *hp with those defaults, eps 1e-7 and the ORIGINAL scale;
+ * hp NULL: no effect. */
 MUON_API void muon_default_hparams(muon_hparams* hp);
-/* AdamW defaults of the first page: lr 3e-4, betas 0.9 / 0.95, eps 1e-8,
- * weight decay 0.01. */
+/* Source: "Muon: An optimizer for the hidden layers of neural networks",
+ * section "Usage" (AdamW for the non-hidden parameters: lr 3e-4, betas 0.9 /
+ * 0.95, weight decay 0.01).  Fills *hp with those and eps 1e-8. */
 MUON_API void muon_default_adamw_hparams(muon_adamw_hparams* hp);
 
-/* Create a context on CUDA device `device`.  workspace_bytes == 0: the
+/* Source: "Muon: An optimizer for the hidden layers of neural networks",
+ * section "Usage" (the optimizer is constructed once over the parameter
+ * groups and stepped every iteration); the context is that optimizer's
+ * device-side state.
+ * Create a context on CUDA device `device`.  workspace_bytes == 0: the
  * library allocates and grows its own workspace as needed.  Otherwise the
  * library allocates exactly that much once and splits larger requests into
  * chunks that fit; a single matrix that does not fit returns
- * MUON_ERR_WORKSPACE.  *ctx is NULL on failure. */
+ * MUON_ERR_WORKSPACE.  *ctx is NULL on failure.  Errors: ctx NULL or a bad
+ * device -> MUON_ERR_INVALID_ARG; a device that is not sm_100 ->
+ * MUON_ERR_UNSUPPORTED; a failed CUDA call -> MUON_ERR_CUDA. */
 MUON_API muon_status muon_init(muon_ctx** ctx, int device, size_t workspace_bytes);
 
-/* Release the context, its workspace and tables (synchronises the device). */
+/* No counterpart on the pages (resource management).  Release the context,
+ * its workspace and tables (synchronises the device).  NULL: no effect. */
 MUON_API void muon_destroy(muon_ctx* ctx);
 
-/* Human-readable description of the context's last error ("" if none). */
+/* No counterpart on the pages (error reporting).  Human-readable
+ * description of the context's last error ("" if none); the string is owned
+ * by the context and valid until its next call. */
 MUON_API const char* muon_last_error(const muon_ctx* ctx);
+/* No counterpart on the pages (error reporting).  Static name of a status
+ * code ("MUON_OK", ...). */
 MUON_API const char* muon_status_string(muon_status s);
 
-/* Workspace bytes a muon_step / muon_orthogonalize over these groups needs
- * to run in one chunk. */
+/* No counterpart on the pages (memory planning).  Workspace bytes a
+ * muon_step / muon_orthogonalize over these groups needs to run in one
+ * chunk, written to *bytes; host only.  Errors as muon_step's argument
+ * checks. */
 MUON_API muon_status muon_query_workspace(const muon_group* groups, int32_t ngroups, size_t* bytes);
 
-/* Hand the context a caller-owned device workspace (e.g. a torch tensor).
+/* No counterpart on the pages (memory planning).
+ * Hand the context a caller-owned device workspace (e.g. a torch tensor).
  * It is used instead of the library's own until replaced; the caller keeps
  * it alive and unmodified while work enqueued with it may run.  ptr must be
  * 256-byte aligned.  ptr == NULL returns to library-owned workspace. */
 MUON_API muon_status muon_set_workspace(muon_ctx* ctx, void* ptr, size_t bytes);
 
-/* One Muon step over ngroups groups: for every matrix, Nesterov momentum,
+/* Source: "Muon: An optimizer for the hidden layers of neural networks",
+ * sections "Usage" and "Hyperparameter tuning"; "Muon: when the LLM
+ * optimizer treats weight matrices as matrices", section 1 (the moving-
+ * average form of momentum), section 3 (Frobenius normalisation and the
+ * quintic iteration in bf16) and the PyTorch set-up after section 4 (shape
+ * scale, decoupled weight decay).
+ * One Muon step over ngroups groups: for every matrix, Nesterov momentum,
  * Frobenius normalisation, hp->ns_steps quintic Newton-Schulz iterations in
  * bf16 with fp32 accumulation (on the transpose when rows > cols), then
  * W <- W (1 - lr wd) - lr scale O.
@@ -212,21 +236,47 @@ MUON_API muon_status muon_set_workspace(muon_ctx* ctx, void* ptr, size_t bytes);
 MUON_API muon_status muon_step(muon_ctx* ctx, const muon_group* groups, int32_t ngroups,
                       const muon_hparams* hp, void* stream);
 
-/* Frobenius normalisation plus hp->ns_steps Newton-Schulz iterations only
- * (uses hp->eps, ns_a/b/c, ns_steps). */
+/* Source: "Muon: when the LLM optimizer treats weight matrices as
+ * matrices", section 3 (X = G / ||G||_F, then the quintic iteration).
+ * Frobenius normalisation plus hp->ns_steps Newton-Schulz iterations only
+ * (uses hp->eps, ns_a/b/c, ns_steps): outputs[i] (fp32) = NS(inputs[i]),
+ * computed as in muon_step.  Errors as muon_step. */
 MUON_API muon_status muon_orthogonalize(muon_ctx* ctx, const muon_ns_group* groups, int32_t ngroups,
                                const muon_hparams* hp, void* stream);
 
-/* Aux AdamW over n tensors; step counts from 1 (bias correction). */
+/* Source: "Muon: An optimizer for the hidden layers of neural networks",
+ * section "Usage" (every parameter that is not a hidden 2-D weight goes to
+ * AdamW); "Muon: when the LLM optimizer treats weight matrices as
+ * matrices", section 1 (the first and second moments).  Bias-corrected
+ * AdamW with decoupled weight decay over n tensors, in place on param,
+ * exp_avg, exp_avg_sq; step counts from 1.  Errors: step < 1, betas outside
+ * [0, 1), eps <= 0, NULL pointers -> MUON_ERR_INVALID_ARG, before any
+ * launch. */
 MUON_API muon_status muon_adamw_step(muon_ctx* ctx, const muon_adamw_tensor* tensors, int32_t n,
                             const muon_adamw_hparams* hp, int64_t step, void* stream);
 
-/* Newton-Muon refresh: for each descriptor, the second moment of each
- * column block and its inverse (Cholesky in fp32). */
+/* Source: "The Newton-Muon Optimizer", section "What Is Newton-Muon?" (the
+ * refresh half of the refresh/apply step: the activation second moment,
+ * one d x d estimate per layer input, four d x d blocks for the MLP
+ * contraction, and its inverse).
+ * For each descriptor, S_b = X_b^T X_b / tokens (+ damping I) of every
+ * d-wide column block b and S_b^-1 (fp32 Cholesky, fp32 inverse) into
+ * s_inv.  The signature takes an array of activation descriptors and one
+ * damping instead of a single activation, so that every layer input of a
+ * model refreshes in one call and same-shape blocks share one batched
+ * second-moment launch.  bf16 activations are read in place when every
+ * width and block width is a multiple of 8 (else through transposed
+ * copies); fp32 activations are split into bf16 high and low parts whose
+ * three significant cross products are accumulated in fp32.  Errors: NULL
+ * or unaligned pointers, a bad shape, damping < 0 -> MUON_ERR_INVALID_ARG;
+ * a block width above 4096 -> MUON_ERR_UNSUPPORTED; all before any launch.
+ * A second moment that is not positive definite is reported by
+ * muon_check_device(). */
 MUON_API muon_status muon_newton_refresh(muon_ctx* ctx, const muon_act_desc* acts, int32_t n,
                                 float damping, void* stream);
 
-/* Newton-Muon right-preconditioning on its own ("What Is Newton-Muon?",
+/* Source: "The Newton-Muon Optimizer", section "What Is Newton-Muon?".
+ * Newton-Muon right-preconditioning on its own ("What Is Newton-Muon?",
  * the update rule with the gradient replaced by G S^-1, block-diagonal over
  * precond_blocks column blocks): for every matrix of every group,
  *   update_out[i] (fp32 rows x cols) = grads[i] [S_1^-1, ..., S_nb^-1]
@@ -245,22 +295,33 @@ MUON_API muon_status muon_newton_refresh(muon_ctx* ctx, const muon_act_desc* act
 MUON_API muon_status muon_newton_precondition(muon_ctx* ctx, const muon_group* groups, int32_t ngroups,
                                      void* stream);
 
-/* Failure-detection self test: enqueues one kernel whose single bounded
+/* No counterpart on the pages (failure detection).
+ * Failure-detection self test: enqueues one kernel whose single bounded
  * wait (an mbarrier that nothing completes) runs out after its 2 s limit,
  * records the timeout in the context's device flags and returns; nothing
  * faults or hangs and the context stays usable.  The next
  * muon_check_device() returns MUON_ERR_TIMEOUT and clears the flag. */
 MUON_API muon_status muon_selftest_wait(muon_ctx* ctx, void* stream);
 
-/* Synchronise the context's last stream and report device-side flags:
- * MUON_ERR_TIMEOUT if a bounded wait gave up since the last check (the flag
- * is cleared), MUON_ERR_CUDA on an asynchronous CUDA error, else MUON_OK. */
+/* No counterpart on the pages (failure detection).
+ * Synchronise the device and report the context's device-side flags:
+ * MUON_ERR_TIMEOUT if a bounded wait gave up since the last check,
+ * MUON_ERR_INVALID_ARG if a refreshed second moment was not positive
+ * definite, MUON_ERR_CUDA on an asynchronous CUDA error, else MUON_OK.  The
+ * flags are cleared.  While a flag is set, every kernel of later muon_step,
+ * muon_orthogonalize, muon_adamw_step and muon_newton_precondition calls on
+ * this context returns without writing, so a step that lost a product
+ * part-way never applies a half-computed update; call this function to
+ * learn of the error and resume. */
 MUON_API muon_status muon_check_device(muon_ctx* ctx);
 
-/* Number of kernels this context has launched since creation. */
+/* No counterpart on the pages (instrumentation).  Number of kernels this
+ * context has launched since creation. */
 MUON_API uint64_t muon_launch_count(const muon_ctx* ctx);
 
-/* Owner-computes sharding across `world` ranks (host only, no GPU needed):
+/* No counterpart on the pages (multi-GPU placement; the pages train on one
+ * GPU).
+ * Owner-computes sharding across `world` ranks (host only, no GPU needed):
  * every matrix i of shape rows[i] x cols[i] is an independent unit of the
  * step, so each goes to one owner rank, which alone keeps its momentum and
  * runs its Muon step; owners then send the updated weights to the other
@@ -286,7 +347,8 @@ typedef enum {
   MUON_K_PRECONDITION = 7,
   MUON_K_OTHER = 8,      /* finite scan                                    */
   MUON_K_UPDATE_APPLY = 9, /* last update with the weight step in its epilogue */
-  MUON_K_COUNT = 10
+  MUON_K_NS_SMALL = 10,  /* every iteration of matrices up to 256 x 256 in one launch */
+  MUON_K_COUNT = 11
 } muon_kernel_kind;
 
 typedef struct {
@@ -294,14 +356,17 @@ typedef struct {
   uint64_t launches[MUON_K_COUNT];
 } muon_kernel_times;
 
-/* enable != 0: bracket every launch with CUDA events on its stream (a few
+/* No counterpart on the pages (instrumentation).
+ * enable != 0: bracket every launch with CUDA events on its stream (a few
  * microseconds of host time per launch; the GPU work is unchanged). */
 MUON_API muon_status muon_profile_enable(muon_ctx* ctx, int enable);
-/* Wait for the recorded launches, add their event-measured durations into
+/* No counterpart on the pages (instrumentation).
+ * Wait for the recorded launches, add their event-measured durations into
  * *out (zeroed first) and reset the accumulators. */
 MUON_API muon_status muon_profile_read(muon_ctx* ctx, muon_kernel_times* out);
 
-/* Newton-Schulz of ONE matrix for callers that cannot allocate device
+/* No counterpart on the pages (an allocation-free variant).
+ * Newton-Schulz of ONE matrix for callers that cannot allocate device
  * memory -- code running where cudaMalloc is off limits, such as inside a
  * host that manages every device byte itself, a custom allocator's
  * callback, or a process whose memory pool must not grow.  The sources have
@@ -331,8 +396,11 @@ MUON_API muon_status muon_profile_read(muon_ctx* ctx, muon_kernel_times* out);
  * device: calls whose work overlaps on one GPU (different streams, or
  * threads without ordering) race and corrupt each other's results, so order
  * them on one stream.  The array keeps the last call's contents; each call
- * clears the parts that must start at zero.  Device-side wait timeouts are
- * not reported by this entry point. */
+ * clears the parts that must start at zero.  The call copies nothing from
+ * the host: its one descriptor travels as a kernel parameter.  If a bounded
+ * device-side wait gives up during the call, its remaining kernels do
+ * nothing and the output is filled with NaN, so the caller can tell a
+ * result that is not valid from the output alone. */
 MUON_API muon_status muon_orthogonalize_noalloc(const void* input, int32_t in_dtype, int64_t rows,
                                                 int64_t cols, float* output, const muon_hparams* hp,
                                                 void* stream);

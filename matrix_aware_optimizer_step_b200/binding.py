@@ -39,7 +39,7 @@ EXPORTED = [
 ]
 
 KERNEL_KINDS = ["momentum", "gram", "poly", "update", "apply", "adamw", "newton_refresh",
-                "precondition", "other", "update_apply"]
+                "precondition", "other", "update_apply", "ns_small"]
 
 
 class MuonError(RuntimeError):
@@ -363,7 +363,7 @@ class MuonContext:
     def newton_refresh(self, acts: Sequence, s_invs: Sequence, nblocks: Sequence[int],
                        damping: float = 0.0, stream=None):
         """s_invs[i] (fp32, nblocks[i] x d x d) = inverse second moments of
-        the column blocks of acts[i] (bf16 tokens x width)."""
+        the column blocks of acts[i] (bf16 or fp32 tokens x width)."""
         n = len(acts)
         arr = (ActDesc * max(1, n))()
         for i in range(n):

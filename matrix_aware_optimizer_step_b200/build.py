@@ -18,7 +18,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmuon_b200.so")
 SOURCES = ["muon_abi.cu"]
-HEADERS = ["sm100_ptx.cuh", "ns_gemm.cuh", "elementwise.cuh", "newton.cuh"]
+HEADERS = ["sm100_ptx.cuh", "ns_gemm.cuh", "elementwise.cuh", "newton.cuh", "small_ns.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

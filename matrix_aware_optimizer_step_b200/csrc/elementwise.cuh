@@ -121,7 +121,7 @@ __global__ void __launch_bounds__(EW_THREADS)
     momentum_kernel(const MatDesc* __restrict__ descs, const __grid_constant__ SegTable segs, int64_t tile_base,
                     float beta, int nesterov, const int* skip) {
   pdl_wait();      // previous kernel's results visible (no-op without PDL)
-  if (skip != nullptr && *skip) return;
+  if (halted(skip)) return;
   __shared__ __align__(16) __nv_bfloat16 tile[EW_TILE][EW_TILE];
   __shared__ float red[EW_THREADS / 32];
   const int64_t gt = tile_base + blockIdx.x;
@@ -136,26 +136,41 @@ __global__ void __launch_bounds__(EW_THREADS)
     // 256 consecutive elements (the matrix has at least as many 64x64 tiles
     // as 4096-element runs; the blocks past its end store a zero partial).
     const int64_t n = d.rows * d.cols;
+    // both vectors' loads are issued before any store (the stores could
+    // alias the loads as far as the compiler knows, so it would not hoist
+    // them), doubling the bytes each thread has in flight
+    float g[2][8], b[2][8];
+    bool in[2];
 #pragma unroll
     for (int it = 0; it < 2; ++it) {
       const int64_t e = lt * (EW_TILE * EW_TILE) + (threadIdx.x + it * EW_THREADS) * 8;
-      if (e >= n) continue;
-      float g[8], u[8];
-      load8_grad(d.grad, d.grad_dtype, e, g);
+      in[it] = e < n;
+      if (!in[it]) continue;
+      load8_grad(d.grad, d.grad_dtype, e, g[it]);
       if (MODE == 0) {
-        float4* bp = reinterpret_cast<float4*>(d.momentum + e);
+        const float4* bp = reinterpret_cast<const float4*>(d.momentum + e);
         const float4 b0 = bp[0], b1 = bp[1];
-        float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+        b[it][0] = b0.x; b[it][1] = b0.y; b[it][2] = b0.z; b[it][3] = b0.w;
+        b[it][4] = b1.x; b[it][5] = b1.y; b[it][6] = b1.z; b[it][7] = b1.w;
+      }
+    }
+#pragma unroll
+    for (int it = 0; it < 2; ++it) {
+      if (!in[it]) continue;
+      const int64_t e = lt * (EW_TILE * EW_TILE) + (threadIdx.x + it * EW_THREADS) * 8;
+      float u[8];
+      if (MODE == 0) {
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          b[k] = beta * b[k] + (1.f - beta) * g[k];
-          u[k] = nesterov ? (1.f - beta) * g[k] + beta * b[k] : b[k];
+          b[it][k] = beta * b[it][k] + (1.f - beta) * g[it][k];
+          u[k] = nesterov ? (1.f - beta) * g[it][k] + beta * b[it][k] : b[it][k];
         }
-        bp[0] = make_float4(b[0], b[1], b[2], b[3]);
-        bp[1] = make_float4(b[4], b[5], b[6], b[7]);
+        float4* bp = reinterpret_cast<float4*>(d.momentum + e);
+        bp[0] = make_float4(b[it][0], b[it][1], b[it][2], b[it][3]);
+        bp[1] = make_float4(b[it][4], b[it][5], b[it][6], b[it][7]);
       } else {
 #pragma unroll
-        for (int k = 0; k < 8; ++k) u[k] = g[k];
+        for (int k = 0; k < 8; ++k) u[k] = g[it][k];
       }
 #pragma unroll
       for (int k = 0; k < 8; ++k) ss += u[k] * u[k];
@@ -169,7 +184,25 @@ __global__ void __launch_bounds__(EW_THREADS)
     return;
   }
   const bool vec_ok = (d.cols % 8 == 0) && (d.ld % 8 == 0);
-  // 64 rows x 8 vectors of 8 columns = 512 vectors, 2 per thread
+  // 64 rows x 8 vectors of 8 columns = 512 vectors, 2 per thread; the loads
+  // of both are issued before any store
+  float gv[2][8], bv[2][8];
+  bool full[2];
+#pragma unroll
+  for (int it = 0; it < 2; ++it) {
+    const int v = threadIdx.x + it * EW_THREADS;
+    const int64_t r = r0 + (v >> 3), c = c0 + (v & 7) * 8;
+    full[it] = r < d.rows && vec_ok && c + 8 <= d.cols;
+    if (!full[it]) continue;
+    const int64_t idx = r * d.cols + c;
+    load8_grad(d.grad, d.grad_dtype, idx, gv[it]);
+    if (MODE == 0) {
+      const float4* bp = reinterpret_cast<const float4*>(d.momentum + idx);
+      const float4 b0 = bp[0], b1 = bp[1];
+      bv[it][0] = b0.x; bv[it][1] = b0.y; bv[it][2] = b0.z; bv[it][3] = b0.w;
+      bv[it][4] = b1.x; bv[it][5] = b1.y; bv[it][6] = b1.z; bv[it][7] = b1.w;
+    }
+  }
 #pragma unroll
   for (int it = 0; it < 2; ++it) {
     const int v = threadIdx.x + it * EW_THREADS;
@@ -177,24 +210,22 @@ __global__ void __launch_bounds__(EW_THREADS)
     const int64_t r = r0 + rl, c = c0 + cl;
     if (r >= d.rows) continue;
     float u[8];
-    if (vec_ok && c + 8 <= d.cols) {
+    if (full[it]) {
       const int64_t idx = r * d.cols + c;
-      float g[8];
-      load8_grad(d.grad, d.grad_dtype, idx, g);
       if (MODE == 0) {
-        float4* bp = reinterpret_cast<float4*>(d.momentum + idx);
-        float4 b0 = bp[0], b1 = bp[1];
-        float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+        float* b = bv[it];
+        const float* g = gv[it];
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           b[k] = beta * b[k] + (1.f - beta) * g[k];
           u[k] = nesterov ? (1.f - beta) * g[k] + beta * b[k] : b[k];
         }
+        float4* bp = reinterpret_cast<float4*>(d.momentum + idx);
         bp[0] = make_float4(b[0], b[1], b[2], b[3]);
         bp[1] = make_float4(b[4], b[5], b[6], b[7]);
       } else {
 #pragma unroll
-        for (int k = 0; k < 8; ++k) u[k] = g[k];
+        for (int k = 0; k < 8; ++k) u[k] = gv[it][k];
       }
 #pragma unroll
       for (int k = 0; k < 8; ++k) ss += u[k] * u[k];
@@ -255,7 +286,7 @@ __global__ void __launch_bounds__(EW_THREADS)
 // result is the same run to run.
 __global__ void __launch_bounds__(EW_THREADS) norm_reduce_kernel(const MatDesc* __restrict__ descs, const int* skip) {
   pdl_wait();      // previous kernel's results visible (no-op without PDL)
-  if (skip != nullptr && *skip) return;
+  if (halted(skip)) return;
   __shared__ float red[EW_THREADS / 32];
   const MatDesc& d = descs[blockIdx.x];
   const int64_t ntiles = ((d.rows + EW_TILE - 1) / EW_TILE) * d.tiles_c;
@@ -292,7 +323,7 @@ __global__ void __launch_bounds__(EW_THREADS)
     apply_kernel(const MatDesc* __restrict__ descs, const __grid_constant__ SegTable segs, int64_t tile_base,
                  int normalise, float eps, const int* skip) {
   pdl_wait();      // previous kernel's results visible (no-op without PDL)
-  if (skip != nullptr && *skip) return;
+  if (halted(skip)) return;
   __shared__ __align__(16) __nv_bfloat16 tile[EW_TILE][EW_TILE];
   const int64_t gt = tile_base + blockIdx.x;
   const MatDesc& d = descs[seg_find(segs, gt)];
@@ -462,8 +493,9 @@ __device__ __forceinline__ void adam_one(float& p, float g, float& m, float& v, 
 }
 
 __global__ void __launch_bounds__(EW_THREADS)
-    adamw_kernel(const AdamDesc* __restrict__ descs, int n, AdamScalars s) {
+    adamw_kernel(const AdamDesc* __restrict__ descs, int n, AdamScalars s, const int* skip) {
   pdl_wait();      // previous kernel's results visible (no-op without PDL)
+  if (halted(skip)) return;
   const int64_t ch = blockIdx.x;
   const AdamDesc& d = descs[find_adam(descs, n, ch)];
   const int64_t base = (ch - d.chunk_start) * ADAM_CHUNK;

@@ -28,6 +28,7 @@
 #include "elementwise.cuh"
 #include "newton.cuh"
 #include "ns_gemm.cuh"
+#include "small_ns.cuh"
 
 using namespace muon;
 
@@ -108,6 +109,21 @@ bool encode_bf16_3d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t 
   cuuint32_t estr[3] = {1, 1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// bf16 tensor of `batch` matrices rows x ld, `zstride` elements apart,
+// viewed as (cols, rows, batch), 128-byte swizzle.
+bool encode_bf16_3d_strided(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, uint64_t batch,
+                            uint64_t ld, uint64_t zstride, uint32_t box_cols, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {cols, rows, batch};
+  cuuint64_t strides[2] = {ld * 2, zstride * 2};
+  cuuint32_t box[3] = {box_cols, box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -478,13 +494,89 @@ bool encode_run(uint8_t* ws, const Run& r, RunMaps& mp) {
   return ok;
 }
 
+// Runs whose wide shape fits one CTA pair go through small_ns_kernel: all
+// iterations in one launch.
+inline bool small_run(const Run& r) { return r.m <= small_cfg::MAXD && r.n <= small_cfg::MAXD; }
+
+// All ns_steps iterations of the matrices of one small run in one launch;
+// the last update stores the final X at x[ns_steps % 2], or applies the
+// weight step of matrix k from mdesc[k] when mdesc is given.
+muon_status run_small_ns(muon_ctx* ctx, uint8_t* ws, const Run& r, const float* norm2, const muon_hparams* hp,
+                         const int* skip, cudaStream_t st, const MatDesc* mdesc) {
+  static bool attr_done[64] = {};
+  static int max_pairs[64] = {};
+  const int dev = ctx->device & 63;
+  if (!attr_done[dev]) {
+    CUDA_TRY(ctx, cudaFuncSetAttribute(small_ns_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       small_cfg::SMEM));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (device_sms(ctx->device) / 2));
+    cfg.blockDim = dim3(small_cfg::THREADS);
+    cfg.dynamicSmemBytes = small_cfg::SMEM;
+    int np = 0;
+    if (cudaOccupancyMaxActiveClusters(&np, small_ns_kernel, &cfg) != cudaSuccess || np <= 0) {
+      cudaGetLastError();
+      np = device_sms(ctx->device) / 2;
+    }
+    max_pairs[dev] = np;
+    attr_done[dev] = true;
+  }
+  if (hp->ns_steps < 1 || r.count < 1) return MUON_OK;
+  SmallNsArgs a{};
+  a.x_in = reinterpret_cast<const __nv_bfloat16*>(ws + r.off_x0);
+  a.x_out = reinterpret_cast<__nv_bfloat16*>(ws + (hp->ns_steps % 2 ? r.off_x1 : r.off_x0));
+  a.ld = r.ld_n;
+  a.bs = r.m * r.ld_n;
+  a.norm2 = norm2;
+  a.apply = mdesc;
+  a.m = int(r.m);
+  a.n = int(r.n);
+  a.count = r.count;
+  a.steps = hp->ns_steps;
+  a.a = hp->ns_a;
+  a.b = hp->ns_b;
+  a.c = hp->ns_c;
+  a.eps = hp->eps;
+  a.err = ctx->dflags;
+  a.skip = skip;
+  const int pairs = std::min(r.count, max_pairs[dev]);
+  ProfScope ps(ctx, MUON_K_NS_SMALL, st);
+  CUDA_TRY(ctx, launch_pdl(small_ns_kernel, dim3(unsigned(2 * pairs)), dim3(small_cfg::THREADS),
+                           size_t(small_cfg::SMEM), st, a));
+  ctx->launches++;
+  CUDA_TRY(ctx, cudaGetLastError());
+  return MUON_OK;
+}
+
 // ns_steps quintic iterations on the runs of one chunk (X of each run starts
 // in its x0; after the call it is in x[ns_steps % 2]).  norm2s[j] is run j's
-// per-matrix ||U||^2.  Each product of an iteration is one launch over up to
-// MAX_PROBLEMS runs.
-muon_status run_newton_schulz(muon_ctx* ctx, uint8_t* ws, const Run* runs, int nruns,
-                              const float* const* norm2s, const muon_hparams* hp, const int* skip,
-                              cudaStream_t st, const ApplyDesc* const* run_apply = nullptr) {
+// per-matrix ||U||^2.  Runs that fit one CTA pair take one small_ns_kernel
+// launch each; for the others each product of an iteration is one launch
+// over up to MAX_PROBLEMS runs.  When run_apply is given the last product
+// applies the weight step (run_mdesc[j]: the small kernel's per-matrix
+// descriptors of run j).
+muon_status run_newton_schulz(muon_ctx* ctx, uint8_t* ws, const Run* all_runs, int nall,
+                              const float* const* all_norm2s, const muon_hparams* hp, const int* skip,
+                              cudaStream_t st, const ApplyDesc* const* all_apply = nullptr,
+                              const MatDesc* const* run_mdesc = nullptr) {
+  std::vector<Run> big;
+  std::vector<const float*> big_norm2;
+  std::vector<const ApplyDesc*> big_apply;
+  for (int j = 0; j < nall; ++j) {
+    if (small_run(all_runs[j])) {
+      muon_status s = run_small_ns(ctx, ws, all_runs[j], all_norm2s[j], hp, skip, st,
+                                   all_apply != nullptr && run_mdesc != nullptr ? run_mdesc[j] : nullptr);
+      if (s != MUON_OK) return s;
+    } else {
+      big.push_back(all_runs[j]);
+      big_norm2.push_back(all_norm2s[j]);
+      big_apply.push_back(all_apply != nullptr ? all_apply[j] : nullptr);
+    }
+  }
+  const Run* runs = big.data();
+  const int nruns = int(big.size());
+  const float* const* norm2s = big_norm2.data();
+  const ApplyDesc* const* run_apply = all_apply != nullptr ? big_apply.data() : nullptr;
   std::vector<RunMaps> mp(nruns);
   for (int j = 0; j < nruns; ++j)
     if (!encode_run(ws, runs[j], mp[j]))
@@ -750,12 +842,13 @@ muon_status run_precondition_items(muon_ctx* ctx, const std::vector<Item>& items
     launch_pdl(precond_prep_kernel, grid, dim3(256), size_t(0), st, dprep + p0);
     ctx->launches++;
     CUDA_TRY(ctx, cudaGetLastError());
-    s = run_precondition(ctx, std::vector<PreProblem>(probs.begin() + q0, probs.begin() + q1), dpm, nullptr, st);
+    s = run_precondition(ctx, std::vector<PreProblem>(probs.begin() + q0, probs.begin() + q1), dpm, ctx->dflags,
+                         st);
     if (s != MUON_OK) return s;
   }
   if (!pdescs.empty()) {
     launch_pdl(precond_kernel, dim3(unsigned(ptiles)), dim3(PRE_THREADS), size_t(0), st, dpdesc,
-               int(pdescs.size()), static_cast<const int*>(nullptr));
+               int(pdescs.size()), static_cast<const int*>(ctx->dflags));
     ctx->launches++;
     CUDA_TRY(ctx, cudaGetLastError());
   }
@@ -1015,7 +1108,10 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
   const PrecondDesc* dpdesc = reinterpret_cast<const PrecondDesc*>(static_cast<uint8_t*>(dtab) + mat_bytes);
   const PrepDesc* dprep = reinterpret_cast<const PrepDesc*>(static_cast<uint8_t*>(dtab) + mat_bytes + pd_bytes);
 
-  const int* skip = nullptr;
+  // Every kernel of the step gets the context's flags and does nothing once
+  // an error bit (an earlier bounded wait that gave up, a second moment that
+  // was not positive definite) or this step's non-finite flag is set.
+  const int* skip = ctx->dflags;
   if (check) {
     CUDA_TRY(ctx, cudaMemsetAsync(ctx->dflags + 1, 0, sizeof(int), st));
     int64_t tiles = 0;
@@ -1049,7 +1145,6 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
     }
     }
     CUDA_TRY(ctx, cudaGetLastError());
-    skip = ctx->dflags + 1;
   }
 
   for (size_t ci = 0; ci < chunks.size(); ++ci) {
@@ -1097,12 +1192,14 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
       std::vector<const float*> n2(c.runs.size());
       for (size_t j = 0; j < c.runs.size(); ++j) n2[j] = norm2 + (c.runs[j].first - c.first);
       std::vector<const ApplyDesc*> ra;
+      std::vector<const MatDesc*> rm;
       if (chunk_fused[ci]) {
         const ApplyDesc* dapply = reinterpret_cast<const ApplyDesc*>(static_cast<uint8_t*>(dtab) + ap_off);
         for (int64_t k : run_apply_idx[ci]) ra.push_back(dapply + k);
+        for (const Run& r : c.runs) rm.push_back(ddesc + r.first);
       }
       s = run_newton_schulz(ctx, ws, c.runs.data(), int(c.runs.size()), n2.data(), hp, skip, st,
-                            chunk_fused[ci] ? ra.data() : nullptr);
+                            chunk_fused[ci] ? ra.data() : nullptr, chunk_fused[ci] ? rm.data() : nullptr);
       if (s != MUON_OK) return s;
     }
     if (!chunk_fused[ci]) {
@@ -1124,7 +1221,12 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
     int flag = 0;
     CUDA_TRY(ctx, cudaMemcpyAsync(&flag, ctx->dflags + 1, sizeof(int), cudaMemcpyDeviceToHost, st));
     CUDA_TRY(ctx, cudaStreamSynchronize(st));
-    if (flag) return fail(ctx, MUON_ERR_NONFINITE, "a gradient holds NaN or Inf; nothing was updated");
+    if (flag) {
+      // the flag only halts this step's kernels: clear it for the next call
+      CUDA_TRY(ctx, cudaMemsetAsync(ctx->dflags + 1, 0, sizeof(int), st));
+      CUDA_TRY(ctx, cudaStreamSynchronize(st));
+      return fail(ctx, MUON_ERR_NONFINITE, "a gradient holds NaN or Inf; nothing was updated");
+    }
   }
   return MUON_OK;
 }
@@ -1173,6 +1275,24 @@ __global__ void selftest_wait_kernel(int* err) {
   }
   __syncthreads();
   if (threadIdx.x == 0) mbar_wait(&bar, 0, err, &abort_flag);
+}
+
+// muon_orthogonalize_noalloc set-up: the matrix descriptor arrives as a
+// kernel parameter and is stored where the kernels read it; the flags of the
+// previous call are cleared.
+__global__ void noalloc_setup_kernel(const __grid_constant__ MatDesc d, MatDesc* dst, int* flags) {
+  if (threadIdx.x == 0) *dst = d;
+  if (threadIdx.x < 4) flags[threadIdx.x] = 0;
+}
+
+// muon_orthogonalize_noalloc epilogue: when a bounded wait gave up during the
+// call (flags[0] set), the output is filled with NaN, so a caller that cannot
+// query the library's flags still sees that the result is not valid.
+__global__ void noalloc_poison_kernel(const int* flags, float* out, int64_t n) {
+  if (flags[0] == 0) return;
+  const float nan = __int_as_float(0x7fffffff);
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x)
+    out[i] = nan;
 }
 
 extern "C" {
@@ -1395,7 +1515,7 @@ muon_status muon_adamw_step(muon_ctx* ctx, const muon_adamw_tensor* tensors, int
   {
     ProfScope ps(ctx, MUON_K_ADAMW, st);
     launch_pdl(adamw_kernel, dim3(unsigned(chunks)), dim3(EW_THREADS), size_t(0), st,
-        static_cast<const AdamDesc*>(dtab), int(descs.size()), sc);
+        static_cast<const AdamDesc*>(dtab), int(descs.size()), sc, static_cast<const int*>(ctx->dflags));
   }
   ctx->launches++;
   CUDA_TRY(ctx, cudaGetLastError());
@@ -1408,39 +1528,46 @@ muon_status muon_newton_refresh(muon_ctx* ctx, const muon_act_desc* acts, int32_
   if (n < 0 || (n > 0 && !acts)) return fail(ctx, MUON_ERR_INVALID_ARG, "bad activation list");
   if (!(damping >= 0.f) || !std::isfinite(damping)) return fail(ctx, MUON_ERR_INVALID_ARG, "damping must be >= 0");
   // Per d-wide activation block: the fp32 second moment S (then its
-  // Cholesky factor) and the output S^-1.  When every width and block width
-  // is a multiple of 8 elements (16 bytes, the TMA coordinate granule) the
-  // second-moment product reads the activations in place; otherwise each
-  // block is first copied transposed (d x tokens bf16).
+  // Cholesky factor) and the output S^-1.  When every bf16 activation's
+  // width and block width is a multiple of 8 elements (16 bytes, the TMA
+  // coordinate granule) the second-moment product reads the bf16
+  // activations in place; otherwise each bf16 block is first copied
+  // transposed (d x tokens bf16).  An fp32 activation block is split into
+  // bf16 high and low parts, laid out as the two operands of one product
+  // over 3 x tokens (act_split_kernel).
   struct GramProb {
     int64_t tokens, d, ldt;
     int count, nb, pmap_base;
-    size_t xt_off, s_off;
+    int mode;                  // 0: transposed bf16 copy, 1: bf16 in place, 2: split fp32
+    size_t xt_off, xb_off, s_off;
     int64_t s_stride;          // floats between consecutive blocks' S
   };
   bool direct = true;
   for (int i = 0; i < n; ++i)
-    direct = direct && acts[i].nblocks >= 1 && acts[i].width % 8 == 0 && (acts[i].width / acts[i].nblocks) % 8 == 0;
+    if (acts[i].act_dtype == MUON_BF16)
+      direct = direct && acts[i].nblocks >= 1 && acts[i].width % 8 == 0 && (acts[i].width / acts[i].nblocks) % 8 == 0;
   std::vector<ActBlock> ab;
+  std::vector<ActSplitBlock> sbk;
   std::vector<CholDesc> cd;
   std::vector<GramProb> gp;
   size_t s_total = 0, xt_total = 0;
   int max_d = 0;
-  int64_t max_tiles = 0;
-  // activations of one (tokens, d, nblocks) next to each other, so each
-  // shape is one batched problem of the second-moment product
+  int64_t max_tiles = 0, max_split_tiles = 0;
+  // activations of one (dtype, tokens, d, nblocks) next to each other, so
+  // each shape is one batched problem of the second-moment product
   std::vector<int> order(n);
   for (int i = 0; i < n; ++i) order[i] = i;
   auto key = [&](int i) {
     const int64_t nb = acts[i].nblocks >= 1 ? acts[i].nblocks : 1;
-    return std::make_tuple(acts[i].tokens, acts[i].width / nb, acts[i].nblocks);
+    return std::make_tuple(acts[i].act_dtype, acts[i].tokens, acts[i].width / nb, acts[i].nblocks);
   };
   std::stable_sort(order.begin(), order.end(), [&](int x, int y) { return key(x) < key(y); });
   for (int oi = 0; oi < n; ++oi) {
     const int i = order[oi];
     const muon_act_desc& a = acts[i];
     if (!a.acts || !a.s_inv) return fail(ctx, MUON_ERR_INVALID_ARG, "activation %d: NULL pointer", i);
-    if (a.act_dtype != MUON_BF16) return fail(ctx, MUON_ERR_UNSUPPORTED, "activation %d: bf16 only", i);
+    if (a.act_dtype != MUON_BF16 && a.act_dtype != MUON_F32)
+      return fail(ctx, MUON_ERR_INVALID_ARG, "activation %d: act_dtype %d", i, a.act_dtype);
     if (a.tokens < 1 || a.width < 1 || a.nblocks < 1 || a.width % a.nblocks != 0)
       return fail(ctx, MUON_ERR_INVALID_ARG, "activation %d: bad shape", i);
     const int64_t d = a.width / a.nblocks;
@@ -1448,38 +1575,65 @@ muon_status muon_newton_refresh(muon_ctx* ctx, const muon_act_desc* acts, int32_
       return fail(ctx, MUON_ERR_UNSUPPORTED, "activation %d: block width %lld > %d", i, (long long)d, CHOL_MAX_D);
     if (!aligned16(a.acts) || !aligned16(a.s_inv))
       return fail(ctx, MUON_ERR_INVALID_ARG, "activation %d: not 16-byte aligned", i);
-    const int64_t ldt = round_up(a.tokens, 8);
+    const bool split = a.act_dtype == MUON_F32;
+    if (split && 3 * a.tokens > INT32_MAX)
+      return fail(ctx, MUON_ERR_UNSUPPORTED, "activation %d: too many tokens", i);
+    const int mode = split ? 2 : direct ? 1 : 0;
+    // K extent of the operands: tokens, or three segments of tokens (split)
+    const int64_t ldt = round_up(split ? 3 * a.tokens : a.tokens, 8);
     // each block's S starts 256-byte aligned, whatever d is (the Cholesky
     // kernels take 16-byte vector paths when d is a multiple of 4)
     const size_t s_bytes = round_up(size_t(d) * d * 4, kAlign);
+    const size_t op_bytes = round_up(size_t(d) * ldt * 2, kAlign);
     for (int b = 0; b < a.nblocks; ++b) {
-      ActBlock x{};
-      x.acts = static_cast<const __nv_bfloat16*>(a.acts);
-      x.xt = reinterpret_cast<__nv_bfloat16*>(xt_total);    // offset, rebased below
-      x.tokens = a.tokens;
-      x.width = a.width;
-      x.col0 = b * d;
-      x.d = d;
-      x.ldt = ldt;
-      ab.push_back(x);
+      size_t xa_off = xt_total, xb_off = xt_total;
+      if (split) {
+        ActSplitBlock x{};
+        x.acts = static_cast<const float*>(a.acts);
+        xb_off = xt_total + op_bytes;
+        x.xa = reinterpret_cast<__nv_bfloat16*>(xa_off);   // offsets, rebased below
+        x.xb = reinterpret_cast<__nv_bfloat16*>(xb_off);
+        x.tokens = a.tokens;
+        x.width = a.width;
+        x.col0 = b * d;
+        x.d = d;
+        x.ld3 = ldt;
+        sbk.push_back(x);
+        xt_total += 2 * op_bytes;
+        max_split_tiles = std::max<int64_t>(max_split_tiles, cdiv(a.tokens, TPOSE_T) * cdiv(d, TPOSE_T));
+      } else if (!direct) {
+        ActBlock x{};
+        x.acts = static_cast<const __nv_bfloat16*>(a.acts);
+        x.xt = reinterpret_cast<__nv_bfloat16*>(xa_off);    // offset, rebased below
+        x.tokens = a.tokens;
+        x.width = a.width;
+        x.col0 = b * d;
+        x.d = d;
+        x.ldt = ldt;
+        ab.push_back(x);
+        xt_total += op_bytes;
+        max_tiles = std::max<int64_t>(max_tiles, cdiv(a.tokens, TPOSE_T) * cdiv(d, TPOSE_T));
+      }
       CholDesc c{};
       c.a = reinterpret_cast<float*>(s_total);               // offset, rebased below
       c.inv = a.s_inv + size_t(b) * d * d;
       c.d = int(d);
       cd.push_back(c);
-      if (!gp.empty() && gp.back().tokens == a.tokens && gp.back().d == d && (!direct || gp.back().nb == a.nblocks)) {
+      // consecutive blocks of one problem sit op_bytes (or 2 op_bytes) apart
+      // in the operand region and s_bytes apart in the S region
+      if (!gp.empty() && gp.back().mode == mode && gp.back().tokens == a.tokens && gp.back().d == d &&
+          (mode != 1 || gp.back().nb == a.nblocks)) {
         gp.back().count++;
       } else {
-        gp.push_back(GramProb{a.tokens, d, ldt, 1, a.nblocks, oi, xt_total, s_total, int64_t(s_bytes / 4)});
+        gp.push_back(GramProb{a.tokens, d, ldt, 1, a.nblocks, oi, mode, xa_off, xb_off, s_total,
+                              int64_t(s_bytes / 4)});
       }
-      if (!direct) xt_total += size_t(d) * ldt * 2;
       s_total += s_bytes;
       max_d = std::max(max_d, int(d));
-      max_tiles = std::max<int64_t>(max_tiles, cdiv(a.tokens, TPOSE_T) * cdiv(d, TPOSE_T));
     }
   }
-  if (ab.empty()) return MUON_OK;
-  if (ab.size() > 65535) return fail(ctx, MUON_ERR_UNSUPPORTED, "more than 65535 activation blocks");
+  if (cd.empty()) return MUON_OK;
+  if (cd.size() > 65535) return fail(ctx, MUON_ERR_UNSUPPORTED, "more than 65535 activation blocks");
   muon_status s = set_device(ctx);
   if (s != MUON_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -1488,60 +1642,86 @@ muon_status muon_newton_refresh(muon_ctx* ctx, const muon_act_desc* acts, int32_
   const size_t s_region = round_up(s_total, kAlign);
   void* wsv = nullptr;
   // S / L per block, then the recursive L^-1's T per block (same layout),
-  // then the transposed activation copies
+  // then the transposed or split activation copies
   s = ensure_workspace(ctx, 2 * s_region + xt_total, &wsv);
   if (s != MUON_OK) return s;
   uint8_t* ws = static_cast<uint8_t*>(wsv);
-  for (auto& x : ab) x.xt = reinterpret_cast<__nv_bfloat16*>(ws + 2 * s_region + reinterpret_cast<size_t>(x.xt));
+  uint8_t* xt_base = ws + 2 * s_region;
+  for (auto& x : ab) x.xt = reinterpret_cast<__nv_bfloat16*>(xt_base + reinterpret_cast<size_t>(x.xt));
+  for (auto& x : sbk) {
+    x.xa = reinterpret_cast<__nv_bfloat16*>(xt_base + reinterpret_cast<size_t>(x.xa));
+    x.xb = reinterpret_cast<__nv_bfloat16*>(xt_base + reinterpret_cast<size_t>(x.xb));
+  }
   for (auto& c : cd) {
     c.t = reinterpret_cast<float*>(ws + s_region + reinterpret_cast<size_t>(c.a));
     c.a = reinterpret_cast<float*>(ws + reinterpret_cast<size_t>(c.a));
   }
-  // in place: one map per activation over its whole tokens x width matrix,
-  // in the sorted order
+  // in place: one map per bf16 activation over its whole tokens x width
+  // matrix, in the sorted order (fp32 activations leave their slot unused)
   std::vector<PrecondMaps> pmaps(direct ? n : 0);
   for (int oi = 0; direct && oi < n; ++oi) {
     const muon_act_desc& a = acts[order[oi]];
+    if (a.act_dtype != MUON_BF16) continue;
     if (!encode_bf16_3d(&pmaps[oi].a, a.acts, a.width, a.tokens, 1, a.width, 64, 64))
       return fail(ctx, MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed (second moment)");
   }
   const size_t ab_bytes = round_up(ab.size() * sizeof(ActBlock), kAlign);
-  const size_t pm_off = round_up(ab_bytes + cd.size() * sizeof(CholDesc), kAlign);
+  const size_t sb_off = round_up(ab_bytes + cd.size() * sizeof(CholDesc), kAlign);
+  const size_t pm_off = round_up(sb_off + sbk.size() * sizeof(ActSplitBlock), kAlign);
   std::vector<uint8_t> table(pm_off + pmaps.size() * sizeof(PrecondMaps));
-  std::memcpy(table.data(), ab.data(), ab.size() * sizeof(ActBlock));
+  if (!ab.empty()) std::memcpy(table.data(), ab.data(), ab.size() * sizeof(ActBlock));
   std::memcpy(table.data() + ab_bytes, cd.data(), cd.size() * sizeof(CholDesc));
+  if (!sbk.empty()) std::memcpy(table.data() + sb_off, sbk.data(), sbk.size() * sizeof(ActSplitBlock));
   if (!pmaps.empty()) std::memcpy(table.data() + pm_off, pmaps.data(), pmaps.size() * sizeof(PrecondMaps));
   void* dtab = nullptr;
   s = upload_table(ctx, table.data(), table.size(), st, &dtab);
   if (s != MUON_OK) return s;
   const ActBlock* dab = static_cast<const ActBlock*>(dtab);
   const CholDesc* dc = reinterpret_cast<const CholDesc*>(static_cast<uint8_t*>(dtab) + ab_bytes);
+  const ActSplitBlock* dsb = reinterpret_cast<const ActSplitBlock*>(static_cast<uint8_t*>(dtab) + sb_off);
   ProfScope ps(ctx, MUON_K_NEWTON_REFRESH, st);
-  if (!direct) {
+  if (!ab.empty()) {
     launch_pdl(act_transpose_kernel, dim3(unsigned(max_tiles), unsigned(ab.size())), dim3(256), size_t(0), st, dab);
     ctx->launches++;
     CUDA_TRY(ctx, cudaGetLastError());
   }
-  // S = Xt Xt^T / tokens on the tensor cores, up to MAX_PROBLEMS shapes per launch
-  for (size_t b0 = 0; b0 < gp.size(); b0 += MAX_PROBLEMS) {
-    const int nb = int(std::min<size_t>(MAX_PROBLEMS, gp.size() - b0));
+  if (!sbk.empty()) {
+    launch_pdl(act_split_kernel, dim3(unsigned(max_split_tiles), unsigned(sbk.size())), dim3(256), size_t(0), st,
+               dsb);
+    ctx->launches++;
+    CUDA_TRY(ctx, cudaGetLastError());
+  }
+  // S = Xt Xt^T / tokens on the tensor cores, up to MAX_PROBLEMS problems
+  // of one operand mode per launch
+  for (size_t b0 = 0; b0 < gp.size();) {
+    const int mode = gp[b0].mode;
+    int nb = 0;
+    while (nb < MAX_PROBLEMS && b0 + nb < gp.size() && gp[b0 + nb].mode == mode) ++nb;
     GemmMaps maps{};
     GemmArgs g{};
     g.nprob = nb;
     g.err = ctx->dflags;
-    if (direct) g.pmaps = reinterpret_cast<const PrecondMaps*>(static_cast<uint8_t*>(dtab) + pm_off);
+    g.ab_distinct = mode == 2;
+    if (mode == 1) g.pmaps = reinterpret_cast<const PrecondMaps*>(static_cast<uint8_t*>(dtab) + pm_off);
     int tile = 0;
     for (int j = 0; j < nb; ++j) {
       const GramProb& q = gp[b0 + j];
-      if (!direct) {
-        if (!encode_bf16_3d(&maps.a[j], ws + 2 * s_region + q.xt_off, q.tokens, q.d, q.count, q.ldt, 64, 128))
-          return fail(ctx, MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed (second moment)");
-        maps.b[j] = maps.a[j];
+      const int64_t kx = mode == 2 ? 3 * q.tokens : q.tokens;   // K extent
+      if (mode != 1) {
+        // consecutive blocks of the problem: one (or, split, two) operand
+        // copies apart
+        const uint64_t zstride = (mode == 2 ? 2 : 1) * round_up(size_t(q.d) * q.ldt * 2, kAlign) / 2;
+        bool ok = encode_bf16_3d_strided(&maps.a[j], xt_base + q.xt_off, kx, q.d, q.count, q.ldt, zstride, 64, 128);
+        if (mode == 2)
+          ok &= encode_bf16_3d_strided(&maps.b[j], xt_base + q.xb_off, kx, q.d, q.count, q.ldt, zstride, 64, 128);
+        else
+          maps.b[j] = maps.a[j];
+        if (!ok) return fail(ctx, MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed (second moment)");
         maps.aux[j] = maps.a[j];
         maps.out[j] = maps.a[j];
       }
       GemmProblem& P = g.p[j];
-      P.M = int(q.d); P.N = int(q.d); P.K = int(q.tokens);
+      P.M = int(q.d); P.N = int(q.d); P.K = int(kx);
       P.batch = q.count;
       P.tiles_m = P.tiles_n = int(cdiv(q.d, gemm_cfg::TM));
       P.tiles_per_mat = gemm_tiles_per_mat(EPI_GRAM32, P.tiles_m, P.tiles_n);
@@ -1549,7 +1729,7 @@ muon_status muon_newton_refresh(muon_ctx* ctx, const muon_act_desc* acts, int32_
       P.out32 = reinterpret_cast<float*>(ws + q.s_off);
       P.out32_ld = q.d;
       P.out32_bs = q.s_stride;
-      P.nblocks = direct ? q.nb : 1;
+      P.nblocks = mode == 1 ? q.nb : 1;
       P.pmap_base = q.pmap_base;
       P.scale = 1.0f / float(q.tokens);
       const int64_t tt = int64_t(tile) + int64_t(P.batch) * P.tiles_per_mat;
@@ -1557,8 +1737,9 @@ muon_status muon_newton_refresh(muon_ctx* ctx, const muon_act_desc* acts, int32_
       tile = int(tt);
     }
     g.total = tile;
-    if (direct) CUDA_TRY(ctx, (launch_gemm<EPI_GRAM32, true>(ctx, maps, g, st)));
+    if (mode == 1) CUDA_TRY(ctx, (launch_gemm<EPI_GRAM32, true>(ctx, maps, g, st)));
     else CUDA_TRY(ctx, (launch_gemm<EPI_GRAM32, false>(ctx, maps, g, st)));
+    b0 += nb;
   }
   if (max_d <= CHOL_BLOCKED_MAX_D) {
     // blocked factorisation, panels of 32: panel, then trailing update
@@ -1756,23 +1937,26 @@ muon_status muon_orthogonalize_noalloc(const void* input, int32_t in_dtype, int6
   const int64_t tiles = cdiv(rows, EW_TILE) * d.tiles_c;
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  // The descriptor is copied from this stack frame; the runtime stages a
-  // pageable source before the call returns.
-  if (cudaMemcpyAsync(ddesc, &d, sizeof(MatDesc), cudaMemcpyHostToDevice, st) != cudaSuccess) return MUON_ERR_CUDA;
-  // Previous calls leave their values behind: zero the flags (everything
-  // else is fully overwritten before it is read).
-  if (cudaMemsetAsync(flags, 0, sizeof(int) * 4, st) != cudaSuccess) return MUON_ERR_CUDA;
+  // The descriptor travels as a kernel parameter and is stored into the
+  // scratch array on the device, together with zeroed flags (a previous
+  // call leaves its values behind; everything else is fully overwritten
+  // before it is read), so the call makes no host-to-device copy.
+  noalloc_setup_kernel<<<1, 32, 0, st>>>(d, ddesc, flags);
   const std::vector<SegLaunch> segl = build_seg_launches(&d, 1);
-  momentum_kernel<1><<<unsigned(tiles), EW_THREADS, 0, st>>>(ddesc, segl[0].t, 0, 0.f, 0, nullptr);
-  norm_reduce_kernel<<<1, EW_THREADS, 0, st>>>(ddesc, nullptr);
+  momentum_kernel<1><<<unsigned(tiles), EW_THREADS, 0, st>>>(ddesc, segl[0].t, 0, 0.f, 0, flags);
+  norm_reduce_kernel<<<1, EW_THREADS, 0, st>>>(ddesc, flags);
   if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;
   tmp.dflags = flags;
   const float* n2 = d.norm2;
-  s = run_newton_schulz(&tmp, ws, &r, 1, &n2, hp, nullptr, st);
+  // a product whose bounded wait gives up raises flags[0]; the later
+  // products and the export then do nothing, and the output is poisoned
+  s = run_newton_schulz(&tmp, ws, &r, 1, &n2, hp, flags, st);
   tmp.dflags = nullptr;
   if (s != MUON_OK) return s;
   apply_kernel<1><<<unsigned(tiles), EW_THREADS, 0, st>>>(ddesc, segl[0].t, 0, hp->ns_steps == 0, hp->eps,
-                                                          nullptr);
+                                                          flags);
+  const int64_t n = rows * cols;
+  noalloc_poison_kernel<<<unsigned(std::min<int64_t>(cdiv(n, 256), 1024)), 256, 0, st>>>(flags, output, n);
   if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;
   return MUON_OK;
 }

@@ -7,6 +7,10 @@
 //   act_transpose_kernel  a d-wide activation block, transposed to bf16
 //                         d x tokens: the K-major operand of S = Xt Xt^T / N,
 //                         which the tensor-core engine computes (GRAM32).
+//   act_split_kernel      the same for fp32 activations, split into bf16
+//                         high and low parts laid out so that one GRAM32
+//                         product over three times the tokens sums the
+//                         three significant cross products.
 //   chol_panel_kernel, chol_update_kernel  S = L L^T in place (fp32),
 //                         panels of 32, two batched launches per panel
 //                         (d <= 1536).
@@ -531,7 +535,7 @@ struct PrecondDesc {
 __global__ void __launch_bounds__(PRE_THREADS)
     precond_kernel(const PrecondDesc* __restrict__ descs, int n, const int* skip) {
   pdl_wait();      // previous kernel's results visible (no-op without PDL)
-  if (skip != nullptr && *skip) return;
+  if (halted(skip)) return;
   __shared__ float gs[PRE_BK][PRE_BM + 4];   // G tile, transposed (k, row)
   __shared__ float ss[PRE_BK][PRE_BN + 4];   // S^-1 tile (k, col)
   const int64_t gt = blockIdx.x;
@@ -637,6 +641,81 @@ __global__ void __launch_bounds__(256) act_transpose_kernel(const ActBlock* __re
       *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(&t[jj][tsw(jj, tv)]);
     } else {
       for (int k = 0; k < 8 && tok + k < b.tokens; ++k) dst[k] = t[jj][tsw(jj, tv + k)];
+    }
+  }
+}
+
+// One d-wide column block of an fp32 tokens x width activation, written as
+// the two K-major operands of its second moment on the tensor cores: with
+// H = bf16(x) and L = bf16(x - H) (so x - H - L is below 2^-16 |x|),
+//   xa (d rows of 3 tokens, leading dimension ld3) = [H^T | H^T | L^T],
+//   xb (same shape)                                 = [H^T | L^T | H^T],
+// and xa xb^T = H^T H + H^T L + L^T H = X^T X up to the dropped L^T L term
+// and the rounding of L, both below 2^-16 relative per product.
+struct ActSplitBlock {
+  const float* acts;
+  __nv_bfloat16* xa;
+  __nv_bfloat16* xb;
+  int64_t tokens, width, col0, d, ld3;
+};
+
+__global__ void __launch_bounds__(256) act_split_kernel(const ActSplitBlock* __restrict__ blocks) {
+  pdl_wait();      // previous kernel's results visible (no-op without PDL)
+  __shared__ __align__(16) __nv_bfloat16 th[TPOSE_T][TPOSE_T];   // th[j][tsw(j, tok)]: H
+  __shared__ __align__(16) __nv_bfloat16 tl[TPOSE_T][TPOSE_T];   //                     L
+  const ActSplitBlock& b = blocks[blockIdx.y];
+  const int64_t tiles_j = (b.d + TPOSE_T - 1) / TPOSE_T;
+  const int64_t t0 = (blockIdx.x / tiles_j) * TPOSE_T, j0 = (blockIdx.x % tiles_j) * TPOSE_T;
+  if (t0 >= b.tokens) return;
+  const bool vin = (b.width % 4 == 0) && (b.col0 % 4 == 0);
+#pragma unroll
+  for (int it = 0; it < 2; ++it) {
+    const int v = threadIdx.x + it * 256;
+    const int tt = v >> 3, jv = (v & 7) * 8;
+    const int64_t tok = t0 + tt, j = j0 + jv;
+    float x[8];
+    if (vin && tok < b.tokens && j + 8 <= b.d) {
+      const float4* p = reinterpret_cast<const float4*>(b.acts + tok * b.width + b.col0 + j);
+      const float4 u = p[0], w = p[1];
+      x[0] = u.x; x[1] = u.y; x[2] = u.z; x[3] = u.w; x[4] = w.x; x[5] = w.y; x[6] = w.z; x[7] = w.w;
+    } else {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) x[k] = (tok < b.tokens && j + k < b.d) ? b.acts[tok * b.width + b.col0 + j + k] : 0.f;
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const __nv_bfloat16 h = __float2bfloat16_rn(x[k]);
+      th[jv + k][tsw(jv + k, tt)] = h;
+      tl[jv + k][tsw(jv + k, tt)] = __float2bfloat16_rn(x[k] - __bfloat162float(h));
+    }
+  }
+  __syncthreads();
+  // segment offsets along K: xa = [H, H, L], xb = [H, L, H]
+  const int64_t T = b.tokens;
+  const bool vout = (T % 8 == 0) && (b.ld3 % 8 == 0);
+#pragma unroll
+  for (int it = 0; it < 2; ++it) {
+    const int v = threadIdx.x + it * 256;
+    const int jj = v >> 3, tv = (v & 7) * 8;
+    const int64_t j = j0 + jj, tok = t0 + tv;
+    if (j >= b.d) continue;
+    __nv_bfloat16* ra = b.xa + j * b.ld3 + tok;
+    __nv_bfloat16* rb = b.xb + j * b.ld3 + tok;
+    if (vout && tok + 8 <= T) {
+      const uint4 h = *reinterpret_cast<const uint4*>(&th[jj][tsw(jj, tv)]);
+      const uint4 l = *reinterpret_cast<const uint4*>(&tl[jj][tsw(jj, tv)]);
+      *reinterpret_cast<uint4*>(ra) = h;
+      *reinterpret_cast<uint4*>(ra + T) = h;
+      *reinterpret_cast<uint4*>(ra + 2 * T) = l;
+      *reinterpret_cast<uint4*>(rb) = h;
+      *reinterpret_cast<uint4*>(rb + T) = l;
+      *reinterpret_cast<uint4*>(rb + 2 * T) = h;
+    } else {
+      for (int k = 0; k < 8 && tok + k < T; ++k) {
+        const __nv_bfloat16 h = th[jj][tsw(jj, tv + k)], l = tl[jj][tsw(jj, tv + k)];
+        ra[k] = h; ra[T + k] = h; ra[2 * T + k] = l;
+        rb[k] = h; rb[T + k] = l; rb[2 * T + k] = h;
+      }
     }
   }
 }

@@ -60,7 +60,11 @@
 //            in fp32).  Launched with MN-major operands it reads the tokens
 //            x width activation in place: A and B are both MN-major, with
 //            the block's column offset added to the MN coordinate, and the
-//            per-activation maps come from device memory.
+//            per-activation maps come from device memory.  For fp32
+//            activations X = H + L (bf16 high and low parts) it runs over
+//            K = 3N with A = [H | H | L] and B = [H | L | H] (transposed):
+//            the sum H^T H + H^T L + L^T H, symmetric, but with A and B
+//            different tensors (args.ab_distinct).
 //   PRECOND  G' = G [S_hi; S_lo]         M = rows, N = d, K = 2d
 //            (S^-1 = S_hi + S_lo split into two bf16 matrices stacked along
 //            K, G's column block read twice, so the product keeps close to
@@ -84,14 +88,18 @@ constexpr int BK = 64;
 // chunks (below) and spend the space saved on a fifth / sixth stage; the
 // update also has no mirrored blocks.
 __host__ __device__ constexpr int stages_for(int kind) {
-  return kind == 0 ? 5 : kind == 1 ? 4 : kind == 2 ? 6 : kind == 5 ? 5 : 7;
+  return kind == 0 ? 5 : kind == 1 ? 4 : kind == 2 ? 6 : kind == 5 ? 4 : 7;
 }
 // GRAM32 and PRECOND write fp32 straight from registers: no epilogue buffers,
 // so their pipelines take the shared memory.
 __host__ __device__ constexpr bool fp32_out(int kind) { return kind == 3 || kind == 4; }
 // The last update of an optimizer step may apply W <- W (1 - lr wd) - lr
-// scale O in its epilogue (EPI_UPDATE_APPLY): W moves through two 4 KB
-// 32x32 fp32 chunk buffers per warp by TMA, and O never reaches memory.
+// scale O in its epilogue (EPI_UPDATE_APPLY): W moves through a ring of
+// W_NBUF 4 KB 32x32 fp32 chunk buffers per warp by TMA, and O never reaches
+// memory.  Each buffer is refilled with the warp's next chunk (possibly of a
+// later tile) as soon as the store before it has read it, so weight loads
+// run W_NBUF - 1 chunks ahead of the stores.
+constexpr int W_NBUF = 3;
 __host__ __device__ constexpr bool apply_out(int kind) { return kind == 5; }
 __host__ __device__ constexpr bool mirrors(int kind) { return kind == 0 || kind == 1; }
 // Output leaves through two alternating 32x32 chunk buffers per warp
@@ -114,13 +122,22 @@ constexpr int WCH_BYTES = 32 * 128;                  // 32 x 32 fp32 weight chun
 constexpr int BAR_BYTES = 384;
 __host__ __device__ constexpr int smem_bytes(int kind) {
   return stages_for(kind) * STAGE_BYTES +
-         EPI_WARPS * ((apply_out(kind)     ? 2 * WCH_BYTES
+         EPI_WARPS * ((apply_out(kind)     ? W_NBUF * WCH_BYTES
                        : chunked_out(kind) ? CH_BUFS * CH_BYTES
                        : fp32_out(kind)    ? 0
                                            : EPI_BYTES) +
                       (mirrors(kind) ? STG_BYTES : 0)) +
          BAR_BYTES + 1024;   // + alignment slack
 }
+// GRAM32 sums a long K (thousands of tokens): the tensor cores accumulate
+// K in chunks of this many 64-deep blocks into alternating accumulators and
+// the epilogue adds the chunks in fp32 registers, so no fp32 sum in TMEM
+// runs over more than 4 x 16 = 64 MMA accumulation steps.
+constexpr int G32_CHUNK_KB = 4;
+__host__ __device__ constexpr int chunk_kb(int kind) { return kind == 3 ? G32_CHUNK_KB : 1 << 30; }
+// full + empty per stage (at most 7), two tfull, two tempty, drain, the aux
+// barriers, then the TMEM slot and the abort flag
+static_assert((2 * 7 + 5 + W_NBUF * EPI_WARPS) * 8 + 8 <= BAR_BYTES, "barrier area");
 constexpr int ACC_COLS = 256;                        // one fp32 128x256 accumulator per CTA
 constexpr int TMEM_COLS = 2 * ACC_COLS;              // double-buffered
 static_assert(smem_bytes(0) <= 232448 && smem_bytes(1) <= 232448 && smem_bytes(2) <= 232448 &&
@@ -181,10 +198,12 @@ struct GemmArgs {
   float eps;
   float c0, c1, c2;          // POLY: b, c, and a (added on the diagonal)
   int* err;                  // device error flags
-  const int* skip;           // non-null and set: do nothing (non-finite gradient)
+  const int* skip;           // the context's device flags: halted() -> do nothing
   int reverse;               // walk the tile list from its end (see run_newton_schulz)
   const ApplyDesc* apply;    // UPDATE_APPLY: per-matrix weights (device memory)
   const PrecondMaps* pmaps;  // PRECOND: per-matrix operand maps (device memory)
+  int ab_distinct;           // GRAM32 of split fp32 activations: A and B are
+                             // different tensors, so a diagonal tile loads both
 };
 
 // Per problem: A operand rows (box 64 x 128), B operand (K-major box 64 x 128
@@ -268,7 +287,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* smem_epi = smem + STAGES * STAGE_BYTES;             // 1024-aligned slices
-  constexpr int SLICE = apply_out(KIND) ? 2 * WCH_BYTES : chunked_out(KIND) ? CH_BUFS * CH_BYTES
+  constexpr int SLICE = apply_out(KIND) ? W_NBUF * WCH_BYTES : chunked_out(KIND) ? CH_BUFS * CH_BYTES
                         : fp32_out(KIND)  ? 0 : EPI_BYTES;
   uint8_t* smem_stg = smem_epi + EPI_WARPS * SLICE;
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem_stg + (mirrors(KIND) ? EPI_WARPS * STG_BYTES : 0));
@@ -276,8 +295,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
   uint64_t* tfull_bar = empty_bar + STAGES;     // accumulator ready   (leader MMA -> both epilogues)
   uint64_t* tempty_bar = tfull_bar + 2;         // accumulator drained (both epilogues -> leader MMA)
   uint64_t* drain_bar = tempty_bar + 2;
-  uint64_t* aux_bar = drain_bar + 1;            // two per epilogue warp (POLY uses the first)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(aux_bar + 2 * EPI_WARPS);
+  uint64_t* aux_bar = drain_bar + 1;            // W_NBUF per epilogue warp (POLY uses the first)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(aux_bar + W_NBUF * EPI_WARPS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -297,7 +316,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
       mbar_init(&tempty_bar[a], 2 * EPI_WARPS);
     }
     mbar_init(drain_bar, 1);
-    for (int w = 0; w < 2 * EPI_WARPS; ++w) mbar_init(&aux_bar[w], 1);
+    for (int w = 0; w < W_NBUF * EPI_WARPS; ++w) mbar_init(&aux_bar[w], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -320,8 +339,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
   // everything above touches only shared memory, TMEM and the parameter
   // space, so it runs before the wait for the previous kernel
   pdl_wait();
-  // a non-finite gradient flag (uniform over the grid) leaves an empty tile list
-  const int total = (args.skip != nullptr && *args.skip) ? 0 : args.total;
+  // a non-finite gradient or an earlier device error (uniform over the grid)
+  // leaves an empty tile list
+  const int total = halted(args.skip) ? 0 : args.total;
 
   if (warp == 0) {
     // ---------------- TMA producer (both CTAs load their halves) ----------------
@@ -355,7 +375,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
         const int nk = (args.p[pi].K + BK - 1) / BK;
         // diagonal tile of a symmetric product: each CTA's B rows are its A
         // rows, so only A is loaded and the MMA reads it for both operands
-        const bool diag = symmetric_kind(KIND) && ti == tj;
+        const bool diag = symmetric_kind(KIND) && ti == tj && !args.ab_distinct;
         for (int kb = 0; kb < nk; ++kb) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
@@ -400,36 +420,41 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
     // ---------------- MMA issuer (leader CTA only) ----------------
     if (leader && lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(TM, TN, B_MN_MAJOR, A_MN);
-      int it = 0, lt = 0;
+      constexpr int CHUNK = chunk_kb(KIND);
+      int it = 0, la = 0;                   // stages consumed, accumulators filled
       bool ok = true;
-      for (int t = pair; t < total && ok; t += npairs, ++lt) {
+      for (int t = pair; t < total && ok; t += npairs) {
         int pi, bidx, ti, tj;
         decode_tile(KIND, args, t, pi, bidx, ti, tj);
         const int nk = (args.p[pi].K + BK - 1) / BK;
-        const bool diag = symmetric_kind(KIND) && ti == tj;
-        const int acc = lt & 1;
-        if (!mbar_wait(&tempty_bar[acc], ((lt >> 1) & 1) ^ 1, args.err, abort_flag)) break;
-        tc_fence_after();
-        const uint32_t d_tmem = tmem + acc * ACC_COLS;
-        for (int kb = 0; kb < nk; ++kb) {
-          const int s = it % STAGES;
-          const uint32_t ph = (it / STAGES) & 1;
-          if (!mbar_wait(&full_bar[s], ph, args.err, abort_flag)) { ok = false; break; }
+        const bool diag = symmetric_kind(KIND) && ti == tj && !args.ab_distinct;
+        // one accumulator per K chunk (the whole K except for GRAM32)
+        for (int k0 = 0; k0 < nk && ok; k0 += CHUNK, ++la) {
+          const int acc = la & 1;
+          if (!mbar_wait(&tempty_bar[acc], ((la >> 1) & 1) ^ 1, args.err, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a_base = smem_u32(smem + s * STAGE_BYTES);
-          const uint32_t b_base = diag ? a_base : a_base + A_BYTES;
+          const uint32_t d_tmem = tmem + acc * ACC_COLS;
+          const int k1 = min(nk, k0 + CHUNK);
+          for (int kb = k0; kb < k1; ++kb) {
+            const int s = it % STAGES;
+            const uint32_t ph = (it / STAGES) & 1;
+            if (!mbar_wait(&full_bar[s], ph, args.err, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t a_base = smem_u32(smem + s * STAGE_BYTES);
+            const uint32_t b_base = diag ? a_base : a_base + A_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t adesc = A_MN ? sdesc_mnmajor_sw128(a_base + kk * 16 * 128, MN_CHUNK_BYTES)
-                                        : sdesc_kmajor_sw128(a_base + kk * 32);
-            const uint64_t bdesc = B_MN_MAJOR ? sdesc_mnmajor_sw128(b_base + kk * 16 * 128, MN_CHUNK_BYTES)
-                                              : sdesc_kmajor_sw128(b_base + kk * 32);
-            mma_bf16_ss_pair(d_tmem, adesc, bdesc, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              const uint64_t adesc = A_MN ? sdesc_mnmajor_sw128(a_base + kk * 16 * 128, MN_CHUNK_BYTES)
+                                          : sdesc_kmajor_sw128(a_base + kk * 32);
+              const uint64_t bdesc = B_MN_MAJOR ? sdesc_mnmajor_sw128(b_base + kk * 16 * 128, MN_CHUNK_BYTES)
+                                                : sdesc_kmajor_sw128(b_base + kk * 32);
+              mma_bf16_ss_pair(d_tmem, adesc, bdesc, idesc, (kb > k0 || kk > 0) ? 1u : 0u);
+            }
+            mma_commit_pair_mc(&empty_bar[s], 0x3);
+            ++it;
           }
-          mma_commit_pair_mc(&empty_bar[s], 0x3);
-          ++it;
+          if (ok) mma_commit_pair_mc(&tfull_bar[acc], 0x3);
         }
-        if (ok) mma_commit_pair_mc(&tfull_bar[acc], 0x3);
       }
       if (*abort_flag) {
         // wait for the MMAs already issued before TMEM is released
@@ -439,14 +464,211 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
       }
     }
     __syncwarp();
+  } else if constexpr (KIND == EPI_GRAM32) {
+    // ---------------- GRAM32 epilogue: K chunks summed in registers ----------------
+    const int ew = warp - 2;
+    const int q = warp & 3;                 // TMEM lane quarter this warp may read
+    const int half = ew >> 2;               // 128-column half of the tile
+    const uint32_t tempty0 = map_to_cta(smem_u32(tempty_bar), 0);
+    int la = 0;
+    for (int t = pair; t < total; t += npairs) {
+      int pi, bidx, ti, tj;
+      decode_tile(KIND, args, t, pi, bidx, ti, tj);
+      const GemmProblem& P = args.p[pi];
+      const int rb = ti * 2 + static_cast<int>(rank);   // 128-row block index of this CTA
+      const int rbase = rb * HM + q * 32;
+      const int cb = tj * 2 + half;          // 128-column block index
+      const int col0 = cb * 128;
+      // below the diagonal: mirrored by another block
+      const bool active = col0 < P.N && rbase < P.M && cb >= rb;
+      const bool mirror = cb > rb;
+      const int nk = (P.K + BK - 1) / BK;
+      float run[4][32];
+#pragma unroll
+      for (int c32 = 0; c32 < 4; ++c32)
+#pragma unroll
+        for (int k = 0; k < 32; ++k) run[c32][k] = 0.f;
+      bool ok = true;
+      for (int k0 = 0; k0 < nk; k0 += G32_CHUNK_KB, ++la) {
+        const int acc = la & 1;
+        // warp-uniform decision: tcgen05.ld below is warp-collective
+        const bool got = mbar_wait(&tfull_bar[acc], (la >> 1) & 1, args.err, abort_flag);
+        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+        tc_fence_after();
+        if (active) {
+          // eight columns at a time: the 128 running sums already hold most
+          // of the registers a thread may have
+#pragma unroll
+          for (int c8 = 0; c8 < 16; ++c8) {
+            uint32_t raw[8];
+            tmem_ld_32x32b_x8(tmem + acc * ACC_COLS + (static_cast<uint32_t>(q * 32) << 16) + half * 128 + c8 * 8,
+                              raw);
+            tmem_ld_wait();
+#pragma unroll
+            for (int k = 0; k < 8; ++k) run[c8 >> 2][(c8 & 3) * 8 + k] += __uint_as_float(raw[k]);
+          }
+        }
+        // this warp's reads of the chunk completed (tcgen05.wait::ld)
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster_relaxed(tempty0 + acc * 8);   // leader's tempty_bar[acc]
+      }
+      if (!ok) break;
+      const int r = rbase + lane;
+      if (active && r < P.M) {
+        const int64_t zoff = static_cast<int64_t>(bidx) * P.out32_bs;
+#pragma unroll
+        for (int c32 = 0; c32 < 4; ++c32) {
+          const int cbase = col0 + c32 * 32;
+          if (cbase < P.N) {
+            float* v = run[c32];
+#pragma unroll
+            for (int k = 0; k < 32; ++k) v[k] *= P.scale;
+            float* dst = P.out32 + zoff + static_cast<int64_t>(r) * P.out32_ld + cbase;
+            if (cbase + 32 <= P.N && (P.out32_ld & 3) == 0) {
+#pragma unroll
+              for (int u = 0; u < 8; ++u)
+                reinterpret_cast<float4*>(dst)[u] = make_float4(v[u * 4], v[u * 4 + 1], v[u * 4 + 2], v[u * 4 + 3]);
+            } else {
+              for (int k = 0; k < 32 && cbase + k < P.N; ++k) dst[k] = v[k];
+            }
+            if (mirror) {
+              // (r, c) also goes to (c, r): lanes write consecutive r
+#pragma unroll
+              for (int k = 0; k < 32; ++k)
+                if (cbase + k < P.N) P.out32[zoff + static_cast<int64_t>(cbase + k) * P.out32_ld + r] = v[k];
+            }
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if constexpr (apply_out(KIND)) {
+    // ---------------- UPDATE_APPLY epilogue: W chunks through a ring ----------------
+    const int ew = warp - 2;
+    const int q = warp & 3;                 // TMEM lane quarter this warp may read
+    const int half = ew >> 2;               // 128-column half of the tile
+    uint8_t* ring = smem_epi + ew * SLICE;  // W_NBUF chunk buffers
+    uint64_t* wbar = aux_bar + W_NBUF * ew;
+    const uint32_t tempty0 = map_to_cta(smem_u32(tempty_bar), 0);
+    // The warp's chunk sequence: for each of its tiles on which it is active,
+    // the 32-column chunks of its 32 x 128 slice that lie inside the matrix.
+    // lane 0 loads chunk k into buffer k % W_NBUF; the cursor (ct, cc) is the
+    // next chunk to load.
+    int ct = pair, cc = 0;
+    uint32_t issued = 0, used = 0;
+    auto issue_next = [&]() {
+      while (ct < total) {
+        int pi, bidx, ti, tj;
+        decode_tile(KIND, args, ct, pi, bidx, ti, tj);
+        const GemmProblem& P = args.p[pi];
+        const int rbase = (ti * 2 + static_cast<int>(rank)) * HM + q * 32;
+        const int cbase = (tj * 2 + half) * 128 + cc * 32;
+        if (rbase < P.M && cc < 4 && cbase < P.N) {
+          const ApplyDesc& ad = args.apply[P.apply_base + bidx];
+          const int b = static_cast<int>(issued % W_NBUF);
+          mbar_arrive_expect_tx(&wbar[b], WCH_BYTES);
+          if (ad.transposed) tma_load_3d(ring + b * WCH_BYTES, &ad.w, &wbar[b], rbase, cbase, 0);
+          else tma_load_3d(ring + b * WCH_BYTES, &ad.w, &wbar[b], cbase, rbase, 0);
+          ++issued;
+          ++cc;
+          return;
+        }
+        ct += npairs;
+        cc = 0;
+      }
+    };
+    if (lane == 0)
+      for (int k = 0; k < W_NBUF; ++k) issue_next();
+    int lt = 0;
+    for (int t = pair; t < total; t += npairs, ++lt) {
+      int pi, bidx, ti, tj;
+      decode_tile(KIND, args, t, pi, bidx, ti, tj);
+      const GemmProblem& P = args.p[pi];
+      const int acc = lt & 1;
+      const int rbase = (ti * 2 + static_cast<int>(rank)) * HM + q * 32;
+      const int col0 = (tj * 2 + half) * 128;
+      const bool active = col0 < P.N && rbase < P.M;
+      // warp-uniform decision: tcgen05.ld below is warp-collective
+      const bool got = mbar_wait(&tfull_bar[acc], (lt >> 1) & 1, args.err, abort_flag);
+      if (!__all_sync(0xffffffffu, got)) break;
+      tc_fence_after();
+      bool ok = true;
+      if (active) {
+        float alpha = 1.0f;
+        if (P.norm2 != nullptr) alpha = 1.0f / (sqrtf(P.norm2[bidx]) + args.eps);
+        const ApplyDesc& ad = args.apply[P.apply_base + bidx];
+        const float dec = ad.decay, lrs = ad.lr_scale;
+#pragma unroll 1
+        for (int c32 = 0; c32 < 4; ++c32) {
+          const int cbase = col0 + c32 * 32;
+          if (cbase >= P.N) break;
+          uint32_t raw[32];
+          tmem_ld_32x32b_x32(tmem + acc * ACC_COLS + (static_cast<uint32_t>(q * 32) << 16) + half * 128 + c32 * 32,
+                             raw);
+          tmem_ld_wait();
+          const int b = static_cast<int>(used % W_NBUF);
+          uint8_t* wbuf = ring + b * WCH_BYTES;
+          // lane 0 issued the load; all lanes wait on its barrier
+          const bool okw = mbar_wait(&wbar[b], (used / W_NBUF) & 1u, args.err, abort_flag);
+          if (!__all_sync(0xffffffffu, okw)) { ok = false; break; }
+          if (!ad.transposed) {
+            // row `lane` of the chunk: 16-byte unit u at unit u ^ (lane % 8)
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              float4* pw = reinterpret_cast<float4*>(wbuf + lane * 128 + ((u ^ (lane & 7)) << 4));
+              float4 w = *pw;
+              w.x = w.x * dec - lrs * (alpha * __uint_as_float(raw[u * 4 + 0]));
+              w.y = w.y * dec - lrs * (alpha * __uint_as_float(raw[u * 4 + 1]));
+              w.z = w.z * dec - lrs * (alpha * __uint_as_float(raw[u * 4 + 2]));
+              w.w = w.w * dec - lrs * (alpha * __uint_as_float(raw[u * 4 + 3]));
+              *pw = w;
+            }
+          } else {
+            // W is X'^T: element k of this lane's row is W[cbase + k][rbase + lane],
+            // row k of the chunk, column `lane`
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+              float* pw = reinterpret_cast<float*>(wbuf + k * 128 + ((((lane >> 2) ^ k) & 7) << 4) + (lane & 3) * 4);
+              *pw = *pw * dec - lrs * (alpha * __uint_as_float(raw[k]));
+            }
+          }
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (ad.transposed) tma_store_3d(&ad.w, wbuf, rbase, cbase, 0);
+            else tma_store_3d(&ad.w, wbuf, cbase, rbase, 0);
+            bulk_commit_group();
+            // the store before this one has read its buffer: refill that
+            // buffer with the next chunk of the sequence
+            if (used >= 1) {
+              bulk_wait_group_read1();
+              issue_next();
+            }
+          }
+          ++used;
+          __syncwarp();
+        }
+      }
+      if (!ok) break;
+      // this warp's tcgen05.ld reads of the accumulator have completed
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster_relaxed(tempty0 + acc * 8);   // leader's tempty_bar[acc]
+    }
+    if (lane == 0) {
+      // loads issued but not consumed (after an abort) land before exit
+      volatile int no_abort = 0;
+      for (uint32_t k = used; k < issued; ++k) mbar_wait(&wbar[k % W_NBUF], (k / W_NBUF) & 1u, args.err, &no_abort);
+      bulk_wait_group0();
+    }
+    __syncwarp();
   } else {
     // ---------------- epilogue (warps 2..9, both CTAs) ----------------
     const int ew = warp - 2;
     const int q = warp & 3;                 // TMEM lane quarter this warp may read
     const int half = ew >> 2;               // 128-column half of the tile
     uint8_t* slice = smem_epi + ew * SLICE;
-    uint32_t wph = 0;                       // UPDATE_APPLY: phase bit per weight buffer (bits 0, 1)
-    uint32_t wpend = 0;                     // UPDATE_APPLY: weight loads in flight per buffer
     uint32_t nch = 0;                       // output chunks stored so far (buffer = nch & 1)
     uint8_t* stg = smem_stg + ew * STG_BYTES;
     const uint32_t tempty0 = map_to_cta(smem_u32(tempty_bar), 0);
@@ -473,21 +695,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
       const bool two_boxes = col0 + 64 < P.N;
       // the slice is free once the previous tile's TMA store has read it;
       // then fetch this tile's epilogue input into it
-      if constexpr (apply_out(KIND)) {
-        // weight chunks 0 and 1 of this tile into the two buffers, once the
-        // previous tile's stores have read them
-        if (lane == 0 && active) {
-          bulk_wait_group_read0();
-          const ApplyDesc& ad = args.apply[P.apply_base + bidx];
-          for (int c = 0; c < 2 && col0 + c * 32 < P.N; ++c) {
-            const int cb = col0 + c * 32;
-            mbar_arrive_expect_tx(&aux_bar[2 * ew + c], WCH_BYTES);
-            if (ad.transposed) tma_load_3d(slice + c * WCH_BYTES, &ad.w, &aux_bar[2 * ew + c], rbase, cb, 0);
-            else tma_load_3d(slice + c * WCH_BYTES, &ad.w, &aux_bar[2 * ew + c], cb, rbase, 0);
-            wpend |= 1u << c;
-          }
-        }
-      }
       if (lane == 0 && KIND == EPI_POLY) {
         bulk_wait_group_read0();
         if (active) {
@@ -551,54 +758,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
                   if (cbase + k < P.N) P.out32[zoff + static_cast<int64_t>(cbase + k) * P.out32_ld + r] = v[k];
               }
             }
-          } else if constexpr (apply_out(KIND)) {
-            const ApplyDesc& ad = args.apply[P.apply_base + bidx];
-            const int wb = c32 & 1;
-            uint8_t* wbuf = slice + wb * WCH_BYTES;
-            // lane 0 issued the load; all lanes wait on its barrier
-            const bool okw = mbar_wait(&aux_bar[2 * ew + wb], (wph >> wb) & 1u, args.err, abort_flag);
-            if (!__all_sync(0xffffffffu, okw)) break;
-            wph ^= 1u << wb;
-            wpend &= ~(1u << wb);
-            const float dec = ad.decay, lrs = ad.lr_scale;
-            if (!ad.transposed) {
-              // row `lane` of the chunk: 16-byte unit u at unit u ^ (lane % 8)
-#pragma unroll
-              for (int u = 0; u < 8; ++u) {
-                float4* pw = reinterpret_cast<float4*>(wbuf + lane * 128 + ((u ^ (lane & 7)) << 4));
-                float4 w = *pw;
-                w.x = w.x * dec - lrs * (alpha * __uint_as_float(raw[u * 4 + 0]));
-                w.y = w.y * dec - lrs * (alpha * __uint_as_float(raw[u * 4 + 1]));
-                w.z = w.z * dec - lrs * (alpha * __uint_as_float(raw[u * 4 + 2]));
-                w.w = w.w * dec - lrs * (alpha * __uint_as_float(raw[u * 4 + 3]));
-                *pw = w;
-              }
-            } else {
-              // W is X'^T: element k of this lane's row is W[cbase + k][rbase + lane],
-              // row k of the chunk, column `lane`
-#pragma unroll
-              for (int k = 0; k < 32; ++k) {
-                float* pw = reinterpret_cast<float*>(wbuf + k * 128 + ((((lane >> 2) ^ k) & 7) << 4) + (lane & 3) * 4);
-                *pw = *pw * dec - lrs * (alpha * __uint_as_float(raw[k]));
-              }
-            }
-            fence_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-              if (ad.transposed) tma_store_3d(&ad.w, wbuf, rbase, cbase, 0);
-              else tma_store_3d(&ad.w, wbuf, cbase, rbase, 0);
-              bulk_commit_group();
-              // chunk c32 + 2 into this buffer once the store has read it
-              const int cn = cbase + 64;
-              if (c32 + 2 < 4 && cn < P.N) {
-                bulk_wait_group_read0();
-                mbar_arrive_expect_tx(&aux_bar[2 * ew + wb], WCH_BYTES);
-                if (ad.transposed) tma_load_3d(wbuf, &ad.w, &aux_bar[2 * ew + wb], rbase, cn, 0);
-                else tma_load_3d(wbuf, &ad.w, &aux_bar[2 * ew + wb], cn, rbase, 0);
-                wpend |= 1u << wb;
-              }
-            }
-            wpend = __shfl_sync(0xffffffffu, wpend, 0);
           } else if constexpr (chunked_out(KIND)) {
             float v[32];
 #pragma unroll
@@ -705,11 +864,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
         volatile int no_abort = 0;
         mbar_wait(&aux_bar[ew], aux_phase, args.err, &no_abort);   // let the copy land
       }
-      for (int b = 0; b < 2; ++b)
-        if (wpend & (1u << b)) {
-          volatile int no_abort = 0;
-          mbar_wait(&aux_bar[2 * ew + b], (wph >> b) & 1u, args.err, &no_abort);
-        }
       bulk_wait_group0();
     }
     __syncwarp();

@@ -28,9 +28,15 @@ class MuonWithAuxAdam(torch.optim.Optimizer):
     """Muon for groups with use_muon=True (parameters of two or more
     dimensions, stepped as rows x prod(other dims) matrices), AdamW for the
     rest.  Parameters must be contiguous fp32 CUDA tensors on one device;
-    gradients fp32 or bf16."""
+    gradients fp32 or bf16.
 
-    def __init__(self, param_groups: Iterable[dict], device: int = None):
+    Device-side failures (a bounded wait inside a kernel that gave up) are
+    flagged on the GPU; from then on the library leaves every parameter and
+    state tensor untouched until the flag is read.  step() reads it every
+    `check_every` steps (0: never; each read synchronises the device) and
+    raises MuonError when it is set; check() reads it on demand."""
+
+    def __init__(self, param_groups: Iterable[dict], device: int = None, check_every: int = 100):
         groups = []
         for g in param_groups:
             g = dict(g)
@@ -49,6 +55,13 @@ class MuonWithAuxAdam(torch.optim.Optimizer):
                     raise ValueError("Muon parameters need two or more dimensions")
         first = next(p for g in self.param_groups for p in g["params"])
         self.ctx = MuonContext(first.device.index if device is None else device)
+        self.check_every = int(check_every)
+        self._steps = 0
+
+    def check(self):
+        """Synchronise and raise MuonError if a device-side wait gave up since
+        the last check (the library then skipped every update)."""
+        self.ctx.check_device()
 
     @torch.no_grad()
     def step(self, closure=None):
@@ -64,6 +77,9 @@ class MuonWithAuxAdam(torch.optim.Optimizer):
                 self._muon(g, params)
             else:
                 self._adamw(g, params)
+        self._steps += 1
+        if self.check_every and self._steps % self.check_every == 0:
+            self.check()
         return loss
 
     def _muon(self, g, params):

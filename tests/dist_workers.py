@@ -35,8 +35,10 @@ def _inputs():
     return ws, gs
 
 
-def sharded_step_worker(rank, world, port, out_dir):
-    """Three sharded steps; every rank writes its final weights."""
+def sharded_step_worker(rank, world, port, out_dir, stages=2):
+    """Three sharded steps (each owner's matrices in `stages` slices whose
+    exchange is issued right after the slice's step); every rank writes its
+    final weights and the issue order of its last step."""
     try:
         import numpy as np
         import torch
@@ -46,7 +48,10 @@ def sharded_step_worker(rank, world, port, out_dir):
         dist = _init(rank, world, port)
         ws, gs = _inputs()
         weights = [torch.from_numpy(w.copy()) for w in ws]
-        sm = ShardedMuon(weights)
+        storages = {w.untyped_storage().data_ptr() for w in weights}
+        sm = ShardedMuon(weights, stages=stages)
+        # the weights now live in one flat buffer per (owner, stage)
+        assert len({w.untyped_storage().data_ptr() for w in weights}) < len(storages)
         momentum = [torch.zeros_like(w) if i in sm.owned else None for i, w in enumerate(weights)]
 
         def local_step(owned, grads, mom):
@@ -60,6 +65,8 @@ def sharded_step_worker(rank, world, port, out_dir):
             sm.step([torch.from_numpy(g) for g in gs[k]], momentum)
         np.savez(os.path.join(out_dir, f"rank{rank}.npz"), owner=np.array(sm.owner),
                  *[w.numpy() for w in weights])
+        with open(os.path.join(out_dir, f"trace{rank}.txt"), "w") as f:
+            f.write(repr(sm.trace))
         dist.barrier()
         dist.destroy_process_group()
     except Exception:

@@ -33,3 +33,6 @@ def ns_tol(shape):
     return 4e-2 if m >= 16 else 8e-2
 # * fp32 elementwise stages (momentum buffer, staged apply, AdamW).
 EW_TOL = 1e-5
+# * Newton-Muon stages in fp32 (S^-1, G S^-1, the preconditioned momentum)
+#   against the fp64 oracle of the same inputs.
+NEWTON_TOL = 1e-5

@@ -33,6 +33,42 @@ def test_header_declares_the_boundary():
         assert must in names
 
 
+PAGE_TITLES = ("Muon: An optimizer for the hidden layers of neural networks",
+               "Muon: when the LLM optimizer treats weight matrices as",
+               "The Newton-Muon Optimizer")
+
+
+def declaration_comments():
+    """(name, comment text) of every MUON_API declaration: the comment block
+    that ends right above it (or above the declaration before it, for a
+    pair declared back to back)."""
+    src = open(os.path.join(ROOT, "include", "muon.h")).read()
+    out = []
+    for m in re.finditer(r"MUON_API\s+[\w\s\*]+?\b(muon_\w+)\s*\(", src):
+        head = src[:m.start()]
+        end = head.rstrip().rfind("*/")
+        start = head.rfind("/*", 0, end)
+        between = head[end + 2:]
+        assert end >= 0 and start >= 0 and between.count(";") == 0, m.group(1)
+        out.append((m.group(1), " ".join(head[start:end].split())))
+    return out
+
+
+def test_every_declaration_cites_its_source():
+    """Each entry point's comment names the page and section that define the
+    operation, or says that the pages have no counterpart."""
+    found = declaration_comments()
+    assert {n for n, _ in found} == set(declared_symbols())
+    for name, text in found:
+        cited = any(t in text for t in PAGE_TITLES)
+        assert cited or "No counterpart on the pages" in text, name
+    must_cite = {"muon_init", "muon_step", "muon_adamw_step", "muon_newton_refresh",
+                 "muon_newton_precondition", "muon_orthogonalize", "muon_default_hparams"}
+    for name, text in found:
+        if name in must_cite:
+            assert any(t in text for t in PAGE_TITLES), name
+
+
 def test_library_exports_every_declared_symbol(mx):
     lib = mx.load_library()
     names = declared_symbols()

@@ -30,7 +30,7 @@ def bench():
 def test_ns_flops_match_the_metric_definition(bench, name):
     w, aux = bench.workload_def(name)
     work, elems, aux_el = bench.step_work(w, aux)
-    ns = work["gram"][1] + work["poly"][1] + work["update"][1]
+    ns = work["gram"][1] + work["poly"][1] + work["update"][1] + work["ns_small"][1]
     assert ns == sum(oracle.ns_nominal_flops(m.rows, m.cols, 5) for m in w.mats)
     assert elems == sum(m.rows * m.cols for m in w.mats)
     assert aux_el == sum(n for _, n in aux)
@@ -70,3 +70,56 @@ def test_newton_refresh_counts(bench):
     assert kind == "seq"
     assert t_tc == pytest.approx(tc / w.refresh_every)
     assert t_alu == pytest.approx(alu / w.refresh_every, rel=1e-6)
+
+
+def test_executed_flops_follow_the_tile_enumeration(bench):
+    """Executed tensor-core work: whole 256 x 256 pair tiles, the symmetric
+    products only on and above the diagonal.  For m a multiple of 256 with
+    T = m / 256 tiles per side, executed / nominal is (T + 1) / (2 T) for
+    the Gram and polynomial products and 1 for the update."""
+    w, aux = bench.workload_def("llama3-8b")
+    work, _, _ = bench.step_work(w, aux)
+    exe = bench.executed_flops(w)
+    assert exe["update"] == work["update"][1]
+    # per shape class the ratio is (T+1)/(2T); over the set it is the
+    # nominal-weighted mix of those ratios
+    want_g = sum(2 * min(m.rows, m.cols) ** 2 * max(m.rows, m.cols) * 5
+                 * (min(m.rows, m.cols) // 256 + 1) / (2 * (min(m.rows, m.cols) // 256)) for m in w.mats)
+    want_p = sum(2 * min(m.rows, m.cols) ** 3 * 5
+                 * (min(m.rows, m.cols) // 256 + 1) / (2 * (min(m.rows, m.cols) // 256)) for m in w.mats)
+    assert exe["gram"] == pytest.approx(want_g, rel=1e-12)
+    assert exe["poly"] == pytest.approx(want_p, rel=1e-12)
+
+
+def test_executed_flops_round_ragged_shapes_up_to_tiles(bench):
+    """A 300 x 200 matrix (m = 200, n = 300): one 256-tile per side of the
+    Gram over K = 320 (300 rounded up to 64), one poly tile over K = 256,
+    and two update tiles over K = 256; five iterations."""
+    import workloads as wl
+    w = wl.Workload("t", [wl.Mat("a", 300, 200)], "f32", 1.0, 0.02, 1)
+    exe = bench.executed_flops(w)
+    t = 2 * 256 * 256
+    assert exe == {"gram": t * 320 * 5, "poly": t * 256 * 5, "update": 2 * t * 256 * 5, "ns_small": 0}
+
+
+def test_shape_classes_merge_a_shape_with_its_transpose(bench):
+    """The oracle orthogonalises a tall matrix through its transpose, so the
+    CPU baseline samples one matrix per wide shape: three for Llama-3-8B
+    (4096^2 x64, 1024x4096 x64, 4096x14336 x96), two for GPT-2-small."""
+    w, _ = bench.workload_def("llama3-8b")
+    cls = {k: c for k, _, c in bench.shape_classes(w)}
+    assert cls == {(4096, 4096): 64, (1024, 4096): 64, (4096, 14336): 96}
+    w, _ = bench.workload_def("gpt2-small")
+    cls = {k: c for k, _, c in bench.shape_classes(w)}
+    assert cls == {(768, 768): 48, (768, 3072): 24}
+
+
+def test_small_matrices_form_their_own_class(bench):
+    """A 256 x 256 matrix runs every iteration in one launch: its nominal
+    FLOPs (6 m^3 per iteration) and its executed work (three 256-tile
+    products over K = 256) go to the small-matrix class."""
+    w, aux = bench.workload_def("single-256")
+    work, _, _ = bench.step_work(w, aux)
+    assert work["gram"][1] == work["poly"][1] == work["update"][1] == 0
+    assert work["ns_small"][1] == 6 * 256 ** 3 * 5
+    assert bench.executed_flops(w)["ns_small"] == 3 * 2 * 256 ** 3 * 5

@@ -147,3 +147,70 @@ def test_square_sweep_full_size(mx, size):
     if size <= 2048:
         err = rel_fro(_np(O[5]), oracle.newton_schulz(_np(X[5]), 5))
         assert err < NS_TOL, (size, err)
+
+
+def test_newton_muon_gpt2_small_ten_steps_full_size(mx):
+    """Newton-Muon on the GPT-2-small shapes at full size: per layer the
+    activations feeding Q/K/V (one shared estimate), O, the MLP expansion
+    (8192 x 768 each) and the MLP contraction (8192 x 3072, four 768-wide
+    blocks), N(0,1) bf16; S^-1 refreshed at step 0 for all 84 blocks, then
+    10 steps with momentum carried ("The Newton-Muon Optimizer", "What Is
+    Newton-Muon?").  Every step: the momentum of every matrix (the
+    preconditioned gradient's moving average) against the fp64 oracle within
+    the fp32 bar, the staged apply of every matrix, and the whole
+    Newton-Schulz output of one layer (rotating)."""
+    from helpers import NEWTON_TOL
+    dev = torch.device("cuda")
+    w = wl.newton_gpt2_small()
+    mats = w.mats
+    hp = mx.default_hparams()
+    acts, sinv, nblk = [], [], []
+    for a, (_, tokens, width) in enumerate(w.acts):
+        nb = 4 if width > 768 else 1
+        acts.append(wl.torch_normal((tokens, width), 1.0, 8, 0, a, wl.ROLE_ACT, dtype=torch.bfloat16, device=dev))
+        sinv.append(torch.empty((nb, width // nb, width // nb), device=dev))
+        nblk.append(nb)
+    W = [wl.torch_normal((m.rows, m.cols), 0.02, 8, 0, i, wl.ROLE_WEIGHT, device=dev) for i, m in enumerate(mats)]
+    B = [torch.zeros((m.rows, m.cols), device=dev) for m in mats]
+    O = [torch.empty((m.rows, m.cols), device=dev) for m in mats]
+    groups = {}
+    for i, m in enumerate(mats):
+        groups.setdefault((m.rows, m.cols), []).append(i)
+    # the oracle's inverses from the same bf16 activations, in fp64
+    s_or = []
+    for a, nb in zip(acts, nblk):
+        x = _np(a)
+        d = x.shape[1] // nb
+        s_or.append([oracle.spd_inverse(oracle.second_moment(x[:, b * d:(b + 1) * d])) for b in range(nb)])
+    bufs = [np.zeros((m.rows, m.cols)) for m in mats]
+    with mx.MuonContext(0) as ctx:
+        ctx.newton_refresh(acts, sinv, nblk)
+        torch.cuda.synchronize()
+        ctx.check_device()
+        worst = max(rel_fro(_np(sinv[a][b]), s_or[a][b]) for a in range(len(acts)) for b in range(nblk[a]))
+        assert worst < NEWTON_TOL, worst
+        for step in range(10):
+            G = [wl.torch_normal((m.rows, m.cols), 1e-3, 8, step, i, wl.ROLE_GRAD, dtype=torch.bfloat16,
+                                 device=dev) for i, m in enumerate(mats)]
+            w_prev = [_np(x) for x in W]
+            gs = []
+            for ix in groups.values():
+                a0, nb = w.precond[mats[ix[0]].name]
+                gs.append(dict(weights=[W[i] for i in ix], grads=[G[i] for i in ix], momentum=[B[i] for i in ix],
+                               update_out=[O[i] for i in ix],
+                               precond=[sinv[w.precond[mats[i].name][0]] for i in ix], precond_blocks=nb))
+            ctx.step(gs, hp)
+            torch.cuda.synchronize()
+            ctx.check_device()
+            layer = step % 12
+            for i, m in enumerate(mats):
+                a, _ = w.precond[m.name]
+                pg = oracle.right_precondition(_np(G[i]), s_or[a])
+                nb_, u = oracle.nesterov_momentum(pg, bufs[i])
+                assert rel_fro(_np(B[i]), nb_) < NEWTON_TOL, (m.name, step)
+                bufs[i] = nb_
+                o = _np(O[i])
+                want = oracle.apply_update(w_prev[i], o, hp.lr, hp.weight_decay, oracle.shape_scale(m.rows, m.cols))
+                assert rel_fro(_np(W[i]), want) < EW_TOL, (m.name, step)
+                if i // 6 == layer:
+                    assert rel_fro(o, oracle.newton_schulz(u, 5)) < NS_TOL, (m.name, step)

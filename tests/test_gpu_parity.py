@@ -10,7 +10,7 @@ import pytest
 
 import oracle
 import workloads as wl
-from helpers import EW_TOL, NS_TOL, ns_tol, rel_fro, to_np
+from helpers import EW_TOL, NEWTON_TOL, NS_TOL, ns_tol, rel_fro, to_np
 
 torch = pytest.importorskip("torch")
 
@@ -91,6 +91,58 @@ def test_orthogonalize_custom_coefficients(ctx, mx, coeffs):
     torch.cuda.synchronize()
     want = oracle.newton_schulz(wl.bf16_round_np(x), 8, a=a, b=b, c=c)
     assert rel_fro(to_np(out), want) < NS_TOL
+
+
+def test_small_matrix_step_is_three_launches(ctx, mx):
+    """A 256 x 256 step: momentum, the norm reduction and ONE launch for all
+    five iterations with the weight step applied from the fp32 accumulator;
+    momentum within 1e-5 and the applied update within the Newton-Schulz
+    tolerance of the oracle."""
+    shape = (256, 256)
+    g = wl.np_normal(shape, 1.0, seed=40, index=0)
+    w0 = wl.np_normal(shape, 0.02, seed=40, index=0, role=wl.ROLE_WEIGHT)
+    w, b = dev(w0), torch.zeros(shape, device="cuda")
+    n0 = ctx.launch_count
+    ctx.step([dict(weights=[w], grads=[dev(g)], momentum=[b])])
+    torch.cuda.synchronize()
+    ctx.check_device()
+    assert ctx.launch_count - n0 == 3
+    w1, b1, o1 = oracle.muon_step(w0, g, np.zeros(shape))
+    assert rel_fro(to_np(b), b1) < EW_TOL
+    upd = (w0.astype(np.float64) * (1 - 0.02 * 0.01) - to_np(w)) / 0.02
+    assert rel_fro(upd, o1) < NS_TOL
+
+
+def test_small_matrices_batched_past_the_pair_count(ctx, mx):
+    """More small matrices than CTA pairs (each pair takes several in turn),
+    of several shapes in one call, tall ones included, for the
+    Newton-Schulz-only path and a fused step."""
+    shapes = [(64, 200)] * 160 + [(256, 256)] * 2 + [(252, 20)] * 3 + [(96, 96)] * 5
+    xs = [wl.np_normal(sh, 1.0, seed=41, index=i) for i, sh in enumerate(shapes)]
+    outs = [torch.empty(sh, device="cuda") for sh in shapes]
+    ctx.orthogonalize([dev(x, torch.bfloat16) for x in xs], outs)
+    torch.cuda.synchronize()
+    ctx.check_device()
+    for i in list(range(0, 160, 13)) + list(range(160, len(shapes))):
+        want = oracle.newton_schulz(wl.bf16_round_np(xs[i]), 5)
+        assert rel_fro(to_np(outs[i]), want) < ns_tol(shapes[i]), (i, shapes[i])
+    w0 = [wl.np_normal(sh, 0.02, seed=41, index=i, role=wl.ROLE_WEIGHT) for i, sh in enumerate(shapes)]
+    wt = [dev(x) for x in w0]
+    bt = [torch.zeros(sh, device="cuda") for sh in shapes]
+    gt = [dev(x * 1e-3) for x in xs]
+    by = {}
+    for i, sh in enumerate(shapes):
+        by.setdefault(sh, []).append(i)
+    ctx.step([dict(weights=[wt[i] for i in ix], grads=[gt[i] for i in ix], momentum=[bt[i] for i in ix])
+              for ix in by.values()])
+    torch.cuda.synchronize()
+    ctx.check_device()
+    for i in list(range(0, 160, 29)) + list(range(160, len(shapes))):
+        sh = shapes[i]
+        _, _, o = oracle.muon_step(w0[i], (xs[i] * 1e-3).astype(np.float32), np.zeros(sh))
+        scale = oracle.shape_scale(sh[0], sh[1], "original")
+        upd = (w0[i].astype(np.float64) * (1 - 0.02 * 0.01) - to_np(wt[i])) / (0.02 * scale)
+        assert rel_fro(upd, o) < ns_tol(sh), (i, sh)
 
 
 def _step_case(ctx, mx, shapes, steps, grad_dtype, hp_over=None, seed=0, grad_std=1e-3):
@@ -277,6 +329,53 @@ def test_bounded_wait_reports_timeout_and_context_survives(ctx, mx):
     assert rel_fro(to_np(out), oracle.newton_schulz(g, 5)) < NS_TOL
 
 
+def test_timeout_halts_later_steps_until_checked(ctx, mx):
+    """A bounded wait that gave up leaves the context's error flag set; every
+    kernel of a later step then returns without writing, so the weights and
+    momentum stay as they were (no half-computed update reaches them).
+    check_device reports MUON_ERR_TIMEOUT and clears the flag, and the next
+    step updates normally."""
+    ctx.check_device()
+    shape = (256, 384)
+    w0 = wl.np_normal(shape, 0.02, seed=18, index=0, role=wl.ROLE_WEIGHT)
+    g = wl.bf16_round_np(wl.np_normal(shape, 1e-3, seed=18, index=0))
+    w, b = dev(w0), torch.zeros(shape, device="cuda")
+    gt = dev(g, torch.bfloat16)
+    p, pg = dev(np.ones(1000)), dev(np.ones(1000))
+    pm, pv = torch.zeros(1000, device="cuda"), torch.zeros(1000, device="cuda")
+    ctx.selftest_wait()
+    ctx.step([dict(weights=[w], grads=[gt], momentum=[b])])
+    ctx.adamw_step([p], [pg], [pm], [pv], 1)
+    torch.cuda.synchronize()
+    assert torch.equal(w, dev(w0)) and torch.count_nonzero(b) == 0
+    assert torch.all(p == 1) and torch.count_nonzero(pm) == 0
+    with pytest.raises(mx.MuonError) as e:
+        ctx.check_device()
+    assert e.value.status == mx.binding.MUON_ERR_TIMEOUT
+    o = torch.empty(shape, device="cuda")
+    ctx.step([dict(weights=[w], grads=[gt], momentum=[b], update_out=[o])])
+    torch.cuda.synchronize()
+    ctx.check_device()
+    w1, b1, o1 = oracle.muon_step(w0, g, np.zeros(shape))
+    assert rel_fro(to_np(b), b1) < EW_TOL
+    assert rel_fro(to_np(o), o1) < NS_TOL
+
+
+def test_nonfinite_flag_clears_for_the_next_unchecked_step(ctx, mx):
+    """After a step rejected for a non-finite gradient, a step without the
+    finite check still runs (the flag only halts the step that raised it)."""
+    w = torch.ones((64, 96), device="cuda")
+    g = torch.randn((64, 96), device="cuda")
+    g[0, 0] = float("inf")
+    b = torch.zeros((64, 96), device="cuda")
+    with pytest.raises(mx.MuonError):
+        ctx.step([dict(weights=[w], grads=[g], momentum=[b])], mx.default_hparams(check_finite=1))
+    g[0, 0] = 0.0
+    ctx.step([dict(weights=[w], grads=[g], momentum=[b])])
+    torch.cuda.synchronize()
+    assert not torch.all(w == 1) and torch.count_nonzero(b) > 0
+
+
 def test_workspace_cap_and_caller_workspace(ctx, mx):
     """A bounded workspace (chunked execution) and a caller-owned workspace
     give the same result as the library's own."""
@@ -369,7 +468,7 @@ def test_newton_refresh_vs_oracle(ctx, mx):
         d = a.shape[1] // nb
         for b in range(nb):
             want = oracle.spd_inverse(oracle.second_moment(a[:, b * d:(b + 1) * d]))
-            assert rel_fro(to_np(s[b]), want) < 1e-4
+            assert rel_fro(to_np(s[b]), want) < NEWTON_TOL
 
 
 def _s_inv_blocks(tokens, d, nb, seed, index):
@@ -395,7 +494,7 @@ def test_newton_precondition_vs_oracle(ctx, mx, case):
     torch.cuda.synchronize()
     ctx.check_device()
     for g, o in zip(gs, out):
-        assert rel_fro(to_np(o), oracle.right_precondition(g, blocks)) < 1e-4
+        assert rel_fro(to_np(o), oracle.right_precondition(g, blocks)) < NEWTON_TOL
 
 
 def test_newton_precondition_matches_step_and_batches(ctx, mx):
@@ -463,7 +562,33 @@ def test_newton_refresh_paths(ctx, mx, case):
     for (a, nb, d), s in zip(acts, outs):
         for b in range(nb):
             want = oracle.spd_inverse(oracle.second_moment(a[:, b * d:(b + 1) * d]))
-            assert rel_fro(to_np(s[b]), want) < 1e-4
+            assert rel_fro(to_np(s[b]), want) < NEWTON_TOL
+
+
+@pytest.mark.parametrize("case", [[((2048, 192), 1)], [((1001, 256), 2)], [((777, 100), 1)],
+                                  [((1024, 128), 1, "bf16"), ((1024, 128), 1), ((512, 192), 2)]],
+                         ids=["fp32-2048x192", "fp32-ragged-tokens-two-blocks", "fp32-odd-width",
+                              "bf16-and-fp32-in-one-call"])
+def test_newton_refresh_fp32_activations(ctx, mx, case):
+    """fp32 activations (split into bf16 high and low parts whose three
+    significant cross products the tensor cores sum in fp32) against the
+    oracle's second moment of the same fp32 values; bf16 activations in the
+    same call keep their own path."""
+    acts, outs = [], []
+    for k, spec in enumerate(case):
+        shape, nb = spec[0], spec[1]
+        a = wl.np_normal(shape, 1.0, seed=19, index=shape[1] + 7 * k, role=wl.ROLE_ACT)
+        if len(spec) > 2:
+            a = wl.bf16_round_np(a)
+        acts.append((a, nb, shape[1] // nb, torch.bfloat16 if len(spec) > 2 else torch.float32))
+        outs.append(torch.empty((nb, shape[1] // nb, shape[1] // nb), device="cuda"))
+    ctx.newton_refresh([dev(a, dt) for a, _, _, dt in acts], outs, [nb for _, nb, _, _ in acts])
+    torch.cuda.synchronize()
+    ctx.check_device()
+    for (a, nb, d, _), s in zip(acts, outs):
+        for b in range(nb):
+            want = oracle.spd_inverse(oracle.second_moment(a[:, b * d:(b + 1) * d].astype(np.float64)))
+            assert rel_fro(to_np(s[b]), want) < NEWTON_TOL
 
 
 def test_newton_muon_step_vs_oracle(ctx, mx):
@@ -494,5 +619,5 @@ def test_newton_muon_step_vs_oracle(ctx, mx):
         blocks = s_in if i < 3 else s_out
         pg = oracle.right_precondition(gs[i], blocks)
         nb, u = oracle.nesterov_momentum(pg, np.zeros(s))
-        assert rel_fro(to_np(bt[i]), nb) < 1e-4, f"preconditioned momentum {i}"
+        assert rel_fro(to_np(bt[i]), nb) < NEWTON_TOL, f"preconditioned momentum {i}"
         assert rel_fro(to_np(ot[i]), oracle.newton_schulz(u, 5)) < NS_TOL

@@ -55,3 +55,31 @@ def test_matches_library_calls_and_trains_a_toy_model():
         loss.backward()
         opt.step()
     assert loss.item() < 0.7 * first
+
+
+@pytest.mark.gpu
+def test_device_timeout_leaves_parameters_untouched_and_check_raises():
+    """After a bounded device-side wait gave up, optimizer steps change no
+    parameter and no state; the periodic check raises MUON_ERR_TIMEOUT, and
+    stepping resumes afterwards."""
+    import matrix_aware_optimizer_step_b200 as mx
+    from matrix_aware_optimizer_step_b200.optim import MuonWithAuxAdam
+    torch.manual_seed(1)
+    w = torch.nn.Parameter(torch.randn(128, 192, device="cuda") * 0.02)
+    b = torch.nn.Parameter(torch.zeros(192, device="cuda"))
+    opt = MuonWithAuxAdam([dict(params=[w], use_muon=True), dict(params=[b], use_muon=False)], check_every=2)
+    w.grad = torch.randn_like(w) * 1e-3
+    b.grad = torch.randn_like(b) * 1e-3
+    w0, b0 = w.detach().clone(), b.detach().clone()
+    opt.ctx.selftest_wait()
+    opt.step()                                   # no check yet: halted on the device
+    torch.cuda.synchronize()
+    assert torch.equal(w, w0) and torch.equal(b, b0)
+    assert torch.count_nonzero(opt.state[w]["momentum_buffer"]) == 0
+    with pytest.raises(mx.MuonError) as e:
+        opt.step()                               # second step: the check raises
+    assert e.value.status == mx.binding.MUON_ERR_TIMEOUT
+    assert torch.equal(w, w0) and torch.equal(b, b0)
+    opt.step()
+    torch.cuda.synchronize()
+    assert not torch.equal(w, w0) and not torch.equal(b, b0)

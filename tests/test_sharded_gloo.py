@@ -37,9 +37,10 @@ def test_partition_is_complete_balanced_and_deterministic():
         partition([(0, 3)], 2)
 
 
-def test_sharded_step_matches_single_process(tmp_path):
+@pytest.mark.parametrize("stages", [1, 2, 3])
+def test_sharded_step_matches_single_process(tmp_path, stages):
     import torch.multiprocessing as mp
-    mp.spawn(dw.sharded_step_worker, args=(2, free_port(), str(tmp_path)), nprocs=2, join=True)
+    mp.spawn(dw.sharded_step_worker, args=(2, free_port(), str(tmp_path), stages), nprocs=2, join=True)
     ws, gs = dw._inputs()
     bufs = [np.zeros(s) for s in dw.SHAPES]
     for k in range(3):
@@ -52,6 +53,19 @@ def test_sharded_step_matches_single_process(tmp_path):
     for i in range(len(ws)):
         assert np.array_equal(r0[f"arr_{i}"], r1[f"arr_{i}"])
         assert np.array_equal(r0[f"arr_{i}"], ws[i])
+    # issue order: every stage's broadcasts (all owners, rank order) right
+    # after that stage's local step and before the next stage's, the same
+    # broadcast sequence on both ranks
+    import ast
+    t0 = ast.literal_eval((tmp_path / "trace0.txt").read_text())
+    t1 = ast.literal_eval((tmp_path / "trace1.txt").read_text())
+    assert [e for e in t0 if e[0] == "send"] == [e for e in t1 if e[0] == "send"]
+    for t, rank in ((t0, 0), (t1, 1)):
+        steps = [k for k, e in enumerate(t) if e[0] == "step"]
+        assert [t[k] for k in steps] == [("step", rank, s) for s in range(stages)]
+        for s, k in enumerate(steps):
+            end = steps[s + 1] if s + 1 < len(steps) else len(t)
+            assert all(e[0] == "send" and e[2] == s for e in t[k + 1:end])
 
 
 def test_dead_rank_is_detected_by_timeout(tmp_path):

@@ -103,6 +103,13 @@ def llama3_8b():
     return Workload("llama3-8b-hidden-224", llama3_8b_mats(), "bf16", 1e-3, 0.02, 1)
 
 
+def llama3_8b_layer():
+    """One layer of the Llama-3-8B hidden set (7 matrices): the small case
+    the profiler captures; every launch of the full step processes 32 times
+    its units."""
+    return Workload("llama3-8b-hidden-1-layer", llama3_8b_mats(layers=1), "bf16", 1e-3, 0.02, 1)
+
+
 def newton_gpt2_small(layers=12, d=768, tokens=8192):
     """Newton-Muon on the GPT-2-small shapes: per layer the activations that
     feed QKV, O, the MLP expansion (tokens x d) and the MLP contraction
@@ -125,6 +132,7 @@ WORKLOADS = {
     "single-256": single_256,
     "gpt2-small": gpt2_small,
     "llama3-8b": llama3_8b,
+    "llama3-8b-layer": llama3_8b_layer,
     "newton-gpt2-small": newton_gpt2_small,
     "sweep-1024": lambda: square_sweep(1024),
     "sweep-2048": lambda: square_sweep(2048),
