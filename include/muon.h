@@ -304,6 +304,19 @@ MUON_API muon_status muon_newton_precondition(muon_ctx* ctx, const muon_group* g
 MUON_API muon_status muon_selftest_wait(muon_ctx* ctx, void* stream);
 
 /* No counterpart on the pages (failure detection).
+ * Failure-detection self test of the Newton-Schulz engine: one Gram launch
+ * (a single tile of a zero 256 x 640 matrix in the context's workspace)
+ * whose MMA thread takes the operand stages but never issues a product or
+ * releases a stage.  The TMA producer, the MMA thread and the epilogue warps
+ * of both CTAs of the pair each give up after their 2 s limit, run their
+ * abort sequence (let issued copies land, release TMEM after the cluster
+ * barrier) and return; nothing faults or hangs.  The next
+ * muon_check_device() returns MUON_ERR_TIMEOUT and clears the flag; the
+ * context stays usable.  Needs 458752 bytes of workspace
+ * (MUON_ERR_WORKSPACE if a capped or caller-owned one is smaller). */
+MUON_API muon_status muon_selftest_gemm(muon_ctx* ctx, void* stream);
+
+/* No counterpart on the pages (failure detection).
  * Synchronise the device and report the context's device-side flags:
  * MUON_ERR_TIMEOUT if a bounded wait gave up since the last check,
  * MUON_ERR_INVALID_ARG if a refreshed second moment was not positive

@@ -34,7 +34,8 @@ EXPORTED = [
     "muon_last_error", "muon_status_string", "muon_query_workspace", "muon_set_workspace",
     "muon_step", "muon_orthogonalize", "muon_adamw_step", "muon_newton_refresh",
     "muon_newton_precondition",
-    "muon_check_device", "muon_selftest_wait", "muon_launch_count", "muon_profile_enable", "muon_profile_read",
+    "muon_check_device", "muon_selftest_wait", "muon_selftest_gemm", "muon_launch_count", "muon_profile_enable",
+    "muon_profile_read",
     "muon_orthogonalize_noalloc", "muon_partition",
 ]
 
@@ -123,6 +124,7 @@ def load_library() -> ctypes.CDLL:
         "muon_newton_precondition": (st, [vp, ctypes.POINTER(Group), i32, vp]),
         "muon_check_device": (st, [vp]),
         "muon_selftest_wait": (st, [vp, vp]),
+        "muon_selftest_gemm": (st, [vp, vp]),
         "muon_launch_count": (ctypes.c_uint64, [vp]),
         "muon_profile_enable": (st, [vp, ctypes.c_int]),
         "muon_profile_read": (st, [vp, ctypes.POINTER(KernelTimes)]),
@@ -396,6 +398,13 @@ class MuonContext:
         """Enqueue the failure-detection self test: a bounded device-side
         wait that runs out (2 s); check_device() then raises MUON_ERR_TIMEOUT."""
         self._check(self._lib.muon_selftest_wait(self._ctx, _stream_ptr(stream)), "muon_selftest_wait")
+
+    def selftest_gemm(self, stream=None):
+        """Enqueue the engine's failure-detection self test: a Gram launch
+        whose MMA thread never issues, so its producer, MMA thread and
+        epilogue waits all run out (2 s) and abort; check_device() then
+        raises MUON_ERR_TIMEOUT."""
+        self._check(self._lib.muon_selftest_gemm(self._ctx, _stream_ptr(stream)), "muon_selftest_gemm")
 
     @property
     def launch_count(self) -> int:

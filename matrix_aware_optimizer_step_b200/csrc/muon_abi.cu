@@ -1827,6 +1827,49 @@ muon_status muon_selftest_wait(muon_ctx* ctx, void* stream) {
   return MUON_OK;
 }
 
+muon_status muon_selftest_gemm(muon_ctx* ctx, void* stream) {
+  if (!ctx) return MUON_ERR_INVALID_ARG;
+  muon_status s = set_device(ctx);
+  if (s != MUON_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  ctx->last_stream = st;
+  CUDA_TRY(ctx, cudaGetLastError());
+  // One Gram tile of a zero 256 x 640 X: ten K blocks, more than the
+  // pipeline holds, so the producer also waits for a stage the MMA thread
+  // never releases.
+  constexpr int m = 256, n = 640;
+  const size_t xb = size_t(m) * n * 2, ab = size_t(m) * m * 2;
+  void* wsv = nullptr;
+  s = ensure_workspace(ctx, xb + ab, &wsv);
+  if (s != MUON_OK) return s;
+  uint8_t* ws = static_cast<uint8_t*>(wsv);
+  CUDA_TRY(ctx, cudaMemsetAsync(ws, 0, xb + ab, st));
+  GemmMaps maps{};
+  bool ok = encode_bf16_3d(&maps.a[0], ws, n, m, 1, n, 64, 128);
+  maps.b[0] = maps.a[0];
+  ok &= encode_bf16_3d(&maps.out[0], ws + xb, m, m, 1, m, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+  ok &= encode_bf16_3d(&maps.aux[0], ws + xb, m, m, 1, m, 64, 32);
+  if (!ok) return fail(ctx, MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed (self test)");
+  GemmArgs g{};
+  g.nprob = 1;
+  g.total = 1;
+  GemmProblem& P = g.p[0];
+  P.M = m; P.N = m; P.K = n;
+  P.batch = 1;
+  P.tiles_m = P.tiles_n = 1;
+  P.tiles_per_mat = 1;
+  P.out = reinterpret_cast<__nv_bfloat16*>(ws + xb);
+  P.out_ld = m;
+  P.out_bs = int64_t(m) * m;
+  g.alpha_pow = 2;
+  g.eps = 1e-7f;
+  g.err = ctx->dflags;
+  g.skip = nullptr;          // runs whatever the flags hold
+  g.selftest = 1;
+  CUDA_TRY(ctx, (launch_gemm<EPI_GRAM, false>(ctx, maps, g, st)));
+  return MUON_OK;
+}
+
 uint64_t muon_launch_count(const muon_ctx* ctx) { return ctx ? ctx->launches : 0; }
 
 muon_status muon_partition(const int64_t* rows, const int64_t* cols, int32_t n, int32_t world, int32_t* owner) {

@@ -56,10 +56,13 @@ constexpr int kDevErrNotSPD = 2;
 
 struct CholDesc {
   float* a;          // d x d scratch: S in, L (lower) out; strict upper: L^T
-                     // (unblocked path) or, in each 32x32 diagonal block,
-                     // the transpose of that block's inverse (blocked path)
+                     // (unblocked path); blocked path: the 32x32 diagonal
+                     // blocks keep their input values (see t)
   float* inv;        // d x d output S^-1
-  float* t;          // d x d scratch of the recursive L^-1 (blocked path)
+  float* t;          // d x d scratch (blocked path): each 32x32 diagonal
+                     // block holds that block's factor D (lower) and D^-1
+                     // transposed (strict upper); elsewhere the recursive
+                     // L^-1's products
   int32_t d;
   int32_t pad;
 };
@@ -119,10 +122,13 @@ constexpr int CPR = 64;                     // panel rows per chol_panel_kernel 
 //   chol_panel_kernel   every block factors the panel's 32x32 diagonal block
 //                       D (one warp, in shared memory) and inverts it (lane j
 //                       solves for column j of D^-1); block 0 writes D to the
-//                       lower triangle and D^-1 transposed to the block's
-//                       strict upper triangle (read back by linv_init_kernel);
-//                       each block then forms CPR rows of the panel below D,
-//                       P = A_panel D^-T, as a product over all threads.
+//                       lower triangle and D^-1 transposed to the strict
+//                       upper triangle of the same block of the t scratch
+//                       (read back by linv_init_kernel), never over the
+//                       input that the launch's other blocks are still
+//                       reading; each block then forms CPR rows of the panel
+//                       below D, P = A_panel D^-T, as a product over all
+//                       threads.
 //   chol_update_kernel  the trailing lower triangle minus P P^T, in 64x64
 //                       tiles with 4x4 register tiles (grid.x: tile).
 //
@@ -198,10 +204,12 @@ __global__ void __launch_bounds__(CP_THREADS)
   }
   __syncthreads();
   if (blockIdx.x == 0) {
+    // into t, not a: the other blocks of this launch read D's input from a
+    float* t = c.t;
     for (int e = tid; e < nb * nb; e += CP_THREADS) {
       const int i = e / nb, j = e % nb;
-      if (j <= i) a[int64_t(p0 + i) * d + p0 + j] = dg[i][j];
-      else a[int64_t(p0 + i) * d + p0 + j] = dinv[j][i];     // D^-1[j][i], j > i, at (p0 + i, p0 + j)
+      if (j <= i) t[int64_t(p0 + i) * d + p0 + j] = dg[i][j];
+      else t[int64_t(p0 + i) * d + p0 + j] = dinv[j][i];     // D^-1[j][i], j > i, at (p0 + i, p0 + j)
     }
     if (tid == 0 && bad) atomicOr(err, kDevErrNotSPD);
   }
@@ -311,9 +319,10 @@ __global__ void __launch_bounds__(256) linv_init_kernel(const CholDesc* __restri
       v = 0.f;
     } else if (bc == br) {
       // D^-1 of the 32-block starting at p0: strict lower part stored
-      // transposed above the diagonal of L's diagonal block, diagonal 1/L_ii
+      // transposed above the diagonal of the factor's block in t, diagonal
+      // 1/L_ii
       const int p0 = br * CB;
-      v = col == r ? 1.f / c.a[int64_t(r) * d + r] : c.a[int64_t(col) * d + p0 + (r - p0)];
+      v = col == r ? 1.f / c.t[int64_t(r) * d + r] : c.t[int64_t(col) * d + p0 + (r - p0)];
     } else {
       continue;      // lower-left 32x32 block: level 0
     }

@@ -76,7 +76,10 @@
 
 namespace muon {
 
-enum EpiKind : int { EPI_GRAM = 0, EPI_POLY = 1, EPI_UPDATE = 2, EPI_GRAM32 = 3, EPI_PRECOND = 4, EPI_UPDATE_APPLY = 5 };
+enum EpiKind : int {
+  EPI_GRAM = 0, EPI_POLY = 1, EPI_UPDATE = 2, EPI_GRAM32 = 3, EPI_PRECOND = 4, EPI_UPDATE_APPLY = 5,
+  EPI_UPDATE_WIDE = 6   // the update product on 256 x 512 pair tiles (long K)
+};
 
 namespace gemm_cfg {
 constexpr int TM = 256;                              // pair tile rows (128 per CTA)
@@ -88,8 +91,17 @@ constexpr int BK = 64;
 // chunks (below) and spend the space saved on a fifth / sixth stage; the
 // update also has no mirrored blocks.
 __host__ __device__ constexpr int stages_for(int kind) {
-  return kind == 0 ? 5 : kind == 1 ? 4 : kind == 2 ? 6 : kind == 5 ? 4 : 7;
+  return kind == 0 ? 5 : kind == 1 ? 4 : kind == 2 ? 6 : kind == 5 ? 4 : kind == 6 ? 4 : 7;
 }
+// EPI_UPDATE_WIDE: the pair tile is 256 x 512; each K step issues two
+// N = 256 products that share the A operand, into the two halves of TMEM,
+// so a tile needs 48 KB of operands per CTA and 64-deep K block instead of
+// 2 x 32 KB for two 256 x 256 tiles (a quarter fewer bytes from L2 per
+// FLOP).  Both accumulators hold one tile, so the epilogue is not
+// overlapped with the next tile's products: worth it only for long K.
+__host__ __device__ constexpr bool wide_kind(int kind) { return kind == 6; }
+__host__ __device__ constexpr int tile_n(int kind) { return wide_kind(kind) ? 512 : 256; }
+__host__ __device__ constexpr int n_acc(int kind) { return wide_kind(kind) ? 1 : 2; }
 // GRAM32 and PRECOND write fp32 straight from registers: no epilogue buffers,
 // so their pipelines take the shared memory.
 __host__ __device__ constexpr bool fp32_out(int kind) { return kind == 3 || kind == 4; }
@@ -105,10 +117,11 @@ __host__ __device__ constexpr bool mirrors(int kind) { return kind == 0 || kind 
 // Output leaves through two alternating 32x32 chunk buffers per warp
 // (GRAM, UPDATE) instead of a whole 32x128 slice (POLY reads its input A
 // into the slice and overwrites it in place).
-__host__ __device__ constexpr bool chunked_out(int kind) { return kind == 0 || kind == 2; }
+__host__ __device__ constexpr bool chunked_out(int kind) { return kind == 0 || kind == 2 || kind == 6; }
 constexpr int A_BYTES = HM * BK * 2;                 // 16 KB
 constexpr int B_BYTES = HN * BK * 2;                 // 16 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;       // 32 KB per CTA
+__host__ __device__ constexpr int stage_bytes(int kind) { return A_BYTES + (tile_n(kind) / 2) * BK * 2; }
 constexpr int MN_CHUNK_BYTES = BK * 128;             // one 64-wide MN chunk of B (MN-major)
 constexpr int EPI_WARPS = 8;
 constexpr int THREADS = 64 + EPI_WARPS * 32;         // producer, MMA, 8 epilogue warps
@@ -121,7 +134,7 @@ constexpr int CH_BUFS = 2;
 constexpr int WCH_BYTES = 32 * 128;                  // 32 x 32 fp32 weight chunk, 128-byte swizzle
 constexpr int BAR_BYTES = 384;
 __host__ __device__ constexpr int smem_bytes(int kind) {
-  return stages_for(kind) * STAGE_BYTES +
+  return stages_for(kind) * stage_bytes(kind) +
          EPI_WARPS * ((apply_out(kind)     ? W_NBUF * WCH_BYTES
                        : chunked_out(kind) ? CH_BUFS * CH_BYTES
                        : fp32_out(kind)    ? 0
@@ -141,7 +154,8 @@ static_assert((2 * 7 + 5 + W_NBUF * EPI_WARPS) * 8 + 8 <= BAR_BYTES, "barrier ar
 constexpr int ACC_COLS = 256;                        // one fp32 128x256 accumulator per CTA
 constexpr int TMEM_COLS = 2 * ACC_COLS;              // double-buffered
 static_assert(smem_bytes(0) <= 232448 && smem_bytes(1) <= 232448 && smem_bytes(2) <= 232448 &&
-                  smem_bytes(3) <= 232448 && smem_bytes(4) <= 232448 && smem_bytes(5) <= 232448,
+                  smem_bytes(3) <= 232448 && smem_bytes(4) <= 232448 && smem_bytes(5) <= 232448 &&
+                  smem_bytes(6) <= 232448,
               "shared memory per block");
 }  // namespace gemm_cfg
 
@@ -204,6 +218,9 @@ struct GemmArgs {
   const PrecondMaps* pmaps;  // PRECOND: per-matrix operand maps (device memory)
   int ab_distinct;           // GRAM32 of split fp32 activations: A and B are
                              // different tensors, so a diagonal tile loads both
+  int selftest;              // failure-detection self test: the MMA thread
+                             // waits for the operands but never issues or
+                             // commits, so every role's bounded wait runs out
 };
 
 // Per problem: A operand rows (box 64 x 128), B operand (K-major box 64 x 128
@@ -423,7 +440,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
       constexpr int CHUNK = chunk_kb(KIND);
       int it = 0, la = 0;                   // stages consumed, accumulators filled
       bool ok = true;
-      for (int t = pair; t < total && ok; t += npairs) {
+      for (int t = pair; t < total && ok && args.selftest; t += npairs) {
+        // self test: take the operand stages as they land, issue nothing
+        const int nk = (args.p[0].K + BK - 1) / BK;
+        for (int kb = 0; kb < nk; ++kb, ++it)
+          if (!mbar_wait(&full_bar[it % STAGES], (it / STAGES) & 1, args.err, abort_flag)) { ok = false; break; }
+      }
+      for (int t = pair; t < total && ok && !args.selftest; t += npairs) {
         int pi, bidx, ti, tj;
         decode_tile(KIND, args, t, pi, bidx, ti, tj);
         const int nk = (args.p[pi].K + BK - 1) / BK;

@@ -329,6 +329,28 @@ def test_bounded_wait_reports_timeout_and_context_survives(ctx, mx):
     assert rel_fro(to_np(out), oracle.newton_schulz(g, 5)) < NS_TOL
 
 
+def test_engine_abort_sequence_reports_timeout_and_context_survives(ctx, mx):
+    """Failure detection inside the Newton-Schulz engine without a fault: a
+    Gram launch whose MMA thread never issues makes the TMA producer, the MMA
+    thread and the epilogue of both CTAs give up after their bounded waits
+    and run their abort sequences; MUON_ERR_TIMEOUT is reported once, and the
+    same context then computes correct results (TMEM was released, no copy
+    was left in flight)."""
+    ctx.check_device()
+    ctx.selftest_gemm()
+    with pytest.raises(mx.MuonError) as e:
+        ctx.check_device()
+    assert e.value.status == mx.binding.MUON_ERR_TIMEOUT
+    ctx.check_device()
+    for shape in ((512, 768), (256, 256)):
+        g = wl.np_normal(shape, 1.0, seed=43, index=shape[0])
+        out = torch.empty(shape, device="cuda")
+        ctx.orthogonalize([dev(g)], [out])
+        torch.cuda.synchronize()
+        ctx.check_device()
+        assert rel_fro(to_np(out), oracle.newton_schulz(g, 5)) < NS_TOL
+
+
 def test_timeout_halts_later_steps_until_checked(ctx, mx):
     """A bounded wait that gave up leaves the context's error flag set; every
     kernel of a later step then returns without writing, so the weights and
@@ -469,6 +491,36 @@ def test_newton_refresh_vs_oracle(ctx, mx):
         for b in range(nb):
             want = oracle.spd_inverse(oracle.second_moment(a[:, b * d:(b + 1) * d]))
             assert rel_fro(to_np(s[b]), want) < NEWTON_TOL
+
+
+def test_newton_refresh_many_blocks_repeatable(ctx, mx):
+    """A refresh of 84 blocks of width 768 (the GPT-2-small layer inputs:
+    36 single-block activations and 12 four-block ones) launches far more
+    Cholesky panel blocks than the GPU holds at once, so blocks of one
+    matrix run at different times: three refreshes in a row give the same
+    bits, and sampled blocks match the oracle."""
+    tokens = 4096
+    acts, outs, nbl = [], [], []
+    for a in range(48):
+        width, nb = (3072, 4) if a % 4 == 3 else (768, 1)
+        x = wl.bf16_round_np(wl.np_normal((tokens, width), 1.0, seed=42, index=a, role=wl.ROLE_ACT))
+        acts.append(x)
+        nbl.append(nb)
+    at = [dev(x, torch.bfloat16) for x in acts]
+    runs = []
+    for _ in range(3):
+        outs = [torch.empty((nb, 768, 768), device="cuda") for nb in nbl]
+        ctx.newton_refresh(at, outs, nbl)
+        torch.cuda.synchronize()
+        ctx.check_device()
+        runs.append(outs)
+    for other in runs[1:]:
+        for x, y in zip(runs[0], other):
+            assert torch.equal(x, y)
+    for a in (0, 3, 17, 46, 47):
+        for b in range(nbl[a]):
+            want = oracle.spd_inverse(oracle.second_moment(acts[a][:, b * 768:(b + 1) * 768]))
+            assert rel_fro(to_np(runs[0][a][b]), want) < NEWTON_TOL, (a, b)
 
 
 def _s_inv_blocks(tokens, d, nb, seed, index):
