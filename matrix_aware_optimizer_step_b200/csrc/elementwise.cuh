@@ -136,41 +136,26 @@ __global__ void __launch_bounds__(EW_THREADS)
     // 256 consecutive elements (the matrix has at least as many 64x64 tiles
     // as 4096-element runs; the blocks past its end store a zero partial).
     const int64_t n = d.rows * d.cols;
-    // both vectors' loads are issued before any store (the stores could
-    // alias the loads as far as the compiler knows, so it would not hoist
-    // them), doubling the bytes each thread has in flight
-    float g[2][8], b[2][8];
-    bool in[2];
 #pragma unroll
     for (int it = 0; it < 2; ++it) {
       const int64_t e = lt * (EW_TILE * EW_TILE) + (threadIdx.x + it * EW_THREADS) * 8;
-      in[it] = e < n;
-      if (!in[it]) continue;
-      load8_grad(d.grad, d.grad_dtype, e, g[it]);
+      if (e >= n) continue;
+      float g[8], u[8];
+      load8_grad(d.grad, d.grad_dtype, e, g);
       if (MODE == 0) {
-        const float4* bp = reinterpret_cast<const float4*>(d.momentum + e);
+        float4* bp = reinterpret_cast<float4*>(d.momentum + e);
         const float4 b0 = bp[0], b1 = bp[1];
-        b[it][0] = b0.x; b[it][1] = b0.y; b[it][2] = b0.z; b[it][3] = b0.w;
-        b[it][4] = b1.x; b[it][5] = b1.y; b[it][6] = b1.z; b[it][7] = b1.w;
-      }
-    }
-#pragma unroll
-    for (int it = 0; it < 2; ++it) {
-      if (!in[it]) continue;
-      const int64_t e = lt * (EW_TILE * EW_TILE) + (threadIdx.x + it * EW_THREADS) * 8;
-      float u[8];
-      if (MODE == 0) {
+        float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          b[it][k] = beta * b[it][k] + (1.f - beta) * g[it][k];
-          u[k] = nesterov ? (1.f - beta) * g[it][k] + beta * b[it][k] : b[it][k];
+          b[k] = beta * b[k] + (1.f - beta) * g[k];
+          u[k] = nesterov ? (1.f - beta) * g[k] + beta * b[k] : b[k];
         }
-        float4* bp = reinterpret_cast<float4*>(d.momentum + e);
-        bp[0] = make_float4(b[it][0], b[it][1], b[it][2], b[it][3]);
-        bp[1] = make_float4(b[it][4], b[it][5], b[it][6], b[it][7]);
+        bp[0] = make_float4(b[0], b[1], b[2], b[3]);
+        bp[1] = make_float4(b[4], b[5], b[6], b[7]);
       } else {
 #pragma unroll
-        for (int k = 0; k < 8; ++k) u[k] = g[it][k];
+        for (int k = 0; k < 8; ++k) u[k] = g[k];
       }
 #pragma unroll
       for (int k = 0; k < 8; ++k) ss += u[k] * u[k];
@@ -184,25 +169,7 @@ __global__ void __launch_bounds__(EW_THREADS)
     return;
   }
   const bool vec_ok = (d.cols % 8 == 0) && (d.ld % 8 == 0);
-  // 64 rows x 8 vectors of 8 columns = 512 vectors, 2 per thread; the loads
-  // of both are issued before any store
-  float gv[2][8], bv[2][8];
-  bool full[2];
-#pragma unroll
-  for (int it = 0; it < 2; ++it) {
-    const int v = threadIdx.x + it * EW_THREADS;
-    const int64_t r = r0 + (v >> 3), c = c0 + (v & 7) * 8;
-    full[it] = r < d.rows && vec_ok && c + 8 <= d.cols;
-    if (!full[it]) continue;
-    const int64_t idx = r * d.cols + c;
-    load8_grad(d.grad, d.grad_dtype, idx, gv[it]);
-    if (MODE == 0) {
-      const float4* bp = reinterpret_cast<const float4*>(d.momentum + idx);
-      const float4 b0 = bp[0], b1 = bp[1];
-      bv[it][0] = b0.x; bv[it][1] = b0.y; bv[it][2] = b0.z; bv[it][3] = b0.w;
-      bv[it][4] = b1.x; bv[it][5] = b1.y; bv[it][6] = b1.z; bv[it][7] = b1.w;
-    }
-  }
+  // 64 rows x 8 vectors of 8 columns = 512 vectors, 2 per thread
 #pragma unroll
   for (int it = 0; it < 2; ++it) {
     const int v = threadIdx.x + it * EW_THREADS;
@@ -210,22 +177,24 @@ __global__ void __launch_bounds__(EW_THREADS)
     const int64_t r = r0 + rl, c = c0 + cl;
     if (r >= d.rows) continue;
     float u[8];
-    if (full[it]) {
+    if (vec_ok && c + 8 <= d.cols) {
       const int64_t idx = r * d.cols + c;
+      float g[8];
+      load8_grad(d.grad, d.grad_dtype, idx, g);
       if (MODE == 0) {
-        float* b = bv[it];
-        const float* g = gv[it];
+        float4* bp = reinterpret_cast<float4*>(d.momentum + idx);
+        float4 b0 = bp[0], b1 = bp[1];
+        float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           b[k] = beta * b[k] + (1.f - beta) * g[k];
           u[k] = nesterov ? (1.f - beta) * g[k] + beta * b[k] : b[k];
         }
-        float4* bp = reinterpret_cast<float4*>(d.momentum + idx);
         bp[0] = make_float4(b[0], b[1], b[2], b[3]);
         bp[1] = make_float4(b[4], b[5], b[6], b[7]);
       } else {
 #pragma unroll
-        for (int k = 0; k < 8; ++k) u[k] = gv[it][k];
+        for (int k = 0; k < 8; ++k) u[k] = g[k];
       }
 #pragma unroll
       for (int k = 0; k < 8; ++k) ss += u[k] * u[k];

@@ -76,10 +76,7 @@
 
 namespace muon {
 
-enum EpiKind : int {
-  EPI_GRAM = 0, EPI_POLY = 1, EPI_UPDATE = 2, EPI_GRAM32 = 3, EPI_PRECOND = 4, EPI_UPDATE_APPLY = 5,
-  EPI_UPDATE_WIDE = 6   // the update product on 256 x 512 pair tiles (long K)
-};
+enum EpiKind : int { EPI_GRAM = 0, EPI_POLY = 1, EPI_UPDATE = 2, EPI_GRAM32 = 3, EPI_PRECOND = 4, EPI_UPDATE_APPLY = 5 };
 
 namespace gemm_cfg {
 constexpr int TM = 256;                              // pair tile rows (128 per CTA)
@@ -91,37 +88,26 @@ constexpr int BK = 64;
 // chunks (below) and spend the space saved on a fifth / sixth stage; the
 // update also has no mirrored blocks.
 __host__ __device__ constexpr int stages_for(int kind) {
-  return kind == 0 ? 5 : kind == 1 ? 4 : kind == 2 ? 6 : kind == 5 ? 4 : kind == 6 ? 4 : 7;
+  return kind == 0 ? 5 : kind == 1 ? 4 : kind == 2 ? 6 : kind == 5 ? 5 : 7;
 }
-// EPI_UPDATE_WIDE: the pair tile is 256 x 512; each K step issues two
-// N = 256 products that share the A operand, into the two halves of TMEM,
-// so a tile needs 48 KB of operands per CTA and 64-deep K block instead of
-// 2 x 32 KB for two 256 x 256 tiles (a quarter fewer bytes from L2 per
-// FLOP).  Both accumulators hold one tile, so the epilogue is not
-// overlapped with the next tile's products: worth it only for long K.
-__host__ __device__ constexpr bool wide_kind(int kind) { return kind == 6; }
-__host__ __device__ constexpr int tile_n(int kind) { return wide_kind(kind) ? 512 : 256; }
-__host__ __device__ constexpr int n_acc(int kind) { return wide_kind(kind) ? 1 : 2; }
 // GRAM32 and PRECOND write fp32 straight from registers: no epilogue buffers,
 // so their pipelines take the shared memory.
 __host__ __device__ constexpr bool fp32_out(int kind) { return kind == 3 || kind == 4; }
 // The last update of an optimizer step may apply W <- W (1 - lr wd) - lr
-// scale O in its epilogue (EPI_UPDATE_APPLY): W moves through a ring of
-// W_NBUF 4 KB 32x32 fp32 chunk buffers per warp by TMA, and O never reaches
-// memory.  Each buffer is refilled with the warp's next chunk (possibly of a
-// later tile) as soon as the store before it has read it, so weight loads
-// run W_NBUF - 1 chunks ahead of the stores.
-constexpr int W_NBUF = 3;
+// scale O in its epilogue (EPI_UPDATE_APPLY): W moves through two 4 KB
+// 32x32 fp32 chunk buffers per warp by TMA, and O never reaches memory.
+// (A ring of three buffers refilled across tiles, with one stage fewer to
+// make room, measured slower on GPT-2-small and Llama-3-8B shapes.)
+constexpr int W_NBUF = 2;
 __host__ __device__ constexpr bool apply_out(int kind) { return kind == 5; }
 __host__ __device__ constexpr bool mirrors(int kind) { return kind == 0 || kind == 1; }
 // Output leaves through two alternating 32x32 chunk buffers per warp
 // (GRAM, UPDATE) instead of a whole 32x128 slice (POLY reads its input A
 // into the slice and overwrites it in place).
-__host__ __device__ constexpr bool chunked_out(int kind) { return kind == 0 || kind == 2 || kind == 6; }
+__host__ __device__ constexpr bool chunked_out(int kind) { return kind == 0 || kind == 2; }
 constexpr int A_BYTES = HM * BK * 2;                 // 16 KB
 constexpr int B_BYTES = HN * BK * 2;                 // 16 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;       // 32 KB per CTA
-__host__ __device__ constexpr int stage_bytes(int kind) { return A_BYTES + (tile_n(kind) / 2) * BK * 2; }
 constexpr int MN_CHUNK_BYTES = BK * 128;             // one 64-wide MN chunk of B (MN-major)
 constexpr int EPI_WARPS = 8;
 constexpr int THREADS = 64 + EPI_WARPS * 32;         // producer, MMA, 8 epilogue warps
@@ -134,7 +120,7 @@ constexpr int CH_BUFS = 2;
 constexpr int WCH_BYTES = 32 * 128;                  // 32 x 32 fp32 weight chunk, 128-byte swizzle
 constexpr int BAR_BYTES = 384;
 __host__ __device__ constexpr int smem_bytes(int kind) {
-  return stages_for(kind) * stage_bytes(kind) +
+  return stages_for(kind) * STAGE_BYTES +
          EPI_WARPS * ((apply_out(kind)     ? W_NBUF * WCH_BYTES
                        : chunked_out(kind) ? CH_BUFS * CH_BYTES
                        : fp32_out(kind)    ? 0
@@ -154,8 +140,7 @@ static_assert((2 * 7 + 5 + W_NBUF * EPI_WARPS) * 8 + 8 <= BAR_BYTES, "barrier ar
 constexpr int ACC_COLS = 256;                        // one fp32 128x256 accumulator per CTA
 constexpr int TMEM_COLS = 2 * ACC_COLS;              // double-buffered
 static_assert(smem_bytes(0) <= 232448 && smem_bytes(1) <= 232448 && smem_bytes(2) <= 232448 &&
-                  smem_bytes(3) <= 232448 && smem_bytes(4) <= 232448 && smem_bytes(5) <= 232448 &&
-                  smem_bytes(6) <= 232448,
+                  smem_bytes(3) <= 232448 && smem_bytes(4) <= 232448 && smem_bytes(5) <= 232448,
               "shared memory per block");
 }  // namespace gemm_cfg
 
@@ -566,132 +551,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
       }
     }
     __syncwarp();
-  } else if constexpr (apply_out(KIND)) {
-    // ---------------- UPDATE_APPLY epilogue: W chunks through a ring ----------------
-    const int ew = warp - 2;
-    const int q = warp & 3;                 // TMEM lane quarter this warp may read
-    const int half = ew >> 2;               // 128-column half of the tile
-    uint8_t* ring = smem_epi + ew * SLICE;  // W_NBUF chunk buffers
-    uint64_t* wbar = aux_bar + W_NBUF * ew;
-    const uint32_t tempty0 = map_to_cta(smem_u32(tempty_bar), 0);
-    // The warp's chunk sequence: for each of its tiles on which it is active,
-    // the 32-column chunks of its 32 x 128 slice that lie inside the matrix.
-    // lane 0 loads chunk k into buffer k % W_NBUF; the cursor (ct, cc) is the
-    // next chunk to load.
-    int ct = pair, cc = 0;
-    uint32_t issued = 0, used = 0;
-    auto issue_next = [&]() {
-      while (ct < total) {
-        int pi, bidx, ti, tj;
-        decode_tile(KIND, args, ct, pi, bidx, ti, tj);
-        const GemmProblem& P = args.p[pi];
-        const int rbase = (ti * 2 + static_cast<int>(rank)) * HM + q * 32;
-        const int cbase = (tj * 2 + half) * 128 + cc * 32;
-        if (rbase < P.M && cc < 4 && cbase < P.N) {
-          const ApplyDesc& ad = args.apply[P.apply_base + bidx];
-          const int b = static_cast<int>(issued % W_NBUF);
-          mbar_arrive_expect_tx(&wbar[b], WCH_BYTES);
-          if (ad.transposed) tma_load_3d(ring + b * WCH_BYTES, &ad.w, &wbar[b], rbase, cbase, 0);
-          else tma_load_3d(ring + b * WCH_BYTES, &ad.w, &wbar[b], cbase, rbase, 0);
-          ++issued;
-          ++cc;
-          return;
-        }
-        ct += npairs;
-        cc = 0;
-      }
-    };
-    if (lane == 0)
-      for (int k = 0; k < W_NBUF; ++k) issue_next();
-    int lt = 0;
-    for (int t = pair; t < total; t += npairs, ++lt) {
-      int pi, bidx, ti, tj;
-      decode_tile(KIND, args, t, pi, bidx, ti, tj);
-      const GemmProblem& P = args.p[pi];
-      const int acc = lt & 1;
-      const int rbase = (ti * 2 + static_cast<int>(rank)) * HM + q * 32;
-      const int col0 = (tj * 2 + half) * 128;
-      const bool active = col0 < P.N && rbase < P.M;
-      // warp-uniform decision: tcgen05.ld below is warp-collective
-      const bool got = mbar_wait(&tfull_bar[acc], (lt >> 1) & 1, args.err, abort_flag);
-      if (!__all_sync(0xffffffffu, got)) break;
-      tc_fence_after();
-      bool ok = true;
-      if (active) {
-        float alpha = 1.0f;
-        if (P.norm2 != nullptr) alpha = 1.0f / (sqrtf(P.norm2[bidx]) + args.eps);
-        const ApplyDesc& ad = args.apply[P.apply_base + bidx];
-        const float dec = ad.decay, lrs = ad.lr_scale;
-#pragma unroll 1
-        for (int c32 = 0; c32 < 4; ++c32) {
-          const int cbase = col0 + c32 * 32;
-          if (cbase >= P.N) break;
-          uint32_t raw[32];
-          tmem_ld_32x32b_x32(tmem + acc * ACC_COLS + (static_cast<uint32_t>(q * 32) << 16) + half * 128 + c32 * 32,
-                             raw);
-          tmem_ld_wait();
-          const int b = static_cast<int>(used % W_NBUF);
-          uint8_t* wbuf = ring + b * WCH_BYTES;
-          // lane 0 issued the load; all lanes wait on its barrier
-          const bool okw = mbar_wait(&wbar[b], (used / W_NBUF) & 1u, args.err, abort_flag);
-          if (!__all_sync(0xffffffffu, okw)) { ok = false; break; }
-          if (!ad.transposed) {
-            // row `lane` of the chunk: 16-byte unit u at unit u ^ (lane % 8)
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              float4* pw = reinterpret_cast<float4*>(wbuf + lane * 128 + ((u ^ (lane & 7)) << 4));
-              float4 w = *pw;
-              w.x = w.x * dec - lrs * (alpha * __uint_as_float(raw[u * 4 + 0]));
-              w.y = w.y * dec - lrs * (alpha * __uint_as_float(raw[u * 4 + 1]));
-              w.z = w.z * dec - lrs * (alpha * __uint_as_float(raw[u * 4 + 2]));
-              w.w = w.w * dec - lrs * (alpha * __uint_as_float(raw[u * 4 + 3]));
-              *pw = w;
-            }
-          } else {
-            // W is X'^T: element k of this lane's row is W[cbase + k][rbase + lane],
-            // row k of the chunk, column `lane`
-#pragma unroll
-            for (int k = 0; k < 32; ++k) {
-              float* pw = reinterpret_cast<float*>(wbuf + k * 128 + ((((lane >> 2) ^ k) & 7) << 4) + (lane & 3) * 4);
-              *pw = *pw * dec - lrs * (alpha * __uint_as_float(raw[k]));
-            }
-          }
-          fence_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            if (ad.transposed) tma_store_3d(&ad.w, wbuf, rbase, cbase, 0);
-            else tma_store_3d(&ad.w, wbuf, cbase, rbase, 0);
-            bulk_commit_group();
-            // the store before this one has read its buffer: refill that
-            // buffer with the next chunk of the sequence
-            if (used >= 1) {
-              bulk_wait_group_read1();
-              issue_next();
-            }
-          }
-          ++used;
-          __syncwarp();
-        }
-      }
-      if (!ok) break;
-      // this warp's tcgen05.ld reads of the accumulator have completed
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster_relaxed(tempty0 + acc * 8);   // leader's tempty_bar[acc]
-    }
-    if (lane == 0) {
-      // loads issued but not consumed (after an abort) land before exit
-      volatile int no_abort = 0;
-      for (uint32_t k = used; k < issued; ++k) mbar_wait(&wbar[k % W_NBUF], (k / W_NBUF) & 1u, args.err, &no_abort);
-      bulk_wait_group0();
-    }
-    __syncwarp();
   } else {
     // ---------------- epilogue (warps 2..9, both CTAs) ----------------
     const int ew = warp - 2;
     const int q = warp & 3;                 // TMEM lane quarter this warp may read
     const int half = ew >> 2;               // 128-column half of the tile
     uint8_t* slice = smem_epi + ew * SLICE;
+    uint32_t wph = 0;                       // UPDATE_APPLY: phase bit per weight buffer (bits 0, 1)
+    uint32_t wpend = 0;                     // UPDATE_APPLY: weight loads in flight per buffer
     uint32_t nch = 0;                       // output chunks stored so far (buffer = nch & 1)
     uint8_t* stg = smem_stg + ew * STG_BYTES;
     const uint32_t tempty0 = map_to_cta(smem_u32(tempty_bar), 0);
@@ -718,6 +585,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
       const bool two_boxes = col0 + 64 < P.N;
       // the slice is free once the previous tile's TMA store has read it;
       // then fetch this tile's epilogue input into it
+      if constexpr (apply_out(KIND)) {
+        // weight chunks 0 and 1 of this tile into the two buffers, once the
+        // previous tile's stores have read them
+        if (lane == 0 && active) {
+          bulk_wait_group_read0();
+          const ApplyDesc& ad = args.apply[P.apply_base + bidx];
+          for (int c = 0; c < 2 && col0 + c * 32 < P.N; ++c) {
+            const int cb = col0 + c * 32;
+            mbar_arrive_expect_tx(&aux_bar[2 * ew + c], WCH_BYTES);
+            if (ad.transposed) tma_load_3d(slice + c * WCH_BYTES, &ad.w, &aux_bar[2 * ew + c], rbase, cb, 0);
+            else tma_load_3d(slice + c * WCH_BYTES, &ad.w, &aux_bar[2 * ew + c], cb, rbase, 0);
+            wpend |= 1u << c;
+          }
+        }
+      }
       if (lane == 0 && KIND == EPI_POLY) {
         bulk_wait_group_read0();
         if (active) {
@@ -781,6 +663,54 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
                   if (cbase + k < P.N) P.out32[zoff + static_cast<int64_t>(cbase + k) * P.out32_ld + r] = v[k];
               }
             }
+          } else if constexpr (apply_out(KIND)) {
+            const ApplyDesc& ad = args.apply[P.apply_base + bidx];
+            const int wb = c32 & 1;
+            uint8_t* wbuf = slice + wb * WCH_BYTES;
+            // lane 0 issued the load; all lanes wait on its barrier
+            const bool okw = mbar_wait(&aux_bar[2 * ew + wb], (wph >> wb) & 1u, args.err, abort_flag);
+            if (!__all_sync(0xffffffffu, okw)) break;
+            wph ^= 1u << wb;
+            wpend &= ~(1u << wb);
+            const float dec = ad.decay, lrs = ad.lr_scale;
+            if (!ad.transposed) {
+              // row `lane` of the chunk: 16-byte unit u at unit u ^ (lane % 8)
+#pragma unroll
+              for (int u = 0; u < 8; ++u) {
+                float4* pw = reinterpret_cast<float4*>(wbuf + lane * 128 + ((u ^ (lane & 7)) << 4));
+                float4 w = *pw;
+                w.x = w.x * dec - lrs * (alpha * __uint_as_float(raw[u * 4 + 0]));
+                w.y = w.y * dec - lrs * (alpha * __uint_as_float(raw[u * 4 + 1]));
+                w.z = w.z * dec - lrs * (alpha * __uint_as_float(raw[u * 4 + 2]));
+                w.w = w.w * dec - lrs * (alpha * __uint_as_float(raw[u * 4 + 3]));
+                *pw = w;
+              }
+            } else {
+              // W is X'^T: element k of this lane's row is W[cbase + k][rbase + lane],
+              // row k of the chunk, column `lane`
+#pragma unroll
+              for (int k = 0; k < 32; ++k) {
+                float* pw = reinterpret_cast<float*>(wbuf + k * 128 + ((((lane >> 2) ^ k) & 7) << 4) + (lane & 3) * 4);
+                *pw = *pw * dec - lrs * (alpha * __uint_as_float(raw[k]));
+              }
+            }
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              if (ad.transposed) tma_store_3d(&ad.w, wbuf, rbase, cbase, 0);
+              else tma_store_3d(&ad.w, wbuf, cbase, rbase, 0);
+              bulk_commit_group();
+              // chunk c32 + 2 into this buffer once the store has read it
+              const int cn = cbase + 64;
+              if (c32 + 2 < 4 && cn < P.N) {
+                bulk_wait_group_read0();
+                mbar_arrive_expect_tx(&aux_bar[2 * ew + wb], WCH_BYTES);
+                if (ad.transposed) tma_load_3d(wbuf, &ad.w, &aux_bar[2 * ew + wb], rbase, cn, 0);
+                else tma_load_3d(wbuf, &ad.w, &aux_bar[2 * ew + wb], cn, rbase, 0);
+                wpend |= 1u << wb;
+              }
+            }
+            wpend = __shfl_sync(0xffffffffu, wpend, 0);
           } else if constexpr (chunked_out(KIND)) {
             float v[32];
 #pragma unroll
@@ -887,6 +817,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
         volatile int no_abort = 0;
         mbar_wait(&aux_bar[ew], aux_phase, args.err, &no_abort);   // let the copy land
       }
+      for (int b = 0; b < 2; ++b)
+        if (wpend & (1u << b)) {
+          volatile int no_abort = 0;
+          mbar_wait(&aux_bar[2 * ew + b], (wph >> b) & 1u, args.err, &no_abort);
+        }
       bulk_wait_group0();
     }
     __syncwarp();

@@ -68,6 +68,16 @@ __device__ __forceinline__ void st_cluster_v4(uint32_t local_addr, uint32_t rank
                : "memory");
 }
 
+// 16-byte global -> shared copy that does not pass through registers;
+// src_bytes (0..16) are read, the rest of the 16 bytes is zero-filled.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
 __device__ __forceinline__ void fence_async_cluster() {
   asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
 }
@@ -157,49 +167,47 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(small_cfg::THREADS, 
   };
 
   for (int z = pair; z < count; z += npairs) {
-    // ---- X0 into XR (this CTA's rows) and XC (this CTA's columns), zero padded
+    // ---- X0 into XR (this CTA's rows) and XC (this CTA's columns), zero
+    // padded: every 16-byte piece is an asynchronous copy, all in flight at
+    // once (a piece past the matrix reads nothing and is zero-filled)
     const __nv_bfloat16* x0 = args.x_in + static_cast<int64_t>(z) * args.bs;
+#pragma unroll 4
     for (int v = threadIdx.x; v < 128 * (MAXD / 8); v += THREADS) {
       const int r = v >> 5, c = (v & 31) * 8;                 // XR: row r, columns c..c+7
       const int gr = static_cast<int>(rank) * 128 + r;
-      uint4 w = make_uint4(0, 0, 0, 0);
-      if (gr < m && c < n) {
-        w = *reinterpret_cast<const uint4*>(x0 + static_cast<int64_t>(gr) * args.ld + c);
-        if (c + 8 > n) {
-          __nv_bfloat16* e = reinterpret_cast<__nv_bfloat16*>(&w);
-          for (int k = n - c; k < 8; ++k) e[k] = __float2bfloat16_rn(0.f);
-        }
-      }
-      *reinterpret_cast<uint4*>(XR + kmaj_off(r, c)) = w;
+      const bool in = gr < m && c < n;
+      const uint32_t bytes = in ? static_cast<uint32_t>(min(8, n - c) * 2) : 0u;
+      cp_async16(XR + kmaj_off(r, c), in ? x0 + static_cast<int64_t>(gr) * args.ld + c : x0, bytes);
     }
+#pragma unroll 4
     for (int v = threadIdx.x; v < MAXD * 16; v += THREADS) {
       const int k = v >> 4, c = (v & 15) * 8;                 // XC: row k, local columns c..c+7
       const int gc = static_cast<int>(rank) * 128 + c;
-      uint4 w = make_uint4(0, 0, 0, 0);
-      if (k < m && gc < n) {
-        w = *reinterpret_cast<const uint4*>(x0 + static_cast<int64_t>(k) * args.ld + gc);
-        if (gc + 8 > n) {
-          __nv_bfloat16* e = reinterpret_cast<__nv_bfloat16*>(&w);
-          for (int j = n - gc; j < 8; ++j) e[j] = __float2bfloat16_rn(0.f);
-        }
-      }
-      *reinterpret_cast<uint4*>(XC + mnmaj_off(k, c)) = w;
+      const bool in = k < m && gc < n;
+      const uint32_t bytes = in ? static_cast<uint32_t>(min(8, n - gc) * 2) : 0u;
+      cp_async16(XC + mnmaj_off(k, c), in ? x0 + static_cast<int64_t>(k) * args.ld + gc : x0, bytes);
     }
     const float s = 1.0f / (sqrtf(args.norm2[z]) + args.eps);
+    cp_async_wait_all();
     end_phase();
 
     for (int it = 0; it < args.steps; ++it) {
       const float ag = it == 0 ? s * s : 1.0f, au = it == 0 ? s : 1.0f;
       const bool last = it == args.steps - 1;
       // ---- Gram: acc0 = X X^T (K-major X rows as both operands)
-      if (issuer && *abort_flag == 0) {
-        tc_fence_after();
-        const uint32_t xr = smem_u32(XR);
-        for (int k = 0; k < kx; k += 16) {
-          const uint64_t d = sdesc_kmajor_sw128(xr + (k >> 6) * CHUNK + (k & 63) * 2);
-          mma_bf16_ss_pair(tmem, d, d, idesc_k, k > 0 ? 1u : 0u);
+      if (warp == 0) {
+        if (issuer && *abort_flag == 0) {
+          tc_fence_after();
+          const uint32_t xr = smem_u32(XR);
+          for (int k = 0; k < kx; k += 16) {
+            const uint64_t d = sdesc_kmajor_sw128(xr + (k >> 6) * CHUNK + (k & 63) * 2);
+            mma_bf16_ss_pair(tmem, d, d, idesc_k, k > 0 ? 1u : 0u);
+          }
+          mma_commit_pair_mc(done_bar, 0x3);
         }
-        mma_commit_pair_mc(done_bar, 0x3);
+        // the other lanes of the issuing warp wait here rather than spin
+        // on the barrier beside the issuing lane
+        __syncwarp();
       }
       if (wait_done()) {
         // A = alpha X X^T, rounded to bf16, into AB (row il, columns h*128..)
@@ -218,14 +226,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(small_cfg::THREADS, 
       }
       end_phase();
       // ---- polynomial: acc1 = A A (A symmetric: its rows are both operands)
-      if (issuer && *abort_flag == 0) {
-        tc_fence_after();
-        const uint32_t ab = smem_u32(AB);
-        for (int k = 0; k < km; k += 16) {
-          const uint64_t d = sdesc_kmajor_sw128(ab + (k >> 6) * CHUNK + (k & 63) * 2);
-          mma_bf16_ss_pair(tmem + ACC, d, d, idesc_k, k > 0 ? 1u : 0u);
+      if (warp == 0) {
+        if (issuer && *abort_flag == 0) {
+          tc_fence_after();
+          const uint32_t ab = smem_u32(AB);
+          for (int k = 0; k < km; k += 16) {
+            const uint64_t d = sdesc_kmajor_sw128(ab + (k >> 6) * CHUNK + (k & 63) * 2);
+            mma_bf16_ss_pair(tmem + ACC, d, d, idesc_k, k > 0 ? 1u : 0u);
+          }
+          mma_commit_pair_mc(done_bar, 0x3);
         }
-        mma_commit_pair_mc(done_bar, 0x3);
+        // the other lanes of the issuing warp wait here rather than spin
+        // on the barrier beside the issuing lane
+        __syncwarp();
       }
       if (wait_done()) {
         // B' = b A + c A A + a I from the bf16 A in AB, overwritten in place
@@ -256,15 +269,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(small_cfg::THREADS, 
       }
       end_phase();
       // ---- update: acc0 = B' X (B' rows K-major, X columns MN-major)
-      if (issuer && *abort_flag == 0) {
-        tc_fence_after();
-        const uint32_t ab = smem_u32(AB), xc = smem_u32(XC);
-        for (int k = 0; k < km; k += 16) {
-          const uint64_t da = sdesc_kmajor_sw128(ab + (k >> 6) * CHUNK + (k & 63) * 2);
-          const uint64_t db = sdesc_mnmajor_sw128(xc + (k >> 6) * CHUNK + (k & 63) * 128, CHUNK / 2);
-          mma_bf16_ss_pair(tmem, da, db, idesc_mn, k > 0 ? 1u : 0u);
+      if (warp == 0) {
+        if (issuer && *abort_flag == 0) {
+          tc_fence_after();
+          const uint32_t ab = smem_u32(AB), xc = smem_u32(XC);
+          for (int k = 0; k < km; k += 16) {
+            const uint64_t da = sdesc_kmajor_sw128(ab + (k >> 6) * CHUNK + (k & 63) * 2);
+            const uint64_t db = sdesc_mnmajor_sw128(xc + (k >> 6) * CHUNK + (k & 63) * 128, CHUNK / 2);
+            mma_bf16_ss_pair(tmem, da, db, idesc_mn, k > 0 ? 1u : 0u);
+          }
+          mma_commit_pair_mc(done_bar, 0x3);
         }
-        mma_commit_pair_mc(done_bar, 0x3);
+        // the other lanes of the issuing warp wait here rather than spin
+        // on the barrier beside the issuing lane
+        __syncwarp();
       }
       if (wait_done()) {
         if (!last) {
@@ -317,6 +335,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(small_cfg::THREADS, 
         } else {
           // weight step from the fp32 accumulator: W <- W decay - lr scale O,
           // O = alpha B' X (W is O^T for a tall matrix)
+          // The 32 weights of a chunk are all loaded before any is stored:
+          // one read-modify-write after another would wait a full memory
+          // round trip per element (the stores may alias the next loads as
+          // far as the compiler knows).
           const MatDesc& d = args.apply[z];
 #pragma unroll 1
           for (int c32 = 0; c32 < 4; ++c32) {
@@ -325,14 +347,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(small_cfg::THREADS, 
             tmem_ld_wait();
             const int j0 = h * 128 + c32 * 32;
             if (gi < m && j0 < n) {
+              float w[32];
+              const bool vec = !d.transposed && j0 + 32 <= n && (d.cols & 3) == 0;
+              float* row = d.weight + static_cast<int64_t>(gi) * d.cols + j0;   // !transposed
+              if (vec) {
 #pragma unroll
-              for (int k = 0; k < 32; ++k) {
-                if (j0 + k < n) {
-                  const float o = au * __uint_as_float(raw[k]);
-                  float* w = d.transposed ? d.weight + static_cast<int64_t>(j0 + k) * d.cols + gi
-                                          : d.weight + static_cast<int64_t>(gi) * d.cols + j0 + k;
-                  *w = *w * d.decay - d.lr_scale * o;
+                for (int u = 0; u < 8; ++u) {
+                  const float4 q = reinterpret_cast<const float4*>(row)[u];
+                  w[u * 4] = q.x; w[u * 4 + 1] = q.y; w[u * 4 + 2] = q.z; w[u * 4 + 3] = q.w;
                 }
+              } else {
+#pragma unroll
+                for (int k = 0; k < 32; ++k)
+                  w[k] = j0 + k < n ? (d.transposed ? d.weight[static_cast<int64_t>(j0 + k) * d.cols + gi] : row[k])
+                                    : 0.f;
+              }
+#pragma unroll
+              for (int k = 0; k < 32; ++k) w[k] = w[k] * d.decay - d.lr_scale * (au * __uint_as_float(raw[k]));
+              if (vec) {
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                  reinterpret_cast<float4*>(row)[u] = make_float4(w[u * 4], w[u * 4 + 1], w[u * 4 + 2], w[u * 4 + 3]);
+              } else {
+#pragma unroll
+                for (int k = 0; k < 32; ++k)
+                  if (j0 + k < n) {
+                    if (d.transposed) d.weight[static_cast<int64_t>(j0 + k) * d.cols + gi] = w[k];
+                    else row[k] = w[k];
+                  }
               }
             }
           }
