@@ -500,9 +500,11 @@ inline bool small_run(const Run& r) { return r.m <= small_cfg::MAXD && r.n <= sm
 
 // All ns_steps iterations of the matrices of one small run in one launch;
 // the last update stores the final X at x[ns_steps % 2], or applies the
-// weight step of matrix k from mdesc[k] when mdesc is given.
+// weight step of matrix k from mdesc[k] when mdesc is given; with mom, the
+// kernel also forms X0 itself (Nesterov momentum of matrix k from mom[k] and
+// the Frobenius norm), so the run needs no other launch.
 muon_status run_small_ns(muon_ctx* ctx, uint8_t* ws, const Run& r, const float* norm2, const muon_hparams* hp,
-                         const int* skip, cudaStream_t st, const MatDesc* mdesc) {
+                         const int* skip, cudaStream_t st, const MatDesc* mdesc, const MatDesc* mom) {
   static bool attr_done[64] = {};
   static int max_pairs[64] = {};
   const int dev = ctx->device & 63;
@@ -529,6 +531,9 @@ muon_status run_small_ns(muon_ctx* ctx, uint8_t* ws, const Run& r, const float* 
   a.bs = r.m * r.ld_n;
   a.norm2 = norm2;
   a.apply = mdesc;
+  a.mom = mom;
+  a.beta = hp->momentum;
+  a.nesterov = hp->nesterov;
   a.m = int(r.m);
   a.n = int(r.n);
   a.count = r.count;
@@ -553,19 +558,21 @@ muon_status run_small_ns(muon_ctx* ctx, uint8_t* ws, const Run& r, const float* 
 // per-matrix ||U||^2.  Runs that fit one CTA pair take one small_ns_kernel
 // launch each; for the others each product of an iteration is one launch
 // over up to MAX_PROBLEMS runs.  When run_apply is given the last product
-// applies the weight step (run_mdesc[j]: the small kernel's per-matrix
-// descriptors of run j).
+// applies the weight step (run_mdesc[j]: the per-matrix descriptors of run
+// j).  small_mom: the small kernel also runs the momentum of its matrices
+// (their X0 and norm are not in the workspace).
 muon_status run_newton_schulz(muon_ctx* ctx, uint8_t* ws, const Run* all_runs, int nall,
                               const float* const* all_norm2s, const muon_hparams* hp, const int* skip,
                               cudaStream_t st, const ApplyDesc* const* all_apply = nullptr,
-                              const MatDesc* const* run_mdesc = nullptr) {
+                              const MatDesc* const* run_mdesc = nullptr, bool small_mom = false) {
   std::vector<Run> big;
   std::vector<const float*> big_norm2;
   std::vector<const ApplyDesc*> big_apply;
   for (int j = 0; j < nall; ++j) {
     if (small_run(all_runs[j])) {
       muon_status s = run_small_ns(ctx, ws, all_runs[j], all_norm2s[j], hp, skip, st,
-                                   all_apply != nullptr && run_mdesc != nullptr ? run_mdesc[j] : nullptr);
+                                   all_apply != nullptr && run_mdesc != nullptr ? run_mdesc[j] : nullptr,
+                                   small_mom && run_mdesc != nullptr ? run_mdesc[j] : nullptr);
       if (s != MUON_OK) return s;
     } else {
       big.push_back(all_runs[j]);
@@ -923,7 +930,11 @@ muon_status collect_items(muon_ctx* ctx, const muon_group* groups, int32_t ngrou
       items.push_back(it);
     }
   }
+  // wide shapes largest first, matrices that fit one CTA pair (their whole
+  // step runs in small_ns_kernel) after all others
   std::stable_sort(items.begin(), items.end(), [](const Item& a, const Item& b) {
+    const bool sa = a.n <= small_cfg::MAXD, sb = b.n <= small_cfg::MAXD;
+    if (sa != sb) return sb;
     return a.m != b.m ? a.m > b.m : a.n > b.n;
   });
   return MUON_OK;
@@ -960,6 +971,8 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
   std::vector<int> chunk_prep_begin(chunks.size(), 0), chunk_prep_count(chunks.size(), 0);
   std::vector<std::vector<PreProblem>> chunk_pprob(chunks.size());
   const bool check = mode == 0 && hp->check_finite;
+  // the small-matrix kernel forms its matrices' X0 from the momentum itself
+  const bool small_mom = mode == 0 && hp->ns_steps >= 1;
   for (size_t ci = 0; ci < chunks.size(); ++ci) {
     Chunk& c = chunks[ci];
     int64_t tiles = 0;
@@ -1174,9 +1187,17 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
       CUDA_TRY(ctx, cudaGetLastError());
     }
     const std::vector<SegLaunch> segl = build_seg_launches(descs.data() + c.first, c.count);
-    {
+    // In a step with at least one iteration the small-matrix kernel runs the
+    // momentum of its own matrices (they sort last in the chunk), so the
+    // momentum launches cover only the items before them.
+    int n_mom = c.count;
+    if (small_mom)
+      for (const Run& r : c.runs)
+        if (small_run(r)) n_mom = std::min(n_mom, r.first - c.first);
+    if (n_mom > 0) {
+      const std::vector<SegLaunch> segm = build_seg_launches(descs.data() + c.first, n_mom);
       ProfScope ps(ctx, MUON_K_MOMENTUM, st);
-      for (const SegLaunch& L : segl) {
+      for (const SegLaunch& L : segm) {
         if (mode == 0)
           launch_pdl(momentum_kernel<0>, dim3(unsigned(L.tiles)), dim3(EW_THREADS), size_t(0), st,
               ddesc + c.first, L.t, L.tile_base, hp->momentum, hp->nesterov, skip);
@@ -1184,22 +1205,22 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
           launch_pdl(momentum_kernel<1>, dim3(unsigned(L.tiles)), dim3(EW_THREADS), size_t(0), st,
               ddesc + c.first, L.t, L.tile_base, 0.f, 0, skip);
       }
-      launch_pdl(norm_reduce_kernel, dim3(unsigned(c.count)), dim3(EW_THREADS), size_t(0), st, ddesc + c.first, skip);
+      launch_pdl(norm_reduce_kernel, dim3(unsigned(n_mom)), dim3(EW_THREADS), size_t(0), st, ddesc + c.first, skip);
+      ctx->launches += segm.size() + 1;
     }
-    ctx->launches += segl.size() + 1;
     CUDA_TRY(ctx, cudaGetLastError());
     {
       std::vector<const float*> n2(c.runs.size());
       for (size_t j = 0; j < c.runs.size(); ++j) n2[j] = norm2 + (c.runs[j].first - c.first);
       std::vector<const ApplyDesc*> ra;
       std::vector<const MatDesc*> rm;
+      for (const Run& r : c.runs) rm.push_back(ddesc + r.first);
       if (chunk_fused[ci]) {
         const ApplyDesc* dapply = reinterpret_cast<const ApplyDesc*>(static_cast<uint8_t*>(dtab) + ap_off);
         for (int64_t k : run_apply_idx[ci]) ra.push_back(dapply + k);
-        for (const Run& r : c.runs) rm.push_back(ddesc + r.first);
       }
       s = run_newton_schulz(ctx, ws, c.runs.data(), int(c.runs.size()), n2.data(), hp, skip, st,
-                            chunk_fused[ci] ? ra.data() : nullptr, chunk_fused[ci] ? rm.data() : nullptr);
+                            chunk_fused[ci] ? ra.data() : nullptr, rm.data(), small_mom);
       if (s != MUON_OK) return s;
     }
     if (!chunk_fused[ci]) {

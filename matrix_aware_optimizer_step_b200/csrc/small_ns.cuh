@@ -43,7 +43,7 @@ constexpr int MAXD = 256;                  // m, n <= 256 (wide orientation)
 constexpr int THREADS = 256;               // 8 warps, all epilogue; one thread issues the MMAs
 constexpr int PANEL = 128 * MAXD * 2;      // 64 KB: 128 rows x 256 bf16, or 256 K-rows x 128 bf16
 constexpr int CHUNK = 128 * 64 * 2;        // 16 KB: one 64-wide K chunk of a K-major panel
-constexpr int SMEM = 3 * PANEL + 1024 + 64;
+constexpr int SMEM = 3 * PANEL + 1024 + 128;
 constexpr int ACC = 256;                   // TMEM columns of one accumulator
 }  // namespace small_cfg
 
@@ -53,12 +53,23 @@ struct SmallNsArgs {
   int64_t ld, bs;
   const float* norm2;          // ||U||_F^2 of matrix z at norm2[z]
   const MatDesc* apply;        // non-null: weight step of matrix z from apply[z]
+  const MatDesc* mom;          // non-null: X0 is formed here, Nesterov momentum of
+                               // matrix z (mom[z].grad, .momentum) and ||U||_F in
+                               // the kernel, instead of read from x_in / norm2
+  float beta;
+  int nesterov;
   int m, n, count;
   int steps;
   float a, b, c, eps;
   int* err;                    // device error flags (bounded waits)
   const int* skip;             // halted() -> do nothing
 };
+
+// 4-byte store into the shared memory of CTA `rank` of this cluster.
+__device__ __forceinline__ void st_cluster_f32(uint32_t local_addr, uint32_t rank, float v) {
+  const uint32_t a = map_to_cta(local_addr, rank);
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(a), "f"(v) : "memory");
+}
 
 // 16-byte store into the shared memory of CTA `rank` of this cluster.
 __device__ __forceinline__ void st_cluster_v4(uint32_t local_addr, uint32_t rank, uint4 v) {
@@ -103,6 +114,107 @@ __device__ __forceinline__ uint4 pack8(const float* v) {
   return w;
 }
 
+// Sum over the CTA's threads (valid in every thread): warp shuffles, then
+// one partial per warp in red[], added in warp order.
+__device__ __forceinline__ float cta_sum(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float t = 0.f;
+#pragma unroll
+  for (int w = 0; w < small_cfg::THREADS / 32; ++w) t += red[w];
+  return t;
+}
+
+// One 8-column unit of wide row gi, in two halves so that several units'
+// loads can be in flight: momentum_load reads the gradient and momentum of
+// columns j0..j0+7 (zero past the matrix), momentum_finish forms U (the
+// Nesterov look-ahead of the updated momentum) and stores the momentum.
+// Wide (i, j) is the matrix's (i, j), or (j, i) when it is tall
+// (transposed: the wide rows are its columns).
+__device__ __forceinline__ bool unit_vec(const MatDesc& d, int m, int n, int gi, int j0) {
+  return gi < m && !d.transposed && j0 + 8 <= n && (n & 7) == 0;
+}
+__device__ __forceinline__ int64_t unit_idx(const MatDesc& d, int m, int n, int gi, int j) {
+  return d.transposed ? static_cast<int64_t>(j) * m + gi : static_cast<int64_t>(gi) * n + j;
+}
+__device__ __forceinline__ void momentum_load(const MatDesc& d, int m, int n, int gi, int j0, float (&g)[8],
+                                              float (&b)[8]) {
+  if (unit_vec(d, m, n, gi, j0)) {
+    const int64_t idx = unit_idx(d, m, n, gi, j0);
+    load8_grad(d.grad, d.grad_dtype, idx, g);
+    const float4* bp = reinterpret_cast<const float4*>(d.momentum + idx);
+    const float4 b0 = bp[0], b1 = bp[1];
+    b[0] = b0.x; b[1] = b0.y; b[2] = b0.z; b[3] = b0.w; b[4] = b1.x; b[5] = b1.y; b[6] = b1.z; b[7] = b1.w;
+    return;
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const bool in = gi < m && j0 + e < n;
+    const int64_t idx = unit_idx(d, m, n, gi, j0 + e);
+    g[e] = in ? load1_grad(d.grad, d.grad_dtype, idx) : 0.f;
+    b[e] = in ? d.momentum[idx] : 0.f;
+  }
+}
+__device__ __forceinline__ void momentum_finish(const MatDesc& d, float beta, int nesterov, int m, int n, int gi,
+                                                int j0, const float (&g)[8], float (&b)[8], float (&u)[8]) {
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    b[e] = beta * b[e] + (1.f - beta) * g[e];
+    u[e] = nesterov ? (1.f - beta) * g[e] + beta * b[e] : b[e];
+  }
+  if (unit_vec(d, m, n, gi, j0)) {
+    float4* bp = reinterpret_cast<float4*>(d.momentum + unit_idx(d, m, n, gi, j0));
+    bp[0] = make_float4(b[0], b[1], b[2], b[3]);
+    bp[1] = make_float4(b[4], b[5], b[6], b[7]);
+    return;
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e)
+    if (gi < m && j0 + e < n) d.momentum[unit_idx(d, m, n, gi, j0 + e)] = b[e];
+}
+
+// X0 of this CTA from the gradient and momentum: every (row, 8-column unit)
+// of its 128 wide rows, two units per thread in flight; returns the
+// thread's sum of U^2.  A non-transposed matrix takes units along a row per
+// warp (coalesced along the row), a transposed one units down a column.
+__device__ __forceinline__ float momentum_rows(const MatDesc& d, float beta, int nesterov, int m, int n,
+                                               uint32_t rank, uint8_t* XR, uint8_t* XC) {
+  using namespace small_cfg;
+  float ss = 0.f;
+  const uint32_t xc = smem_u32(XC);
+#pragma unroll 1
+  for (int v0 = threadIdx.x; v0 < 128 * (MAXD / 8); v0 += 2 * THREADS) {
+    float g[2][8], b[2][8], u[2][8];
+    int rl[2], j0[2];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const int v = v0 + q * THREADS;
+      rl[q] = d.transposed ? (v & 127) : (v >> 5);
+      j0[q] = d.transposed ? (v >> 7) * 8 : (v & 31) * 8;
+      momentum_load(d, m, n, static_cast<int>(rank) * 128 + rl[q], j0[q], g[q], b[q]);
+    }
+#pragma unroll
+    for (int q = 0; q < 2; ++q)
+      momentum_finish(d, beta, nesterov, m, n, static_cast<int>(rank) * 128 + rl[q], j0[q], g[q], b[q], u[q]);
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) ss += u[q][e] * u[q][e];
+      const uint4 w = pack8(u[q]);
+      const int gi = static_cast<int>(rank) * 128 + rl[q];
+      *reinterpret_cast<uint4*>(XR + kmaj_off(rl[q], j0[q])) = w;
+      const uint32_t off = mnmaj_off(gi, j0[q] & 127);
+      const uint32_t owner = static_cast<uint32_t>(j0[q] >> 7);
+      if (owner == rank) *reinterpret_cast<uint4*>(XC + off) = w;
+      else st_cluster_v4(xc + off, owner, w);
+    }
+  }
+  return ss;
+}
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(small_cfg::THREADS, 1)
     small_ns_kernel(const __grid_constant__ SmallNsArgs args) {
   using namespace small_cfg;
@@ -116,6 +228,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(small_cfg::THREADS, 
   uint64_t* drain_bar = done_bar + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* nslot = reinterpret_cast<float*>(tmem_slot + 2);   // ||U||^2 partial of CTA 0, CTA 1
+  float* red = nslot + 2;                                    // block reduction, one per warp
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -167,6 +281,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(small_cfg::THREADS, 
   };
 
   for (int z = pair; z < count; z += npairs) {
+    float s;
+    if (args.mom == nullptr) {
     // ---- X0 into XR (this CTA's rows) and XC (this CTA's columns), zero
     // padded: every 16-byte piece is an asynchronous copy, all in flight at
     // once (a piece past the matrix reads nothing and is zero-filled)
@@ -187,9 +303,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(small_cfg::THREADS, 
       const uint32_t bytes = in ? static_cast<uint32_t>(min(8, n - gc) * 2) : 0u;
       cp_async16(XC + mnmaj_off(k, c), in ? x0 + static_cast<int64_t>(k) * args.ld + gc : x0, bytes);
     }
-    const float s = 1.0f / (sqrtf(args.norm2[z]) + args.eps);
+    s = 1.0f / (sqrtf(args.norm2[z]) + args.eps);
     cp_async_wait_all();
     end_phase();
+    } else {
+      // ---- momentum in the kernel: this CTA forms U for its wide rows,
+      // updates their momentum, writes U (bf16) as its XR rows and, by
+      // columns, into both CTAs' XC; the two CTAs' sums of U^2 meet in
+      // nslot and are added in rank order on both sides
+      const float ss = momentum_rows(args.mom[z], args.beta, args.nesterov, m, n, rank, XR, XC);
+      const float tot = cta_sum(ss, red);
+      if (threadIdx.x == 0) {
+        nslot[rank] = tot;
+        st_cluster_f32(smem_u32(&nslot[rank]), rank ^ 1u, tot);
+      }
+      end_phase();
+      s = 1.0f / (sqrtf(nslot[0] + nslot[1]) + args.eps);
+    }
 
     for (int it = 0; it < args.steps; ++it) {
       const float ag = it == 0 ? s * s : 1.0f, au = it == 0 ? s : 1.0f;

@@ -93,11 +93,11 @@ def test_orthogonalize_custom_coefficients(ctx, mx, coeffs):
     assert rel_fro(to_np(out), want) < NS_TOL
 
 
-def test_small_matrix_step_is_three_launches(ctx, mx):
-    """A 256 x 256 step: momentum, the norm reduction and ONE launch for all
-    five iterations with the weight step applied from the fp32 accumulator;
-    momentum within 1e-5 and the applied update within the Newton-Schulz
-    tolerance of the oracle."""
+def test_small_matrix_step_is_one_launch(ctx, mx):
+    """A 256 x 256 step is ONE launch: the kernel forms the momentum and the
+    Frobenius norm, runs all five iterations and applies the weight step
+    from the fp32 accumulator; momentum within 1e-5 and the applied update
+    within the Newton-Schulz tolerance of the oracle."""
     shape = (256, 256)
     g = wl.np_normal(shape, 1.0, seed=40, index=0)
     w0 = wl.np_normal(shape, 0.02, seed=40, index=0, role=wl.ROLE_WEIGHT)
@@ -106,11 +106,41 @@ def test_small_matrix_step_is_three_launches(ctx, mx):
     ctx.step([dict(weights=[w], grads=[dev(g)], momentum=[b])])
     torch.cuda.synchronize()
     ctx.check_device()
-    assert ctx.launch_count - n0 == 3
+    assert ctx.launch_count - n0 == 1
     w1, b1, o1 = oracle.muon_step(w0, g, np.zeros(shape))
     assert rel_fro(to_np(b), b1) < EW_TOL
     upd = (w0.astype(np.float64) * (1 - 0.02 * 0.01) - to_np(w)) / 0.02
     assert rel_fro(upd, o1) < NS_TOL
+
+
+@pytest.mark.parametrize("case", [((256, 256), "f32", 2), ((250, 17), "bf16", 3), ((17, 250), "f32", 2),
+                                  ((1, 1), "f32", 2), ((129, 127), "bf16", 2)],
+                         ids=lambda c: f"{c[0][0]}x{c[0][1]}-{c[1]}")
+def test_small_matrix_momentum_in_kernel_over_steps(ctx, mx, case):
+    """The momentum the small-matrix kernel forms itself, carried over
+    steps, wide and tall, fused weight step or not (widths not a multiple
+    of 4 take the separate apply pass): the buffer within 1e-5 of the
+    oracle's, the update within the Newton-Schulz tolerance."""
+    shape, dt, steps = case
+    _step_case(ctx, mx, [shape], steps, dt, grad_std=1.0)
+    w0 = wl.np_normal(shape, 0.02, seed=44, index=0, role=wl.ROLE_WEIGHT)
+    w, b = dev(w0), torch.zeros(shape, device="cuda")
+    buf = np.zeros(shape)
+    wd = w0.astype(np.float64)
+    for step in range(steps):
+        g = wl.np_normal(shape, 1.0, seed=44, step=step, index=0)
+        if dt == "bf16":
+            g = wl.bf16_round_np(g)
+        ctx.step([dict(weights=[w], grads=[dev(g, torch.bfloat16 if dt == "bf16" else torch.float32)],
+                       momentum=[b])])
+        torch.cuda.synchronize()
+        w_prev = wd
+        wd, buf, o = oracle.muon_step(w_prev, g, buf)
+        assert rel_fro(to_np(b), buf) < EW_TOL, step
+        scale = oracle.shape_scale(shape[0], shape[1], "original")
+        upd = (w_prev * (1 - 0.02 * 0.01) - to_np(w)) / (0.02 * scale)
+        assert rel_fro(upd, o) < ns_tol(shape), step
+        wd = to_np(w)
 
 
 def test_small_matrices_batched_past_the_pair_count(ctx, mx):
