@@ -62,20 +62,39 @@ struct MatDesc {
 
 // Segments of equal-shape matrices in one launch (kernel parameter space,
 // no global memory round trip): tile -> matrix is a short scan plus one
-// division instead of a search through the descriptor table.
+// division instead of a search through the descriptor table.  Tiles are
+// counted from the launch's first block, so the lookup is 32-bit integer
+// arithmetic: every thread of a block repeats it, and a 64-bit division is
+// a long instruction sequence that, repeated per thread, made up about half
+// of the momentum kernel's issued instructions.
 constexpr int MAX_SEGS = 32;
 struct SegTable {
   int n;
-  int first_mat[MAX_SEGS];        // descriptor index of the segment's first matrix
-  int64_t tile_start[MAX_SEGS];   // first tile of the segment (launch numbering)
-  int64_t tiles_per_mat[MAX_SEGS];
+  int first_mat[MAX_SEGS];         // descriptor index of the segment's first matrix
+  uint32_t tile_start[MAX_SEGS];   // first tile of the segment, from the launch's first block
+  uint32_t tiles_per_mat[MAX_SEGS];
 };
 
-__device__ __forceinline__ int seg_find(const SegTable& t, int64_t tile) {
+struct TileLoc {
+  int mat;        // descriptor index
+  uint32_t lt;    // tile index within the matrix
+};
+
+__device__ __forceinline__ TileLoc seg_locate(const SegTable& t, uint32_t b) {
   int s = 0;
 #pragma unroll 1
-  while (s + 1 < t.n && t.tile_start[s + 1] <= tile) ++s;
-  return t.first_mat[s] + static_cast<int>((tile - t.tile_start[s]) / t.tiles_per_mat[s]);
+  while (s + 1 < t.n && t.tile_start[s + 1] <= b) ++s;
+  const uint32_t rel = b - t.tile_start[s];
+  const uint32_t k = rel / t.tiles_per_mat[s];
+  return {t.first_mat[s] + static_cast<int>(k), rel - k * t.tiles_per_mat[s]};
+}
+
+// Origin (row, column) of tile lt of a matrix with tiles_c tile columns.
+__device__ __forceinline__ void tile_origin(uint32_t lt, int32_t tiles_c, int64_t& r0, int64_t& c0) {
+  const uint32_t tc = static_cast<uint32_t>(tiles_c);
+  const uint32_t tr = lt / tc;
+  r0 = static_cast<int64_t>(tr) * EW_TILE;
+  c0 = static_cast<int64_t>(lt - tr * tc) * EW_TILE;
 }
 
 __device__ __forceinline__ void load8_grad(const void* g, int dtype, int64_t idx, float (&x)[8]) {
@@ -125,10 +144,9 @@ __global__ void __launch_bounds__(EW_THREADS)
   __shared__ __align__(16) __nv_bfloat16 tile[EW_TILE][EW_TILE];
   __shared__ float red[EW_THREADS / 32];
   const int64_t gt = tile_base + blockIdx.x;
-  const MatDesc& d = descs[seg_find(segs, gt)];
-  const int64_t lt = gt - d.tile_start;
-  const int64_t r0 = (lt / d.tiles_c) * EW_TILE;
-  const int64_t c0 = (lt % d.tiles_c) * EW_TILE;
+  const TileLoc loc = seg_locate(segs, blockIdx.x);
+  const MatDesc& d = descs[loc.mat];
+  const int64_t lt = loc.lt;
   float ss = 0.f;
   if (!d.transposed && d.ld == d.cols && (d.cols % 8) == 0) {
     // Rows are contiguous in both layouts: block lt takes elements
@@ -168,6 +186,8 @@ __global__ void __launch_bounds__(EW_THREADS)
     if (threadIdx.x == 0) d.partials[gt] = tot;
     return;
   }
+  int64_t r0, c0;
+  tile_origin(loc.lt, d.tiles_c, r0, c0);
   const bool vec_ok = (d.cols % 8 == 0) && (d.ld % 8 == 0);
   // 64 rows x 8 vectors of 8 columns = 512 vectors, 2 per thread
 #pragma unroll
@@ -289,16 +309,16 @@ __device__ __forceinline__ void store_f32x8(float* dst, const float (&o)[8]) {
 // norm_scale: when no iteration ran, O = U / (||U|| + eps) is formed here.
 template <int MODE>
 __global__ void __launch_bounds__(EW_THREADS)
-    apply_kernel(const MatDesc* __restrict__ descs, const __grid_constant__ SegTable segs, int64_t tile_base,
+    apply_kernel(const MatDesc* __restrict__ descs, const __grid_constant__ SegTable segs,
                  int normalise, float eps, const int* skip) {
   pdl_wait();      // previous kernel's results visible (no-op without PDL)
   if (halted(skip)) return;
   __shared__ __align__(16) __nv_bfloat16 tile[EW_TILE][EW_TILE];
-  const int64_t gt = tile_base + blockIdx.x;
-  const MatDesc& d = descs[seg_find(segs, gt)];
-  const int64_t lt = gt - d.tile_start;
-  const int64_t r0 = (lt / d.tiles_c) * EW_TILE;
-  const int64_t c0 = (lt % d.tiles_c) * EW_TILE;
+  const TileLoc loc = seg_locate(segs, blockIdx.x);
+  const MatDesc& d = descs[loc.mat];
+  const int64_t lt = loc.lt;
+  int64_t r0, c0;
+  tile_origin(loc.lt, d.tiles_c, r0, c0);
   const float s = normalise ? 1.0f / (sqrtf(*d.norm2) + eps) : 1.0f;
   if (!d.transposed && d.ld == d.cols && (d.cols % 8) == 0) {
     // contiguous rows: the flat element run of momentum_kernel, loads of both
@@ -408,14 +428,13 @@ __global__ void __launch_bounds__(EW_THREADS)
 // Sets *flag when any gradient element is NaN or Inf.  One 64x64 tile per
 // block, same tiling as momentum_kernel.
 __global__ void __launch_bounds__(EW_THREADS)
-    finite_kernel(const MatDesc* __restrict__ descs, const __grid_constant__ SegTable segs, int64_t tile_base,
+    finite_kernel(const MatDesc* __restrict__ descs, const __grid_constant__ SegTable segs,
                   int* flag) {
   pdl_wait();      // previous kernel's results visible (no-op without PDL)
-  const int64_t gt = tile_base + blockIdx.x;
-  const MatDesc& d = descs[seg_find(segs, gt)];
-  const int64_t lt = gt - d.tile_start;
-  const int64_t r0 = (lt / d.tiles_c) * EW_TILE;
-  const int64_t c0 = (lt % d.tiles_c) * EW_TILE;
+  const TileLoc loc = seg_locate(segs, blockIdx.x);
+  const MatDesc& d = descs[loc.mat];
+  int64_t r0, c0;
+  tile_origin(loc.lt, d.tiles_c, r0, c0);
   bool bad = false;
   for (int e = threadIdx.x; e < EW_TILE * EW_TILE; e += EW_THREADS) {
     const int64_t r = r0 + e / EW_TILE, c = c0 + e % EW_TILE;

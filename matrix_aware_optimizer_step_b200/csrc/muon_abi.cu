@@ -169,6 +169,10 @@ int device_sms(int device) {
 
 // Elementwise launches over descriptors d[0..n) whose tile_start fields are
 // set: each launch covers up to MAX_SEGS segments of equal-shape matrices.
+// The segment table counts tiles from the launch's first block (tile_base)
+// in 32 bits; a launch is one grid, at most 2^31 - 1 blocks, and every
+// tensor the library takes fits in device memory, far below 2^31 tiles of
+// 4096 elements.
 struct SegLaunch {
   SegTable t;
   int64_t tile_base;
@@ -192,8 +196,8 @@ std::vector<SegLaunch> build_seg_launches(const MatDesc* d, int n) {
     if (cur.t.n == 0) cur.tile_base = d[i].tile_start;
     const int s = cur.t.n++;
     cur.t.first_mat[s] = i;
-    cur.t.tile_start[s] = d[i].tile_start;
-    cur.t.tiles_per_mat[s] = desc_tiles(d[i]);
+    cur.t.tile_start[s] = static_cast<uint32_t>(d[i].tile_start - cur.tile_base);
+    cur.t.tiles_per_mat[s] = static_cast<uint32_t>(desc_tiles(d[i]));
   }
   if (n > 0) close(d[n - 1].tile_start + desc_tiles(d[n - 1]));
   return out;
@@ -1153,7 +1157,7 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
       ProfScope ps(ctx, MUON_K_OTHER, st);
       for (const SegLaunch& L : build_seg_launches(raw.data(), int(raw.size()))) {
       launch_pdl(finite_kernel, dim3(unsigned(L.tiles)), dim3(EW_THREADS), size_t(0), st,
-                 draw, L.t, L.tile_base, ctx->dflags + 1);
+                 draw, L.t, ctx->dflags + 1);
       ctx->launches++;
     }
     }
@@ -1228,10 +1232,10 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
       for (const SegLaunch& L : segl) {
         if (mode == 0)
           launch_pdl(apply_kernel<0>, dim3(unsigned(L.tiles)), dim3(EW_THREADS), size_t(0), st,
-              ddesc + c.first, L.t, L.tile_base, hp->ns_steps == 0, hp->eps, skip);
+              ddesc + c.first, L.t, hp->ns_steps == 0, hp->eps, skip);
         else
           launch_pdl(apply_kernel<1>, dim3(unsigned(L.tiles)), dim3(EW_THREADS), size_t(0), st,
-              ddesc + c.first, L.t, L.tile_base, hp->ns_steps == 0, hp->eps, skip);
+              ddesc + c.first, L.t, hp->ns_steps == 0, hp->eps, skip);
       }
       ctx->launches += segl.size();
     }
@@ -2017,7 +2021,7 @@ muon_status muon_orthogonalize_noalloc(const void* input, int32_t in_dtype, int6
   s = run_newton_schulz(&tmp, ws, &r, 1, &n2, hp, flags, st);
   tmp.dflags = nullptr;
   if (s != MUON_OK) return s;
-  apply_kernel<1><<<unsigned(tiles), EW_THREADS, 0, st>>>(ddesc, segl[0].t, 0, hp->ns_steps == 0, hp->eps,
+  apply_kernel<1><<<unsigned(tiles), EW_THREADS, 0, st>>>(ddesc, segl[0].t, hp->ns_steps == 0, hp->eps,
                                                           flags);
   const int64_t n = rows * cols;
   noalloc_poison_kernel<<<unsigned(std::min<int64_t>(cdiv(n, 256), 1024)), 256, 0, st>>>(flags, output, n);
