@@ -95,6 +95,7 @@ def step_work(w, aux, ns_steps=5):
         refresh_tc += nb * 2 * tokens * d * d
         refresh_alu += nb * 3 * (d ** 3 // 3)
     small = 0
+    fused_bytes = 0
     for m in w.mats:
         a, b = min(m.rows, m.cols), max(m.rows, m.cols)
         if b <= SMALL_MAX:
@@ -104,6 +105,9 @@ def step_work(w, aux, ns_steps=5):
             gram += 2 * a * a * b * ns_steps
             poly += 2 * a ** 3 * ns_steps
             upd += 2 * a * a * b * ns_steps
+            # the last update with the weight step: bf16 B' (a x a) and X
+            # (a x b) read, fp32 W read and written
+            fused_bytes += 2 * a * a + 2 * a * b + 8 * a * b
         elems += m.rows * m.cols
     gbytes = 2 if w.grad_dtype == "bf16" else 4
     aux_el = sum(n for _, n in aux)
@@ -112,9 +116,10 @@ def step_work(w, aux, ns_steps=5):
         "gram": ("flop", gram), "poly": ("flop", poly), "update": ("flop", upd),
         "ns_small": ("flop", small),
         # the last update with the weight step fused: one iteration's FLOPs
-        # and the fp32 weights read and written (8 B/element); the update
-        # class then holds the other ns_steps - 1 iterations
-        "update_apply": ("mixed", (per_iter, elems * 8)),
+        # and its compulsory HBM bytes (its operands B' and X read once, the
+        # fp32 weights read and written once); the update class then holds
+        # the other ns_steps - 1 iterations
+        "update_apply": ("mixed", (per_iter, fused_bytes)),
         # momentum: read grad + buf, write buf + bf16 U
         "momentum": ("byte", elems * (gbytes + 4 + 4 + 2)),
         # apply: read bf16 O + W, write W

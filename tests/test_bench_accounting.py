@@ -49,9 +49,12 @@ def test_gpt2_small_counts(bench):
     assert abs(ns / 1e12 - 1.63) < 0.01
     assert work["momentum"] == ("byte", elems * 12)
     assert work["adamw"] == ("byte", aux_el * 26)
-    # the fused last update: one iteration's 2 m^2 n and 8 B of fp32 weight per element
+    # the fused last update: one iteration's 2 m^2 n, and its compulsory
+    # bytes: bf16 B' (m = 768 for all 72 matrices) and X read once, fp32 W
+    # read and written once (2 m^2 + 2 m n + 8 m n)
     per_iter = sum(2 * min(m.rows, m.cols) ** 2 * max(m.rows, m.cols) for m in w.mats)
-    assert work["update_apply"] == ("mixed", (per_iter, elems * 8))
+    assert work["update_apply"] == ("mixed", (per_iter, 2 * 72 * 768 * 768 + 10 * elems))
+    assert 2 * 72 * 768 * 768 + 10 * elems == 934281216
 
 
 def test_newton_refresh_counts(bench):
