@@ -720,23 +720,31 @@ def main():
         # Pipelined like a training loop that streams gradients in and weights
         # out: step k's gradients arrive on a copy-in stream (into the device
         # set the step reads; the set is reused every n_cycle steps), the
-        # updated weights are copied on the device into one of two staging
-        # buffers and leave for the host on a copy-out stream, so PCIe in
-        # both directions overlaps the next step's kernels.
+        # updated weights are copied on the device into a staging buffer and
+        # leave for the host on a copy-out stream, so PCIe in both directions
+        # overlaps the next step's kernels.  Two staging buffers when device
+        # memory holds them, one otherwise (the next step's staging copy then
+        # waits for the previous copy-out); with no room for one, the weights
+        # leave directly and the next step waits for them before it starts.
         s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
-        staging = w_elems * 4 <= (8 << 30)          # large sets copy out of the weights directly
-        stage = [torch.empty(w_elems, dtype=torch.float32, device=dev) for _ in range(2)] if staging else None
+        torch.cuda.synchronize(dev)
+        free_b, _ = torch.cuda.mem_get_info(dev)
+        margin = 4 << 30
+        n_stage = 2 if 2 * w_elems * 4 + margin <= free_b else (1 if w_elems * 4 + margin <= free_b else 0)
+        staging = n_stage > 0
+        stage = [torch.empty(w_elems, dtype=torch.float32, device=dev) for _ in range(n_stage)]
         h_views, off = [], 0
         for t in dev_w:
             h_views.append(h_w[off:off + t.numel()].view(t.shape))
             off += t.numel()
         in_done = [torch.cuda.Event() for _ in range(n_cycle)]
         used = [torch.cuda.Event() for _ in range(n_cycle)]
-        staged = [torch.cuda.Event() for _ in range(2)]
-        out_done = [torch.cuda.Event() for _ in range(2)]
+        n_out = max(1, n_stage)
+        staged = [torch.cuda.Event() for _ in range(n_out)]
+        out_done = [torch.cuda.Event() for _ in range(n_out)]
 
         def e2e_step(k):
-            s, b = k % n_cycle, k & 1
+            s, b = k % n_cycle, k % n_out
             with torch.cuda.stream(s_in):
                 if k >= n_cycle:
                     s_in.wait_event(used[s])          # the step that last read this set is done
@@ -746,12 +754,12 @@ def main():
                 in_done[s].record(s_in)
             stream.wait_event(in_done[s])
             if not staging and k >= 1:
-                stream.wait_event(out_done[b ^ 1])    # the previous weights have left before they change
+                stream.wait_event(out_done[0])        # the previous weights have left before they change
             one_step(k)
             used[s].record(stream)
             if staging:
-                if k >= 2:
-                    stream.wait_event(out_done[b])    # staging buffer b (two steps ago) has left
+                if k >= n_out:
+                    stream.wait_event(out_done[b])    # staging buffer b (n_out steps ago) has left
                 torch.cat([t.view(-1) for t in dev_w], out=stage[b])   # one device kernel
             staged[b].record(stream)
             with torch.cuda.stream(s_out):
@@ -764,16 +772,21 @@ def main():
                 out_done[b].record(s_out)
 
         def e2e_finish():
-            stream.wait_event(out_done[(k_e2e - 1) & 1])
+            stream.wait_event(out_done[(k_e2e - 1) % n_out])
 
         ms_e2e = timed(k_e2e, e2e_step, e2e_finish)
-        # the host holds the last step's weights
-        if not torch.equal(h_w, torch.cat([t.view(-1) for t in dev_w]).cpu()):
+        # the host holds the last step's weights (compared tensor by tensor:
+        # no second device copy of the whole set)
+        if not all(torch.equal(hv, t.cpu()) for hv, t in zip(h_views, dev_w)):
             raise RuntimeError("e2e: host weights differ from the device weights")
+        del stage
+        torch.cuda.empty_cache()
         e2e = {"value": units * 1e3 * k_e2e / ms_e2e, "unit": "Muon step/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h,
-               "note": "every step: gradients host->device (copy-in stream), updated fp32 weights device->device->host "
-                       "(copy-out stream), overlapped with the next step's kernels"}
+               "staging_buffers": n_stage,
+               "note": ("every step: gradients host->device (copy-in stream), updated fp32 weights "
+                        + ("device->device->host (copy-out stream), overlapped with the next step's kernels"
+                           if staging else "device->host (copy-out stream); the next step starts after it"))}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
