@@ -1203,10 +1203,10 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
       ProfScope ps(ctx, MUON_K_MOMENTUM, st);
       for (const SegLaunch& L : segm) {
         if (mode == 0)
-          launch_pdl(momentum_kernel<0>, dim3(unsigned(L.tiles)), dim3(EW_THREADS), size_t(0), st,
+          launch_pdl(momentum_kernel<0>, dim3(unsigned(L.tiles)), dim3(MOM_THREADS), size_t(0), st,
               ddesc + c.first, L.t, L.tile_base, hp->momentum, hp->nesterov, skip);
         else
-          launch_pdl(momentum_kernel<1>, dim3(unsigned(L.tiles)), dim3(EW_THREADS), size_t(0), st,
+          launch_pdl(momentum_kernel<1>, dim3(unsigned(L.tiles)), dim3(MOM_THREADS), size_t(0), st,
               ddesc + c.first, L.t, L.tile_base, 0.f, 0, skip);
       }
       launch_pdl(norm_reduce_kernel, dim3(unsigned(n_mom)), dim3(EW_THREADS), size_t(0), st, ddesc + c.first, skip);
@@ -2011,7 +2011,7 @@ muon_status muon_orthogonalize_noalloc(const void* input, int32_t in_dtype, int6
   // before it is read), so the call makes no host-to-device copy.
   noalloc_setup_kernel<<<1, 32, 0, st>>>(d, ddesc, flags);
   const std::vector<SegLaunch> segl = build_seg_launches(&d, 1);
-  momentum_kernel<1><<<unsigned(tiles), EW_THREADS, 0, st>>>(ddesc, segl[0].t, 0, 0.f, 0, flags);
+  momentum_kernel<1><<<unsigned(tiles), MOM_THREADS, 0, st>>>(ddesc, segl[0].t, 0, 0.f, 0, flags);
   norm_reduce_kernel<<<1, EW_THREADS, 0, st>>>(ddesc, flags);
   if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;
   tmp.dflags = flags;
