@@ -214,3 +214,57 @@ def test_newton_muon_gpt2_small_ten_steps_full_size(mx):
                 assert rel_fro(_np(W[i]), want) < EW_TOL, (m.name, step)
                 if i // 6 == layer:
                     assert rel_fro(o, oracle.newton_schulz(u, 5)) < NS_TOL, (m.name, step)
+
+
+@pytest.mark.parametrize("shape", [(16384, 131136), (131136, 16384)], ids=["wide", "tall"])
+def test_single_matrix_past_2_31_elements(mx, shape):
+    """One matrix of 2.15 G elements (more than 2^31, so every element,
+    tile and byte offset needs 64 bits), bf16 gradient N(0,1e-3), fp32
+    weights N(0,0.02), zero momentum, one step; both orientations (the tall
+    one goes through the transposing momentum tile).  Unfused first, with the
+    update written out: the momentum and the staged apply on sampled elements
+    (among them the first, the last and those around index 2^31) against the
+    oracle, the update finite and in the quintic's band.  Then the same step
+    fused: the applied update on the same elements against the unfused one,
+    up to bf16 rounding, and the momentum bit for bit."""
+    dev = torch.device("cuda")
+    rows, cols = shape
+    numel = rows * cols
+    assert numel > 2 ** 31
+    hp = mx.default_hparams()
+    decay = 1.0 - hp.lr * hp.weight_decay
+    scale = oracle.shape_scale(rows, cols)
+    G = wl.torch_normal(shape, 1e-3, 9, 0, 0, wl.ROLE_GRAD, dtype=torch.bfloat16, device=dev)
+    W = wl.torch_normal(shape, 0.02, 9, 0, 0, wl.ROLE_WEIGHT, device=dev)
+    B = torch.zeros(shape, device=dev)
+    O = torch.empty(shape, device=dev)
+    special = [0, 1, 2 ** 31 - 1, 2 ** 31, 2 ** 31 + 1, 2 ** 31 + 12345, numel - cols, numel - 1]
+    rng = np.random.default_rng(31)
+    idx_np = np.unique(np.concatenate([rng.integers(0, numel, 4096), np.array(special)]))
+    idx = torch.from_numpy(idx_np).to(dev)
+    w0 = W.view(-1)[idx].double().cpu().numpy()
+    g0 = G.view(-1)[idx].double().cpu().numpy()
+    with mx.MuonContext(0) as ctx:
+        ctx.step([dict(weights=[W], grads=[G], momentum=[B], update_out=[O])], hp)
+        torch.cuda.synchronize()
+        ctx.check_device()
+        nb, _ = oracle.nesterov_momentum(g0, np.zeros_like(g0))
+        b1 = B.view(-1)[idx].clone()
+        assert rel_fro(b1.double().cpu().numpy(), nb) < EW_TOL
+        assert bool(torch.isfinite(O).all())
+        ok, r = _band_ok(O, rows, cols)
+        assert ok, r
+        o1 = O.view(-1)[idx].double().cpu().numpy()
+        want = oracle.apply_update(w0, o1, hp.lr, hp.weight_decay, scale)
+        assert rel_fro(W.view(-1)[idx].double().cpu().numpy(), want) < EW_TOL
+        del O
+        torch.cuda.empty_cache()
+        # the same step with the weight update fused into the last product
+        wl.torch_normal(shape, 0.02, 9, 0, 0, wl.ROLE_WEIGHT, device=dev, out=W)
+        B.zero_()
+        ctx.step([dict(weights=[W], grads=[G], momentum=[B])], hp)
+        torch.cuda.synchronize()
+        ctx.check_device()
+        assert torch.equal(B.view(-1)[idx], b1)
+        upd = (w0 * decay - W.view(-1)[idx].double().cpu().numpy()) / (hp.lr * scale)
+        assert rel_fro(upd, o1) < 5e-3
