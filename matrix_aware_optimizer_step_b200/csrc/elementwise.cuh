@@ -6,7 +6,9 @@
 //                     transposing through shared memory for tall matrices,
 //                     and one partial sum of U^2 per tile (block reduction).
 //                     12 B/element with bf16 gradients.
-//   norm_reduce_kernel  ||U||^2 per matrix from its tiles' partials.
+//   norm_reduce_kernel  ||U||^2 per matrix from its tiles' partials (or from
+//                     the preconditioning product's, when that product
+//                     applied the momentum itself).
 //   apply_kernel      W <- W (1 - lr wd) - lr scale O, O read from the final
 //                     wide bf16 X (transposed back through shared memory for
 //                     tall matrices); optionally O to an fp32 output.
@@ -65,7 +67,10 @@ struct MatDesc {
   int32_t grad_dtype;        // 0 f32, 1 bf16
   float lr_scale;            // lr * shape scale
   float decay;               // 1 - lr * wd
-  int32_t pad;
+  int32_t nparts;            // > 0: momentum, U and the partials of ||U||^2 come
+                             // from the preconditioning product's epilogue, the
+                             // partials at partials[0 .. nparts); momentum_kernel
+                             // skips the matrix
 };
 
 // Segments of equal-shape matrices in one launch (kernel parameter space,
@@ -155,6 +160,7 @@ __global__ void __launch_bounds__(MOM_THREADS)
   const int64_t gt = tile_base + blockIdx.x;
   const TileLoc loc = seg_locate(segs, blockIdx.x);
   const MatDesc& d = descs[loc.mat];
+  if (d.nparts > 0) return;   // done in the preconditioning product (uniform per block)
   const int64_t lt = loc.lt;
   float ss = 0.f;
   if (!d.transposed && d.ld == d.cols && (d.cols % 8) == 0) {
@@ -287,9 +293,11 @@ __global__ void __launch_bounds__(EW_THREADS) norm_reduce_kernel(const MatDesc* 
   if (halted(skip)) return;
   __shared__ float red[EW_THREADS / 32];
   const MatDesc& d = descs[blockIdx.x];
-  const int64_t ntiles = ((d.rows + EW_TILE - 1) / EW_TILE) * d.tiles_c;
+  const bool fused = d.nparts > 0;
+  const int64_t ntiles = fused ? d.nparts : ((d.rows + EW_TILE - 1) / EW_TILE) * d.tiles_c;
+  const float* part = fused ? d.partials : d.partials + d.tile_start;
   float acc = 0.f;
-  for (int64_t t = threadIdx.x; t < ntiles; t += EW_THREADS) acc += d.partials[d.tile_start + t];
+  for (int64_t t = threadIdx.x; t < ntiles; t += EW_THREADS) acc += part[t];
   const float all = block_sum(acc, red);
   if (threadIdx.x == 0) *d.norm2 = all;
 }

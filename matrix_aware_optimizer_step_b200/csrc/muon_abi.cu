@@ -228,6 +228,7 @@ struct Chunk {
   size_t off_norm;               // count floats, then per-tile partials
   size_t off_partials;
   size_t off_pgrad;              // preconditioned gradients (fp32), if any
+  size_t off_fparts;             // partials of ||U||^2 from the preconditioning epilogue
   bool tc_pre;                   // preconditioning on the tensor-core engine
   size_t off_sst;                // S^-1 hi/lo stacks (tensor-core preconditioning)
   std::vector<Run> runs;
@@ -240,6 +241,12 @@ inline bool tc_precond_ok(const Item& it) { return (it.cols / it.precond_blocks)
 inline size_t sst_bytes(const Item& it) {
   const size_t d = size_t(it.cols / it.precond_blocks);
   return size_t(it.precond_blocks) * 2 * d * d * 2;
+}
+// Partials of ||U||^2 that the preconditioning product writes when it applies
+// the momentum itself: one per (256 x 256 pair tile, CTA, epilogue warp).
+inline int64_t fused_parts(const Item& it) {
+  const int64_t d = it.cols / it.precond_blocks;
+  return int64_t(it.precond_blocks) * cdiv(it.rows, gemm_cfg::TM) * cdiv(d, gemm_cfg::TN) * 2 * gemm_cfg::EPI_WARPS;
 }
 
 constexpr size_t kAlign = 256;
@@ -254,6 +261,11 @@ size_t layout_chunk(Chunk& c, const std::vector<Item>& items) {
   for (int i = c.first; i < c.first + c.count; ++i)
     tiles += cdiv(items[i].rows, EW_TILE) * cdiv(items[i].cols, EW_TILE);
   off += round_up(size_t(tiles) * sizeof(float), kAlign);
+  c.off_fparts = off;
+  int64_t fparts = 0;
+  for (int i = c.first; i < c.first + c.count; ++i)
+    if (items[i].precond) fparts += fused_parts(items[i]);
+  off += round_up(size_t(fparts) * sizeof(float), kAlign);
   c.off_pgrad = off;
   bool any_pre = false;
   c.tc_pre = true;
@@ -684,6 +696,8 @@ struct PreProblem {
   int pmap_base;
   float* pg;
   int64_t pg_stride;
+  int fused;                 // momentum in the epilogue (PRECOND_MOM); pg unused
+  int momd_base;             // fused: MomDesc of the problem's first matrix
 };
 
 // Operand maps of one preconditioned matrix: its gradient in place and the
@@ -696,17 +710,27 @@ bool encode_precond_maps(PrecondMaps* pm, const void* grad, int64_t rows, int64_
 }
 
 // G' = G [S_hi; S_lo] for every problem, up to MAX_PROBLEMS per launch;
-// pmaps is the device copy of the PrecondMaps table.
+// pmaps is the device copy of the PrecondMaps table.  Fused problems (inside
+// a step) apply the momentum in the epilogue instead of writing G' (their
+// matrices' MomDescs start at momd + momd_base); consecutive problems of one
+// kind share a launch.
 muon_status run_precondition(muon_ctx* ctx, const std::vector<PreProblem>& probs, const PrecondMaps* pmaps,
-                             const int* skip, cudaStream_t st) {
-  for (size_t b0 = 0; b0 < probs.size(); b0 += MAX_PROBLEMS) {
-    const int nb = int(std::min<size_t>(MAX_PROBLEMS, probs.size() - b0));
+                             const int* skip, cudaStream_t st, const MomDesc* momd = nullptr, float beta = 0.f,
+                             int nesterov = 0) {
+  size_t b0 = 0;
+  while (b0 < probs.size()) {
+    const int fused = probs[b0].fused;
+    int nb = 0;
+    while (nb < MAX_PROBLEMS && b0 + nb < probs.size() && probs[b0 + nb].fused == fused) ++nb;
     GemmMaps maps{};           // unused: the operands' maps are in pmaps
     GemmArgs g{};
     g.nprob = nb;
     g.err = ctx->dflags;
     g.skip = skip;
     g.pmaps = pmaps;
+    g.momd = momd;
+    g.beta = beta;
+    g.nesterov = nesterov;
     int tile = 0;
     for (int j = 0; j < nb; ++j) {
       const PreProblem& q = probs[b0 + j];
@@ -721,12 +745,15 @@ muon_status run_precondition(muon_ctx* ctx, const std::vector<PreProblem>& probs
       P.nblocks = q.nb;
       P.scale = 1.0f;
       P.pmap_base = q.pmap_base;
+      P.apply_base = q.momd_base;
       const int64_t tt = int64_t(tile) + int64_t(P.batch) * P.tiles_per_mat;
       if (tt > INT32_MAX) return fail(ctx, MUON_ERR_UNSUPPORTED, "too many tiles in one launch");
       tile = int(tt);
     }
     g.total = tile;
-    CUDA_TRY(ctx, (launch_gemm<EPI_PRECOND, true>(ctx, maps, g, st)));
+    if (fused) CUDA_TRY(ctx, (launch_gemm<EPI_PRECOND_MOM, true>(ctx, maps, g, st)));
+    else CUDA_TRY(ctx, (launch_gemm<EPI_PRECOND, true>(ctx, maps, g, st)));
+    b0 += nb;
   }
   return MUON_OK;
 }
@@ -974,6 +1001,8 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
   std::vector<PrecondMaps> pmaps;
   std::vector<int> chunk_prep_begin(chunks.size(), 0), chunk_prep_count(chunks.size(), 0);
   std::vector<std::vector<PreProblem>> chunk_pprob(chunks.size());
+  // per matrix whose momentum the preconditioning product applies
+  std::vector<MomDesc> momds;
   const bool check = mode == 0 && hp->check_finite;
   // the small-matrix kernel forms its matrices' X0 from the momentum itself
   const bool small_mom = mode == 0 && hp->ns_steps >= 1;
@@ -982,6 +1011,7 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
     int64_t tiles = 0;
     size_t pg_off = c.off_pgrad;
     size_t sst_off = c.off_sst;
+    int64_t fp_off = 0;                       // fused partials used so far
     std::map<StackKey, const __nv_bfloat16*> stacks;
     chunk_pbegin[ci] = int(pdescs.size());
     chunk_prep_begin[ci] = int(prep.size());
@@ -993,6 +1023,9 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
         MatDesc& d = descs[idx];
         d.grad = it.grad;
         d.grad_dtype = it.grad_dtype;
+        // in a step, the tensor-core preconditioning applies the momentum in
+        // its epilogue (the small-matrix kernel forms its own)
+        const bool fused = it.precond && c.tc_pre && mode == 0 && !small_run(r);
         if (it.precond && c.tc_pre) {
           float* pg = reinterpret_cast<float*>(ws + pg_off);
           const size_t pg_bytes = round_up(size_t(it.rows) * it.cols * 4, kAlign);
@@ -1016,7 +1049,7 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
           pmaps.push_back(pm);
           std::vector<PreProblem>& pp = chunk_pprob[ci];
           if (!pp.empty() && pp.back().rows == it.rows && pp.back().cols == it.cols &&
-              pp.back().nb == it.precond_blocks && pp.back().last == idx - 1) {
+              pp.back().nb == it.precond_blocks && pp.back().last == idx - 1 && pp.back().fused == int(fused)) {
             pp.back().count++;
             pp.back().last = idx;
           } else {
@@ -1024,6 +1057,8 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
             q.rows = it.rows; q.cols = it.cols; q.nb = it.precond_blocks; q.d = dd; q.count = 1; q.last = idx;
             q.pmap_base = int(pmaps.size()) - 1;
             q.pg = pg; q.pg_stride = int64_t(pg_bytes / 4);
+            q.fused = fused ? 1 : 0;
+            q.momd_base = int(momds.size());       // this matrix's MomDesc, pushed below
             pp.push_back(q);
           }
           d.grad = pg;
@@ -1055,6 +1090,7 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
                   int64_t(k) * r.m * r.ld_n;
         d.norm2 = reinterpret_cast<float*>(ws + c.off_norm) + (idx - c.first);
         d.partials = reinterpret_cast<float*>(ws + c.off_partials);
+        d.nparts = 0;
         d.rows = it.rows;
         d.cols = it.cols;
         d.ld = r.ld_n;
@@ -1065,6 +1101,19 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
         d.lr_scale = hp->lr * scale;
         d.decay = 1.0f - hp->lr * hp->weight_decay;
         tiles += cdiv(it.rows, EW_TILE) * d.tiles_c;
+        if (fused) {
+          d.nparts = int32_t(fused_parts(it));
+          d.partials = reinterpret_cast<float*>(ws + c.off_fparts) + fp_off;
+          fp_off += d.nparts;
+          MomDesc md{};
+          bool ok = encode_f32_matrix(&md.mom, it.momentum, uint64_t(it.cols), uint64_t(it.rows));
+          ok &= encode_bf16_3d(&md.x, d.x_in, uint64_t(r.n), uint64_t(r.m), 1, uint64_t(r.ld_n), 32, 32,
+                               CU_TENSOR_MAP_SWIZZLE_64B);
+          if (!ok) return fail(ctx, MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed (momentum)");
+          md.partials = d.partials;
+          md.transposed = it.transposed ? 1 : 0;
+          momds.push_back(md);
+        }
       }
     }
     chunk_tiles[ci] = tiles;
@@ -1112,12 +1161,14 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
   const size_t pd_bytes = round_up(pdescs.size() * sizeof(PrecondDesc), kAlign);
   const size_t ap_off = round_up(mat_bytes + pd_bytes + prep.size() * sizeof(PrepDesc), kAlign);
   const size_t pm_off = round_up(ap_off + adescs.size() * sizeof(ApplyDesc), kAlign);
-  std::vector<uint8_t> table(pm_off + pmaps.size() * sizeof(PrecondMaps));
+  const size_t md_off = round_up(pm_off + pmaps.size() * sizeof(PrecondMaps), kAlign);
+  std::vector<uint8_t> table(md_off + momds.size() * sizeof(MomDesc));
   std::memcpy(table.data(), descs.data(), descs.size() * sizeof(MatDesc));
   if (!pdescs.empty()) std::memcpy(table.data() + mat_bytes, pdescs.data(), pdescs.size() * sizeof(PrecondDesc));
   if (!prep.empty()) std::memcpy(table.data() + mat_bytes + pd_bytes, prep.data(), prep.size() * sizeof(PrepDesc));
   if (!adescs.empty()) std::memcpy(table.data() + ap_off, adescs.data(), adescs.size() * sizeof(ApplyDesc));
   if (!pmaps.empty()) std::memcpy(table.data() + pm_off, pmaps.data(), pmaps.size() * sizeof(PrecondMaps));
+  if (!momds.empty()) std::memcpy(table.data() + md_off, momds.data(), momds.size() * sizeof(MomDesc));
   void* dtab = nullptr;
   s = upload_table(ctx, table.data(), table.size(), st, &dtab);
   if (s != MUON_OK) return s;
@@ -1180,7 +1231,9 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
       ctx->launches++;
       CUDA_TRY(ctx, cudaGetLastError());
       s = run_precondition(ctx, chunk_pprob[ci],
-                           reinterpret_cast<const PrecondMaps*>(static_cast<uint8_t*>(dtab) + pm_off), skip, st);
+                           reinterpret_cast<const PrecondMaps*>(static_cast<uint8_t*>(dtab) + pm_off), skip, st,
+                           reinterpret_cast<const MomDesc*>(static_cast<uint8_t*>(dtab) + md_off), hp->momentum,
+                           hp->nesterov);
       if (s != MUON_OK) return s;
     }
     if (chunk_pcount[ci] > 0) {
@@ -1199,18 +1252,26 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
       for (const Run& r : c.runs)
         if (small_run(r)) n_mom = std::min(n_mom, r.first - c.first);
     if (n_mom > 0) {
-      const std::vector<SegLaunch> segm = build_seg_launches(descs.data() + c.first, n_mom);
+      // matrices whose momentum the preconditioning product applied are
+      // skipped by the momentum kernel; when that is all of them, it is not
+      // launched and only their norms are reduced
+      bool all_fused = true;
+      for (int i = c.first; i < c.first + n_mom && all_fused; ++i) all_fused = descs[i].nparts > 0;
       ProfScope ps(ctx, MUON_K_MOMENTUM, st);
-      for (const SegLaunch& L : segm) {
-        if (mode == 0)
-          launch_pdl(momentum_kernel<0>, dim3(unsigned(L.tiles)), dim3(MOM_THREADS), size_t(0), st,
-              ddesc + c.first, L.t, L.tile_base, hp->momentum, hp->nesterov, skip);
-        else
-          launch_pdl(momentum_kernel<1>, dim3(unsigned(L.tiles)), dim3(MOM_THREADS), size_t(0), st,
-              ddesc + c.first, L.t, L.tile_base, 0.f, 0, skip);
+      if (!all_fused) {
+        const std::vector<SegLaunch> segm = build_seg_launches(descs.data() + c.first, n_mom);
+        for (const SegLaunch& L : segm) {
+          if (mode == 0)
+            launch_pdl(momentum_kernel<0>, dim3(unsigned(L.tiles)), dim3(MOM_THREADS), size_t(0), st,
+                ddesc + c.first, L.t, L.tile_base, hp->momentum, hp->nesterov, skip);
+          else
+            launch_pdl(momentum_kernel<1>, dim3(unsigned(L.tiles)), dim3(MOM_THREADS), size_t(0), st,
+                ddesc + c.first, L.t, L.tile_base, 0.f, 0, skip);
+        }
+        ctx->launches += segm.size();
       }
       launch_pdl(norm_reduce_kernel, dim3(unsigned(n_mom)), dim3(EW_THREADS), size_t(0), st, ddesc + c.first, skip);
-      ctx->launches += segm.size() + 1;
+      ctx->launches += 1;
     }
     CUDA_TRY(ctx, cudaGetLastError());
     {

@@ -70,13 +70,24 @@
 //            K, G's column block read twice, so the product keeps close to
 //            fp32 precision; G is read in place and each matrix's operands
 //            come from its own tensor maps in device memory)
+//   PRECOND_MOM  the same product inside an optimizer step, with Nesterov
+//            momentum in the epilogue, so G' never reaches memory: each 32x32
+//            fp32 chunk of the momentum buffer comes in by TMA (two buffers
+//            per warp, requested ahead as the fused weight step does), is
+//            updated with the G' chunk in place and goes back by TMA; U
+//            leaves by TMA as a 32x32 bf16 block of the Newton-Schulz input
+//            (staged transposed for tall matrices, whose wide layout is U^T);
+//            every warp stores one partial of ||U||^2 per tile
 #pragma once
 
 #include "sm100_ptx.cuh"
 
 namespace muon {
 
-enum EpiKind : int { EPI_GRAM = 0, EPI_POLY = 1, EPI_UPDATE = 2, EPI_GRAM32 = 3, EPI_PRECOND = 4, EPI_UPDATE_APPLY = 5 };
+enum EpiKind : int {
+  EPI_GRAM = 0, EPI_POLY = 1, EPI_UPDATE = 2, EPI_GRAM32 = 3, EPI_PRECOND = 4, EPI_UPDATE_APPLY = 5,
+  EPI_PRECOND_MOM = 6
+};
 
 namespace gemm_cfg {
 constexpr int TM = 256;                              // pair tile rows (128 per CTA)
@@ -88,11 +99,13 @@ constexpr int BK = 64;
 // chunks (below) and spend the space saved on a fifth / sixth stage; the
 // update also has no mirrored blocks.
 __host__ __device__ constexpr int stages_for(int kind) {
-  return kind == 0 ? 5 : kind == 1 ? 4 : kind == 2 ? 6 : kind == 5 ? 5 : 7;
+  return kind == 0 ? 5 : kind == 1 ? 4 : kind == 2 ? 6 : kind == 5 ? 5 : kind == 6 ? 4 : 7;
 }
 // GRAM32 and PRECOND write fp32 straight from registers: no epilogue buffers,
 // so their pipelines take the shared memory.
 __host__ __device__ constexpr bool fp32_out(int kind) { return kind == 3 || kind == 4; }
+__host__ __device__ constexpr bool precond_kind(int kind) { return kind == 4 || kind == 6; }
+__host__ __device__ constexpr bool mom_out(int kind) { return kind == 6; }
 // The last update of an optimizer step may apply W <- W (1 - lr wd) - lr
 // scale O in its epilogue (EPI_UPDATE_APPLY): W moves through two 4 KB
 // 32x32 fp32 chunk buffers per warp by TMA, and O never reaches memory.
@@ -119,9 +132,12 @@ constexpr int CH_BYTES = 32 * 64;                    // 32 rows x 32 bf16, 64-by
 constexpr int CH_BUFS = 2;
 constexpr int WCH_BYTES = 32 * 128;                  // 32 x 32 fp32 weight chunk, 128-byte swizzle
 constexpr int BAR_BYTES = 384;
+// PRECOND_MOM, per warp: two momentum chunks (fp32) and two U chunks (bf16)
+constexpr int MOM_SLICE = 2 * WCH_BYTES + 2 * CH_BYTES;
 __host__ __device__ constexpr int smem_bytes(int kind) {
   return stages_for(kind) * STAGE_BYTES +
-         EPI_WARPS * ((apply_out(kind)     ? W_NBUF * WCH_BYTES
+         EPI_WARPS * ((mom_out(kind)       ? MOM_SLICE
+                       : apply_out(kind)   ? W_NBUF * WCH_BYTES
                        : chunked_out(kind) ? CH_BUFS * CH_BYTES
                        : fp32_out(kind)    ? 0
                                            : EPI_BYTES) +
@@ -140,7 +156,8 @@ static_assert((2 * 7 + 5 + W_NBUF * EPI_WARPS) * 8 + 8 <= BAR_BYTES, "barrier ar
 constexpr int ACC_COLS = 256;                        // one fp32 128x256 accumulator per CTA
 constexpr int TMEM_COLS = 2 * ACC_COLS;              // double-buffered
 static_assert(smem_bytes(0) <= 232448 && smem_bytes(1) <= 232448 && smem_bytes(2) <= 232448 &&
-                  smem_bytes(3) <= 232448 && smem_bytes(4) <= 232448 && smem_bytes(5) <= 232448,
+                  smem_bytes(3) <= 232448 && smem_bytes(4) <= 232448 && smem_bytes(5) <= 232448 &&
+                  smem_bytes(6) <= 232448,
               "shared memory per block");
 }  // namespace gemm_cfg
 
@@ -162,6 +179,7 @@ struct GemmProblem {
   int nblocks;
   float scale;               // GRAM32 / PRECOND: result = scale * sum
   int apply_base;            // UPDATE_APPLY: first ApplyDesc of this problem's matrices
+                             // PRECOND_MOM: first MomDesc of this problem's matrices
   int pmap_base;             // PRECOND: first PrecondMaps of this problem's matrices
 };
 
@@ -172,6 +190,18 @@ struct alignas(64) ApplyDesc {
   CUtensorMap w;
   float lr_scale;            // lr * shape scale
   float decay;               // 1 - lr * wd
+  int transposed;
+  int pad;
+};
+
+// Per matrix of a preconditioning product with momentum (PRECOND_MOM): its
+// fp32 momentum buffer (rows x cols, box 32 x 32, 128-byte swizzle), its
+// Newton-Schulz input in the wide layout (bf16, box 32 x 32, 64-byte
+// swizzle), where its partials of ||U||^2 go, and its orientation.
+struct alignas(64) MomDesc {
+  CUtensorMap mom;
+  CUtensorMap x;
+  float* partials;
   int transposed;
   int pad;
 };
@@ -201,6 +231,9 @@ struct GemmArgs {
   int reverse;               // walk the tile list from its end (see run_newton_schulz)
   const ApplyDesc* apply;    // UPDATE_APPLY: per-matrix weights (device memory)
   const PrecondMaps* pmaps;  // PRECOND: per-matrix operand maps (device memory)
+  const MomDesc* momd;       // PRECOND_MOM: per-matrix momentum and output (device memory)
+  float beta;                // PRECOND_MOM: momentum coefficient
+  int nesterov;              // PRECOND_MOM: U = (1 - beta) G' + beta buf, else buf
   int ab_distinct;           // GRAM32 of split fp32 activations: A and B are
                              // different tensors, so a diagonal tile loads both
   int selftest;              // failure-detection self test: the MMA thread
@@ -218,7 +251,7 @@ struct GemmMaps {
 // Launches whose operand tensor maps are per matrix in device memory
 // (args.pmaps) rather than per problem in parameter space.
 __host__ __device__ constexpr bool device_maps(int kind, bool b_mn_major) {
-  return kind == EPI_PRECOND || (kind == EPI_GRAM32 && b_mn_major);
+  return gemm_cfg::precond_kind(kind) || (kind == EPI_GRAM32 && b_mn_major);
 }
 
 __host__ __device__ constexpr bool symmetric_kind(int kind) {
@@ -289,7 +322,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* smem_epi = smem + STAGES * STAGE_BYTES;             // 1024-aligned slices
-  constexpr int SLICE = apply_out(KIND) ? W_NBUF * WCH_BYTES : chunked_out(KIND) ? CH_BUFS * CH_BYTES
+  constexpr int SLICE = mom_out(KIND) ? MOM_SLICE : apply_out(KIND) ? W_NBUF * WCH_BYTES
+                        : chunked_out(KIND) ? CH_BUFS * CH_BYTES
                         : fp32_out(KIND)  ? 0 : EPI_BYTES;
   uint8_t* smem_stg = smem_epi + EPI_WARPS * SLICE;
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem_stg + (mirrors(KIND) ? EPI_WARPS * STG_BYTES : 0));
@@ -357,7 +391,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
         const CUtensorMap* tmB = &maps.b[pi];
         int za = bidx, zb = bidx;              // depth coordinates of the A and B loads
         int xoff = 0;                          // MN offset of both operands (GRAM32 direct)
-        if (KIND == EPI_PRECOND) {
+        if (precond_kind(KIND)) {
           // tile bidx: column block bidx % nblocks of matrix bidx / nblocks
           const int nbk = args.p[pi].nblocks;
           const PrecondMaps& pm = args.pmaps[args.p[pi].pmap_base + bidx / nbk];
@@ -386,7 +420,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
           uint8_t* b_dst = a_dst + A_BYTES;
           const uint32_t fb = full0 + s * 8;
           if (leader) mbar_arrive_expect_tx(&full_bar[s], diag ? 2 * A_BYTES : 2 * STAGE_BYTES);
-          if (KIND == EPI_PRECOND) {
+          if (precond_kind(KIND)) {
             // A: the gradient's column block zb, read twice along K (against
             // S_hi, then S_lo)
             const int d = args.p[pi].N;
@@ -600,6 +634,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
           }
         }
       }
+      if constexpr (mom_out(KIND)) {
+        // momentum chunks 0 and 1 of this tile into the two buffers, once the
+        // previous tile's stores have read them
+        if (lane == 0 && active) {
+          bulk_wait_group_read0();
+          const int z = bidx / P.nblocks, blk = bidx % P.nblocks;
+          const MomDesc& md = args.momd[P.apply_base + z];
+          for (int c = 0; c < 2 && col0 + c * 32 < P.N; ++c) {
+            mbar_arrive_expect_tx(&aux_bar[2 * ew + c], WCH_BYTES);
+            tma_load_3d(slice + c * WCH_BYTES, &md.mom, &aux_bar[2 * ew + c], blk * P.N + col0 + c * 32, rbase, 0);
+            wpend |= 1u << c;
+          }
+        }
+      }
       if (lane == 0 && KIND == EPI_POLY) {
         bulk_wait_group_read0();
         if (active) {
@@ -620,6 +668,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
         aux_phase ^= 1;
         aux_pending = false;
       }
+      float ss_tile = 0.f;                   // PRECOND_MOM: this warp's share of ||U||^2
       if (active) {
         float alpha = 1.0f;
         if (P.norm2 != nullptr) {
@@ -663,6 +712,86 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
                   if (cbase + k < P.N) P.out32[zoff + static_cast<int64_t>(cbase + k) * P.out32_ld + r] = v[k];
               }
             }
+          } else if constexpr (mom_out(KIND)) {
+            // G' chunk (row `lane`, 32 columns of column block blk of matrix
+            // z): momentum updated in its buffer and stored back, U staged
+            // as bf16 and stored into the Newton-Schulz input
+            const int z = bidx / P.nblocks, blk = bidx % P.nblocks;
+            const MomDesc& md = args.momd[P.apply_base + z];
+            const int wb = c32 & 1;
+            uint8_t* wbuf = slice + wb * WCH_BYTES;
+            // lane 0 issued the load; all lanes wait on its barrier
+            const bool okw = mbar_wait(&aux_bar[2 * ew + wb], (wph >> wb) & 1u, args.err, abort_flag);
+            if (!__all_sync(0xffffffffu, okw)) break;
+            wph ^= 1u << wb;
+            wpend &= ~(1u << wb);
+            const int cg = blk * P.N + cbase;          // column in the whole matrix
+            const float beta = args.beta;
+            float u[32];
+            // row `lane` of the chunk: 16-byte unit v at unit v ^ (lane % 8)
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+              float4* pb = reinterpret_cast<float4*>(wbuf + lane * 128 + ((v ^ (lane & 7)) << 4));
+              const float4 b4 = *pb;
+              float b[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float g = P.scale * __uint_as_float(raw[v * 4 + e]);
+                b[e] = beta * b[e] + (1.f - beta) * g;
+                u[v * 4 + e] = args.nesterov ? (1.f - beta) * g + beta * b[e] : b[e];
+              }
+              *pb = make_float4(b[0], b[1], b[2], b[3]);
+            }
+            if (rbase + lane < P.M) {
+#pragma unroll
+              for (int k = 0; k < 32; ++k) ss_tile += u[k] * u[k];
+            }
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_3d(&md.mom, wbuf, cg, rbase, 0);   // rows past the matrix are clipped
+              bulk_commit_group();
+            }
+            // U buffer wb: the store that last read it (two chunks ago) is
+            // at most the fourth most recent group
+            uint8_t* ubuf = slice + 2 * WCH_BYTES + wb * CH_BYTES;
+            if (lane == 0) bulk_wait_group_read3();
+            __syncwarp();
+            if (!md.transposed) {
+              // row `lane`: 16-byte unit v at unit v ^ ((lane / 2) % 4) (64-byte swizzle)
+#pragma unroll
+              for (int v = 0; v < 4; ++v) {
+                uint4 w;
+                w.x = pack_bf16x2(u[v * 8 + 0], u[v * 8 + 1]);
+                w.y = pack_bf16x2(u[v * 8 + 2], u[v * 8 + 3]);
+                w.z = pack_bf16x2(u[v * 8 + 4], u[v * 8 + 5]);
+                w.w = pack_bf16x2(u[v * 8 + 6], u[v * 8 + 7]);
+                *reinterpret_cast<uint4*>(ubuf + lane * 64 + ((v ^ ((lane >> 1) & 3)) << 4)) = w;
+              }
+            } else {
+              // the wide layout is U^T: buffer row k is column cg + k, the
+              // lanes' rows side by side (element `lane` of unit lane / 8)
+#pragma unroll
+              for (int k = 0; k < 32; ++k)
+                *reinterpret_cast<__nv_bfloat16*>(ubuf + k * 64 + ((((lane >> 3) ^ ((k >> 1) & 3)) & 3) << 4) +
+                                                  (lane & 7) * 2) = __float2bfloat16_rn(u[k]);
+            }
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              if (!md.transposed) tma_store_3d(&md.x, ubuf, cg, rbase, 0);
+              else tma_store_3d(&md.x, ubuf, rbase, cg, 0);
+              bulk_commit_group();
+              // momentum chunk c32 + 2 into this buffer once its store has read it
+              const int cn = cbase + 64;
+              if (c32 + 2 < 4 && cn < P.N) {
+                bulk_wait_group_read1();
+                mbar_arrive_expect_tx(&aux_bar[2 * ew + wb], WCH_BYTES);
+                tma_load_3d(wbuf, &md.mom, &aux_bar[2 * ew + wb], blk * P.N + cn, rbase, 0);
+                wpend |= 1u << wb;
+              }
+            }
+            wpend = __shfl_sync(0xffffffffu, wpend, 0);
           } else if constexpr (apply_out(KIND)) {
             const ApplyDesc& ad = args.apply[P.apply_base + bidx];
             const int wb = c32 & 1;
@@ -804,6 +933,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
           tma_store_3d(tmOut, slice, col0, rbase, bidx);
           if (two_boxes) tma_store_3d(tmOut, slice + EPI_BOX_BYTES, col0 + 64, rbase, bidx);
           bulk_commit_group();
+        }
+      }
+      if constexpr (mom_out(KIND)) {
+        // one partial of ||U||^2 per (tile, CTA, warp), zero when the warp's
+        // rows or columns lie outside the matrix; the norm kernel adds a
+        // matrix's partials in this fixed order
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ss_tile += __shfl_xor_sync(0xffffffffu, ss_tile, o);
+        if (lane == 0) {
+          const int z = bidx / P.nblocks, blk = bidx % P.nblocks;
+          args.momd[P.apply_base + z].partials[((static_cast<int64_t>(blk) * P.tiles_m + ti) * P.tiles_n + tj) *
+                                                   (2 * EPI_WARPS) + static_cast<int>(rank) * EPI_WARPS + ew] = ss_tile;
         }
       }
       // this warp's tcgen05.ld reads of the accumulator have completed

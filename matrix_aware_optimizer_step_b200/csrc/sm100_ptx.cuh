@@ -130,6 +130,10 @@ __device__ __forceinline__ void bulk_wait_group_read0() {
 __device__ __forceinline__ void bulk_wait_group_read1() {
   asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
+// ... all but the three most recently committed groups
+__device__ __forceinline__ void bulk_wait_group_read3() {
+  asm volatile("cp.async.bulk.wait_group.read 3;" ::: "memory");
+}
 // wait until all committed bulk stores have completed
 __device__ __forceinline__ void bulk_wait_group0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
