@@ -80,11 +80,22 @@ def step_work(w, aux, ns_steps=5):
     gram = poly = upd = 0
     elems = 0
     pre = 0
+    pre_bytes = 0          # momentum applied in the preconditioning product's epilogue
+    mom_elems = 0          # momentum in the momentum kernel
     for m in w.mats:
+        fused = False
         if m.name in w.precond:
             nb = w.precond[m.name][1]
             d = m.cols // nb
             pre += 2 * m.rows * m.cols * d
+            # tensor-core preconditioning (block width a multiple of 64) of a
+            # matrix the small-matrix kernel does not take: bf16 G read, the
+            # momentum buffer read and written, bf16 U written, in one launch
+            fused = d % 64 == 0 and max(m.rows, m.cols) > SMALL_MAX
+        if fused:
+            pre_bytes += m.rows * m.cols * (2 + 4 + 4 + 2)
+        else:
+            mom_elems += m.rows * m.cols
     refresh_tc = refresh_alu = 0
     for _, tokens, width in w.acts:
         nb = 4 if width > 768 else 1
@@ -112,7 +123,7 @@ def step_work(w, aux, ns_steps=5):
     gbytes = 2 if w.grad_dtype == "bf16" else 4
     aux_el = sum(n for _, n in aux)
     per_iter = upd // max(1, ns_steps)
-    return {
+    work = {
         "gram": ("flop", gram), "poly": ("flop", poly), "update": ("flop", upd),
         "ns_small": ("flop", small),
         # the last update with the weight step fused: one iteration's FLOPs
@@ -121,15 +132,21 @@ def step_work(w, aux, ns_steps=5):
         # the other ns_steps - 1 iterations
         "update_apply": ("mixed", (per_iter, fused_bytes)),
         # momentum: read grad + buf, write buf + bf16 U
-        "momentum": ("byte", elems * (gbytes + 4 + 4 + 2)),
+        "momentum": ("byte", mom_elems * (gbytes + 4 + 4 + 2)),
         # apply: read bf16 O + W, write W
         "apply": ("byte", elems * (2 + 4 + 4)),
         # adamw: read bf16 grad, read+write param, m, v
         "adamw": ("byte", aux_el * (2 + 3 * 8)),
-        # tensor cores: G [S_hi; S_lo] executes twice the algorithmic 2 rows cols d
-        "precondition": ("flop", pre),
+        # tensor cores: G [S_hi; S_lo] executes twice the algorithmic 2 rows cols d;
+        # with the momentum in its epilogue it also moves 12 B per element
+        "precondition": ("mixed", (pre, pre_bytes)) if pre_bytes else ("flop", pre),
         "newton_refresh": ("seq", (refresh_tc / max(1, w.refresh_every), refresh_alu / max(1, w.refresh_every))),
-    }, elems, aux_el
+    }
+    if mom_elems == 0:
+        # every matrix's momentum is applied by the preconditioning product;
+        # what is left in the momentum class is the norm reduction
+        del work["momentum"]
+    return work, elems, aux_el
 
 
 PAIR_TILE = 256     # output tile of the tensor-core engine (a CTA pair)

@@ -126,3 +126,19 @@ def test_small_matrices_form_their_own_class(bench):
     assert work["gram"][1] == work["poly"][1] == work["update"][1] == 0
     assert work["ns_small"][1] == 6 * 256 ** 3 * 5
     assert bench.executed_flops(w)["ns_small"] == 3 * 2 * 256 ** 3 * 5
+
+
+def test_newton_momentum_counted_with_the_preconditioning(bench):
+    """Every GPT-2-small matrix is preconditioned on the tensor cores (block
+    width 768), and that product applies the momentum in its epilogue: its
+    class carries the algorithmic 2 rows cols d FLOPs and 12 B per element
+    (bf16 G read, fp32 buffer read and written, bf16 U written); no
+    momentum-kernel bytes remain."""
+    w, aux = bench.workload_def("newton-gpt2-small")
+    work, elems, _ = bench.step_work(w, aux)
+    flops = 0
+    for m in w.mats:
+        nb = w.precond[m.name][1]
+        flops += 2 * m.rows * m.cols * (m.cols // nb)
+    assert work["precondition"] == ("mixed", (flops, 12 * elems))
+    assert "momentum" not in work
