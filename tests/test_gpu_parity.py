@@ -703,3 +703,41 @@ def test_newton_muon_step_vs_oracle(ctx, mx):
         nb, u = oracle.nesterov_momentum(pg, np.zeros(s))
         assert rel_fro(to_np(bt[i]), nb) < NEWTON_TOL, f"preconditioned momentum {i}"
         assert rel_fro(to_np(ot[i]), oracle.newton_schulz(u, 5)) < NS_TOL
+
+
+def test_newton_momentum_in_preconditioning_epilogue_edges(ctx, mx):
+    """The preconditioning product that applies the momentum in its
+    epilogue, on the shapes that exercise its edges: a tall matrix with a
+    row count that is not a multiple of 32 (the wide layout is U^T and the
+    last row tile is partly outside the matrix), a wide matrix with fewer
+    than 256 rows, and two column blocks; Nesterov off and beta 0.9, two
+    steps with the momentum carried, against the oracle at the fp32 bar (and
+    the Newton-Schulz output at its own)."""
+    hp = mx.default_hparams(momentum=0.9, nesterov=0)
+    cases = [((1001, 256), 1), ((200, 768), 1), ((640, 256), 2)]
+    tokens = 2048
+    sinv_np, sinv_dev = [], []
+    for i, ((rows, cols), nb) in enumerate(cases):
+        d = cols // nb
+        acts = wl.bf16_round_np(wl.np_normal((tokens, cols), 1.0, seed=33, index=i, role=wl.ROLE_ACT))
+        blocks = [oracle.spd_inverse(oracle.second_moment(acts[:, b * d:(b + 1) * d])) for b in range(nb)]
+        sinv_np.append(blocks)
+        sinv_dev.append(dev(np.stack(blocks)))
+    shapes = [c[0] for c in cases]
+    wt = [dev(wl.np_normal(s, 0.02, seed=33, index=i, role=wl.ROLE_WEIGHT)) for i, s in enumerate(shapes)]
+    bt = [torch.zeros(s, device="cuda") for s in shapes]
+    ot = [torch.empty(s, device="cuda") for s in shapes]
+    bufs = [np.zeros(s) for s in shapes]
+    for step in range(2):
+        gs = [wl.bf16_round_np(wl.np_normal(s, 1e-3, seed=33, step=step, index=i)) for i, s in enumerate(shapes)]
+        gt = [dev(x, torch.bfloat16) for x in gs]
+        ctx.step([dict(weights=[wt[i]], grads=[gt[i]], momentum=[bt[i]], update_out=[ot[i]],
+                       precond=[sinv_dev[i]], precond_blocks=cases[i][1]) for i in range(len(cases))], hp)
+        torch.cuda.synchronize()
+        ctx.check_device()
+        for i, s in enumerate(shapes):
+            pg = oracle.right_precondition(gs[i], sinv_np[i])
+            nb_, u = oracle.nesterov_momentum(pg, bufs[i], beta=0.9, nesterov=False)
+            bufs[i] = nb_
+            assert rel_fro(to_np(bt[i]), nb_) < NEWTON_TOL, (s, step)
+            assert rel_fro(to_np(ot[i]), oracle.newton_schulz(u, 5)) < ns_tol(s), (s, step)
