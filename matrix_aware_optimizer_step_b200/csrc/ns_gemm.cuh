@@ -72,9 +72,9 @@
 //            come from its own tensor maps in device memory)
 //   PRECOND_MOM  the same product inside an optimizer step, with Nesterov
 //            momentum in the epilogue, so G' never reaches memory: each 32x32
-//            fp32 chunk of the momentum buffer comes in by TMA (two buffers
-//            per warp, requested ahead as the fused weight step does), is
-//            updated with the G' chunk in place and goes back by TMA; U
+//            fp32 chunk of the momentum buffer comes in by TMA (one buffer
+//            per warp, the next chunk requested once the store has read it),
+//            is updated with the G' chunk in place and goes back by TMA; U
 //            leaves by TMA as a 32x32 bf16 block of the Newton-Schulz input
 //            (staged transposed for tall matrices, whose wide layout is U^T);
 //            every warp stores one partial of ||U||^2 per tile
@@ -99,7 +99,7 @@ constexpr int BK = 64;
 // chunks (below) and spend the space saved on a fifth / sixth stage; the
 // update also has no mirrored blocks.
 __host__ __device__ constexpr int stages_for(int kind) {
-  return kind == 0 ? 5 : kind == 1 ? 4 : kind == 2 ? 6 : kind == 5 ? 5 : kind == 6 ? 4 : 7;
+  return kind == 0 ? 5 : kind == 1 ? 4 : kind == 2 ? 6 : kind == 5 ? 5 : kind == 6 ? 5 : 7;
 }
 // GRAM32 and PRECOND write fp32 straight from registers: no epilogue buffers,
 // so their pipelines take the shared memory.
@@ -133,7 +133,12 @@ constexpr int CH_BUFS = 2;
 constexpr int WCH_BYTES = 32 * 128;                  // 32 x 32 fp32 weight chunk, 128-byte swizzle
 constexpr int BAR_BYTES = 384;
 // PRECOND_MOM, per warp: two momentum chunks (fp32) and two U chunks (bf16)
-constexpr int MOM_SLICE = 2 * WCH_BYTES + 2 * CH_BYTES;
+// One momentum chunk buffer per warp (two U buffers): the slice then leaves
+// room for a fifth pipeline stage, which the product needs more than the
+// epilogue needs a second buffer (its MMA thread waited for operands on 47 %
+// of its cycles with four stages; 0.321 against 0.343 ms per GPT-2-small step)
+constexpr int MOM_NBUF = 1;
+constexpr int MOM_SLICE = MOM_NBUF * WCH_BYTES + 2 * CH_BYTES;
 __host__ __device__ constexpr int smem_bytes(int kind) {
   return stages_for(kind) * STAGE_BYTES +
          EPI_WARPS * ((mom_out(kind)       ? MOM_SLICE
@@ -641,7 +646,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
           bulk_wait_group_read0();
           const int z = bidx / P.nblocks, blk = bidx % P.nblocks;
           const MomDesc& md = args.momd[P.apply_base + z];
-          for (int c = 0; c < 2 && col0 + c * 32 < P.N; ++c) {
+          for (int c = 0; c < MOM_NBUF && col0 + c * 32 < P.N; ++c) {
             mbar_arrive_expect_tx(&aux_bar[2 * ew + c], WCH_BYTES);
             tma_load_3d(slice + c * WCH_BYTES, &md.mom, &aux_bar[2 * ew + c], blk * P.N + col0 + c * 32, rbase, 0);
             wpend |= 1u << c;
@@ -718,7 +723,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
             // as bf16 and stored into the Newton-Schulz input
             const int z = bidx / P.nblocks, blk = bidx % P.nblocks;
             const MomDesc& md = args.momd[P.apply_base + z];
-            const int wb = c32 & 1;
+            const int wb = c32 % MOM_NBUF;
             uint8_t* wbuf = slice + wb * WCH_BYTES;
             // lane 0 issued the load; all lanes wait on its barrier
             const bool okw = mbar_wait(&aux_bar[2 * ew + wb], (wph >> wb) & 1u, args.err, abort_flag);
@@ -754,7 +759,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
             }
             // U buffer wb: the store that last read it (two chunks ago) is
             // at most the fourth most recent group
-            uint8_t* ubuf = slice + 2 * WCH_BYTES + wb * CH_BYTES;
+            uint8_t* ubuf = slice + MOM_NBUF * WCH_BYTES + (c32 & 1) * CH_BYTES;
             if (lane == 0) bulk_wait_group_read3();
             __syncwarp();
             if (!md.transposed) {
@@ -782,9 +787,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::THREADS, 1
               if (!md.transposed) tma_store_3d(&md.x, ubuf, cg, rbase, 0);
               else tma_store_3d(&md.x, ubuf, rbase, cg, 0);
               bulk_commit_group();
-              // momentum chunk c32 + 2 into this buffer once its store has read it
-              const int cn = cbase + 64;
-              if (c32 + 2 < 4 && cn < P.N) {
+              // momentum chunk c32 + MOM_NBUF into this buffer once its store has read it
+              const int cn = cbase + 32 * MOM_NBUF;
+              if (c32 + MOM_NBUF < 4 && cn < P.N) {
                 bulk_wait_group_read1();
                 mbar_arrive_expect_tx(&aux_bar[2 * ew + wb], WCH_BYTES);
                 tma_load_3d(wbuf, &md.mom, &aux_bar[2 * ew + wb], blk * P.N + cn, rbase, 0);
