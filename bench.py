@@ -444,8 +444,9 @@ def main():
                          "from their owners, stage by stage, overlapping the next stage's step")
     ap.add_argument("--stages", type=int, default=2, help="slices per owner in --sharded mode")
     ap.add_argument("--overlap-adamw", action="store_true",
-                    help="run the aux AdamW on a second stream, forked from and joined into the Muon "
-                         "stream every step (per-kernel times are then taken under contention)")
+                    help="run the aux AdamW on a second, low-priority stream, forked from and joined into "
+                         "the (high-priority) Muon stream every step (per-kernel times are then taken "
+                         "under contention)")
     args = ap.parse_args()
     w, aux = workload_def(args.workload)
     if args.impl == "reference":
@@ -541,14 +542,23 @@ def main():
     ctx = mx.MuonContext(local)
     hp = mx.default_hparams()
     ahp = mx.default_adamw_hparams()
-    stream = torch.cuda.current_stream()
     # The aux AdamW runs on the Muon stream, ahead of the Muon step.  It touches
-    # none of the Muon tensors, so --overlap-adamw may run it on a second
-    # stream, forked from and joined back into the Muon stream every step; on
-    # GPT-2-small that gives the same step time (its HBM traffic competes with
-    # the momentum pass), and the per-kernel times get mixed up.
+    # none of the Muon tensors, so --overlap-adamw runs it on a second stream of
+    # the lowest priority, forked from and joined back into the Muon stream
+    # (highest priority) every step: its blocks are then scheduled only where
+    # the Muon kernels leave room (registers and HBM bandwidth beside the
+    # persistent Newton-Schulz CTAs), and the per-kernel times get mixed up.
     serial = not args.overlap_adamw
-    aux_stream = stream if serial else torch.cuda.Stream()
+    if serial:
+        stream = torch.cuda.current_stream()
+        aux_stream = stream
+    else:
+        torch.cuda.synchronize(dev)
+        stream = torch.cuda.Stream(device=dev, priority=-100)
+        aux_stream = torch.cuda.Stream(device=dev, priority=0)
+        # every other torch operation (the end-to-end staging copies) then
+        # runs in order with the Muon step
+        torch.cuda.set_stream(stream)
     fork_ev = [torch.cuda.Event() for _ in range(2)]
     join_ev = [torch.cuda.Event() for _ in range(2)]
     ctx_aux = ctx if serial else mx.MuonContext(local)
@@ -818,7 +828,7 @@ def main():
         "config": {"workload": w.name, "matrices": len(w.mats), "hidden_params": elems,
                    "aux_params": aux_el, "grad_dtype": w.grad_dtype, "ns_steps": hp.ns_steps,
                    "grad_sets_cycled": n_cycle, "l2": "inputs larger than L2 (no flush)",
-                   "aux_adamw": "same stream" if serial else "second stream, joined every step",
+                   "aux_adamw": "same stream" if serial else "second stream of the lowest priority, joined every step",
                    "parallelism": (f"owner-computes x{world}, {args.stages} exchange stages" if args.sharded
                                    else f"replicas x{world}" if world > 1 else "single")},
         "ns_tflops": ns_flops / (ns_ms * 1e-3) / 1e12 if ns_ms else None,
