@@ -443,10 +443,10 @@ def main():
                          "only the matrices muon_partition gives it, and the updated weights are broadcast "
                          "from their owners, stage by stage, overlapping the next stage's step")
     ap.add_argument("--stages", type=int, default=2, help="slices per owner in --sharded mode")
-    ap.add_argument("--overlap-adamw", action="store_true",
-                    help="run the aux AdamW on a second, low-priority stream, forked from and joined into "
-                         "the (high-priority) Muon stream every step (per-kernel times are then taken "
-                         "under contention)")
+    ap.add_argument("--serial-adamw", action="store_true",
+                    help="run the aux AdamW on the Muon stream ahead of the Muon step; by default it runs "
+                         "on a second, lowest-priority stream, forked from and joined into the "
+                         "(highest-priority) Muon stream every step")
     args = ap.parse_args()
     w, aux = workload_def(args.workload)
     if args.impl == "reference":
@@ -542,13 +542,15 @@ def main():
     ctx = mx.MuonContext(local)
     hp = mx.default_hparams()
     ahp = mx.default_adamw_hparams()
-    # The aux AdamW runs on the Muon stream, ahead of the Muon step.  It touches
-    # none of the Muon tensors, so --overlap-adamw runs it on a second stream of
-    # the lowest priority, forked from and joined back into the Muon stream
-    # (highest priority) every step: its blocks are then scheduled only where
-    # the Muon kernels leave room (registers and HBM bandwidth beside the
-    # persistent Newton-Schulz CTAs), and the per-kernel times get mixed up.
-    serial = not args.overlap_adamw
+    # The aux AdamW touches none of the Muon tensors, so it runs through a
+    # second context on a second stream of the lowest priority, forked from
+    # and joined back into the Muon stream (highest priority) every step: its
+    # blocks are scheduled only where the Muon kernels leave room (registers
+    # and HBM bandwidth beside the persistent Newton-Schulz CTAs).  The
+    # per-kernel pass below runs it on the Muon stream instead, so each
+    # kernel's time is taken without contention.  --serial-adamw runs it on the
+    # Muon stream, ahead of the Muon step, throughout.
+    serial = args.serial_adamw or not aux
     if serial:
         stream = torch.cuda.current_stream()
         aux_stream = stream
@@ -570,21 +572,25 @@ def main():
             raise SystemExit("--sharded runs plain Muon workloads")
         sm = ShardedMuon(Ws, ctx=ctx, hp=hp, stages=args.stages)
     adam_step = [0]
+    on_side = [not serial]          # AdamW on the side stream (False: on the Muon stream)
 
     def one_step(k):
         if aux:
-            fork_ev[k & 1].record(stream)
-            aux_stream.wait_event(fork_ev[k & 1])
+            side = on_side[0]
+            if side:
+                fork_ev[k & 1].record(stream)
+                aux_stream.wait_event(fork_ev[k & 1])
             adam_step[0] += 1
-            ctx_aux.adamw_step(Ps, AGs[k % n_cycle], Ms, Vs, adam_step[0], ahp, aux_stream)
-            join_ev[k & 1].record(aux_stream)
+            ctx_aux.adamw_step(Ps, AGs[k % n_cycle], Ms, Vs, adam_step[0], ahp, aux_stream if side else stream)
+            if side:
+                join_ev[k & 1].record(aux_stream)
         if newton and k % w.refresh_every == 0:
             ctx.newton_refresh(Acts, Sinv, nblk, 0.0, stream)
         if sm is not None:
             sm.step(Gs[k % n_cycle], Bs, stream)
         else:
             ctx.step(pre_groups[k % n_cycle], hp, stream)
-        if aux:
+        if aux and side:
             stream.wait_event(join_ev[k & 1])
 
     def barrier():
@@ -636,7 +642,9 @@ def main():
     ctx.profile(True)
     if ctx_aux is not ctx:
         ctx_aux.profile(True)
+    on_side[0] = False
     timed(args.steps, lambda k: one_step(args.warmup + args.steps + k))
+    on_side[0] = not serial
     kt = ctx.profile_read()
     ctx.profile(False)
     if ctx_aux is not ctx:
@@ -828,7 +836,9 @@ def main():
         "config": {"workload": w.name, "matrices": len(w.mats), "hidden_params": elems,
                    "aux_params": aux_el, "grad_dtype": w.grad_dtype, "ns_steps": hp.ns_steps,
                    "grad_sets_cycled": n_cycle, "l2": "inputs larger than L2 (no flush)",
-                   "aux_adamw": "same stream" if serial else "second stream of the lowest priority, joined every step",
+                   "aux_adamw": ("same stream" if serial else
+                                 "second stream of the lowest priority, joined every step"),
+                   "kernels_pass": "aux AdamW on the Muon stream (per-kernel times without contention)",
                    "parallelism": (f"owner-computes x{world}, {args.stages} exchange stages" if args.sharded
                                    else f"replicas x{world}" if world > 1 else "single")},
         "ns_tflops": ns_flops / (ns_ms * 1e-3) / 1e12 if ns_ms else None,
