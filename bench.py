@@ -519,13 +519,17 @@ def main():
 
     # Newton-Muon: activations per layer input, one S^-1 buffer per input
     newton = bool(w.acts)
-    Acts, Sinv, nblk = [], [], []
+    Acts, Sinv, Split, nblk = [], [], [], []
     if newton:
         for a, (_, tokens, width) in enumerate(w.acts):
             nb = 4 if width > 768 else 1
+            d = width // nb
             Acts.append(wl.torch_normal((tokens, width), 1.0, seed, 0, 20000 + a, wl.ROLE_ACT,
                                         dtype=torch.bfloat16, device=dev))
-            Sinv.append(torch.empty((nb, width // nb, width // nb), device=dev))
+            Sinv.append(torch.empty((nb, d, d), device=dev))
+            # the refresh also writes S^-1's bf16 hi/lo split, which the steps
+            # until the next refresh use as it is
+            Split.append(torch.empty((nb, 2 * d, d), dtype=torch.bfloat16, device=dev))
             nblk.append(nb)
 
     def groups_for(s):
@@ -535,6 +539,7 @@ def main():
                      momentum=[Bs[i] for i in ix])
             if newton:
                 g["precond"] = [Sinv[w.precond[w.mats[i].name][0]] for i in ix]
+                g["precond_split"] = [Split[w.precond[w.mats[i].name][0]] for i in ix]
                 g["precond_blocks"] = w.precond[w.mats[ix[0]].name][1]
             gs.append(g)
         return gs
@@ -585,7 +590,7 @@ def main():
             if side:
                 join_ev[k & 1].record(aux_stream)
         if newton and k % w.refresh_every == 0:
-            ctx.newton_refresh(Acts, Sinv, nblk, 0.0, stream)
+            ctx.newton_refresh(Acts, Sinv, nblk, 0.0, stream, splits=Split)
         if sm is not None:
             sm.step(Gs[k % n_cycle], Bs, stream)
         else:

@@ -106,7 +106,14 @@ typedef struct {
  *                d = cols / precond_blocks; the gradient is right-multiplied
  *                block-diagonally by them before momentum (Newton-Muon).
  *                Several matrices may share one S^-1 (the shared QKV
- *                estimate).  Requires grad_dtype == MUON_BF16. */
+ *                estimate).  Requires grad_dtype == MUON_BF16.
+ *   precond_split  optional (NULL = off; only read with precond, by
+ *                muon_step): precond_split[i] is the bf16 high/low split of
+ *                precond[i] that muon_newton_refresh wrote to an activation's
+ *                s_inv_split (layout there), 16-byte aligned.  The step then
+ *                uses it instead of splitting precond[i] again; the caller
+ *                keeps the two consistent (both written by the same
+ *                refresh).  Individual entries may be NULL. */
 typedef struct {
   int64_t rows;
   int64_t cols;
@@ -119,6 +126,7 @@ typedef struct {
   const float* const* precond;
   int32_t precond_blocks;
   int32_t reserved;
+  const void* const* precond_split;
 } muon_group;
 
 /* Newton-Schulz only: outputs[i] (fp32 rows x cols) = NS(inputs[i]). */
@@ -150,7 +158,12 @@ typedef struct {
 /* One activation matrix feeding a Newton-Muon refresh: acts is tokens x
  * width (act_dtype), split into nblocks column blocks of d = width / nblocks;
  * s_inv receives nblocks consecutive fp32 d x d matrices
- * (X_b^T X_b / tokens + damping I)^-1. */
+ * (X_b^T X_b / tokens + damping I)^-1.  s_inv_split, optional (NULL = off,
+ * 16-byte aligned), receives their bf16 high/low split for the tensor-core
+ * preconditioning: per block, S_hi = bf16(S^-1) as d rows of d, then S_lo =
+ * bf16(S^-1 - S_hi) as d more rows (nblocks * 2d * d bf16 in all); pass it to
+ * muon_step as the group's precond_split so that steps until the next
+ * refresh do not split S^-1 again. */
 typedef struct {
   const void* acts;
   int32_t act_dtype;               /* muon_dtype: MUON_BF16 or MUON_F32 */
@@ -158,6 +171,7 @@ typedef struct {
   int64_t tokens;
   int64_t width;
   float* s_inv;
+  void* s_inv_split;
 } muon_act_desc;
 
 typedef struct muon_ctx muon_ctx;

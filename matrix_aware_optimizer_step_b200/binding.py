@@ -62,7 +62,8 @@ class Group(ctypes.Structure):
                 ("grad_dtype", ctypes.c_int32), ("weights", ctypes.c_void_p),
                 ("grads", ctypes.c_void_p), ("momentum", ctypes.c_void_p),
                 ("update_out", ctypes.c_void_p), ("precond", ctypes.c_void_p),
-                ("precond_blocks", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+                ("precond_blocks", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("precond_split", ctypes.c_void_p)]
 
 
 class NsGroup(ctypes.Structure):
@@ -86,7 +87,8 @@ class AdamwHparams(ctypes.Structure):
 class ActDesc(ctypes.Structure):
     _fields_ = [("acts", ctypes.c_void_p), ("act_dtype", ctypes.c_int32),
                 ("nblocks", ctypes.c_int32), ("tokens", ctypes.c_int64),
-                ("width", ctypes.c_int64), ("s_inv", ctypes.c_void_p)]
+                ("width", ctypes.c_int64), ("s_inv", ctypes.c_void_p),
+                ("s_inv_split", ctypes.c_void_p)]
 
 
 class KernelTimes(ctypes.Structure):
@@ -261,8 +263,9 @@ class MuonContext:
     def make_groups(groups: Sequence[dict]):
         """Build muon_group structs from dicts with keys weights, grads,
         momentum (lists of tensors of one shape), optional update_out,
-        precond (list of S^-1 tensors) and precond_blocks.  Returns the ctypes
-        array and the objects that must stay alive during the call."""
+        precond (list of S^-1 tensors), precond_blocks and precond_split
+        (the bf16 hi/lo splits a refresh wrote for those S^-1).  Returns the
+        ctypes array and the objects that must stay alive during the call."""
         keep = []
         arr = (Group * max(1, len(groups)))()
         for i, g in enumerate(groups):
@@ -280,10 +283,14 @@ class MuonContext:
                 for t in g["precond"]:
                     if t.numel() != nb * d * d:
                         raise ValueError(f"precond: {t.numel()} elements != {nb} x {d} x {d}")
+                for t in (g.get("precond_split") or []):
+                    if t.numel() * t.element_size() != nb * 2 * d * d * 2:
+                        raise ValueError(f"precond_split: {t.numel() * t.element_size()} bytes != "
+                                         f"{nb} x 2 x {d} x {d} bf16")
             gs = arr[i]
             gs.rows, gs.cols, gs.count = rows, cols, len(grads)
             gs.grad_dtype = _dtype_code(grads[0])
-            for key in ("weights", "grads", "momentum", "update_out", "precond"):
+            for key in ("weights", "grads", "momentum", "update_out", "precond", "precond_split"):
                 ts = g.get(key)
                 if ts is None:
                     setattr(gs, key, None)
@@ -363,9 +370,11 @@ class MuonContext:
                                               _stream_ptr(stream)), "muon_adamw_step")
 
     def newton_refresh(self, acts: Sequence, s_invs: Sequence, nblocks: Sequence[int],
-                       damping: float = 0.0, stream=None):
+                       damping: float = 0.0, stream=None, splits: Optional[Sequence] = None):
         """s_invs[i] (fp32, nblocks[i] x d x d) = inverse second moments of
-        the column blocks of acts[i] (bf16 or fp32 tokens x width)."""
+        the column blocks of acts[i] (bf16 or fp32 tokens x width).  With
+        splits, splits[i] (bf16, nblocks[i] x 2d x d, or None) also receives
+        their hi/lo split, to pass to step() as a group's precond_split."""
         n = len(acts)
         arr = (ActDesc * max(1, n))()
         for i in range(n):
@@ -375,6 +384,13 @@ class MuonContext:
             arr[i].nblocks = int(nblocks[i])
             arr[i].tokens, arr[i].width = acts[i].shape
             arr[i].s_inv = s_invs[i].data_ptr()
+            sp = splits[i] if splits is not None else None
+            if sp is not None:
+                _check_cuda([sp], "newton_refresh")
+                d = arr[i].width // max(1, arr[i].nblocks)
+                if sp.numel() * sp.element_size() != arr[i].nblocks * 2 * d * d * 2:
+                    raise ValueError("newton_refresh: split buffer size")
+                arr[i].s_inv_split = sp.data_ptr()
         self._check(self._lib.muon_newton_refresh(self._ctx, arr, n, float(damping),
                                                   _stream_ptr(stream)), "muon_newton_refresh")
 

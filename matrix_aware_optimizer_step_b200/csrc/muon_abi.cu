@@ -214,6 +214,7 @@ struct Item {
   float* update_out;
   const float* precond;
   int precond_blocks;
+  const void* precond_split = nullptr;   // caller's bf16 hi/lo split of precond (muon_step)
 };
 
 // A run of matrices sharing one wide shape, inside one chunk.
@@ -952,11 +953,13 @@ muon_status collect_items(muon_ctx* ctx, const muon_group* groups, int32_t ngrou
       it.update_out = g.update_out ? g.update_out[k] : nullptr;
       it.precond = g.precond ? g.precond[k] : nullptr;
       it.precond_blocks = g.precond ? g.precond_blocks : 0;
+      it.precond_split = (for_step && g.precond && g.precond_split) ? g.precond_split[k] : nullptr;
       if (!it.grad || (for_step && (!it.weight || !it.momentum)) || (g.precond && !it.precond) ||
           (g.update_out && !it.update_out))
         return fail(ctx, MUON_ERR_INVALID_ARG, "group %d matrix %d: NULL tensor pointer", gi, k);
       if (!aligned16(it.grad) || (it.weight && !aligned16(it.weight)) || (it.momentum && !aligned16(it.momentum)) ||
-          (it.update_out && !aligned16(it.update_out)) || (it.precond && !aligned16(it.precond)))
+          (it.update_out && !aligned16(it.update_out)) || (it.precond && !aligned16(it.precond)) ||
+          (it.precond_split && !aligned16(it.precond_split)))
         return fail(ctx, MUON_ERR_INVALID_ARG, "group %d matrix %d: tensor not 16-byte aligned", gi, k);
       items.push_back(it);
     }
@@ -1031,20 +1034,26 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
           const size_t pg_bytes = round_up(size_t(it.rows) * it.cols * 4, kAlign);
           pg_off += pg_bytes;
           const int dd = int(it.cols / it.precond_blocks);
-          const StackKey key{it.precond, it.precond_blocks, dd};
-          auto f = stacks.find(key);
-          if (f == stacks.end()) {
-            PrepDesc pd{};
-            pd.s_inv = it.precond;
-            pd.sst = reinterpret_cast<__nv_bfloat16*>(ws + sst_off);
-            pd.nb = it.precond_blocks;
-            pd.d = dd;
-            sst_off += round_up(sst_bytes(it), kAlign);
-            prep.push_back(pd);
-            f = stacks.emplace(key, pd.sst).first;
+          // the caller's split from the refresh, else one split per distinct
+          // S^-1 of the chunk, staged in workspace
+          const __nv_bfloat16* sst = static_cast<const __nv_bfloat16*>(it.precond_split);
+          if (sst == nullptr) {
+            const StackKey key{it.precond, it.precond_blocks, dd};
+            auto f = stacks.find(key);
+            if (f == stacks.end()) {
+              PrepDesc pd{};
+              pd.s_inv = it.precond;
+              pd.sst = reinterpret_cast<__nv_bfloat16*>(ws + sst_off);
+              pd.nb = it.precond_blocks;
+              pd.d = dd;
+              sst_off += round_up(sst_bytes(it), kAlign);
+              prep.push_back(pd);
+              f = stacks.emplace(key, pd.sst).first;
+            }
+            sst = f->second;
           }
           PrecondMaps pm{};
-          if (!encode_precond_maps(&pm, it.grad, it.rows, it.cols, it.precond_blocks, dd, f->second))
+          if (!encode_precond_maps(&pm, it.grad, it.rows, it.cols, it.precond_blocks, dd, sst))
             return fail(ctx, MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed (precondition)");
           pmaps.push_back(pm);
           std::vector<PreProblem>& pp = chunk_pprob[ci];
@@ -1218,18 +1227,21 @@ muon_status run_items(muon_ctx* ctx, const std::vector<Item>& items, const muon_
   for (size_t ci = 0; ci < chunks.size(); ++ci) {
     const Chunk& c = chunks[ci];
     float* norm2 = reinterpret_cast<float*>(ws + c.off_norm);
-    if (chunk_prep_count[ci] > 0) {
+    if (!chunk_pprob[ci].empty()) {
       ProfScope ps(ctx, MUON_K_PRECONDITION, st);
-      int64_t most = 0;
-      for (int k = 0; k < chunk_prep_count[ci]; ++k) {
-        const PrepDesc& pd = prep[chunk_prep_begin[ci] + k];
-        most = std::max<int64_t>(most, int64_t(pd.nb) * pd.d * pd.d);
+      // split each distinct S^-1 the caller gave no split for
+      if (chunk_prep_count[ci] > 0) {
+        int64_t most = 0;
+        for (int k = 0; k < chunk_prep_count[ci]; ++k) {
+          const PrepDesc& pd = prep[chunk_prep_begin[ci] + k];
+          most = std::max<int64_t>(most, int64_t(pd.nb) * pd.d * pd.d);
+        }
+        const dim3 grid(unsigned(std::max<int64_t>(1, std::min<int64_t>(cdiv(most, 256 * 8), 512))),
+                        unsigned(chunk_prep_count[ci]));
+        launch_pdl(precond_prep_kernel, grid, dim3(256), size_t(0), st, dprep + chunk_prep_begin[ci]);
+        ctx->launches++;
+        CUDA_TRY(ctx, cudaGetLastError());
       }
-      const dim3 grid(unsigned(std::max<int64_t>(1, std::min<int64_t>(cdiv(most, 256 * 8), 512))),
-                      unsigned(chunk_prep_count[ci]));
-      launch_pdl(precond_prep_kernel, grid, dim3(256), size_t(0), st, dprep + chunk_prep_begin[ci]);
-      ctx->launches++;
-      CUDA_TRY(ctx, cudaGetLastError());
       s = run_precondition(ctx, chunk_pprob[ci],
                            reinterpret_cast<const PrecondMaps*>(static_cast<uint8_t*>(dtab) + pm_off), skip, st,
                            reinterpret_cast<const MomDesc*>(static_cast<uint8_t*>(dtab) + md_off), hp->momentum,
@@ -1639,6 +1651,7 @@ muon_status muon_newton_refresh(muon_ctx* ctx, const muon_act_desc* acts, int32_
   size_t s_total = 0, xt_total = 0;
   int max_d = 0;
   int64_t max_tiles = 0, max_split_tiles = 0;
+  std::vector<PrepDesc> splits;     // S^-1 to split into the caller's hi/lo stacks
   // activations of one (dtype, tokens, d, nblocks) next to each other, so
   // each shape is one batched problem of the second-moment product
   std::vector<int> order(n);
@@ -1659,8 +1672,16 @@ muon_status muon_newton_refresh(muon_ctx* ctx, const muon_act_desc* acts, int32_
     const int64_t d = a.width / a.nblocks;
     if (d > CHOL_MAX_D)
       return fail(ctx, MUON_ERR_UNSUPPORTED, "activation %d: block width %lld > %d", i, (long long)d, CHOL_MAX_D);
-    if (!aligned16(a.acts) || !aligned16(a.s_inv))
+    if (!aligned16(a.acts) || !aligned16(a.s_inv) || (a.s_inv_split && !aligned16(a.s_inv_split)))
       return fail(ctx, MUON_ERR_INVALID_ARG, "activation %d: not 16-byte aligned", i);
+    if (a.s_inv_split) {
+      PrepDesc pd{};
+      pd.s_inv = a.s_inv;
+      pd.sst = static_cast<__nv_bfloat16*>(a.s_inv_split);
+      pd.nb = a.nblocks;
+      pd.d = int(d);
+      splits.push_back(pd);
+    }
     const bool split = a.act_dtype == MUON_F32;
     if (split && 3 * a.tokens > INT32_MAX)
       return fail(ctx, MUON_ERR_UNSUPPORTED, "activation %d: too many tokens", i);
@@ -1754,17 +1775,32 @@ muon_status muon_newton_refresh(muon_ctx* ctx, const muon_act_desc* acts, int32_
   const size_t ab_bytes = round_up(ab.size() * sizeof(ActBlock), kAlign);
   const size_t sb_off = round_up(ab_bytes + cd.size() * sizeof(CholDesc), kAlign);
   const size_t pm_off = round_up(sb_off + sbk.size() * sizeof(ActSplitBlock), kAlign);
-  std::vector<uint8_t> table(pm_off + pmaps.size() * sizeof(PrecondMaps));
+  const size_t sp_off = round_up(pm_off + pmaps.size() * sizeof(PrecondMaps), kAlign);
+  std::vector<uint8_t> table(sp_off + splits.size() * sizeof(PrepDesc));
   if (!ab.empty()) std::memcpy(table.data(), ab.data(), ab.size() * sizeof(ActBlock));
   std::memcpy(table.data() + ab_bytes, cd.data(), cd.size() * sizeof(CholDesc));
   if (!sbk.empty()) std::memcpy(table.data() + sb_off, sbk.data(), sbk.size() * sizeof(ActSplitBlock));
   if (!pmaps.empty()) std::memcpy(table.data() + pm_off, pmaps.data(), pmaps.size() * sizeof(PrecondMaps));
+  if (!splits.empty()) std::memcpy(table.data() + sp_off, splits.data(), splits.size() * sizeof(PrepDesc));
   void* dtab = nullptr;
   s = upload_table(ctx, table.data(), table.size(), st, &dtab);
   if (s != MUON_OK) return s;
   const ActBlock* dab = static_cast<const ActBlock*>(dtab);
   const CholDesc* dc = reinterpret_cast<const CholDesc*>(static_cast<uint8_t*>(dtab) + ab_bytes);
   const ActSplitBlock* dsb = reinterpret_cast<const ActSplitBlock*>(static_cast<uint8_t*>(dtab) + sb_off);
+  // after S^-1 is written: the hi/lo splits the caller asked for
+  auto emit_splits = [&]() -> muon_status {
+    if (splits.empty()) return MUON_OK;
+    int64_t most = 0;
+    for (const PrepDesc& pd : splits) most = std::max<int64_t>(most, int64_t(pd.nb) * pd.d * pd.d);
+    const dim3 grid(unsigned(std::max<int64_t>(1, std::min<int64_t>(cdiv(most, 256 * 8), 512))),
+                    unsigned(splits.size()));
+    launch_pdl(precond_prep_kernel, grid, dim3(256), size_t(0), st,
+               reinterpret_cast<const PrepDesc*>(static_cast<uint8_t*>(dtab) + sp_off));
+    ctx->launches++;
+    CUDA_TRY(ctx, cudaGetLastError());
+    return MUON_OK;
+  };
   ProfScope ps(ctx, MUON_K_NEWTON_REFRESH, st);
   if (!ab.empty()) {
     launch_pdl(act_transpose_kernel, dim3(unsigned(max_tiles), unsigned(ab.size())), dim3(256), size_t(0), st, dab);
@@ -1871,7 +1907,7 @@ muon_status muon_newton_refresh(muon_ctx* ctx, const muon_act_desc* acts, int32_
                dim3(256), size_t(0), st, dc);
     ctx->launches++;
     CUDA_TRY(ctx, cudaGetLastError());
-    return MUON_OK;
+    return emit_splits();
   }
   cholesky_kernel<<<unsigned(cd.size()), CHOL_THREADS, 0, st>>>(dc, damping, ctx->dflags);
   ctx->launches++;
@@ -1880,7 +1916,7 @@ muon_status muon_newton_refresh(muon_ctx* ctx, const muon_act_desc* acts, int32_
   chol_solve_kernel<<<unsigned(cd.size() * parts), SOLVE_THREADS, 0, st>>>(dc, parts);
   ctx->launches++;
   CUDA_TRY(ctx, cudaGetLastError());
-  return MUON_OK;
+  return emit_splits();
 }
 
 muon_status muon_check_device(muon_ctx* ctx) {

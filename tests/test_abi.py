@@ -175,3 +175,39 @@ def test_product_path_does_not_touch_the_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
                 src = open(os.path.join(dirpath, f)).read()
                 assert "oracle" not in src.lower(), f
+
+
+def test_binding_structs_match_the_header(tmp_path):
+    """Every ctypes struct of the binding has the size and field offsets the
+    C compiler gives the matching struct of include/muon.h (a host program
+    built with gcc prints them; no GPU involved)."""
+    import ctypes
+    import shutil
+    import subprocess
+    from matrix_aware_optimizer_step_b200 import binding as b
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    pairs = {"muon_hparams": b.Hparams, "muon_group": b.Group, "muon_ns_group": b.NsGroup,
+             "muon_adamw_tensor": b.AdamwTensor, "muon_adamw_hparams": b.AdamwHparams,
+             "muon_act_desc": b.ActDesc, "muon_kernel_times": b.KernelTimes}
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "muon.h"', "int main(void) {"]
+    for cname, cls in pairs.items():
+        lines.append(f'  printf("{cname} size %zu\\n", sizeof({cname}));')
+        for fname, _ in cls._fields_:
+            lines.append(f'  printf("{cname} {fname} %zu\\n", offsetof({cname}, {fname}));')
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    inc = os.path.join(ROOT, "include")
+    subprocess.run(["gcc", "-std=c99", "-I", inc, str(src), "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split("\n")
+    got = {}
+    for ln in out:
+        if ln:
+            parts = ln.split()
+            got[(parts[0], parts[1])] = int(parts[2])
+    for cname, cls in pairs.items():
+        assert got[(cname, "size")] == ctypes.sizeof(cls), cname
+        for fname, _ in cls._fields_:
+            assert got[(cname, fname)] == getattr(cls, fname).offset, (cname, fname)

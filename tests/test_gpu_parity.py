@@ -741,3 +741,52 @@ def test_newton_momentum_in_preconditioning_epilogue_edges(ctx, mx):
             bufs[i] = nb_
             assert rel_fro(to_np(bt[i]), nb_) < NEWTON_TOL, (s, step)
             assert rel_fro(to_np(ot[i]), oracle.newton_schulz(u, 5)) < ns_tol(s), (s, step)
+
+
+def test_newton_refresh_writes_split_and_step_uses_it(ctx, mx):
+    """A refresh asked for the bf16 hi/lo split of each S^-1 writes exactly
+    S_hi = bf16(S^-1) and S_lo = bf16(S^-1 - S_hi), block by block; a step
+    given that split as precond_split is bit-identical to one that splits
+    S^-1 itself (weights and momentum), over two steps, for a one-block and a
+    four-block preconditioner shared by several matrices."""
+    tokens = 2048
+    specs = [(768, 1), (512, 4)]
+    acts, sinv, splits, nblk = [], [], [], []
+    for a, (width, nb) in enumerate(specs):
+        d = width // nb
+        acts.append(dev(wl.bf16_round_np(wl.np_normal((tokens, width), 1.0, seed=35, index=a, role=wl.ROLE_ACT)),
+                        torch.bfloat16))
+        sinv.append(torch.empty((nb, d, d), device="cuda"))
+        splits.append(torch.empty((nb, 2 * d, d), dtype=torch.bfloat16, device="cuda"))
+        nblk.append(nb)
+    ctx.newton_refresh(acts, sinv, nblk, splits=splits)
+    torch.cuda.synchronize()
+    ctx.check_device()
+    for s, sp, (width, nb) in zip(sinv, splits, specs):
+        d = width // nb
+        hi = s.to(torch.bfloat16)
+        lo = (s - hi.float()).to(torch.bfloat16)
+        assert torch.equal(sp[:, :d, :], hi)
+        assert torch.equal(sp[:, d:, :], lo)
+    shapes = [(768, 768), (768, 768), (1024, 768), (640, 512)]
+    use = [0, 0, 0, 1]
+    w0 = [dev(wl.np_normal(s, 0.02, seed=35, index=i, role=wl.ROLE_WEIGHT)) for i, s in enumerate(shapes)]
+    wa, wb = [t.clone() for t in w0], [t.clone() for t in w0]
+    ba, bb = [torch.zeros(s, device="cuda") for s in shapes], [torch.zeros(s, device="cuda") for s in shapes]
+    for step in range(2):
+        gt = [dev(wl.bf16_round_np(wl.np_normal(s, 1e-3, seed=35, step=step, index=i)), torch.bfloat16)
+              for i, s in enumerate(shapes)]
+        for w, bufs, with_split in ((wa, ba, False), (wb, bb, True)):
+            groups = []
+            for i, s in enumerate(shapes):
+                g = dict(weights=[w[i]], grads=[gt[i]], momentum=[bufs[i]], precond=[sinv[use[i]]],
+                         precond_blocks=nblk[use[i]])
+                if with_split:
+                    g["precond_split"] = [splits[use[i]]]
+                groups.append(g)
+            ctx.step(groups)
+        torch.cuda.synchronize()
+        ctx.check_device()
+        for i in range(len(shapes)):
+            assert torch.equal(ba[i], bb[i]), (shapes[i], step)
+            assert torch.equal(wa[i], wb[i]), (shapes[i], step)
