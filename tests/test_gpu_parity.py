@@ -55,6 +55,37 @@ def test_orthogonalize_vs_oracle(ctx, shape, dtype):
     assert err < ns_tol(shape), f"{shape} {dtype}: {err}"
 
 
+@pytest.mark.parametrize("case", [((3072, 768), "f32"), ((3072, 768), "bf16"), ((1000, 336), "f32"),
+                                  ((520, 264), "bf16"), ((264, 520), "f32")],
+                         ids=lambda c: f"{c[0][0]}x{c[0][1]}-{c[1]}")
+def test_orthogonalize_zero_steps_exact_layout(ctx, mx, case):
+    """With no iteration the output is U / (||U||_F + eps) where U is stored
+    in bf16 in the wide layout and read back.  Element for element it is the
+    bf16-rounded input times one scale, so a misplaced element of the layout
+    write (transposing for the tall shapes, whole and ragged tiles) fails
+    here even where the Newton-Schulz tolerance could absorb it."""
+    shape, dt = case
+    x = wl.np_normal(shape, 1.0, seed=10, index=shape[0]).astype(np.float32)
+    if dt == "bf16":
+        x = wl.bf16_round_np(x)
+    out = torch.empty(shape, dtype=torch.float32, device="cuda")
+    ctx.orthogonalize([dev(x, torch.bfloat16 if dt == "bf16" else torch.float32)], [out],
+                      mx.default_hparams(ns_steps=0))
+    torch.cuda.synchronize()
+    ctx.check_device()
+    want = wl.bf16_round_np(x).astype(np.float64) / (np.linalg.norm(x.astype(np.float64)) + oracle.NS_EPS)
+    got = to_np(out)
+    assert np.max(np.abs(got - want)) <= 1e-5 * np.max(np.abs(want)), shape
+
+
+def test_step_tall_f32_gradients(ctx, mx):
+    """fp32 gradients on tall matrices past the single-launch size (whole
+    and ragged 64 x 64 tiles), two steps, with and without Nesterov."""
+    shapes = [(1000, 336), (3072, 768), (520, 264)]
+    _step_case(ctx, mx, shapes, 2, "f32")
+    _step_case(ctx, mx, shapes, 2, "f32", hp_over=dict(nesterov=0), seed=1)
+
+
 def test_orthogonalize_batched_groups(ctx):
     """Many matrices of mixed shapes in one call: every one matches."""
     shapes = [(384, 384)] * 5 + [(384, 1536)] * 3 + [(1536, 384)] * 3 + [(64, 64)] * 7
