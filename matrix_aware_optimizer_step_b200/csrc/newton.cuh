@@ -149,6 +149,7 @@ __global__ void __launch_bounds__(CP_THREADS)
   __shared__ float dg[CB][CBP];
   __shared__ float dinv[CB][CBP];
   __shared__ float ap[CPR][CBP];
+  __shared__ float rdiag[CB];                          // 1 / L_ii of D
   __shared__ int bad;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid == 0) bad = 0;
@@ -165,7 +166,11 @@ __global__ void __launch_bounds__(CP_THREADS)
   __syncthreads();
   if (warp == 0) {
     // unblocked Cholesky of D in registers: lane i holds row i (zero above
-    // the diagonal and past nb); column k travels by shuffle
+    // the diagonal and past nb); column k travels by shuffle.  This warp's
+    // serial chain is the panel launch's critical path, so the pivot's
+    // reciprocal square root q (rsqrtf, within 2 ulp) gives both L_kk =
+    // a_kk q and the column scaling by one multiply each, and the
+    // inverse below multiplies by the stored q instead of dividing.
     float a[CB];
 #pragma unroll
     for (int j = 0; j < CB; ++j) a[j] = dg[lane][j];
@@ -175,9 +180,9 @@ __global__ void __launch_bounds__(CP_THREADS)
       if (k < nb) {
         float akk = __shfl_sync(0xffffffffu, a[k], k);
         if (!(akk > 0.f)) { neg = true; akk = 1.f; }
-        const float lkk = sqrtf(akk);
-        if (lane == k) a[k] = lkk;
-        else if (lane > k) a[k] = a[k] / lkk;
+        const float q = rsqrtf(akk);
+        if (lane == k) { a[k] = akk * q; rdiag[k] = q; }
+        else if (lane > k) a[k] *= q;
         const float lik = a[k];
 #pragma unroll
         for (int j = k + 1; j < CB; ++j) {
@@ -190,14 +195,23 @@ __global__ void __launch_bounds__(CP_THREADS)
 #pragma unroll
     for (int j = 0; j < CB; ++j) dg[lane][j] = a[j];
     __syncwarp();
-    // D x = e_lane: x = column `lane` of D^-1
+    // D x = e_lane: x = column `lane` of D^-1, forward substitution with
+    // four independent partial sums per row (the chain of dependent adds is
+    // a quarter as long)
     float x[CB];
 #pragma unroll
     for (int i = 0; i < CB; ++i) {
-      float sum = (i == lane) ? 1.f : 0.f;
+      float s0 = (i == lane) ? 1.f : 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
 #pragma unroll
-      for (int k = 0; k < i; ++k) sum -= dg[i][k] * x[k];
-      x[i] = (i < nb) ? sum / dg[i][i] : 0.f;
+      for (int k = 0; k + 3 < i; k += 4) {
+        s0 -= dg[i][k] * x[k];
+        s1 -= dg[i][k + 1] * x[k + 1];
+        s2 -= dg[i][k + 2] * x[k + 2];
+        s3 -= dg[i][k + 3] * x[k + 3];
+      }
+#pragma unroll
+      for (int k = i & ~3; k < i; ++k) s0 -= dg[i][k] * x[k];
+      x[i] = (i < nb) ? ((s0 + s1) + (s2 + s3)) * rdiag[i] : 0.f;
     }
 #pragma unroll
     for (int i = 0; i < CB; ++i) dinv[i][lane] = x[i];
@@ -330,10 +344,34 @@ __global__ void __launch_bounds__(256) linv_init_kernel(const CholDesc* __restri
   }
 }
 
+// 8x8 register tile of a 64x64 output tile over 64 threads: thread (ty, tx)
+// owns rows {4ty .. 4ty+3, 32+4ty .. 32+4ty+3} and the same columns with tx,
+// so each 16-byte shared-memory load of a warp reads contiguous bytes, and a
+// thread issues 64 FMAs per four loads (a 4x4 tile over 256 threads issues
+// 16 per two, which leaves the FMA pipes waiting on shared memory).
+__device__ __forceinline__ int rc8(int t, int u) { return (u < 4) ? t * 4 + u : 32 + t * 4 + (u - 4); }
+
+template <int LD>
+__device__ __forceinline__ void fma_tile8(const float (*xs)[LD], const float (*ys)[LD], int kk, int ty, int tx,
+                                          float (&acc)[8][8]) {
+  const float4 x0 = *reinterpret_cast<const float4*>(&xs[kk][ty * 4]);
+  const float4 x1 = *reinterpret_cast<const float4*>(&xs[kk][32 + ty * 4]);
+  const float4 y0 = *reinterpret_cast<const float4*>(&ys[kk][tx * 4]);
+  const float4 y1 = *reinterpret_cast<const float4*>(&ys[kk][32 + tx * 4]);
+  const float xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+  const float yv[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
+#pragma unroll
+  for (int u = 0; u < 8; ++u)
+#pragma unroll
+    for (int v = 0; v < 8; ++v) acc[u][v] += xv[u] * yv[v];
+}
+
 // One product of a doubling level (grid.x: pair x output tile, grid.y:
-// matrix), 64x64 output tiles, 4x4 per thread, K staged 32 at a time.
-// mode 0: T = C A^-1, mode 1: X21 = -B^-1 T.
-constexpr int LV_T = 64, LV_K = 32, LV_THREADS = 256;
+// matrix), 64x64 output tiles, 8x8 per thread, K staged 32 at a time.
+// mode 0: T = C A^-1, mode 1: X21 = -B^-1 T.  Each output is summed over k
+// in increasing order, one FMA per k, whatever the register tiling.
+constexpr int LV_T = 64, LV_K = 32, LV_THREADS = 64;
+constexpr int LV_LOADS = LV_T * LV_K / 4 / LV_THREADS;   // 16-byte loads per thread per panel
 __global__ void __launch_bounds__(LV_THREADS) linv_level_kernel(const CholDesc* __restrict__ descs, int s, int mode) {
   pdl_wait();      // previous kernel's results visible (no-op without PDL)
   const CholDesc& c = descs[blockIdx.y];
@@ -357,39 +395,67 @@ __global__ void __launch_bounds__(LV_THREADS) linv_level_kernel(const CholDesc* 
   float* O = mode == 0 ? c.t + int64_t(r0 + s) * d + r0 : c.inv + int64_t(r0 + s) * d + r0;
   const int kdim = mode == 0 ? s : s2;                    // valid k of the operands
   __shared__ __align__(16) float ps[LV_K][LV_T + 4];     // P transposed: ps[k][i]
-  __shared__ __align__(16) float qs[LV_K][LV_T];
-  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
-  float acc[4][4] = {};
+  __shared__ __align__(16) float qs[LV_K][LV_T + 4];
+  const int tid = threadIdx.x, ty = tid >> 3, tx = tid & 7;
+  float acc[8][8] = {};
+  // 16-byte loads need rows that start 16-byte aligned; every operand view
+  // starts at a column that is a multiple of 32
+  const bool vec = (d % 4) == 0;
+  const int klim = min(khi, kdim);
+  // The next panel pair is loaded into registers while this one is
+  // multiplied: each thread issues its 16 loads (16 bytes each) together,
+  // one latency per panel, hidden behind 2048 FMAs.  Loaded one element at a
+  // time into shared memory, with 64 accumulators per thread, the compiler
+  // spaced the loads out and exposed each one's latency (measured 2.5x
+  // slower at the same instruction count).
+  float4 pv[LV_LOADS], qv[LV_LOADS];
+  auto load = [&](int k0) {
+#pragma unroll
+    for (int n = 0; n < LV_LOADS; ++n) {
+      const int e = tid + n * LV_THREADS;
+      const int i = e >> 3, k4 = (e & 7) * 4;             // P: row i, k4 .. k4 + 3 of the panel
+      const int gi = i0 + i, gk = k0 + k4;
+      if (vec && gi < s2 && gk + 3 < klim) {
+        pv[n] = *reinterpret_cast<const float4*>(P + int64_t(gi) * d + gk);
+      } else {
+        float* pp = reinterpret_cast<float*>(&pv[n]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) pp[c] = (gi < s2 && gk + c < klim) ? P[int64_t(gi) * d + gk + c] : 0.f;
+      }
+      const int qk = e >> 4, qj4 = (e & 15) * 4;          // Q: row qk, columns qj4 .. qj4 + 3
+      const int hk = k0 + qk, hj = j0 + qj4;
+      if (vec && hk < klim && hj + 3 < s) {
+        qv[n] = *reinterpret_cast<const float4*>(Q + int64_t(hk) * d + hj);
+      } else {
+        float* qq = reinterpret_cast<float*>(&qv[n]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) qq[c] = (hk < klim && hj + c < s) ? Q[int64_t(hk) * d + hj + c] : 0.f;
+      }
+    }
+  };
+  if (klo < khi) load(klo);
   for (int k0 = klo; k0 < khi; k0 += LV_K) {
-    for (int e = tid; e < LV_T * LV_K; e += LV_THREADS) {
-      const int i = e >> 5, k = e & 31;                   // P: 32 consecutive k per row
-      const int gi = i0 + i, gk = k0 + k;
-      ps[k][i] = (gi < s2 && gk < khi && gk < kdim) ? P[int64_t(gi) * d + gk] : 0.f;
-      const int qk = e >> 6, qj = e & 63;                 // Q: 64 consecutive j per row
-      const int hk = k0 + qk, hj = j0 + qj;
-      qs[qk][qj] = (hk < khi && hk < kdim && hj < s) ? Q[int64_t(hk) * d + hj] : 0.f;
+#pragma unroll
+    for (int n = 0; n < LV_LOADS; ++n) {
+      const int e = tid + n * LV_THREADS;
+      const int i = e >> 3, k4 = (e & 7) * 4;
+      ps[k4][i] = pv[n].x; ps[k4 + 1][i] = pv[n].y; ps[k4 + 2][i] = pv[n].z; ps[k4 + 3][i] = pv[n].w;
+      *reinterpret_cast<float4*>(&qs[e >> 4][(e & 15) * 4]) = qv[n];
     }
     __syncthreads();
-#pragma unroll 8
-    for (int kk = 0; kk < LV_K; ++kk) {
-      const float4 a = *reinterpret_cast<const float4*>(&ps[kk][ty * 4]);
-      const float4 b = *reinterpret_cast<const float4*>(&qs[kk][tx * 4]);
-      const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-#pragma unroll
-        for (int v = 0; v < 4; ++v) acc[u][v] += av[u] * bv[v];
-    }
+    if (k0 + LV_K < khi) load(k0 + LV_K);
+#pragma unroll 4
+    for (int kk = 0; kk < LV_K; ++kk) fma_tile8<LV_T + 4>(ps, qs, kk, ty, tx, acc);
     __syncthreads();
   }
   const float sign = mode == 0 ? 1.f : -1.f;
 #pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const int i = i0 + ty * 4 + u;
+  for (int u = 0; u < 8; ++u) {
+    const int i = i0 + rc8(ty, u);
     if (i >= s2) continue;
 #pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      const int j = j0 + tx * 4 + v;
+    for (int v = 0; v < 8; ++v) {
+      const int j = j0 + rc8(tx, v);
       if (j < s) O[int64_t(i) * d + j] = sign * acc[u][v];
     }
   }
