@@ -655,14 +655,18 @@ def test_newton_precondition_rejects_bad_arguments(ctx, mx):
     assert torch.all(o == 7.0)
 
 
-@pytest.mark.parametrize("case", [[((1001, 256), 2)], [((1001, 100), 1)], [((640, 90), 2), ((512, 128), 1)]],
-                         ids=["in-place-ragged-tokens", "transposed-width-100", "transposed-odd-block-then-even"])
+@pytest.mark.parametrize("case", [[((1001, 256), 2)], [((1001, 100), 1)], [((640, 90), 2), ((512, 128), 1)],
+                                  [((1500, 301), 1)]],
+                         ids=["in-place-ragged-tokens", "transposed-width-100", "transposed-odd-block-then-even",
+                              "odd-width-301"])
 def test_newton_refresh_paths(ctx, mx, case):
     """The second moment read in place (widths multiples of 8, here with a
     token count that is not) and through transposed copies (a width or block
     width that is not a multiple of 8; an odd block width followed, in the
     same call, by a block whose kernels take 16-byte vector paths) all match
-    the oracle."""
+    the oracle.  Width 301 runs doubling levels of 32, 64, 128 and 256 rows
+    (ragged second blocks of 13 and 45 rows) on the element-by-element load
+    paths of the inverse's kernels."""
     acts, outs = [], []
     for k, (shape, nb) in enumerate(case):
         a = wl.bf16_round_np(wl.np_normal(shape, 1.0, seed=16, index=shape[1] + k, role=wl.ROLE_ACT))
